@@ -1,0 +1,179 @@
+/*
+ * Lean-P / power-of-two block-scale emulator, plain C, bit level.
+ * TEST INFRASTRUCTURE ONLY (see oracle/__init__.py): only the tests, the smoke check and
+ * the bench's CPU-baseline leg load this file's library.  It shares no code with the CUDA
+ * path and includes nothing from it.
+ *
+ * What the pages say ([ZYFA-mb] "Como o motor de atenção FP8 da Zyphra funciona";
+ * [ZYFA-pt] "Como o ZYFA funciona?", cut off at the first technique; [ZYFA-fr] "Ce que
+ * couvrent les noyaux"):
+ *   - each FP8 probability is produced by one multiply-add and one integer conversion
+ *     that yields the FP8 bit pattern, exploiting the bit structure of the format, with
+ *     no exponential;
+ *   - each 64-key block is scaled by a power of two before the FP8 rounding, and the
+ *     scaled matrix instruction removes that factor;
+ *   - the row normaliser is the sum of the *rounded* probabilities, formed by one extra
+ *     matrix instruction per block.
+ *
+ * Reading (the plainest one the pages support; all arithmetic float32 with one rounding
+ * per operation, fmaf = fused multiply-add with a single rounding):
+ *   The e4m3 code n = 8e + m (exponent field e, mantissa m) decodes to about
+ *   2^(n/8 - 7) (the logarithm of 1 + m/8 taken as m/8: Mitchell 1962), so the code
+ *   of 2^y is about 8 (y + 7) -- linear in y, which is linear in the score.  With
+ *   a = 8 log2(e) * scale * dq * dk (byte units per raw score unit), per row:
+ *     m      running maximum in byte units, an integer:
+ *            m <- max(m, ceil(float32(a * mu_tile)))   mu_tile = tile max of raw scores
+ *     k_b    per 64-key block b with block max mu_b:
+ *            t = fmaf(mu_b, a, -m);  k_b = clamp(floor(-t / 8), 0, KMAX)
+ *            (the block maximum lands in code range (112, 120], i.e. value 2^7..2^8)
+ *     code   r = fmaf(s, a, MAGIC + (120 + 8 k_b - m)),  MAGIC = 1.5 * 2^23
+ *            (the single rounding of the fma at magnitude 2^23 is the round-to-nearest-
+ *            even integer conversion: the low bits of r hold the integer), then
+ *            byte = low 8 bits of max(r, MAGIC)   (negative codes clamp to 0)
+ *     value  decode(byte) ~ 2^((a s - m)/8) * 2^(8 + k_b); the matrix instruction
+ *            applies 2^-(8 + k_b) per (row, 64-key block) through UE8M0 scale factors
+ *     l      l <- alpha l + sum_j decode(byte_j) 2^-(8+k_b(j));   O likewise with v_j
+ *     alpha  2^((m_old - m_new)/8) when m grows (0 on the first tile)
+ *   final:   o = O * dv / l,  lse = ln 2 * (m / 8 + log2 l)
+ * Masked scores are -inf: their code is 0.  A fully masked block gets k_b = KMAX (its
+ * codes are all 0, so its scale multiplies zeros).
+ *
+ * Build: gcc -O2 -ffp-contract=off -fno-fast-math -shared -fPIC (every a*b+c here is
+ * written as the operation it is; the compiler must not fuse or reorder them).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#define LEANP_MAGIC 12582912.0f /* 1.5 * 2^23 */
+
+/* ---- e4m3fn decode by the format definition (independent of the Python codec) ---- */
+double leanp_e4m3_decode(uint8_t c) {
+    int e = (c >> 3) & 15, m = c & 7;
+    double mag;
+    if ((c & 0x7F) == 0x7F) return NAN;
+    if (e == 0) mag = ldexp((double)m, -9);
+    else mag = ldexp(1.0 + m / 8.0, e - 7);
+    return (c & 0x80) ? -mag : mag;
+}
+
+/* exposed for the tests' exact-rounding pin */
+float leanp_fmaf(float x, float y, float z) { return fmaf(x, y, z); }
+
+/* running max in byte units after seeing a tile whose raw-score maximum is mu_tile */
+int leanp_update_max(float mu_tile, float a, int m_old, int m_valid) {
+    if (isinf(mu_tile) && mu_tile < 0) return m_old;  /* no visible key in the tile */
+    float prod = a * mu_tile;                          /* one float32 rounding */
+    int cand = (int)ceilf(prod);
+    if (!m_valid) return cand;
+    return cand > m_old ? cand : m_old;
+}
+
+/* power-of-two shift of one 64-key block */
+int leanp_kshift(float mu_b, float a, int m, int kmax) {
+    if (isinf(mu_b) && mu_b < 0) return kmax;          /* fully masked block */
+    float t = fmaf(mu_b, a, -(float)m);
+    float g = -t * 0.125f;                             /* exact */
+    if (g >= (float)kmax) return kmax;
+    float f = floorf(g);
+    if (f <= 0.0f) return 0;
+    return (int)f;
+}
+
+/* code of one score given the block constant */
+uint8_t leanp_code(float s, float a, int m, int kb) {
+    float c = LEANP_MAGIC + (float)(120 + 8 * kb - m); /* exact: small integers */
+    float r = fmaf(s, a, c);
+    r = fmaxf(r, LEANP_MAGIC);
+    uint32_t bits;
+    memcpy(&bits, &r, 4);
+    return (uint8_t)(bits & 0xFF);
+}
+
+/*
+ * Encode one row of one key tile.  s: n raw scores (n a multiple of 64, -inf = masked),
+ * m: the running max already updated with this tile.  Writes n codes and n/64 shifts.
+ */
+void leanp_encode_row_tile(const float* s, int n, float a, int m, int kmax,
+                           uint8_t* codes, uint8_t* kshift) {
+    for (int b = 0; b < n / 64; ++b) {
+        float mu = -INFINITY;
+        for (int j = 0; j < 64; ++j) mu = fmaxf(mu, s[b * 64 + j]);
+        int kb = leanp_kshift(mu, a, m, kmax);
+        kshift[b] = (uint8_t)kb;
+        for (int j = 0; j < 64; ++j) codes[b * 64 + j] = leanp_code(s[b * 64 + j], a, m, kb);
+    }
+}
+
+/*
+ * Replay the kernel's per-row state machine over a row of raw scores, tile by tile in
+ * ascending key order, and return codes, shifts and the reference max used per tile.
+ *   s       [ntiles * tile] raw scores of one query row (-inf where masked)
+ *   codes   [ntiles * tile] out, kshift [ntiles * tile / 64] out, mref [ntiles] out
+ * Tiles with no visible key are skipped (their codes are 0 and shifts KMAX).
+ */
+void leanp_encode_row(const float* s, int ntiles, int tile, float a, int kmax,
+                      uint8_t* codes, uint8_t* kshift, int* mref) {
+    int m = 0, m_valid = 0;
+    for (int t = 0; t < ntiles; ++t) {
+        const float* st = s + (size_t)t * tile;
+        float mu = -INFINITY;
+        for (int j = 0; j < tile; ++j) mu = fmaxf(mu, st[j]);
+        m = leanp_update_max(mu, a, m, m_valid);
+        if (!(isinf(mu) && mu < 0)) m_valid = 1;
+        mref[t] = m_valid ? m : 0;
+        if (!m_valid) {
+            memset(codes + (size_t)t * tile, 0, tile);
+            for (int b = 0; b < tile / 64; ++b) kshift[(size_t)t * tile / 64 + b] = (uint8_t)kmax;
+            continue;
+        }
+        leanp_encode_row_tile(st, tile, a, m, kmax, codes + (size_t)t * tile,
+                              kshift + (size_t)t * tile / 64);
+    }
+}
+
+/*
+ * End-to-end tile driver for one query row: from the row's raw scores (float32) and the
+ * value rows (float64, already dequantised), the lean-P output row and lse.
+ *   s [S_k] raw scores (-inf masked), v [S_k * dv] dequantised values (row-major),
+ *   scale_nat = softmax scale * dq * dk (natural units per raw score unit) for lse.
+ * The products and sums of this step are formed in float64 (the tensor core's float32
+ * accumulation order is not specified), so this predicts the kernel within float32
+ * accumulation error, not bit for bit.
+ */
+void leanp_attention_row(const float* s, int S_k, int tile, const double* v, int dv,
+                         float a, int kmax, double* o_out, double* lse_out) {
+    int ntiles = (S_k + tile - 1) / tile;
+    double acc[1024];
+    double l = 0.0;
+    int m = 0, m_valid = 0;
+    float buf[512];
+    uint8_t codes[512], ks[8];
+    for (int d = 0; d < dv; ++d) acc[d] = 0.0;
+    for (int t = 0; t < ntiles; ++t) {
+        int n = tile;
+        for (int j = 0; j < n; ++j) {
+            int key = t * tile + j;
+            buf[j] = key < S_k ? s[key] : -INFINITY;
+        }
+        float mu = -INFINITY;
+        for (int j = 0; j < n; ++j) mu = fmaxf(mu, buf[j]);
+        if (isinf(mu) && mu < 0) continue;
+        int m_new = leanp_update_max(mu, a, m, m_valid);
+        double alpha = m_valid ? exp2((double)(m - m_new) / 8.0) : 0.0;
+        m = m_new;
+        m_valid = 1;
+        leanp_encode_row_tile(buf, n, a, m, kmax, codes, ks);
+        l *= alpha;
+        for (int d = 0; d < dv; ++d) acc[d] *= alpha;
+        for (int j = 0; j < n; ++j) {
+            int key = t * tile + j;
+            if (key >= S_k || codes[j] == 0) continue;
+            double w = leanp_e4m3_decode(codes[j]) * ldexp(1.0, -(8 + ks[j / 64]));
+            l += w;
+            for (int d = 0; d < dv; ++d) acc[d] += w * v[(size_t)key * dv + d];
+        }
+    }
+    for (int d = 0; d < dv; ++d) o_out[d] = acc[d] / l;
+    *lse_out = log(2.0) * ((double)m / 8.0 + log2(l));
+}

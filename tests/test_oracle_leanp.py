@@ -1,0 +1,141 @@
+"""Pins of the lean-P emulator: exact rounding, closed forms, the Mitchell bound,
+monotonicity, and the end-to-end tile driver against fp64 attention."""
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import synth
+from oracle import attention, e4m3, leanp, quantize
+
+MAGIC = 12582912.0
+
+
+def _round_f32_exact(fr):
+    """Nearest float32 to a rational, ties to even, by checking neighbours exactly."""
+    c = np.float32(float(fr))
+    cands = [c, np.nextafter(c, np.float32(np.inf)), np.nextafter(c, np.float32(-np.inf))]
+    best = None
+    for v in cands:
+        d = abs(Fraction(float(v)) - fr)
+        key = (d, int(np.float32(v).view(np.uint32)) & 1)
+        if best is None or key < best[0]:
+            best = (key, v)
+    return np.float32(best[1])
+
+
+def test_fmaf_single_rounding():
+    rng = np.random.default_rng(0)
+    for _ in range(3000):
+        x = np.float32(rng.standard_normal() * 50)
+        y = np.float32(rng.standard_normal() * 20)
+        z = np.float32(MAGIC + rng.integers(-500, 500))
+        exact = Fraction(float(x)) * Fraction(float(y)) + Fraction(float(z))
+        assert leanp.fmaf(x, y, z) == _round_f32_exact(exact)
+    # a case where two roundings differ from one: x*y just above a .5 boundary
+    x = np.float32(1.0 + 2 ** -23)
+    y = np.float32(0.5)
+    z = np.float32(MAGIC)
+    exact = Fraction(float(x)) * Fraction(float(y)) + Fraction(float(z))
+    assert leanp.fmaf(x, y, z) == _round_f32_exact(exact) == np.float32(MAGIC + 1)
+
+
+def test_closed_form_block_max_code():
+    # with a power-of-two slope a*s is exact, so a score equal to the running max (in byte
+    # units) codes to 120 = 8*(7+8), i.e. 2^8, and the scale 2^-(8+0) gives weight 1
+    checked = 0
+    for a in (np.float32(0.25), np.float32(2.0), leanp.slope(128, 1.0, 1.0)):
+        for m in (-40, 0, 7, 333):
+            s = np.float32(m / float(a))
+            if float(np.float32(a * s)) != float(m) or float(a) * float(s) != m:
+                continue
+            kb = leanp.kshift(s, a, m)
+            assert kb == 0
+            c = leanp.code(s, a, m, kb)
+            assert c == 120 == 8 * (7 + 8)
+            assert e4m3.e4m3_decode(np.array([c]))[0] * 2.0 ** -(8 + kb) == 1.0
+            # one block below: k = 1 keeps the code in range and the weight 2^-1
+            s2 = np.float32((m - 8) / float(a))
+            if float(a) * float(s2) == m - 8:
+                assert leanp.kshift(s2, a, m) == 1
+                assert leanp.code(s2, a, m, 1) == 120
+            checked += 1
+    assert checked >= 8
+
+
+def test_codes_follow_log_linear_rule_within_mitchell_bound():
+    rng = np.random.default_rng(1)
+    a = leanp.slope(128, 0.01, 0.02)
+    s = (rng.standard_normal(128 * 16) * 300).astype(np.float32)
+    codes, ks, mref = leanp.encode_row(s, a)
+    for t in range(16):
+        m = mref[t]
+        for j in range(128):
+            idx = t * 128 + j
+            c = int(codes[idx])
+            kb = int(ks[idx // 64])
+            y = (float(a) * float(s[idx]) - m) / 8.0 + 8 + kb     # wanted log2 of the value
+            if c >= 8:                                          # normal e4m3 codes
+                got = np.log2(e4m3.e4m3_decode(np.array([c]))[0])
+                assert abs(got - y) <= 0.0861 + 1.0 / 16 + 1e-6
+            elif c == 0:
+                assert y < 0.5 / 8 - 6                          # below the smallest code
+            assert c <= 120
+
+
+def test_block_shift_rule_and_monotonicity():
+    rng = np.random.default_rng(2)
+    a = leanp.slope(128, 0.02, 0.02)
+    for trial in range(50):
+        s = (rng.standard_normal(128) * 200 - rng.uniform(0, 3000) * (np.arange(128) >= 64)).astype(np.float32)
+        codes, ks, mref = leanp.encode_row(s, a)
+        m = mref[0]
+        for b in range(2):
+            blk = s[b * 64:(b + 1) * 64]
+            mu = blk.max()
+            kb = int(ks[b])
+            top = int(codes[b * 64 + int(np.argmax(blk))])
+            if 0 < kb < leanp.KMAX:
+                assert 112 <= top <= 120
+            if kb == 0:
+                assert top <= 120
+            # monotone within a block
+            order = np.argsort(blk, kind="stable")
+            assert np.all(np.diff(codes[b * 64:(b + 1) * 64][order].astype(int)) >= 0)
+        assert m == int(np.ceil(np.float32(a * s.max())))
+
+
+def test_masked_scores_code_zero_and_full_mask_shift():
+    a = leanp.slope(128, 1.0, 1.0)
+    s = np.full(128, -np.inf, dtype=np.float32)
+    s[:10] = np.linspace(-5, 5, 10)
+    codes, ks, mref = leanp.encode_row(s, a)
+    assert not codes[10:].any()
+    assert ks[1] == leanp.KMAX
+
+
+def test_running_max_rescale_sequence():
+    a = leanp.slope(128, 1.0, 1.0)
+    s = np.concatenate([np.full(128, 1.0), np.full(128, 3.0), np.full(128, 2.0)]).astype(np.float32)
+    _, _, mref = leanp.encode_row(s, a)
+    assert list(mref) == [int(np.ceil(np.float32(a * 1))), int(np.ceil(np.float32(a * 3))), int(np.ceil(np.float32(a * 3)))]
+
+
+@pytest.mark.parametrize("dist", ["gaussian", "outlier"])
+def test_tile_driver_within_fp8_tolerance_of_fp64(dist):
+    B, S, Hq, Hkv, D = 1, 384, 4, 2, 128
+    q, k, v = synth.make_qkv(B, S, Hq, Hkv, D, D, seed=3, dist=dist)
+    qf, kf, vf = [t.float().numpy() for t in (q, k, v)]
+    (qc, dq), (kc, dk), (vc, dv) = [quantize.quantize_e4m3(t) for t in (qf, kf, vf)]
+    qd, kd, vd = [quantize.dequantize(c, s) for c, s in ((qc, dq), (kc, dk), (vc, dv))]
+    o_ref, lse_ref = attention.causal_attention(qd, kd, vd)
+    rows = np.arange(S)
+    heads = list(range(Hq))
+    o_lp, lse_lp = leanp.attention_rows(qc, kc, vc, dq, dk, dv, rows, heads)
+    ref = o_ref[0].transpose(1, 0, 2)
+    rel = np.sqrt(((o_lp - ref) ** 2).sum() / (ref ** 2).sum())
+    assert rel <= 3e-2
+    # lse carries the log-linear code error: at most the Mitchell bound plus half a step
+    assert np.abs(lse_lp - lse_ref[0]).max() <= np.log(2) * (0.0861 + 1 / 16)
+    # row 0: a single key of weight one -> o = v0 exactly
+    np.testing.assert_allclose(o_lp[:, 0, :], vd[0, 0, [h // 2 for h in heads], :], rtol=0, atol=1e-12)
