@@ -1,0 +1,175 @@
+"""Python binding of libattn_b200.so (include/attn.h): argument marshalling only.
+
+Every step of the computation runs in the library's CUDA kernels; this module turns torch
+tensors into device pointers and sizes, allocates outputs with torch when the caller
+does not pass them, and raises on a non-zero status.  There is no fallback: if the
+library is missing or fails to load, the calls raise.
+"""
+import ctypes
+import os
+
+import torch
+
+from .build import LIB as LIB_PATH
+
+ATTN_OK = 0
+ATTN_ERR_INVALID_ARG = 1
+ATTN_ERR_UNSUPPORTED = 2
+ATTN_ERR_ALIGNMENT = 3
+ATTN_ERR_CUDA = 4
+ATTN_ERR_TIMEOUT = 5
+ATTN_BF16 = 0
+ATTN_FP8_E4M3 = 1
+ATTN_FLAG_UNROTATE_O = 1
+
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+def lib():
+    """Load the shared library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"CUDA library {LIB_PATH} is not built; run "
+                "`python -m bf16_causal_prefill_attn_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, u32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint
+        fwd_args = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, vp, vp, i32]
+        L.attn_fwd.argtypes = fwd_args + [vp]
+        L.attn_fwd.restype = i32
+        L.attn_fwd_ex.argtypes = fwd_args + [u32, vp]
+        L.attn_fwd_ex.restype = i32
+        L.attn_fwd_fp8_dump.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                        vp, vp, vp, i32, vp, vp, vp, vp]
+        L.attn_fwd_fp8_dump.restype = i32
+        L.attn_quantize_e4m3.argtypes = [vp, vp, vp, ctypes.c_int64, i32, i32, i32, vp,
+                                         ctypes.c_size_t, vp]
+        L.attn_quantize_e4m3.restype = i32
+        L.attn_quantize_workspace_size.argtypes = [ctypes.c_int64, i32, i32]
+        L.attn_quantize_workspace_size.restype = ctypes.c_size_t
+        L.attn_device_status.argtypes = [vp]
+        L.attn_device_status.restype = i32
+        L.attn_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
+        L.attn_set_wait_timeout_ns.restype = None
+        L.attn_status_string.argtypes = [i32]
+        L.attn_status_string.restype = ctypes.c_char_p
+        L.attn_version.argtypes = []
+        L.attn_version.restype = i32
+        _lib = L
+    return _lib
+
+
+def status_string(status):
+    return lib().attn_status_string(int(status)).decode()
+
+
+def version():
+    return lib().attn_version()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(status, what):
+    if status != ATTN_OK:
+        raise AttnError(status, what)
+
+
+def _codes(t):
+    """e4m3 tensors may be passed as uint8 codes or torch.float8_e4m3fn."""
+    return t.view(torch.uint8) if t.dtype == torch.float8_e4m3fn else t
+
+
+def attn_fwd(q, k, v, causal=True, descale_q=None, descale_k=None, descale_v=None, out=None,
+             lse=None, return_lse=True, unrotate=False, stream=None):
+    """Causal prefill attention.  q [B,S,Hq,d_qk], k [B,S,Hkv,d_qk], v [B,S,Hkv,d_v] on the
+    GPU: bf16, or e4m3 codes (uint8 / float8_e4m3fn) with fp32 descale tensors.
+    Returns (o bf16 [B,S,Hq,d_v], lse fp32 [B,Hq,S] or None)."""
+    fp8 = q.dtype in (torch.uint8, torch.float8_e4m3fn)
+    q, k, v = (_codes(x) for x in (q, k, v)) if fp8 else (q, k, v)
+    for x in (q, k, v):
+        if not x.is_contiguous():
+            raise ValueError("q, k, v must be contiguous [B, S, H, d]")
+    B, S, Hq, d_qk = q.shape
+    Hkv = k.shape[2]
+    d_v = v.shape[3]
+    if out is None:
+        out = torch.empty((B, S, Hq, d_v), dtype=torch.bfloat16, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, S), dtype=torch.float32, device=q.device)
+    flags = ATTN_FLAG_UNROTATE_O if unrotate else 0
+    st = lib().attn_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, S,
+                           d_qk, d_v, ATTN_FP8_E4M3 if fp8 else ATTN_BF16, _ptr(descale_q),
+                           _ptr(descale_k), _ptr(descale_v), 1 if causal else 0, flags,
+                           _stream(stream))
+    _check(st, "attn_fwd")
+    return out, lse
+
+
+def attn_fwd_fp8_dump(q, k, v, descale_q, descale_k, descale_v, causal=True, stream=None):
+    """Test-only FP8 forward that also returns the raw scores, lean-P codes and shifts."""
+    q, k, v = (_codes(x) for x in (q, k, v))
+    B, S, Hq, d_qk = q.shape
+    Hkv = k.shape[2]
+    d_v = v.shape[3]
+    dev = q.device
+    out = torch.empty((B, S, Hq, d_v), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, Hq, S), dtype=torch.float32, device=dev)
+    ds = torch.full((B, Hq, S, S), float("nan"), dtype=torch.float32, device=dev)
+    dc = torch.zeros((B, Hq, S, S), dtype=torch.uint8, device=dev)
+    dk = torch.full((B, Hq, S, S // 64), 255, dtype=torch.uint8, device=dev)
+    st = lib().attn_fwd_fp8_dump(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv,
+                                 S, d_qk, d_v, _ptr(descale_q), _ptr(descale_k),
+                                 _ptr(descale_v), 1 if causal else 0, _ptr(ds), _ptr(dc),
+                                 _ptr(dk), _stream(stream))
+    _check(st, "attn_fwd_fp8_dump")
+    return out, lse, ds, dc, dk
+
+
+def attn_quantize_workspace_size(tokens, H, d):
+    return lib().attn_quantize_workspace_size(tokens, H, d)
+
+
+def attn_quantize_e4m3(x, hadamard=False, out=None, descale=None, workspace=None, stream=None):
+    """Per-tensor e4m3 quantisation of a contiguous bf16 tensor [tokens, H, d] (or
+    [B, S, H, d]).  Returns (codes uint8 with x's shape, descale fp32 [1])."""
+    if x.dtype != torch.bfloat16 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous bf16 tensor")
+    d = x.shape[-1]
+    H = x.shape[-2]
+    tokens = x.numel() // (H * d) if x.numel() else 0
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    if descale is None:
+        descale = torch.empty((1,), dtype=torch.float32, device=x.device)
+    ws_bytes = attn_quantize_workspace_size(tokens, H, d)
+    if workspace is None:
+        workspace = torch.empty((ws_bytes + 3) // 4, dtype=torch.int32, device=x.device)
+    st = lib().attn_quantize_e4m3(_ptr(x), _ptr(out), _ptr(descale), tokens, H, d,
+                                  1 if hadamard else 0, _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "attn_quantize_e4m3")
+    return out, descale
+
+
+def attn_device_status(stream=None):
+    """Synchronise the stream and return the device status code (ATTN_OK, ATTN_ERR_*)."""
+    return lib().attn_device_status(_stream(stream))
+
+
+def attn_set_wait_timeout_ns(ns):
+    lib().attn_set_wait_timeout_ns(int(ns))

@@ -1,0 +1,259 @@
+// C ABI of libattn_b200.so (declared in include/attn.h): argument validation, TMA tensor
+// maps, kernel selection and launch.  No device memory is allocated here.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/attn.h"
+#include "attn_fwd.cuh"
+#include "quantize.cuh"
+
+namespace {
+
+constexpr int kVersion = 1;
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s per bounded wait
+
+// Device error word of every GPU that loads the library (set by bounded waits).
+__device__ uint32_t g_dev_err = 0;
+
+uint64_t g_timeout_ns = kDefaultTimeoutNs;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool dev_err_ptr(uint32_t** out) {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_dev_err) != cudaSuccess) return false;
+  *out = static_cast<uint32_t*>(p);
+  return true;
+}
+
+// 3-D tiled map over [T, H, d] (d innermost), box = (box_cols, 1, 128), 128-B swizzle.
+bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, uint64_t d,
+              uint64_t H, uint64_t T, uint32_t box_cols) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d, H, T};
+  cuuint64_t strides[2] = {d * esize, H * d * esize};
+  cuuint32_t box[3] = {box_cols, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <bool FP8, int DQK, bool DUMP>
+attn_status_t launch_fwd(const void* q, const void* k, const void* v, attn::FwdParams& prm,
+                         cudaStream_t stream) {
+  using C = attn::FwdCfg<FP8, DQK>;
+  const CUtensorMapDataType dt =
+      FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const uint64_t T = static_cast<uint64_t>(prm.B) * prm.S;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, dt, C::E, DQK, prm.Hq, T, C::BOX_COLS) ||
+      !make_map(&mk, k, dt, C::E, DQK, prm.Hkv, T, C::BOX_COLS) ||
+      !make_map(&mv, v, dt, C::E, attn::DV, prm.Hkv, T, C::BOX_COLS))
+    return ATTN_ERR_CUDA;
+  auto kern = attn::attn_fwd_kernel<FP8, DQK, DUMP>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC) !=
+      cudaSuccess)
+    return ATTN_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(prm.n_q_tiles) * prm.B * prm.Hq;
+  kern<<<grid, attn::NUM_THREADS, C::SMEM_ALLOC, stream>>>(mq, mk, mv, prm);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                       int Hq, int Hkv, int S, int d_qk, int d_v, attn_dtype_t dtype,
+                       const float* dq, const float* dk, const float* dv, int causal,
+                       unsigned flags, float* dump_s, uint8_t* dump_codes,
+                       uint8_t* dump_kshift, bool dump, void* stream) {
+  if (B < 0 || S < 0 || Hq <= 0 || Hkv <= 0 || (Hq % Hkv) != 0) return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if ((flags & ~static_cast<unsigned>(ATTN_FLAG_UNROTATE_O)) != 0) return ATTN_ERR_INVALID_ARG;
+  if (dtype != ATTN_BF16 && dtype != ATTN_FP8_E4M3) return ATTN_ERR_INVALID_ARG;
+  if ((d_qk != 128 && d_qk != 192) || d_v != 128) return ATTN_ERR_UNSUPPORTED;
+  if (B == 0 || S == 0) return ATTN_OK;
+  if (!q || !k || !v || !o) return ATTN_ERR_INVALID_ARG;
+  if (dtype == ATTN_FP8_E4M3 && (!dq || !dk || !dv)) return ATTN_ERR_INVALID_ARG;
+  if (dump && (dtype != ATTN_FP8_E4M3 || !dump_s || !dump_codes || !dump_kshift))
+    return ATTN_ERR_INVALID_ARG;
+  if (S % 128 != 0) return ATTN_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(B) * S > INT32_MAX ||
+      static_cast<int64_t>(S / 128) * B * Hq > INT32_MAX)
+    return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_ALIGNMENT;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATTN_ERR_ALIGNMENT;
+
+  attn::FwdParams prm{};
+  prm.B = B;
+  prm.S = S;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.G = Hq / Hkv;
+  prm.n_q_tiles = S / 128;
+  prm.causal = causal;
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.lse = lse;
+  const double scale = 1.0 / std::sqrt(static_cast<double>(d_qk));
+  const double log2e = 1.4426950408889634;
+  prm.c1 = static_cast<float>(scale * log2e);
+  prm.leanp_c = 8.0 * log2e * scale;
+  prm.descale_q = dq;
+  prm.descale_k = dk;
+  prm.descale_v = dv;
+  prm.unrotate = (flags & ATTN_FLAG_UNROTATE_O) ? 1 : 0;
+  prm.timeout_ns = g_timeout_ns;
+  prm.dump_s = dump_s;
+  prm.dump_codes = dump_codes;
+  prm.dump_kshift = dump_kshift;
+  if (!dev_err_ptr(&prm.err)) return ATTN_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  if (dtype == ATTN_BF16) {
+    if (d_qk == 128) return launch_fwd<false, 128, false>(q, k, v, prm, st);
+    return launch_fwd<false, 192, false>(q, k, v, prm, st);
+  }
+  if (dump) {
+    if (d_qk == 128) return launch_fwd<true, 128, true>(q, k, v, prm, st);
+    return launch_fwd<true, 192, true>(q, k, v, prm, st);
+  }
+  if (d_qk == 128) return launch_fwd<true, 128, false>(q, k, v, prm, st);
+  return launch_fwd<true, 192, false>(q, k, v, prm, st);
+}
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+}  // namespace
+
+extern "C" {
+
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                       int Hq, int Hkv, int S, int d_qk, int d_v, attn_dtype_t dtype,
+                       const float* descale_q, const float* descale_k, const float* descale_v,
+                       int causal, void* stream) {
+  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, S, d_qk, d_v, dtype, descale_q, descale_k,
+                  descale_v, causal, 0u, nullptr, nullptr, nullptr, false, stream);
+}
+
+attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int B, int Hq, int Hkv, int S, int d_qk, int d_v, attn_dtype_t dtype,
+                          const float* descale_q, const float* descale_k,
+                          const float* descale_v, int causal, unsigned flags, void* stream) {
+  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, S, d_qk, d_v, dtype, descale_q, descale_k,
+                  descale_v, causal, flags, nullptr, nullptr, nullptr, false, stream);
+}
+
+attn_status_t attn_fwd_fp8_dump(const void* q, const void* k, const void* v, void* o, float* lse,
+                                int B, int Hq, int Hkv, int S, int d_qk, int d_v,
+                                const float* descale_q, const float* descale_k,
+                                const float* descale_v, int causal, float* dump_s,
+                                uint8_t* dump_codes, uint8_t* dump_kshift, void* stream) {
+  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, S, d_qk, d_v, ATTN_FP8_E4M3, descale_q, descale_k,
+                  descale_v, causal, 0u, dump_s, dump_codes, dump_kshift, true, stream);
+}
+
+size_t attn_quantize_workspace_size(int64_t tokens, int H, int d) {
+  (void)tokens;
+  (void)H;
+  (void)d;
+  return 16;
+}
+
+attn_status_t attn_quantize_e4m3(const void* x_bf16, void* x_e4m3, float* descale_out,
+                                 int64_t tokens, int H, int d, int hadamard, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  if (tokens < 0 || H <= 0 || d <= 0 || (d % 8) != 0) return ATTN_ERR_INVALID_ARG;
+  if (hadamard != 0 && hadamard != 1) return ATTN_ERR_INVALID_ARG;
+  if (hadamard && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!descale_out || !workspace) return ATTN_ERR_INVALID_ARG;
+  if (workspace_bytes < attn_quantize_workspace_size(tokens, H, d)) return ATTN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 3u) ||
+      (reinterpret_cast<uintptr_t>(descale_out) & 3u))
+    return ATTN_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t rows = tokens * H;
+  uint32_t* amax = static_cast<uint32_t*>(workspace);
+  if (rows == 0) {
+    const float one = 1.0f;
+    return cudaMemcpyAsync(descale_out, &one, sizeof(float), cudaMemcpyHostToDevice, st) ==
+                   cudaSuccess
+               ? ATTN_OK
+               : ATTN_ERR_CUDA;
+  }
+  if (!x_bf16 || !x_e4m3) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(x_bf16) || !aligned16(x_e4m3)) return ATTN_ERR_ALIGNMENT;
+  if (cudaMemsetAsync(amax, 0, sizeof(uint32_t), st) != cudaSuccess) return ATTN_ERR_CUDA;
+  const int threads = 256;
+  const int sms = num_sms();
+  const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(x_bf16);
+  uint8_t* y = static_cast<uint8_t*>(x_e4m3);
+  if (hadamard) {
+    const int64_t want = (rows + 7) / 8;  // 8 warps (rows) per block
+    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(want, int64_t(sms) * 16));
+    attn::amax_rot_kernel<<<grid, threads, 0, st>>>(x, rows, amax);
+    attn::convert_rot_kernel<<<grid, threads, 0, st>>>(x, y, rows, amax, descale_out);
+  } else {
+    const int64_t n8 = rows * d / 8;
+    const int64_t want = (n8 + threads - 1) / threads;
+    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(want, int64_t(sms) * 16));
+    attn::amax_flat_kernel<<<grid, threads, 0, st>>>(x, n8, amax);
+    attn::convert_flat_kernel<<<grid, threads, 0, st>>>(x, y, n8, amax, descale_out);
+  }
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status_t attn_device_status(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return ATTN_ERR_CUDA;
+  uint32_t host = 0;
+  if (cudaMemcpyFromSymbol(&host, g_dev_err, sizeof(host)) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (host != attn::DEV_OK) {
+    const uint32_t zero = 0;
+    if (cudaMemcpyToSymbol(g_dev_err, &zero, sizeof(zero)) != cudaSuccess) return ATTN_ERR_CUDA;
+    return ATTN_ERR_TIMEOUT;
+  }
+  return ATTN_OK;
+}
+
+void attn_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns = ns ? ns : kDefaultTimeoutNs; }
+
+const char* attn_status_string(attn_status_t s) {
+  switch (s) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported shape or option";
+    case ATTN_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case ATTN_ERR_CUDA: return "CUDA error";
+    case ATTN_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+int attn_version(void) { return kVersion; }
+
+}  // extern "C"

@@ -1,0 +1,160 @@
+// Per-tensor e4m3 quantisation of bf16 activations, optionally after a 128-point
+// Hadamard rotation along the head dimension ([ZYFA-mb] "Precisão, estabilidade e efeito
+// na prática": most FP8 error comes from quantising Q, K and V; a Hadamard rotation of
+// those tensors halves it).
+//
+// Two HBM-bound passes over x [rows, d] (rows = tokens * heads, d contiguous):
+//   1. amax = max |y| with y = x or y = (x H_128) * float32(1/sqrt(128)), the rotation done
+//      in float32 by the butterfly stages h = 1, 2, ..., 64, (u, w) -> (u + w, u - w).
+//      Reduced with an integer atomicMax on the bit pattern (exact and order-free for
+//      non-negative floats, so the result is deterministic).
+//   2. scale = 448 / amax (float32, correctly rounded); code = e4m3 RNE-satfinite of
+//      float32(y * scale); descale = amax / 448 written once.
+// The rounding of every step is fixed, so the codes are a defined function of x.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace attn {
+
+constexpr float HAD_R = 0.08838834764831845f;  // float32(1/sqrt(128))
+
+__device__ __forceinline__ uint32_t f32_to_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// ---- rotated rows: one warp per 128-element row, 4 consecutive elements per lane
+__device__ __forceinline__ void load_row4(const __nv_bfloat16* x, int64_t row, int lane,
+                                          float v[4]) {
+  const uint2 raw = __ldg(reinterpret_cast<const uint2*>(x + row * 128) + lane);
+  const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
+  const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
+  v[0] = __low2float(a);
+  v[1] = __high2float(a);
+  v[2] = __low2float(b);
+  v[3] = __high2float(b);
+}
+
+__device__ __forceinline__ void hadamard_row4(float v[4], int lane) {
+  // stages h = 1, 2 inside the lane
+  float u, w;
+  u = v[0]; w = v[1]; v[0] = __fadd_rn(u, w); v[1] = __fsub_rn(u, w);
+  u = v[2]; w = v[3]; v[2] = __fadd_rn(u, w); v[3] = __fsub_rn(u, w);
+  u = v[0]; w = v[2]; v[0] = __fadd_rn(u, w); v[2] = __fsub_rn(u, w);
+  u = v[1]; w = v[3]; v[1] = __fadd_rn(u, w); v[3] = __fsub_rn(u, w);
+  // stages h = 4 .. 64 across lanes (partner lane = lane ^ (h / 4))
+#pragma unroll
+  for (int m = 1; m < 32; m <<= 1) {
+    const bool upper = (lane & m) != 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float other = __shfl_xor_sync(0xffffffffu, v[i], m);
+      v[i] = upper ? __fsub_rn(other, v[i]) : __fadd_rn(v[i], other);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) v[i] = __fmul_rn(v[i], HAD_R);
+}
+
+__device__ __forceinline__ void block_amax_atomic(float m, uint32_t* amax_bits) {
+  __shared__ float red[32];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[warp] = m;
+  __syncthreads();
+  if (warp == 0) {
+    m = lane < (blockDim.x >> 5) ? red[lane] : 0.0f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) atomicMax(amax_bits, __float_as_uint(m));
+  }
+}
+
+__global__ void amax_rot_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows,
+                                uint32_t* amax_bits) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  float m = 0.0f;
+  for (int64_t row = warp_g; row < rows; row += nwarps) {
+    float v[4];
+    load_row4(x, row, lane, v);
+    hadamard_row4(v, lane);
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3]))));
+  }
+  block_amax_atomic(m, amax_bits);
+}
+
+__global__ void amax_flat_kernel(const __nv_bfloat16* __restrict__ x, int64_t n8,
+                                 uint32_t* amax_bits) {
+  float m = 0.0f;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += stride) {
+    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(x) + i);
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      m = fmaxf(m, fmaxf(fabsf(__low2float(h2[k])), fabsf(__high2float(h2[k]))));
+    }
+  }
+  block_amax_atomic(m, amax_bits);
+}
+
+__device__ __forceinline__ float quant_scale(uint32_t amax_bits) {
+  const float amax = __uint_as_float(amax_bits);
+  return amax > 0.0f ? __fdiv_rn(448.0f, amax) : 1.0f;
+}
+
+__device__ __forceinline__ void write_descale(uint32_t amax_bits, float* descale_out) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    const float amax = __uint_as_float(amax_bits);
+    *descale_out = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+  }
+}
+
+__global__ void convert_rot_kernel(const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ y,
+                                   int64_t rows, const uint32_t* amax_bits, float* descale_out) {
+  const uint32_t ab = *amax_bits;
+  const float sc = quant_scale(ab);
+  write_descale(ab, descale_out);
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t row = warp_g; row < rows; row += nwarps) {
+    float v[4];
+    load_row4(x, row, lane, v);
+    hadamard_row4(v, lane);
+    const uint32_t lo = f32_to_e4m3x2(__fmul_rn(v[0], sc), __fmul_rn(v[1], sc));
+    const uint32_t hi = f32_to_e4m3x2(__fmul_rn(v[2], sc), __fmul_rn(v[3], sc));
+    reinterpret_cast<uint32_t*>(y + row * 128)[lane] = lo | (hi << 16);
+  }
+}
+
+__global__ void convert_flat_kernel(const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ y,
+                                    int64_t n8, const uint32_t* amax_bits, float* descale_out) {
+  const uint32_t ab = *amax_bits;
+  const float sc = quant_scale(ab);
+  write_descale(ab, descale_out);
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += stride) {
+    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(x) + i);
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+    uint32_t w[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      w[k] = f32_to_e4m3x2(__fmul_rn(__low2float(h2[k]), sc), __fmul_rn(__high2float(h2[k]), sc));
+    uint2 out;
+    out.x = w[0] | (w[1] << 16);
+    out.y = w[2] | (w[3] << 16);
+    reinterpret_cast<uint2*>(y)[i] = out;
+  }
+}
+
+}  // namespace attn

@@ -1,0 +1,130 @@
+/*
+ * C ABI of the B200 (sm_100a) causal prefill attention library, libattn_b200.so.
+ *
+ * The operation ([ZYFA-fr] = ai-daily-news.org article
+ * "zyphra-zyfa-fp8-flashattention-amd-mi355x", section "Ce que couvrent les noyaux";
+ * [ZYFA-pt] = acheiumaia.com.br news item "zyphra-zyfa-flashattention-fp8-para-amd-mi355x",
+ * TL;DR; [ZYFA-mb] = miraibroadcast.com, "Zyphra lança ZYFA e acelera GPUs AMD em até
+ * 1,76x IA", sections "Como o motor de atenção FP8 da Zyphra funciona" and "Precisão,
+ * estabilidade e efeito na prática"):
+ *
+ *   forward causal (prefill) attention  O = softmax(mask(Q K^T * scale)) V
+ *   in BF16 or FP8 e4m3, head dim 128 with grouped-query heads, or the MLA shape
+ *   (qk dim 192, v dim 128).  The FP8 path forms probabilities with the exp-free lean-P
+ *   encoding, scales each 64-key block by a power of two removed by the block-scaled MMA,
+ *   and takes the row normaliser from the tensor-core sum of the rounded probabilities.
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers unless stated; the caller allocates and
+ *     frees them.  The library never allocates device memory (TMEM is allocated and
+ *     released inside each kernel).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are asynchronous
+ *     and stream-ordered; they do not synchronise.  They are thread-safe and reentrant.
+ *   - Layouts: token-major BSHD, i.e. [B, S, H, d] contiguous with d innermost.
+ *   - Synchronous argument checks return an error code before anything is launched; no
+ *     exception crosses the ABI.  Kernels never trap: a bounded wait that expires sets a
+ *     device error word, reported by attn_device_status().
+ *   - Scale = 1/sqrt(d_qk).  Query head h reads key/value head h / (Hq / Hkv).
+ *     Causal: key j is visible from query i iff j <= i (Sq == Sk == S).
+ */
+#ifndef ATTN_B200_H
+#define ATTN_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum attn_status {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1, /* null pointer, negative size, Hq % Hkv != 0, bad flag */
+  ATTN_ERR_UNSUPPORTED = 2, /* head dims other than 128/192 (qk) and 128 (v); S % 128 != 0 */
+  ATTN_ERR_ALIGNMENT = 3,   /* a tensor pointer not 16-byte aligned */
+  ATTN_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed */
+  ATTN_ERR_TIMEOUT = 5      /* a device-side bounded wait expired (see attn_device_status) */
+} attn_status_t;
+
+typedef enum attn_dtype { ATTN_BF16 = 0, ATTN_FP8_E4M3 = 1 } attn_dtype_t;
+
+/* flags of attn_fwd_ex */
+#define ATTN_FLAG_UNROTATE_O 1u /* V was Hadamard-rotated: apply x H/sqrt(128) to O rows */
+
+/*
+ * attn_fwd: forward causal prefill attention.
+ *   q         [B, S, Hq,  d_qk]  bf16 (ATTN_BF16) or e4m3 codes (ATTN_FP8_E4M3)
+ *   k         [B, S, Hkv, d_qk]  same type as q
+ *   v         [B, S, Hkv, d_v ]  same type as q
+ *   o         [B, S, Hq,  d_v ]  bf16 output (round to nearest even)
+ *   lse       [B, Hq, S] fp32 natural-log sum-exp of the scaled scores, or NULL
+ *   d_qk      128 or 192;  d_v  128
+ *   dtype     ATTN_BF16 or ATTN_FP8_E4M3
+ *   descale_q/k/v  DEVICE pointers to one fp32 each (x = code * descale), as written by
+ *             attn_quantize_e4m3; required for FP8, ignored (may be NULL) for BF16
+ *   causal    1 = causal mask (the contract), 0 = full attention
+ * Requirements: S % 128 == 0, Hq % Hkv == 0, pointers 16-byte aligned.
+ * B == 0 or S == 0 is a no-op.
+ */
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                       int Hq, int Hkv, int S, int d_qk, int d_v, attn_dtype_t dtype,
+                       const float* descale_q, const float* descale_k, const float* descale_v,
+                       int causal, void* stream);
+
+/* attn_fwd with option flags (ATTN_FLAG_*). */
+attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int B, int Hq, int Hkv, int S, int d_qk, int d_v, attn_dtype_t dtype,
+                          const float* descale_q, const float* descale_k,
+                          const float* descale_v, int causal, unsigned flags, void* stream);
+
+/*
+ * attn_quantize_e4m3: per-tensor e4m3 quantisation of a bf16 tensor [tokens, H, d]
+ * ([ZYFA-mb], "Precisão, estabilidade e efeito na prática").
+ *   y = x, or with hadamard = 1, y = (x H_128) * float32(1/sqrt(128)) along d (d must be
+ *   128), computed in float32 by butterfly stages h = 1, 2, ..., 64;
+ *   amax = max|y|; scale = 448/amax; codes = e4m3 round-to-nearest-even, saturating, of
+ *   float32(y * scale); *descale_out = amax/448 (both 1 when amax == 0).
+ *   x_bf16     device, [tokens, H, d] bf16, 16-byte aligned
+ *   x_e4m3     device, [tokens, H, d] uint8 output, 16-byte aligned
+ *   descale_out device, one fp32
+ *   workspace  device scratch of at least attn_quantize_workspace_size() bytes, 4-byte
+ *              aligned, owned by the caller; must not be shared by calls running
+ *              concurrently
+ * Requirements: d % 8 == 0.  Deterministic.
+ */
+attn_status_t attn_quantize_e4m3(const void* x_bf16, void* x_e4m3, float* descale_out,
+                                 int64_t tokens, int H, int d, int hadamard, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+size_t attn_quantize_workspace_size(int64_t tokens, int H, int d);
+
+/*
+ * Test-only: FP8 attn_fwd that also dumps, for every (query row, visible key tile), the
+ * raw fp32 scores after masking, the lean-P e4m3 codes and the per-64-key shifts:
+ *   dump_s      [B, Hq, S, S] fp32      dump_codes [B, Hq, S, S] uint8
+ *   dump_kshift [B, Hq, S, S/64] uint8  (entries of key tiles that are not visible are
+ *   left untouched).  d_qk must be 128 or 192; slow; for small S only.
+ */
+attn_status_t attn_fwd_fp8_dump(const void* q, const void* k, const void* v, void* o, float* lse,
+                                int B, int Hq, int Hkv, int S, int d_qk, int d_v,
+                                const float* descale_q, const float* descale_k,
+                                const float* descale_v, int causal, float* dump_s,
+                                uint8_t* dump_codes, uint8_t* dump_kshift, void* stream);
+
+/*
+ * Synchronises `stream` and reports (then clears) the device error word of the current
+ * device: ATTN_ERR_TIMEOUT if a kernel's bounded wait expired, ATTN_ERR_CUDA if the stream
+ * reported an error, ATTN_OK otherwise.
+ */
+attn_status_t attn_device_status(void* stream);
+
+/* Test-only: sets the bounded-wait limit in nanoseconds (0 restores the default, 2 s). */
+void attn_set_wait_timeout_ns(uint64_t ns);
+
+const char* attn_status_string(attn_status_t status);
+int attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_H */

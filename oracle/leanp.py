@@ -64,9 +64,9 @@ def _ptr(a, ct):
 
 
 def slope(d_qk, descale_q, descale_k):
-    """a = float32(8 log2(e) / sqrt(d_qk) * dq * dk): byte units per raw-score unit.
-    The product is formed in float64 in this order and rounded once."""
-    c = 8.0 * LOG2E / np.sqrt(np.float64(d_qk))
+    """a = float32(8 log2(e) * (1/sqrt(d_qk)) * dq * dk): byte units per raw-score unit.
+    The product is formed in float64, left to right in this order, and rounded once."""
+    c = 8.0 * LOG2E * (1.0 / np.sqrt(np.float64(d_qk)))
     return np.float32(c * np.float64(np.float32(descale_q)) * np.float64(np.float32(descale_k)))
 
 

@@ -1,0 +1,91 @@
+"""The C-ABI library loads, exports every symbol include/attn.h declares, and rejects bad
+arguments before touching the GPU (host logic only: no kernel runs here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import bf16_causal_prefill_attn_b200 as pkg
+from bf16_causal_prefill_attn_b200 import build as B
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "attn.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    B.build()
+    return pkg.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(attn_[a-z0-9_]+)\s*\(", text, flags=re.M)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert "attn_fwd" in names and "attn_quantize_e4m3" in names and len(names) >= 9
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_version_and_status_strings(L):
+    assert pkg.version() >= 1
+    assert pkg.status_string(0) == "ok"
+    assert "timed out" in pkg.status_string(pkg.ATTN_ERR_TIMEOUT)
+    assert pkg.status_string(99) == "unknown status"
+
+
+def _fwd(L, q=1, k=1, v=1, o=1, B=1, Hq=2, Hkv=1, S=128, dqk=128, dv=128, dtype=0, ds=(0, 0, 0),
+         causal=1, flags=0):
+    vp = ctypes.c_void_p
+    p = lambda x: vp(x * 256) if x else None  # fake, aligned, never dereferenced
+    return L.attn_fwd_ex(p(q), p(k), p(v), p(o), None, B, Hq, Hkv, S, dqk, dv, dtype,
+                         p(ds[0]), p(ds[1]), p(ds[2]), causal, flags, None)
+
+
+def test_fwd_argument_validation(L):
+    assert _fwd(L, Hq=3, Hkv=2) == pkg.ATTN_ERR_INVALID_ARG
+    assert _fwd(L, Hkv=0) == pkg.ATTN_ERR_INVALID_ARG
+    assert _fwd(L, B=-1) == pkg.ATTN_ERR_INVALID_ARG
+    assert _fwd(L, causal=2) == pkg.ATTN_ERR_INVALID_ARG
+    assert _fwd(L, flags=8) == pkg.ATTN_ERR_INVALID_ARG
+    assert _fwd(L, dtype=7) == pkg.ATTN_ERR_INVALID_ARG
+    assert _fwd(L, dqk=64) == pkg.ATTN_ERR_UNSUPPORTED
+    assert _fwd(L, dv=192) == pkg.ATTN_ERR_UNSUPPORTED
+    assert _fwd(L, S=100) == pkg.ATTN_ERR_UNSUPPORTED
+    assert _fwd(L, q=0) == pkg.ATTN_ERR_INVALID_ARG
+    assert _fwd(L, o=0) == pkg.ATTN_ERR_INVALID_ARG
+    assert _fwd(L, dtype=1) == pkg.ATTN_ERR_INVALID_ARG      # FP8 without descales
+    # empty problems are no-ops that never touch the device
+    assert _fwd(L, S=0, q=0, k=0, v=0, o=0) == pkg.ATTN_OK
+    assert _fwd(L, B=0, q=0, k=0, v=0, o=0) == pkg.ATTN_OK
+    # misaligned pointers
+    vp = ctypes.c_void_p
+    st = L.attn_fwd(vp(256 + 8), vp(256), vp(256), vp(256), None, 1, 1, 1, 128, 128, 128, 0,
+                    None, None, None, 1, None)
+    assert st == pkg.ATTN_ERR_ALIGNMENT
+
+
+def test_quantize_argument_validation(L):
+    vp = ctypes.c_void_p
+    ws = L.attn_quantize_workspace_size(10, 2, 128)
+    assert ws >= 4
+    q = L.attn_quantize_e4m3
+    assert q(vp(256), vp(256), vp(256), 10, 2, 100, 0, vp(256), ws, None) == pkg.ATTN_ERR_INVALID_ARG
+    assert q(vp(256), vp(256), vp(256), 10, 2, 64, 1, vp(256), ws, None) == pkg.ATTN_ERR_UNSUPPORTED
+    assert q(vp(256), vp(256), None, 10, 2, 128, 0, vp(256), ws, None) == pkg.ATTN_ERR_INVALID_ARG
+    assert q(vp(256), vp(256), vp(256), 10, 2, 128, 0, None, ws, None) == pkg.ATTN_ERR_INVALID_ARG
+    assert q(vp(256), vp(256), vp(256), 10, 2, 128, 0, vp(256), 0, None) == pkg.ATTN_ERR_INVALID_ARG
+    assert q(vp(256), vp(256), vp(256), -1, 2, 128, 0, vp(256), ws, None) == pkg.ATTN_ERR_INVALID_ARG
+    assert q(vp(256), vp(256), vp(256), 10, 2, 128, 3, vp(256), ws, None) == pkg.ATTN_ERR_INVALID_ARG
+    assert q(vp(256), vp(256), vp(258), 10, 2, 128, 0, vp(256), ws, None) == pkg.ATTN_ERR_ALIGNMENT
+
+
+def test_binding_raises_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(pkg, "_lib", None)
+    monkeypatch.setattr(pkg, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="not built"):
+        pkg.lib()
