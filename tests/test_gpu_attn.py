@@ -20,6 +20,18 @@ def rel_rms(got, ref):
     return float(np.sqrt(((got - ref) ** 2).sum() / (ref ** 2).sum()))
 
 
+def assert_bf16_close(got, ref):
+    """max-abs 1e-2 and rel-RMS 5e-3 against fp64.  The output is bf16, whose rounding
+    alone is up to 2^-9 |o|, so an absolute 1e-2 is only attainable where |o| <= 2.56;
+    elementwise the bound is 1e-2 * max(1, |o_ref|) (identical to max-abs 1e-2 for the
+    unit-scale Gaussian cases)."""
+    err = np.abs(got - ref)
+    bound = BF16_MAX_ABS * np.maximum(1.0, np.abs(ref))
+    worst = float((err / bound).max())
+    rr = rel_rms(got, ref)
+    assert worst <= 1.0 and rr <= BF16_REL_RMS, (float(err.max()), worst, rr)
+
+
 def quantize_dev(ts, rotate=False):
     return [pkg.attn_quantize_e4m3(t.cuda(), hadamard=rotate) for t in ts]
 
@@ -40,8 +52,7 @@ def test_bf16_matches_fp64(B, S, Hq, Hkv, dqk, causal, dist):
     ref, lref = attention.causal_attention(q.float().numpy(), k.float().numpy(),
                                            v.float().numpy(), causal=causal)
     got = o.float().cpu().numpy()
-    assert np.abs(got - ref).max() <= BF16_MAX_ABS
-    assert rel_rms(got, ref) <= BF16_REL_RMS
+    assert_bf16_close(got, ref)
     assert np.abs(lse.cpu().numpy() - lref).max() <= 2e-3
     if causal:
         # row 0 sees key 0 only: o = v0 exactly (after bf16 rounding of v0, which v already is)
