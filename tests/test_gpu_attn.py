@@ -20,13 +20,14 @@ def rel_rms(got, ref):
     return float(np.sqrt(((got - ref) ** 2).sum() / (ref ** 2).sum()))
 
 
-def assert_bf16_close(got, ref):
-    """max-abs 1e-2 and rel-RMS 5e-3 against fp64.  The output is bf16, whose rounding
-    alone is up to 2^-9 |o|, so an absolute 1e-2 is only attainable where |o| <= 2.56;
-    elementwise the bound is 1e-2 * max(1, |o_ref|) (identical to max-abs 1e-2 for the
-    unit-scale Gaussian cases)."""
+def assert_bf16_close(got, ref, mag):
+    """max-abs 1e-2 and rel-RMS 5e-3 against fp64.  P and O are rounded to bf16, so the
+    error of o_id is up to about 2^-9 (sum_j p_ij |v_jd| + |o_id|): an absolute 1e-2 only
+    holds where those magnitudes are O(1).  Elementwise the bound is therefore
+    1e-2 * max(1, mag_id) with mag = attention applied to |V| (>= |o|); for unit-scale
+    inputs mag <= max|v| ~ 1 and this is the plain max-abs 1e-2."""
     err = np.abs(got - ref)
-    bound = BF16_MAX_ABS * np.maximum(1.0, np.abs(ref))
+    bound = BF16_MAX_ABS * np.maximum(1.0, mag)
     worst = float((err / bound).max())
     rr = rel_rms(got, ref)
     assert worst <= 1.0 and rr <= BF16_REL_RMS, (float(err.max()), worst, rr)
@@ -51,8 +52,12 @@ def test_bf16_matches_fp64(B, S, Hq, Hkv, dqk, causal, dist):
     assert pkg.attn_device_status() == pkg.ATTN_OK
     ref, lref = attention.causal_attention(q.float().numpy(), k.float().numpy(),
                                            v.float().numpy(), causal=causal)
+    mag, _ = attention.causal_attention(q.float().numpy(), k.float().numpy(),
+                                        np.abs(v.float().numpy()), causal=causal)
     got = o.float().cpu().numpy()
-    assert_bf16_close(got, ref)
+    assert_bf16_close(got, ref, mag)
+    if dist == "gaussian":
+        assert np.abs(got - ref).max() <= BF16_MAX_ABS
     assert np.abs(lse.cpu().numpy() - lref).max() <= 2e-3
     if causal:
         # row 0 sees key 0 only: o = v0 exactly (after bf16 rounding of v0, which v already is)
