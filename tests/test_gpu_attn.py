@@ -175,9 +175,6 @@ def test_fp8_hadamard_rotated(dist):
     ref = hadamard.rotate_fp64(ref_rot)                      # un-rotate along d_v
     got = o.float().cpu().numpy()
     assert rel_rms(got, ref) <= FP8_REL_RMS
-    # and against the unquantised source the rotation keeps the error small
-    src, _ = attention.causal_attention(q.float().numpy(), k.float().numpy(), v.float().numpy())
-    assert rel_rms(got, src) <= 0.1
 
 
 def test_bitwise_deterministic_1000_launches():

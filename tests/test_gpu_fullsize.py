@@ -1,0 +1,96 @@
+"""Parity at the full benchmark sizes, in the launch configuration the bench times (one
+attn_fwd call over the whole problem), on sampled query rows the oracle computes one by
+one: first/last rows of tiles, the middle and the end of the sequence, plus seeded random
+rows, on the first, a middle and the last query heads."""
+import numpy as np
+import pytest
+import torch
+
+import bf16_causal_prefill_attn_b200 as pkg
+import synth
+from oracle import attention, hadamard, leanp, quantize
+
+pytestmark = pytest.mark.gpu
+
+
+def sample_rows(S, seed=0):
+    fixed = [0, 1, 127, 128, 255, S // 2 - 1, S // 2, S - 129, S - 128, S - 1]
+    rnd = np.random.default_rng(seed).integers(0, S, size=6).tolist()
+    return sorted(set(r for r in fixed + rnd if 0 <= r < S))
+
+
+def rel_rms(got, ref):
+    return float(np.sqrt(((got - ref) ** 2).sum() / (ref ** 2).sum()))
+
+
+CONFIGS = {
+    # name: (B, S, Hq, Hkv, d_qk, dist)
+    "gqa16k_outlier": (1, 16384, 32, 8, 128, "outlier"),
+    "mha32k_gaussian": (1, 32768, 32, 32, 128, "gaussian"),
+    "mla16k_outlier": (1, 16384, 16, 16, 192, "outlier"),
+    "mla32k_outlier": (1, 32768, 16, 16, 192, "outlier"),
+    "sweep_s1k_b32": (32, 1024, 32, 8, 128, "gaussian"),
+    "sweep_s8k_b4": (4, 8192, 32, 8, 128, "outlier"),
+}
+
+
+def _heads(Hq):
+    return sorted(set([0, 1, Hq // 2, Hq - 1]))
+
+
+@pytest.mark.parametrize("name", ["gqa16k_outlier", "mha32k_gaussian", "sweep_s1k_b32"])
+def test_bf16_fullsize(name):
+    B, S, Hq, Hkv, dqk, dist = CONFIGS[name]
+    q, k, v = synth.make_qkv(B, S, Hq, Hkv, dqk, 128, seed=0, dist=dist)
+    o, lse = pkg.attn_fwd(q.cuda(), k.cuda(), v.cuda())
+    torch.cuda.synchronize()
+    assert pkg.attn_device_status() == pkg.ATTN_OK
+    o = o.float().cpu().numpy()
+    lse = lse.cpu().numpy()
+    rows, heads = sample_rows(S), _heads(Hq)
+    for b in sorted(set([0, B - 1])):
+        ref, lref = attention.causal_attention_rows(q.float().numpy(), k.float().numpy(),
+                                                    v.float().numpy(), rows, heads, batch=b)
+        mag, _ = attention.causal_attention_rows(q.float().numpy(), k.float().numpy(),
+                                                 np.abs(v.float().numpy()), rows, heads, batch=b)
+        got = o[b][rows][:, heads, :].transpose(1, 0, 2)
+        err = np.abs(got - ref)
+        assert (err / (1e-2 * np.maximum(1.0, mag))).max() <= 1.0
+        assert rel_rms(got, ref) <= 5e-3
+        assert np.abs(lse[b][heads][:, rows] - lref).max() <= 2e-3
+
+
+@pytest.mark.parametrize("name,rotate", [("gqa16k_outlier", False), ("mha32k_gaussian", False),
+                                         ("mla16k_outlier", False), ("mla32k_outlier", False),
+                                         ("sweep_s1k_b32", True), ("sweep_s8k_b4", True)])
+def test_fp8_fullsize(name, rotate):
+    B, S, Hq, Hkv, dqk, dist = CONFIGS[name]
+    q, k, v = synth.make_qkv(B, S, Hq, Hkv, dqk, 128, seed=0, dist=dist)
+    dev = [pkg.attn_quantize_e4m3(t.cuda(), hadamard=rotate) for t in (q, k, v)]
+    (q8, dq), (k8, dk), (v8, dv) = dev
+    o, lse = pkg.attn_fwd(q8, k8, v8, descale_q=dq, descale_k=dk, descale_v=dv, unrotate=rotate)
+    torch.cuda.synchronize()
+    assert pkg.attn_device_status() == pkg.ATTN_OK
+    o = o.float().cpu().numpy()
+    host = []
+    for t, (c, d) in zip((q, k, v), dev):
+        hc, hd = quantize.quantize_e4m3(t.float().numpy(), rotate=rotate)
+        assert d.item() == float(hd)
+        # codes: bit-exact on the sampled rows' slices of every tensor
+        cc = c.cpu().numpy()
+        sel = np.asarray(sample_rows(S))
+        assert np.array_equal(cc[:, sel], hc[:, sel])
+        host.append((hc, hd))
+    rows, heads = sample_rows(S), _heads(Hq)
+    deq = [quantize.dequantize(c, s) for c, s in host]
+    for b in sorted(set([0, B - 1])):
+        ref, _ = attention.causal_attention_rows(*deq, rows, heads, batch=b)
+        if rotate:
+            ref = hadamard.rotate_fp64(ref)
+        emu, _ = leanp.attention_rows(host[0][0], host[1][0], host[2][0], host[0][1],
+                                      host[1][1], host[2][1], rows, heads, batch=b)
+        if rotate:
+            emu = hadamard.rotate_fp64(emu)
+        got = o[b][rows][:, heads, :].transpose(1, 0, 2)
+        assert rel_rms(got, emu) <= 5e-3
+        assert rel_rms(got, ref) <= 3e-2
