@@ -1,0 +1,392 @@
+"""Benchmark: causal prefill attention TFLOP/s on B200 through the C-ABI library.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+  FP8   per-tensor e4m3 quantisation of Q, K and V, then the lean-P attention kernel;
+  BF16  the attention kernel.
+The headline `value` is the FP8 step on the workload (default: GQA Hq=32/Hkv=8,
+S=16384, d=128, outlier-channel inputs); the BF16 step is timed on the same workload
+and reported under "bf16".  Throughput counts causal FLOPs 2*B*Hq*S^2/2*(d_qk+d_v).
+
+Timing: W warm-up steps, then K steps, each bracketed by CUDA events on the launching
+stream, with a 256 MiB L2 flush written between steps outside the events; a barrier and
+a device synchronisation bracket the whole timed region; multi-GPU runs take the max over
+ranks.  `e2e` repeats the FP8 step through the same calls with pinned host buffers: the
+host->device copies of Q, K, V and the device->host copy of O are inside its timing.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                       [--impl reference] [--no-cpu-baseline]
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "causal prefill attn TFLOP/s (FP8 e4m3, BF16) at 16K/32K; % of B200 tensor peak"
+UNIT = "TFLOP/s"
+NOMINAL_FP8_TFLOPS = 4500.0
+NOMINAL_BF16_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+WORKLOADS = {
+    # name: (B, S, Hq, Hkv, d_qk, d_v, distribution, description)
+    "gqa16k_outlier": (1, 16384, 32, 8, 128, 128, "outlier",
+                       "GQA causal prefill B=1 Hq=32 Hkv=8 S=16384 d=128, outlier-channel inputs"),
+    "mha32k_gaussian": (1, 32768, 32, 32, 128, 128, "gaussian",
+                        "causal prefill B=1 H=32 S=32768 d=128, Gaussian inputs"),
+    "mla16k_outlier": (1, 16384, 16, 16, 192, 128, "outlier",
+                       "MLA-shaped causal prefill B=1 H=16 S=16384 d_qk=192 d_v=128, outlier inputs"),
+    "mla32k_outlier": (1, 32768, 16, 16, 192, 128, "outlier",
+                       "MLA-shaped causal prefill B=1 H=16 S=32768 d_qk=192 d_v=128, outlier inputs"),
+}
+for _s in (1024, 2048, 4096, 8192, 16384, 32768):
+    WORKLOADS[f"sweep_s{_s // 1024}k"] = (
+        32768 // _s, _s, 32, 8, 128, 128, "gaussian",
+        f"sweep B*S=32768 S={_s} Hq=32 Hkv=8 d=128, Gaussian inputs")
+
+
+def causal_flops(B, Hq, S, d_qk, d_v):
+    return 2.0 * B * Hq * S * S / 2.0 * (d_qk + d_v)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 50 ms while active."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) == 7:
+                    rows.append(parts)
+        except OSError:
+            pass
+        finally:
+            try:
+                os.unlink(self.path)
+            except OSError:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[3 + i] == "Active"})
+        # samples under load: SM clock above idle
+        loaded = [x for x in sm if x > 600] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- GPU leg
+def gpu_bench(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import bf16_causal_prefill_attn_b200 as pkg
+    import synth
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    B, S, Hq, Hkv, dqk, dv, distn, desc = WORKLOADS[args.workload]
+    flops = causal_flops(B, Hq, S, dqk, dv)
+    q_h, k_h, v_h = synth.make_qkv(B, S, Hq, Hkv, dqk, dv, seed=rank, dist=distn)
+    q_h, k_h, v_h = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    stream = torch.cuda.current_stream(dev)
+    # outputs and scratch allocated once (the library never allocates)
+    q8 = torch.empty(q.shape, dtype=torch.uint8, device=dev)
+    k8 = torch.empty(k.shape, dtype=torch.uint8, device=dev)
+    v8 = torch.empty(v.shape, dtype=torch.uint8, device=dev)
+    ds = [torch.empty(1, dtype=torch.float32, device=dev) for _ in range(3)]
+    ws = [torch.empty(4, dtype=torch.int32, device=dev) for _ in range(3)]
+    o = torch.empty((B, S, Hq, dv), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, Hq, S), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.int32, device=dev)
+    o_h = torch.empty(o.shape, dtype=torch.bfloat16).pin_memory()
+
+    def fp8_step(ev_a=None, ev_b=None):
+        pkg.attn_quantize_e4m3(q, hadamard=args.hadamard, out=q8, descale=ds[0], workspace=ws[0])
+        pkg.attn_quantize_e4m3(k, hadamard=args.hadamard, out=k8, descale=ds[1], workspace=ws[1])
+        pkg.attn_quantize_e4m3(v, hadamard=args.hadamard, out=v8, descale=ds[2], workspace=ws[2])
+        if ev_a is not None:
+            ev_a.record(stream)
+        pkg.attn_fwd(q8, k8, v8, descale_q=ds[0], descale_k=ds[1], descale_v=ds[2], out=o, lse=lse,
+                     unrotate=args.hadamard)
+        if ev_b is not None:
+            ev_b.record(stream)
+
+    def bf16_step(ev_a=None, ev_b=None):
+        if ev_a is not None:
+            ev_a.record(stream)
+        pkg.attn_fwd(q, k, v, out=o, lse=lse)
+        if ev_b is not None:
+            ev_b.record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    def timed(step, K, W):
+        for _ in range(W):
+            flush.zero_()
+            step()
+        barrier()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+        for i in range(K):
+            flush.zero_()
+            s0, k0, k1, s1 = evs[i]
+            s0.record(stream)
+            step(k0, k1)
+            s1.record(stream)
+        barrier()
+        step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+        kern_ms = [e[1].elapsed_time(e[2]) for e in evs]
+        st = pkg.attn_device_status()
+        if st != pkg.ATTN_OK:
+            raise RuntimeError(f"device status {pkg.status_string(st)}")
+        return step_ms, kern_ms
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    peaks, peak_src = load_peaks()
+    with ClockSampler(local_rank) as clk:
+        fp8_step_ms, fp8_kern_ms = timed(fp8_step, args.steps, args.warmup)
+        bf16_step_ms, bf16_kern_ms = timed(bf16_step, args.steps, args.warmup)
+    clocks = clk.summary()
+
+    # end to end: pinned host buffers, H2D of the inputs and D2H of O inside the timing
+    def e2e_step(ev_a=None, ev_b=None):
+        q.copy_(q_h, non_blocking=True)
+        k.copy_(k_h, non_blocking=True)
+        v.copy_(v_h, non_blocking=True)
+        fp8_step(ev_a, ev_b)
+        o_h.copy_(o, non_blocking=True)
+
+    e2e_ms, _ = timed(e2e_step, max(3, args.steps // 4), max(1, args.warmup // 2))
+    h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h))
+    d2h = o_h.numel() * o_h.element_size()
+
+    fp8_ms = max_over_ranks(statistics.mean(fp8_step_ms))
+    fp8_kern = max_over_ranks(statistics.mean(fp8_kern_ms))
+    bf16_ms = max_over_ranks(statistics.mean(bf16_step_ms))
+    bf16_kern = max_over_ranks(statistics.mean(bf16_kern_ms))
+    e2e_mean = max_over_ranks(statistics.mean(e2e_ms))
+    total_flops = flops * world
+    bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    fp8_peak = 2.0 * bf16_peak  # measured bf16 peak x the nominal fp8/bf16 ratio (2)
+    fp8_kern_tf = flops / (fp8_kern * 1e-3) / 1e12
+    bf16_kern_tf = flops / (bf16_kern * 1e-3) / 1e12
+    traffic = load_traffic(args.workload)
+    result = {
+        "metric": METRIC,
+        "value": round(total_flops / (fp8_ms * 1e-3) / 1e12, 2),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(fp8_ms, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e4m3",
+        "data": "synthetic",
+        "config": {"workload": desc, "name": args.workload, "B": B, "S": S, "Hq": Hq, "Hkv": Hkv,
+                   "d_qk": dqk, "d_v": dv, "hadamard": bool(args.hadamard),
+                   "step": "e4m3 quantisation of Q, K, V + lean-P attention",
+                   "l2": "256 MiB L2 flush written between steps, outside the timed step",
+                   "parallelism": f"replicas x{world} (independent problems per GPU)"},
+        "roofline": {"bound": "tensor", "achieved": round(fp8_kern_tf, 2),
+                     "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
+                     "frac": round(fp8_kern_tf / fp8_peak, 4),
+                     "peak_source": f"{peak_src} bf16 cuBLAS burst x2 (fp8/bf16 nominal ratio)",
+                     "frac_of_nominal_4500": round(fp8_kern_tf / NOMINAL_FP8_TFLOPS, 4),
+                     "kernel": "attn_fwd_kernel<fp8>", "kernel_ms": round(fp8_kern, 4),
+                     "traffic": traffic.get("fp8")},
+        "bf16": {"value": round(total_flops / (bf16_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+                 "ms_per_step": round(bf16_ms, 4), "dtype": "bf16",
+                 "roofline": {"bound": "tensor", "achieved": round(bf16_kern_tf, 2),
+                              "peak": round(bf16_peak, 1), "unit": "TFLOP/s",
+                              "frac": round(bf16_kern_tf / bf16_peak, 4),
+                              "peak_source": f"{peak_src} bf16 cuBLAS burst",
+                              "frac_of_nominal_2250": round(bf16_kern_tf / NOMINAL_BF16_TFLOPS, 4),
+                              "traffic": traffic.get("bf16")}},
+        "e2e": {"value": round(total_flops / (e2e_mean * 1e-3) / 1e12, 2), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_mean, 4)},
+        "gpu_launches": args.steps * 7 + args.steps,
+        "clocks": clocks,
+    }
+    return result
+
+
+def load_traffic(workload):
+    """DRAM bytes per launch from the committed ncu summary, if it covers this workload
+    and the current kernel source (else null)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return {}
+    return d.get(workload, {})
+
+
+# ----------------------------------------------------------------------------- CPU leg
+def cpu_reference(workload, budget_s, rank=0):
+    """The oracle (fp64 attention on the dequantised FP8 inputs), as it stands, on a bounded
+    sample of query rows of the workload, on this host's cores."""
+    import numpy as np
+
+    import synth
+    from oracle import attention, quantize
+
+    B, S, Hq, Hkv, dqk, dv, distn, desc = WORKLOADS[workload]
+    q, k, v = synth.make_qkv(B, S, Hq, Hkv, dqk, dv, seed=rank, dist=distn)
+    deq = [quantize.dequantize(*quantize.quantize_e4m3(t.float().numpy())) for t in (q, k, v)]
+    rng = np.random.default_rng(0)
+    done_flops = 0.0
+    rows_done = 0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < budget_s:
+        h = int(rng.integers(0, Hq))
+        rows = np.sort(rng.integers(0, S, size=8))
+        attention.causal_attention_rows(*deq, rows, [h], batch=int(rng.integers(0, B)))
+        done_flops += sum(2.0 * (int(i) + 1) * (dqk + dv) for i in rows)
+        rows_done += len(rows)
+    dt = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    return {"value": done_flops / dt / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{rows_done} random causal query rows (fp64, all visible keys) of {desc}; "
+                      f"{dt:.1f} s; quantisation and input generation not timed",
+            "seconds": dt}
+
+
+def reference_main(args, rank, world):
+    if rank != 0:
+        return 0
+    budget = max(1.0, 20.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        cpu_reference(args.workload, budget / 4)
+    vals, secs = [], 0.0
+    last = None
+    for _ in range(args.steps):
+        last = cpu_reference(args.workload, budget)
+        vals.append(last["value"])
+        secs += last["seconds"]
+    B, S, Hq, Hkv, dqk, dv, distn, desc = WORKLOADS[args.workload]
+    value = statistics.mean(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": secs * 1e3 / max(1, args.steps), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": desc, "name": args.workload},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": last["cores"],
+                             "kind": "oracle", "sample": last["sample"]},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="gqa16k_outlier", choices=sorted(WORKLOADS))
+    ap.add_argument("--hadamard", action="store_true")
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return reference_main(args, rank, world)
+    # the oracle baseline is measured before any CUDA call (no fork after CUDA init)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_reference(args.workload, args.cpu_seconds)
+        cpu.pop("seconds", None)
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        res = gpu_bench(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    if rank == 0:
+        res["cpu_baseline"] = cpu
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
