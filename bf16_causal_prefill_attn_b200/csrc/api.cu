@@ -257,3 +257,55 @@ const char* attn_status_string(attn_status_t s) {
 int attn_version(void) { return kVersion; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------
+// Quantiser entry point for callers that cannot allocate device memory.
+//
+// attn_quantize_e4m3 needs a few bytes of device scratch (the running amax).  Some callers
+// cannot provide it: a plugin running inside an engine whose device memory is planned and
+// owned entirely by the host framework, or a latency-critical loop where a cudaMalloc
+// (which may synchronise the device) is not allowed.  attn_quantize_e4m3_static takes the
+// scratch from a fixed array compiled into this library instead.  Every GPU that loads the
+// library holds the array until the process exits.
+namespace {
+
+constexpr size_t kStaticScratchBytes = 256;  // maximum scratch this entry point can use
+static __device__ __align__(256) uint32_t g_static_scratch[kStaticScratchBytes / 4];
+
+constexpr int kMaxDevices = 128;
+std::mutex g_static_mu;
+uint32_t* g_static_ptr[kMaxDevices] = {};
+
+// Device address of g_static_scratch on the current device.  In host code the array's
+// name only stands in for the symbol; the address is looked up once per device, with that
+// device current, on the first call made on it.
+attn_status_t static_scratch(uint32_t** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (g_static_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr)
+      return ATTN_ERR_CUDA;
+    g_static_ptr[dev] = static_cast<uint32_t*>(p);
+  }
+  *out = g_static_ptr[dev];
+  return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" attn_status_t attn_quantize_e4m3_static(const void* x_bf16, void* x_e4m3,
+                                                   float* descale_out, int64_t tokens, int H,
+                                                   int d, int hadamard, void* stream) {
+  if (tokens < 0 || H <= 0 || d <= 0) return ATTN_ERR_INVALID_ARG;
+  if (attn_quantize_workspace_size(tokens, H, d) > kStaticScratchBytes)
+    return ATTN_ERR_UNSUPPORTED;  // would need more scratch than the fixed array holds
+  uint32_t* scratch = nullptr;
+  const attn_status_t st = static_scratch(&scratch);
+  if (st != ATTN_OK) return st;
+  // same kernels as attn_quantize_e4m3; the amax word is cleared at the start of every call
+  return attn_quantize_e4m3(x_bf16, x_e4m3, descale_out, tokens, H, d, hadamard, scratch,
+                            kStaticScratchBytes, stream);
+}

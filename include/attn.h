@@ -98,6 +98,25 @@ attn_status_t attn_quantize_e4m3(const void* x_bf16, void* x_e4m3, float* descal
 size_t attn_quantize_workspace_size(int64_t tokens, int H, int d);
 
 /*
+ * attn_quantize_e4m3_static: attn_quantize_e4m3 for callers that cannot allocate device
+ * memory (e.g. a plugin inside an engine that owns and pre-plans all device memory, or a
+ * latency-critical loop where cudaMalloc's possible device synchronisation is not allowed).
+ * The pages have no counterpart: it is an interface convenience of this library.
+ *   Same arguments, results and codes as attn_quantize_e4m3, minus the workspace: the
+ *   scratch is a fixed 256-byte array compiled into the library, held on every GPU that
+ *   loads it until the process exits.  A problem whose scratch need
+ *   (attn_quantize_workspace_size) exceeds 256 bytes returns ATTN_ERR_UNSUPPORTED.
+ *   The first call on a device looks up the array's device address (with that device
+ *   current); make that first call before any stream capture.  All calls share the array
+ *   (it keeps the last call's contents; the amax word is cleared at the start of each call),
+ *   so calls that may overlap on the GPU -- on different streams, or from different host
+ *   threads -- race and must be serialised by the caller.  Allocates nothing.
+ */
+attn_status_t attn_quantize_e4m3_static(const void* x_bf16, void* x_e4m3, float* descale_out,
+                                        int64_t tokens, int H, int d, int hadamard,
+                                        void* stream);
+
+/*
  * Test-only: FP8 attn_fwd that also dumps, for every (query row, visible key tile), the
  * raw fp32 scores after masking, the lean-P e4m3 codes and the per-64-key shifts:
  *   dump_s      [B, Hq, S, S] fp32      dump_codes [B, Hq, S, S] uint8
