@@ -77,7 +77,15 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, attn::FwdP
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC) !=
       cudaSuccess)
     return ATTN_ERR_CUDA;
-  const unsigned grid = static_cast<unsigned>(prm.n_q_tiles) * prm.B * prm.Hq;
+  // The kernel moves registers from its producer/MMA warps to its softmax warps
+  // (setmaxnreg); the increase only succeeds if the block was launched with at least
+  // REGS_NEEDED_AT_LAUNCH registers per thread, so never launch with fewer.
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (fa.numRegs < attn::REGS_NEEDED_AT_LAUNCH ||
+      fa.numRegs * attn::NUM_THREADS > 65536)
+    return ATTN_ERR_UNSUPPORTED;
+  const unsigned grid = static_cast<unsigned>(prm.n_pairs) * prm.B * prm.Hq;
   kern<<<grid, attn::NUM_THREADS, C::SMEM_ALLOC, stream>>>(mq, mk, mv, prm);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -99,7 +107,7 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, flo
     return ATTN_ERR_INVALID_ARG;
   if (S % 128 != 0) return ATTN_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(B) * S > INT32_MAX ||
-      static_cast<int64_t>(S / 128) * B * Hq > INT32_MAX)
+      static_cast<int64_t>((S / 128 + 1) / 2) * B * Hq > INT32_MAX)
     return ATTN_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_ALIGNMENT;
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATTN_ERR_ALIGNMENT;
@@ -111,6 +119,7 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, flo
   prm.Hkv = Hkv;
   prm.G = Hq / Hkv;
   prm.n_q_tiles = S / 128;
+  prm.n_pairs = (prm.n_q_tiles + 1) / 2;
   prm.causal = causal;
   prm.o = static_cast<__nv_bfloat16*>(o);
   prm.lse = lse;

@@ -1,30 +1,36 @@
 // Forward causal (prefill) attention on sm_100a: TMA-fed tcgen05 MMAs with TMEM
-// accumulators, warp-specialised.
+// accumulators, warp-specialised, two query tiles per CTA in ping-pong.
 //
-// Computes O = softmax(mask(Q K^T * scale)) V for one 128-row query tile per CTA
-// (the forward causal attention of the prefill phase, [ZYFA-fr] "Ce que couvrent les
-// noyaux"), in two precisions:
+// Computes O = softmax(mask(Q K^T * scale)) V (the forward causal attention of the
+// prefill phase, [ZYFA-fr] "Ce que couvrent les noyaux") in two precisions:
 //   BF16  S = Q K^T (kind::f16, fp32 accumulate); P = exp2((S - M) * scale * log2 e) in
-//         fp32, rounded to bf16 for O += P V; the row sum is accumulated in fp32.
+//         fp32 (three quarters on the MUFU, one quarter by a polynomial on the FMA pipe),
+//         rounded to bf16 for O += P V; the row sum is accumulated in fp32.
 //   FP8   S = Q K^T on e4m3 codes (kind::f8f6f4); P is produced without an exponential by
 //         the lean-P encoding ([ZYFA-mb] "Como o motor de atenção FP8 da Zyphra
-//         funciona": one multiply-add and an integer conversion write the e4m3 bit
-//         pattern), each 64-key block carries a power-of-two shift that the block-scaled
-//         MMA (kind::mxf8f6f4.block_scale, UE8M0 scale per 32 keys) removes, and the row
-//         normaliser is the sum of the rounded probabilities formed by one extra MMA per
+//         funciona": a multiply-add and an integer conversion write the e4m3 bit pattern);
+//         each 64-key block carries a power-of-two shift that the block-scaled MMA
+//         (kind::mxf8f6f4.block_scale, UE8M0 scale per 32 keys) removes, and the row
+//         normaliser is the sum of the rounded probabilities, formed by one extra MMA per
 //         key tile against a matrix of ones.
 //
-// Roles (192 threads):
-//   warps 0-3  softmax: thread r owns query row r of the tile (TMEM lane r); reads S,
-//              updates the running max, rescales O in TMEM when the max grows, writes P
-//              (and the FP8 scale factors) to TMEM, and finally writes O and lse.
-//   warp 4     TMA producer: Q once, then K and V tiles through an NST-stage ring.
-//   warp 5     TMEM allocator and MMA issuer (one thread): S(j+1) is issued before
-//              PV(j) so the tensor core computes the next scores while the softmax warps
-//              turn S(j) into P(j).
-// TMEM (512 columns x 128 lanes, fp32): S double buffer [0,256), O [256,384), P at 384
-// (bf16: 64 columns, e4m3: 32), and for FP8 the row-sum accumulator at 448 (16 columns),
-// scale factors of P at 464 (4 columns) and of V / ones at 468 (4 columns).
+// A CTA owns two 128-row query tiles t = 0, 1 of one (batch, head): rows
+// [256 p + 128 t, +128) of query-tile pair p.  They share every K/V tile in shared memory.
+// Roles (384 threads, 12 warps):
+//   warps 0-3   softmax of tile 0, warps 4-7 softmax of tile 1: thread r of the group owns
+//               query row r (TMEM lane r); reads S, updates the reference max (lazily:
+//               only when the tile max exceeds it by more than the headroom), rescales O
+//               in TMEM when it does, writes P (and the FP8 scale factors) into the S
+//               columns it has consumed, and finally writes O and lse;
+//   warp 8      TMA producer: both Q tiles once, then K and V through NK / NV stages;
+//   warp 9      MMA issuer (warp-wide control flow, one elected lane issues), in the fixed
+//               order PV_0(j), S_0(j+1), PV_1(j), S_1(j+1): one tile's softmax overlaps
+//               the other tile's MMAs (ping-pong);
+//   warp 10     idle; warp 11 TMEM allocator.
+// TMEM (512 columns x 128 lanes): S_0 [0,128), S_1 [128,256), O_0 [256,384),
+// O_1 [384,512).  P_t overwrites the first columns of S_t (bf16: 64, e4m3: 32); for FP8
+// the scale factors of P_t sit at S_t + 32 (4 columns), those of B at S_t + 36 (4) and the
+// row-sum MMA writes S_t + 64 (16), read back by the softmax group before S_t(j+1).
 //
 // Every wait is bounded (mbar_wait): on expiry the CTA records DEV_TIMEOUT and unwinds.
 #pragma once
@@ -39,14 +45,30 @@ namespace attn {
 constexpr int BLOCK_M = 128;
 constexpr int BLOCK_N = 128;
 constexpr int DV = 128;
-constexpr int NUM_THREADS = 192;
-constexpr uint32_t TM_S0 = 0, TM_O = 256, TM_P = 384, TM_RS = 448, TM_SFA = 464, TM_SFB = 468;
+constexpr int NUM_THREADS = 384;
+constexpr int REGS_SOFTMAX = 208;  // per thread of warps 0-7 after setmaxnreg
+constexpr int REGS_OTHER = 88;     // per thread of warps 8-11
+// registers per thread the launch must provide at least for that split
+constexpr int REGS_NEEDED_AT_LAUNCH =
+    (2 * 128 * REGS_SOFTMAX + 128 * REGS_OTHER + NUM_THREADS - 1) / NUM_THREADS;
+constexpr uint32_t TM_O = 256;
+constexpr uint32_t TM_SFA_OFF = 32, TM_SFB_OFF = 36, TM_RS_OFF = 64;
 constexpr float LEANP_MAGIC = 12582912.0f;  // 1.5 * 2^23
 constexpr int LEANP_KMAX = 16;
+constexpr int LEANP_TOP = 112;       // code of a block maximum at the reference
+constexpr int LEANP_HEADROOM = 14;   // 126 - LEANP_TOP
+constexpr float BF16_HEADROOM = 8.0f;  // log2 units the reference max may lag the true max
+
+// 2^f on [-0.5, 0.5], degree 3, coefficients fitted here to minimise the relative error
+// (max 7.5e-5, well under the bf16 rounding of P)
+constexpr float EXP2_C0 = 0.99992817640304565f;
+constexpr float EXP2_C1 = 0.69326096773147583f;
+constexpr float EXP2_C2 = 0.24260970950126648f;
+constexpr float EXP2_C3 = 0.05517097562551498f;
 
 struct FwdParams {
   int B, S, Hq, Hkv, G;
-  int n_q_tiles;
+  int n_q_tiles, n_pairs;
   int causal;
   __nv_bfloat16* o;   // [B, S, Hq, DV]
   float* lse;         // [B, Hq, S] or null
@@ -58,7 +80,7 @@ struct FwdParams {
   int unrotate;       // apply x H / sqrt(128) to each output row (Hadamard-rotated V)
   uint32_t* err;
   uint64_t timeout_ns;
-  float* dump_s;      // FP8 debug: raw scores [B, Hq, S, S]
+  float* dump_s;         // FP8 debug: raw scores [B, Hq, S, S]
   uint8_t* dump_codes;   // FP8 debug: P codes   [B, Hq, S, S]
   uint8_t* dump_kshift;  // FP8 debug: shifts    [B, Hq, S, S/64]
 };
@@ -73,33 +95,54 @@ struct FwdCfg {
   static constexpr int Q_BYTES = Q_BOXES * BOX_BYTES;
   static constexpr int K_BYTES = Q_BYTES;
   static constexpr int V_BYTES = V_BOXES * BOX_BYTES;
-  static constexpr int NST = FP8 ? 3 : 2;                       // K/V ring depth
+  static constexpr int NK = FP8 ? (DQK == 128 ? 4 : 3) : 2;     // K ring depth
+  static constexpr int NV = FP8 ? (DQK == 128 ? 4 : 3) : (DQK == 128 ? 2 : 1);
   static constexpr int KSTEP = FP8 ? 32 : 16;                   // MMA K per instruction
   static constexpr int QK_STEPS = DQK / KSTEP;
   static constexpr int PV_STEPS = BLOCK_N / KSTEP;
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + NST * K_BYTES;
-  static constexpr int OFF_ONES = OFF_V + NST * V_BYTES;        // FP8: 16 x 128 B of 1.0
+  static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
+  static constexpr int OFF_V = OFF_K + NK * K_BYTES;
+  static constexpr int OFF_ONES = OFF_V + NV * V_BYTES;         // FP8: 16 x 128 B of 1.0
   static constexpr int OFF_BAR = OFF_ONES + (FP8 ? 2048 : 0);
-  // barriers: q_full, k_full[NST], k_empty[NST], v_full[NST], v_empty[NST], s_full[2],
-  //           s_empty[2], p_full, o_done, sf_bar, mma_done
-  static constexpr int NUM_BARS = 1 + 4 * NST + 4 + 4;
+  // barriers: q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], and per tile:
+  //           s_full, p_full, pv_done, s_free, sf_bar, mma_done
+  static constexpr int NUM_BARS = 1 + 2 * NK + 2 * NV + 2 * 6;
   static constexpr int OFF_TMEMPTR = OFF_BAR + NUM_BARS * 8;
-  static constexpr int OFF_SF = (OFF_TMEMPTR + 4 + 15) / 16 * 16;  // [2][128] u32
-  static constexpr int SMEM_BYTES = OFF_SF + 2 * 128 * 4;
+  static constexpr int OFF_SF = (OFF_TMEMPTR + 4 + 15) / 16 * 16;  // [2 tiles][2][128] u32
+  static constexpr int SMEM_BYTES = OFF_SF + (FP8 ? 2 * 2 * 128 * 4 : 0);
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;           // 1024-B alignment slack
   static constexpr uint32_t IDESC_S =
       idesc_dense(FP8 ? 0u : 1u, FP8 ? 0u : 1u, 0u, 0u, BLOCK_M, BLOCK_N);
   static constexpr uint32_t IDESC_PV_BF16 = idesc_dense(1u, 1u, 0u, 1u, BLOCK_M, DV);
 };
 
-// k'_b: power-of-two shift of one 64-key block (block max mu, reference m in byte units)
+// k_b: power-of-two shift of one 64-key block (block max mu, reference m in code units)
 __device__ __forceinline__ int leanp_kshift(float mu, float a, int m) {
   float t = __fmaf_rn(mu, a, -__int2float_rn(m));
   float g = -t * 0.125f;
   int k = __float2int_rd(g);  // saturating: +inf -> INT_MAX
   return min(max(k, 0), LEANP_KMAX);
+}
+
+__device__ __forceinline__ float fma_sat(float a, float b, float c) {
+  float d;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for x <= 8 on the FMA pipe: x = n + f, f in [-0.5, 0.5], 2^f by the polynomial,
+// 2^n added to the exponent field.  Inputs below -125 give 2^-125.
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -125.0f);
+  const float j = __fadd_rn(x, LEANP_MAGIC);   // round to the nearest integer n
+  const float n = __fsub_rn(j, LEANP_MAGIC);
+  const float f = __fsub_rn(x, n);
+  float p = __fmaf_rn(EXP2_C3, f, EXP2_C2);
+  p = __fmaf_rn(p, f, EXP2_C1);
+  p = __fmaf_rn(p, f, EXP2_C0);
+  // low bits of j hold n (two's complement); n << 23 added to the exponent of p
+  return __int_as_float(__float_as_int(j) * (1 << 23) + __float_as_int(p));
 }
 
 template <bool FP8, int DQK, bool DUMP>
@@ -114,15 +157,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
-  uint64_t* k_empty = k_full + C::NST;
-  uint64_t* v_full = k_empty + C::NST;
-  uint64_t* v_empty = v_full + C::NST;
-  uint64_t* s_full = v_empty + C::NST;
-  uint64_t* s_empty = s_full + 2;
-  uint64_t* p_full = s_empty + 2;
-  uint64_t* o_done = p_full + 1;
-  uint64_t* sf_bar = o_done + 1;
-  uint64_t* mma_done = sf_bar + 1;
+  uint64_t* k_empty = k_full + C::NK;
+  uint64_t* v_full = k_empty + C::NK;
+  uint64_t* v_empty = v_full + C::NV;
+  uint64_t* tbar = v_empty + C::NV;  // per tile: 6 barriers
+  auto s_full = [&](int t) { return tbar + 6 * t + 0; };
+  auto p_full = [&](int t) { return tbar + 6 * t + 1; };
+  auto pv_done = [&](int t) { return tbar + 6 * t + 2; };
+  auto s_free = [&](int t) { return tbar + 6 * t + 3; };
+  auto sf_bar = [&](int t) { return tbar + 6 * t + 4; };
+  auto mma_done = [&](int t) { return tbar + 6 * t + 5; };
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEMPTR);
   uint32_t* sf_x = reinterpret_cast<uint32_t*>(smem + C::OFF_SF);
 
@@ -130,39 +174,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
-  // longest-processing-time order: the longest query tiles (largest causal extent) first
+  // longest-processing-time order: the pairs with the largest causal extent first
   const int nbh = p.B * p.Hq;
-  const int qt = p.n_q_tiles - 1 - static_cast<int>(blockIdx.x) / nbh;
+  const int pr = p.n_pairs - 1 - static_cast<int>(blockIdx.x) / nbh;
   const int bh = static_cast<int>(blockIdx.x) % nbh;
   const int b = bh / p.Hq;
   const int h = bh % p.Hq;
   const int g = h / p.G;
-  const int n_kv = p.causal ? qt + 1 : p.n_q_tiles;
+  const int qt0 = 2 * pr;                               // query tile of t = 0
+  const bool has1 = qt0 + 1 < p.n_q_tiles;              // t = 1 exists
+  const int n_t0 = p.causal ? qt0 + 1 : p.n_q_tiles;     // key tiles of each query tile
+  const int n_t1 = has1 ? (p.causal ? qt0 + 2 : p.n_q_tiles) : 0;
+  const int n_max = n_t1 > n_t0 ? n_t1 : n_t0;
   const int tok0 = b * p.S;  // first token of this batch entry
 
   if (tid == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < C::NST; ++i) {
+    for (int i = 0; i < C::NK; ++i) {
       mbar_init(k_full + i, 1);
       mbar_init(k_empty + i, 1);
+    }
+    for (int i = 0; i < C::NV; ++i) {
       mbar_init(v_full + i, 1);
       mbar_init(v_empty + i, 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(s_full + i, 1);
-      mbar_init(s_empty + i, 128);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(s_full(t), 1);
+      mbar_init(p_full(t), 128);
+      mbar_init(pv_done(t), 1);
+      mbar_init(s_free(t), 128);
+      mbar_init(sf_bar(t), 128);
+      mbar_init(mma_done(t), 1);
     }
-    mbar_init(p_full, 128);
-    mbar_init(o_done, 1);
-    mbar_init(sf_bar, 128);
-    mbar_init(mma_done, 1);
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == 11) {
     tmem_alloc(tmem_ptr, 512);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
@@ -177,146 +227,184 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_ptr;
 
-  if (warp == 4) {
-    // ------------------------------------------------------------- TMA producer
-    if (lane == 0) {
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_OTHER));
+    if (warp == 8) {
+      // ----------------------------------------------------------- TMA producer (warp-wide,
+      // one elected lane issues)
       bool ok = true;
-      mbar_arrive_expect_tx(q_full, C::Q_BYTES);
-      for (int i = 0; i < C::Q_BOXES; ++i)
-        tma_load_3d(smem + C::OFF_Q + i * C::BOX_BYTES, &tm_q, q_full, i * C::BOX_COLS, h,
-                    tok0 + qt * BLOCK_M);
-      int j = 0;
-      bool v_issued_last = true;  // whether the V load of tile j-1 was issued
-      for (; j < n_kv && ok; ++j) {
-        const int st = j % C::NST;
-        const uint32_t use = j / C::NST;
-        if (j >= C::NST) ok = mbar_wait(k_empty + st, (use - 1) & 1, p.err, p.timeout_ns);
-        if (!ok) break;
-        mbar_arrive_expect_tx(k_full + st, C::K_BYTES);
-        for (int i = 0; i < C::Q_BOXES; ++i)
-          tma_load_3d(smem + C::OFF_K + st * C::K_BYTES + i * C::BOX_BYTES, &tm_k, k_full + st,
-                      i * C::BOX_COLS, g, tok0 + j * BLOCK_N);
-        if (j >= C::NST) ok = mbar_wait(v_empty + st, (use - 1) & 1, p.err, p.timeout_ns);
-        if (!ok) {
-          ++j;  // the K load of this tile is in flight, its V load is not
-          v_issued_last = false;
-          break;
-        }
-        mbar_arrive_expect_tx(v_full + st, C::V_BYTES);
-        for (int i = 0; i < C::V_BOXES; ++i)
-          tma_load_3d(smem + C::OFF_V + st * C::V_BYTES + i * C::BOX_BYTES, &tm_v, v_full + st,
-                      i * C::BOX_COLS, g, tok0 + j * BLOCK_N);
+      if (elect_one()) {
+        mbar_arrive_expect_tx(q_full, (has1 ? 2 : 1) * C::Q_BYTES);
+        for (int t = 0; t < (has1 ? 2 : 1); ++t)
+          for (int i = 0; i < C::Q_BOXES; ++i)
+            tma_load_3d(smem + C::OFF_Q + t * C::Q_BYTES + i * C::BOX_BYTES, &tm_q, q_full,
+                        i * C::BOX_COLS, h, tok0 + (qt0 + t) * BLOCK_M);
       }
-      // drain: make sure no copy issued by this CTA is still in flight at exit
+      __syncwarp();
+      int jk = 0, jv = 0;  // K and V tiles issued
+      for (int j = 0; j < n_max && ok; ++j) {
+        const int sk = j % C::NK;
+        if (j >= C::NK) ok = mbar_wait(k_empty + sk, ((j / C::NK) - 1) & 1, p.err, p.timeout_ns);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        if (elect_one()) {
+          mbar_arrive_expect_tx(k_full + sk, C::K_BYTES);
+          for (int i = 0; i < C::Q_BOXES; ++i)
+            tma_load_3d(smem + C::OFF_K + sk * C::K_BYTES + i * C::BOX_BYTES, &tm_k, k_full + sk,
+                        i * C::BOX_COLS, g, tok0 + j * BLOCK_N);
+        }
+        __syncwarp();
+        jk = j + 1;
+        const int sv = j % C::NV;
+        if (j >= C::NV) ok = mbar_wait(v_empty + sv, ((j / C::NV) - 1) & 1, p.err, p.timeout_ns);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        if (elect_one()) {
+          mbar_arrive_expect_tx(v_full + sv, C::V_BYTES);
+          for (int i = 0; i < C::V_BOXES; ++i)
+            tma_load_3d(smem + C::OFF_V + sv * C::V_BYTES + i * C::BOX_BYTES, &tm_v, v_full + sv,
+                        i * C::BOX_COLS, g, tok0 + j * BLOCK_N);
+        }
+        __syncwarp();
+        jv = j + 1;
+      }
+      // drain: no copy issued by this CTA may still be in flight at exit
       mbar_wait(q_full, 0, p.err, DRAIN_TIMEOUT_NS, false);
-      for (int jj = (j > C::NST ? j - C::NST : 0); jj < j; ++jj) {
-        const int st = jj % C::NST;
-        mbar_wait(k_full + st, (jj / C::NST) & 1, p.err, DRAIN_TIMEOUT_NS, false);
-        if (jj < j - 1 || v_issued_last)
-          mbar_wait(v_full + st, (jj / C::NST) & 1, p.err, DRAIN_TIMEOUT_NS, false);
-      }
-    }
-  } else if (warp == 5) {
-    // ------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      bool ok = mbar_wait(q_full, 0, p.err, p.timeout_ns);
-      const uint32_t q_base = smem_addr(smem + C::OFF_Q);
-      auto issue_pv = [&](int jj) -> bool {
-        const int st = jj % C::NST;
-        if (!mbar_wait(p_full, jj & 1, p.err, p.timeout_ns)) return false;
-        if (!mbar_wait(v_full + st, (jj / C::NST) & 1, p.err, p.timeout_ns)) return false;
-        tc_fence_after();
-        const uint32_t v_base = smem_addr(smem + C::OFF_V + st * C::V_BYTES);
-        if constexpr (!FP8) {
+      for (int jj = (jk > C::NK ? jk - C::NK : 0); jj < jk; ++jj)
+        mbar_wait(k_full + jj % C::NK, (jj / C::NK) & 1, p.err, DRAIN_TIMEOUT_NS, false);
+      for (int jj = (jv > C::NV ? jv - C::NV : 0); jj < jv; ++jj)
+        mbar_wait(v_full + jj % C::NV, (jj / C::NV) & 1, p.err, DRAIN_TIMEOUT_NS, false);
+    } else if (warp == 9) {
+      // ----------------------------------------------------------- MMA issuer (warp-wide
+      // control flow, one elected lane issues).  Fixed order per key tile j:
+      //   PV_0(j), S_0(j+1), PV_1(j), S_1(j+1)
+      // so tile 1's softmax of j overlaps PV_0(j) + S_0(j+1) and tile 0's softmax of j+1
+      // overlaps PV_1(j) + S_1(j+1) (ping-pong).
+      auto nt = [&](int t) { return t == 0 ? n_t0 : n_t1; };
+      const uint32_t ones_base = smem_addr(smem + C::OFF_ONES);
+      auto issue_s = [&](int t, int j) {
+        const int sk = j % C::NK;
+        const uint32_t q_base = smem_addr(smem + C::OFF_Q + t * C::Q_BYTES);
+        const uint32_t k_base = smem_addr(smem + C::OFF_K + sk * C::K_BYTES);
+        const uint32_t tm_s = tmem + t * 128;
+        if (elect_one()) {
 #pragma unroll
-          for (int s = 0; s < C::PV_STEPS; ++s) {
-            // V is [keys x d] with d contiguous: B operand MN-major; 8-key groups 1 KB apart,
-            // 64-column atoms 16 KB apart
-            const uint64_t bdesc = smem_desc_sw128(v_base + s * 2048, C::BOX_BYTES, 1024);
-            mma_ts_f16(tmem + TM_O, tmem + TM_P + s * 8, bdesc, C::IDESC_PV_BF16,
-                       (jj > 0 || s > 0) ? 1u : 0u);
+          for (int s = 0; s < C::QK_STEPS; ++s) {
+            const uint32_t off = (s / 4) * C::BOX_BYTES + (s % 4) * 32;
+            mma_ss<FP8 ? 1 : 0>(tm_s, smem_desc_sw128(q_base + off, 16, 1024),
+                                smem_desc_sw128(k_base + off, 16, 1024), C::IDESC_S,
+                                s > 0 ? 1u : 0u);
           }
-        } else {
-          const uint32_t ones_base = smem_addr(smem + C::OFF_ONES);
-#pragma unroll
-          for (int s = 0; s < C::PV_STEPS; ++s) {
-            const uint64_t bdesc = smem_desc_sw128(v_base + s * 4096, C::BOX_BYTES, 1024);
-            const uint32_t sfa = (tmem + TM_SFA) | (static_cast<uint32_t>(s) << 30);
-            const uint32_t sfb = (tmem + TM_SFB) | (static_cast<uint32_t>(s) << 30);
-            mma_ts_mxf8(tmem + TM_O, tmem + TM_P + s * 8, bdesc, idesc_mxf8(0, 1, BLOCK_M, DV, s, s),
-                        sfa, sfb, (jj > 0 || s > 0) ? 1u : 0u);
-          }
-#pragma unroll
-          for (int s = 0; s < C::PV_STEPS; ++s) {
-            // row sum of the rounded probabilities: P x ones (16 x 128 keys, K-major)
-            const uint64_t odesc = smem_desc_sw128(ones_base + s * 32, 16, 1024);
-            const uint32_t sfa = (tmem + TM_SFA) | (static_cast<uint32_t>(s) << 30);
-            const uint32_t sfb = (tmem + TM_SFB) | (static_cast<uint32_t>(s) << 30);
-            mma_ts_mxf8(tmem + TM_RS, tmem + TM_P + s * 8, odesc, idesc_mxf8(0, 0, BLOCK_M, 16, s, s),
-                        sfa, sfb, (jj > 0 || s > 0) ? 1u : 0u);
-          }
+          tc_commit(s_full(t));
+          // K(j) is free once its last S has run: tile 1's, or tile 0's if tile 1 skips j
+          if (t == 1 || j >= n_t1) tc_commit(k_empty + sk);
         }
-        tc_commit(o_done);
-        tc_commit(v_empty + st);
-        return true;
+        __syncwarp();
       };
-      int j = 0;
-      for (; j < n_kv && ok; ++j) {
-        const int st = j % C::NST;
-        const int sb = j & 1;
-        ok = mbar_wait(k_full + st, (j / C::NST) & 1, p.err, p.timeout_ns);
-        if (ok && j >= 2) ok = mbar_wait(s_empty + sb, ((j >> 1) - 1) & 1, p.err, p.timeout_ns);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t k_base = smem_addr(smem + C::OFF_K + st * C::K_BYTES);
+      auto issue_pv = [&](int t, int j) {
+        const int sv = j % C::NV;
+        const uint32_t v_base = smem_addr(smem + C::OFF_V + sv * C::V_BYTES);
+        const uint32_t tm_s = tmem + t * 128;
+        const uint32_t tm_o = tmem + TM_O + t * 128;
+        if (elect_one()) {
+          if constexpr (!FP8) {
 #pragma unroll
-        for (int s = 0; s < C::QK_STEPS; ++s) {
-          const uint32_t off = (s / 4) * C::BOX_BYTES + (s % 4) * 32;
-          const uint64_t adesc = smem_desc_sw128(q_base + off, 16, 1024);
-          const uint64_t bdesc = smem_desc_sw128(k_base + off, 16, 1024);
-          mma_ss<FP8 ? 1 : 0>(tmem + TM_S0 + sb * 128, adesc, bdesc, C::IDESC_S, s > 0 ? 1u : 0u);
+            for (int s = 0; s < C::PV_STEPS; ++s) {
+              // V is [keys x d] with d contiguous: B operand MN-major; 8-key groups 1 KB
+              // apart, 64-column atoms 16 KB apart
+              mma_ts_f16(tm_o, tm_s + s * 8,
+                         smem_desc_sw128(v_base + s * 2048, C::BOX_BYTES, 1024),
+                         C::IDESC_PV_BF16, (j > 0 || s > 0) ? 1u : 0u);
+            }
+          } else {
+#pragma unroll
+            for (int s = 0; s < C::PV_STEPS; ++s) {
+              const uint32_t sfa = (tm_s + TM_SFA_OFF) | (static_cast<uint32_t>(s) << 30);
+              const uint32_t sfb = (tm_s + TM_SFB_OFF) | (static_cast<uint32_t>(s) << 30);
+              mma_ts_mxf8(tm_o, tm_s + s * 8,
+                          smem_desc_sw128(v_base + s * 4096, C::BOX_BYTES, 1024),
+                          idesc_mxf8(0, 1, BLOCK_M, DV, s, s), sfa, sfb,
+                          (j > 0 || s > 0) ? 1u : 0u);
+            }
+#pragma unroll
+            for (int s = 0; s < C::PV_STEPS; ++s) {
+              // row sum of the rounded probabilities: P x ones (16 x 128 keys, K-major)
+              const uint32_t sfa = (tm_s + TM_SFA_OFF) | (static_cast<uint32_t>(s) << 30);
+              const uint32_t sfb = (tm_s + TM_SFB_OFF) | (static_cast<uint32_t>(s) << 30);
+              mma_ts_mxf8(tm_s + TM_RS_OFF, tm_s + s * 8,
+                          smem_desc_sw128(ones_base + s * 32, 16, 1024),
+                          idesc_mxf8(0, 0, BLOCK_M, 16, s, s), sfa, sfb, s > 0 ? 1u : 0u);
+            }
+          }
+          tc_commit(pv_done(t));
+          if (t == 1 || j >= n_t1) tc_commit(v_empty + sv);
         }
-        tc_commit(s_full + sb);
-        tc_commit(k_empty + st);
-        if (j >= 1) ok = issue_pv(j - 1);
+        __syncwarp();
+      };
+      bool ok = mbar_wait(q_full, 0, p.err, p.timeout_ns);
+      if (__all_sync(0xffffffffu, ok)) {
+        ok = mbar_wait(k_full, 0, p.err, p.timeout_ns);
+        if (__all_sync(0xffffffffu, ok)) {
+          tc_fence_after();
+          if (n_t0 > 0) issue_s(0, 0);
+          if (n_t1 > 0) issue_s(1, 0);
+        }
       }
-      if (ok && j == n_kv) issue_pv(n_kv - 1);
-      // all MMAs issued by this thread complete before TMEM is released
-      tc_commit(mma_done);
-      mbar_wait(mma_done, 0, p.err, DRAIN_TIMEOUT_NS, false);
+      for (int j = 0; j < n_max && __all_sync(0xffffffffu, ok); ++j) {
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (j >= nt(t)) continue;
+          ok = mbar_wait(p_full(t), j & 1, p.err, p.timeout_ns);
+          if (ok) ok = mbar_wait(v_full + j % C::NV, (j / C::NV) & 1, p.err, p.timeout_ns);
+          if (!__all_sync(0xffffffffu, ok)) break;
+          tc_fence_after();
+          issue_pv(t, j);
+          if (j + 1 < nt(t)) {
+            if (FP8) ok = mbar_wait(s_free(t), j & 1, p.err, p.timeout_ns);
+            if (ok) ok = mbar_wait(k_full + (j + 1) % C::NK, ((j + 1) / C::NK) & 1, p.err, p.timeout_ns);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            issue_s(t, j + 1);
+          }
+        }
+      }
+      // every MMA issued by this warp completes before TMEM is released
+      if (elect_one()) tc_commit(mma_done(0));
+      __syncwarp();
+      mbar_wait(mma_done(0), 0, p.err, DRAIN_TIMEOUT_NS, false);
     }
   } else {
-    // ------------------------------------------------------------- softmax warps 0-3
-    const int r = tid;                       // row within the tile == TMEM lane
-    const int q_pos = qt * BLOCK_M + r;      // query position in the sequence
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    float a = 0.0f;  // FP8 slope, byte units per raw score
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_SOFTMAX));
+    // ------------------------------------------------------------- softmax of tile t
+    const int t = warp >> 2;
+    const int n_t = t == 0 ? n_t0 : n_t1;
+    const int qt = qt0 + t;
+    const int r = tid & 127;                      // row within the tile == TMEM lane
+    const int q_pos = qt * BLOCK_M + r;           // query position in the sequence
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t ts = lane_base + t * 128;      // S_t / P_t columns of this lane
+    const uint32_t to = lane_base + TM_O + t * 128;
+    float a = 0.0f, a256 = 0.0f;  // FP8 slope in code units per raw score (and / 256)
     if constexpr (FP8) {
       a = static_cast<float>(p.leanp_c * static_cast<double>(*p.descale_q) *
                              static_cast<double>(*p.descale_k));
-      // B-operand scale factors: 2^0 everywhere (V and the ones matrix)
-      tmem_st4(lane_base + TM_SFB, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
-      tmem_wait_st();
+      a256 = a * 0.00390625f;
     }
-    float m_f = -INFINITY;  // BF16 running max (raw scores)
-    int m_i = 0;            // FP8 running max (byte units)
-    float l = 0.0f;         // BF16 running row sum
+    float ms = -INFINITY;  // BF16 reference max, scaled to log2 units
+    int m_i = 0;           // FP8 reference max, code units
+    float l = 0.0f;        // running row sum
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      const int sb = j & 1;
-      ok = mbar_wait(s_full + sb, (j >> 1) & 1, p.err, p.timeout_ns);
+    for (int j = 0; j < n_t; ++j) {
+      ok = mbar_wait(s_full(t), j & 1, p.err, p.timeout_ns);
       if (!ok) break;
       tc_fence_after();
       uint32_t sraw[BLOCK_N];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + TM_S0 + sb * 128 + c * 32, sraw + c * 32);
+      for (int c = 0; c < 4; ++c) tmem_ld32(ts + c * 32, sraw + c * 32);
       tmem_wait_ld();
       float s[BLOCK_N];
 #pragma unroll
       for (int c = 0; c < BLOCK_N; ++c) s[c] = __uint_as_float(sraw[c]);
-      tc_fence_before();
-      mbar_arrive(s_empty + sb);
-      if (p.causal && j == qt) {
+      const bool diag = p.causal && j == qt;
+      if (diag) {
 #pragma unroll
         for (int c = 0; c < BLOCK_N; ++c)
           if (c > r) s[c] = -INFINITY;
@@ -331,43 +419,60 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mu1 = fmaxf(mu1, s[127]);
 
       uint32_t pw[FP8 ? 32 : 64];
-      float alpha;
-      uint32_t sf_word = 0;
+      float alpha = 1.0f;
       if constexpr (!FP8) {
-        const float m_new = fmaxf(m_f, fmaxf(mu0, mu1));
-        alpha = ex2_approx((m_f - m_new) * p.c1);
-        const float mc = m_new * p.c1;
-        float lsum = 0.0f;
+        const float cand = fmaxf(mu0, mu1) * p.c1;
+        const float ms_new = (j == 0 || cand > ms + BF16_HEADROOM) ? cand : ms;
+        if (j > 0) alpha = ex2_approx(ms - ms_new);
+        ms = ms_new;
+        float lsum0 = 0.0f, lsum1 = 0.0f;
+        if (diag) {
 #pragma unroll
-        for (int c = 0; c < BLOCK_N; c += 2) {
-          const float p0 = ex2_approx(__fmaf_rn(s[c], p.c1, -mc));
-          const float p1 = ex2_approx(__fmaf_rn(s[c + 1], p.c1, -mc));
-          lsum += p0 + p1;
-          pw[c >> 1] = pack_bf16x2(p0, p1);
+          for (int c = 0; c < BLOCK_N; c += 2) {
+            const float p0 = ex2_approx(__fmaf_rn(s[c], p.c1, -ms));
+            const float p1 = ex2_approx(__fmaf_rn(s[c + 1], p.c1, -ms));
+            lsum0 += p0;
+            lsum1 += p1;
+            pw[c >> 1] = pack_bf16x2(p0, p1);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < BLOCK_N; c += 2) {
+            const float x0 = __fmaf_rn(s[c], p.c1, -ms);
+            const float x1 = __fmaf_rn(s[c + 1], p.c1, -ms);
+            // one element pair in four on the FMA pipe, the rest on the MUFU
+            const bool poly = (c & 7) == 6;
+            const float p0 = poly ? exp2_poly(x0) : ex2_approx(x0);
+            const float p1 = poly ? exp2_poly(x1) : ex2_approx(x1);
+            lsum0 += p0;
+            lsum1 += p1;
+            pw[c >> 1] = pack_bf16x2(p0, p1);
+          }
         }
-        l = l * alpha + lsum;
-        m_f = m_new;
+        l = l * alpha + (lsum0 + lsum1);
       } else {
         const float mu = fmaxf(mu0, mu1);
         const int cand = __float2int_ru(__fmul_rn(a, mu));
-        const int m_new = (j == 0) ? cand : max(m_i, cand);
-        alpha = (j == 0) ? 0.0f : ex2_approx(static_cast<float>(m_i - m_new) * 0.125f);
+        const int m_new = (j == 0 || cand > m_i + LEANP_HEADROOM) ? cand : m_i;
+        if (j > 0) alpha = ex2_approx(static_cast<float>(m_i - m_new) * 0.125f);
+        m_i = m_new;
+        l *= alpha;
         const int k0 = leanp_kshift(mu0, a, m_new);
         const int k1 = leanp_kshift(mu1, a, m_new);
-        const float cb0 = LEANP_MAGIC + __int2float_rn(120 + 8 * k0 - m_new);
-        const float cb1 = LEANP_MAGIC + __int2float_rn(120 + 8 * k1 - m_new);
+        const float cb0 = __int2float_rn(LEANP_TOP + 8 * k0 - m_new) * 0.00390625f;
+        const float cb1 = __int2float_rn(LEANP_TOP + 8 * k1 - m_new) * 0.00390625f;
 #pragma unroll
         for (int c = 0; c < BLOCK_N; c += 4) {
           const float cb = c < 64 ? cb0 : cb1;
-          const uint32_t b0 = __float_as_uint(fmaxf(__fmaf_rn(s[c + 0], a, cb), LEANP_MAGIC));
-          const uint32_t b1 = __float_as_uint(fmaxf(__fmaf_rn(s[c + 1], a, cb), LEANP_MAGIC));
-          const uint32_t b2 = __float_as_uint(fmaxf(__fmaf_rn(s[c + 2], a, cb), LEANP_MAGIC));
-          const uint32_t b3 = __float_as_uint(fmaxf(__fmaf_rn(s[c + 3], a, cb), LEANP_MAGIC));
+          // multiply-add (saturating to [0,1]) and the integer conversion by a magic fma
+          const uint32_t b0 = __float_as_uint(__fmaf_rn(fma_sat(s[c + 0], a256, cb), 256.0f, LEANP_MAGIC));
+          const uint32_t b1 = __float_as_uint(__fmaf_rn(fma_sat(s[c + 1], a256, cb), 256.0f, LEANP_MAGIC));
+          const uint32_t b2 = __float_as_uint(__fmaf_rn(fma_sat(s[c + 2], a256, cb), 256.0f, LEANP_MAGIC));
+          const uint32_t b3 = __float_as_uint(__fmaf_rn(fma_sat(s[c + 3], a256, cb), 256.0f, LEANP_MAGIC));
           pw[c >> 2] = pack_low_bytes(b0, b1, b2, b3);
         }
-        const uint32_t e0 = static_cast<uint32_t>(119 - k0), e1 = static_cast<uint32_t>(119 - k1);
-        sf_word = e0 | (e0 << 8) | (e1 << 16) | (e1 << 24);
-        m_i = m_new;
+        const uint32_t e0 = static_cast<uint32_t>(120 - k0), e1 = static_cast<uint32_t>(120 - k1);
+        const uint32_t sf_word = e0 | (e0 << 8) | (e1 << 16) | (e1 << 24);  // UE8M0 2^-(7+k)
         if constexpr (DUMP) {
           const size_t row = (static_cast<size_t>(b) * p.Hq + h) * p.S + q_pos;
           float* ds = p.dump_s + row * p.S + static_cast<size_t>(j) * BLOCK_N;
@@ -378,72 +483,65 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           dk[0] = static_cast<uint8_t>(k0);
           dk[1] = static_cast<uint8_t>(k1);
         }
-      }
-      if constexpr (FP8) {
-        // scale factors of P: the word for row R lives in column TM_SFA + R/32 at lane R%32
+        // scale factors of P: the word for row R lives in column SFA + R/32 at lane R%32
         // of every 32-lane quadrant (byte k = 32-key block k of the tile), so each warp
         // writes the words of all 128 rows for its own quadrant: exchange through smem
-        sf_x[(j & 1) * 128 + r] = sf_word;
-        mbar_arrive(sf_bar);
+        sf_x[(t * 2 + (j & 1)) * 128 + r] = sf_word;
+        mbar_arrive(sf_bar(t));
       }
-      if (j >= 1) {
-        // PV(j-1) must be complete before P, its scale factors and O are touched again
-        ok = mbar_wait(o_done, (j - 1) & 1, p.err, p.timeout_ns);
-        if (!ok) break;
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+      // the previous PV of this tile is complete here (BF16: S_t(j) completed after it;
+      // FP8: the row sum was read back before S_t(j) was issued), so O_t may be rescaled
+      if (__any_sync(0xffffffffu, alpha != 1.0f)) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t o[32];
-            tmem_ld32(lane_base + TM_O + c * 32, o);
-            tmem_wait_ld();
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld32(to + c * 32, o);
+          tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(lane_base + TM_O + c * 32, o);
-          }
-          if constexpr (FP8) {
-            uint32_t rs;
-            tmem_ld1(lane_base + TM_RS, rs);
-            tmem_wait_ld();
-            tmem_st1(lane_base + TM_RS, __float_as_uint(__uint_as_float(rs) * alpha));
-          }
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(to + c * 32, o);
         }
       }
       if constexpr (!FP8) {
-        tmem_st32(lane_base + TM_P, pw);
-        tmem_st32(lane_base + TM_P + 32, pw + 32);
+        tmem_st32(ts, pw);
+        tmem_st32(ts + 32, pw + 32);
       } else {
-        tmem_st32(lane_base + TM_P, pw);
-        ok = mbar_wait(sf_bar, j & 1, p.err, p.timeout_ns);
+        tmem_st32(ts, pw);
+        tmem_st4(ts + TM_SFB_OFF, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+        ok = mbar_wait(sf_bar(t), j & 1, p.err, p.timeout_ns);
         if (!ok) break;
-        const uint32_t* x = sf_x + (j & 1) * 128;
-        tmem_st4(lane_base + TM_SFA, x[lane], x[32 + lane], x[64 + lane], x[96 + lane]);
+        const uint32_t* x = sf_x + (t * 2 + (j & 1)) * 128;
+        tmem_st4(ts + TM_SFA_OFF, x[lane], x[32 + lane], x[64 + lane], x[96 + lane]);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(p_full(t));
+      if constexpr (FP8) {
+        // the row sum of this tile's rounded probabilities, read back before S_t(j+1)
+        ok = mbar_wait(pv_done(t), j & 1, p.err, p.timeout_ns);
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t rs;
+        tmem_ld1(ts + TM_RS_OFF, rs);
+        tmem_wait_ld();
+        l += __uint_as_float(rs);
+        tc_fence_before();
+        mbar_arrive(s_free(t));
+      }
     }
     tmem_wait_st();  // nothing of this thread may still be writing TMEM on any exit path
     // ------------------------------------------------------------- epilogue
-    if (ok) ok = mbar_wait(o_done, (n_kv - 1) & 1, p.err, p.timeout_ns);
-    if (ok) {
+    if (ok && n_t > 0 && !FP8) ok = mbar_wait(pv_done(t), (n_t - 1) & 1, p.err, p.timeout_ns);
+    if (ok && n_t > 0) {
       tc_fence_after();
       uint32_t oraw[DV];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + TM_O + c * 32, oraw + c * 32);
-      float lrow = l;
-      if constexpr (FP8) {
-        uint32_t rs;
-        tmem_ld1(lane_base + TM_RS, rs);
-        tmem_wait_ld();
-        lrow = __uint_as_float(rs);
-      } else {
-        tmem_wait_ld();
-      }
+      for (int c = 0; c < 4; ++c) tmem_ld32(to + c * 32, oraw + c * 32);
+      tmem_wait_ld();
       float o[DV];
 #pragma unroll
       for (int c = 0; c < DV; ++c) o[c] = __uint_as_float(oraw[c]);
-      float inv = 1.0f / lrow;
+      float inv = 1.0f / l;
       if constexpr (FP8) inv *= *p.descale_v;
       if (p.unrotate) {
         // x -> x H_128 / sqrt(128), butterfly stages h = 1, 2, ..., 64
@@ -460,8 +558,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         inv *= 0.08838834764831845f;
       }
-      __nv_bfloat16* orow =
-          p.o + ((static_cast<size_t>(tok0) + q_pos) * p.Hq + h) * DV;
+      __nv_bfloat16* orow = p.o + ((static_cast<size_t>(tok0) + q_pos) * p.Hq + h) * DV;
 #pragma unroll
       for (int c = 0; c < DV; c += 8) {
         uint4 v;
@@ -474,15 +571,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (p.lse != nullptr) {
         float lse_v;
         if constexpr (FP8)
-          lse_v = 0.69314718055994531f * (static_cast<float>(m_i) * 0.125f + __log2f(lrow));
+          lse_v = 0.69314718055994531f * (static_cast<float>(m_i) * 0.125f + __log2f(l));
         else
-          lse_v = 0.69314718055994531f * (m_f * p.c1 + __log2f(lrow));
+          lse_v = 0.69314718055994531f * (ms + __log2f(l));
         p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.S + q_pos] = lse_v;
       }
     }
   }
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 11) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

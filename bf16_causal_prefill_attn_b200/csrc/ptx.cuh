@@ -53,10 +53,10 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{.reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, "
+      "{.reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, "
       "0, p;}"
       : "=r"(ok)
-      : "r"(smem_addr(bar)), "r"(parity), "r"(1000000u)
+      : "r"(smem_addr(bar)), "r"(parity)
       : "memory");
   return ok != 0;
 }
@@ -86,6 +86,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
 // Limit of the drain waits (copies and MMAs already issued), independent of the
 // configurable limit of ordinary waits.
 constexpr uint64_t DRAIN_TIMEOUT_NS = 2000000000ull;
+
+// One lane of the (fully active) warp: issue single-thread async ops from warp-uniform
+// values so their operands stay in uniform registers.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{.reg .pred P; elect.sync _|P, 0xffffffff; selp.b32 %0, 1, 0, P;}" : "=r"(pred)::"memory");
+  return pred != 0;
+}
 
 // ------------------------------------------------------------------ named barriers
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {

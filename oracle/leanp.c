@@ -18,22 +18,27 @@
  * Reading (the plainest one the pages support; all arithmetic float32 with one rounding
  * per operation, fmaf = fused multiply-add with a single rounding):
  *   The e4m3 code n = 8e + m (exponent field e, mantissa m) decodes to about
- *   2^(n/8 - 7) (the logarithm of 1 + m/8 taken as m/8: Mitchell 1962), so the code
- *   of 2^y is about 8 (y + 7) -- linear in y, which is linear in the score.  With
- *   a = 8 log2(e) * scale * dq * dk (byte units per raw score unit), per row:
- *     m      running maximum in byte units, an integer:
- *            m <- max(m, ceil(float32(a * mu_tile)))   mu_tile = tile max of raw scores
+ *   2^(n/8 - 7) (the logarithm of 1 + m/8 taken as m/8: Mitchell 1962), so a code
+ *   linear in the score approximates the exponential (the exponential-by-integer idea of
+ *   Schraudolph 1999).  With a = 8 log2(e) * scale * dq * dk (code units per raw score
+ *   unit), per row and per 128-key tile in ascending key order:
+ *     m      reference max in code units, an integer, raised lazily:
+ *            cand = ceil(float32(a * mu_tile)) (mu_tile = tile max of the raw scores);
+ *            m = cand on the first tile, afterwards m = cand only if cand > m + H
+ *            (H = 14, the headroom between the block-max code 112 and the largest
+ *            finite code 126); otherwise m is kept
  *     k_b    per 64-key block b with block max mu_b:
  *            t = fmaf(mu_b, a, -m);  k_b = clamp(floor(-t / 8), 0, KMAX)
- *            (the block maximum lands in code range (112, 120], i.e. value 2^7..2^8)
- *     code   r = fmaf(s, a, MAGIC + (120 + 8 k_b - m)),  MAGIC = 1.5 * 2^23
- *            (the single rounding of the fma at magnitude 2^23 is the round-to-nearest-
- *            even integer conversion: the low bits of r hold the integer), then
- *            byte = low 8 bits of max(r, MAGIC)   (negative codes clamp to 0)
- *     value  decode(byte) ~ 2^((a s - m)/8) * 2^(8 + k_b); the matrix instruction
- *            applies 2^-(8 + k_b) per (row, 64-key block) through UE8M0 scale factors
- *     l      l <- alpha l + sum_j decode(byte_j) 2^-(8+k_b(j));   O likewise with v_j
- *     alpha  2^((m_old - m_new)/8) when m grows (0 on the first tile)
+ *            (a block whose max sits below m by 8 k_b or more is lifted by 2^k_b)
+ *     code   the multiply-add, saturating to [0, 1] (negative codes clamp to 0):
+ *              u = sat(fmaf(s, a / 256, (112 + 8 k_b - m) / 256))
+ *            and the integer conversion, one fma whose rounding at magnitude 2^23 is the
+ *            round-to-nearest-even integer:  r = fmaf(u, 256, 1.5 * 2^23);
+ *            byte = low 8 bits of r  (at most 126: never the NaN code 127)
+ *     value  decode(byte) ~ 2^((a s - m)/8) * 2^(7 + k_b); the matrix instruction
+ *            applies 2^-(7 + k_b) per (row, 64-key block) through UE8M0 scale factors
+ *     l      l <- alpha l + sum_j decode(byte_j) 2^-(7+k_b(j));   O likewise with v_j
+ *     alpha  2^((m_old - m_new)/8) when m is raised (0 on the first tile)
  *   final:   o = O * dv / l,  lse = ln 2 * (m / 8 + log2 l)
  * Masked scores are -inf: their code is 0.  A fully masked block gets k_b = KMAX (its
  * codes are all 0, so its scale multiplies zeros).
@@ -46,6 +51,8 @@
 #include <string.h>
 
 #define LEANP_MAGIC 12582912.0f /* 1.5 * 2^23 */
+#define LEANP_TOP 112          /* code of a block maximum at the reference */
+#define LEANP_HEADROOM 14      /* 126 - LEANP_TOP */
 
 /* ---- e4m3fn decode by the format definition (independent of the Python codec) ---- */
 double leanp_e4m3_decode(uint8_t c) {
@@ -60,13 +67,13 @@ double leanp_e4m3_decode(uint8_t c) {
 /* exposed for the tests' exact-rounding pin */
 float leanp_fmaf(float x, float y, float z) { return fmaf(x, y, z); }
 
-/* running max in byte units after seeing a tile whose raw-score maximum is mu_tile */
+/* reference max in code units after seeing a tile whose raw-score maximum is mu_tile */
 int leanp_update_max(float mu_tile, float a, int m_old, int m_valid) {
     if (isinf(mu_tile) && mu_tile < 0) return m_old;  /* no visible key in the tile */
     float prod = a * mu_tile;                          /* one float32 rounding */
     int cand = (int)ceilf(prod);
     if (!m_valid) return cand;
-    return cand > m_old ? cand : m_old;
+    return cand > m_old + LEANP_HEADROOM ? cand : m_old;
 }
 
 /* power-of-two shift of one 64-key block */
@@ -80,11 +87,14 @@ int leanp_kshift(float mu_b, float a, int m, int kmax) {
     return (int)f;
 }
 
-/* code of one score given the block constant */
+/* code of one score given the block shift */
 uint8_t leanp_code(float s, float a, int m, int kb) {
-    float c = LEANP_MAGIC + (float)(120 + 8 * kb - m); /* exact: small integers */
-    float r = fmaf(s, a, c);
-    r = fmaxf(r, LEANP_MAGIC);
+    const float inv256 = 0.00390625f;
+    float c = (float)(LEANP_TOP + 8 * kb - m) * inv256; /* exact: small integer / 256 */
+    float u = fmaf(s, a * inv256, c);                  /* a / 256 exact */
+    if (!(u > 0.0f)) u = 0.0f;                         /* saturate (NaN, -inf, <= 0 -> 0) */
+    if (u > 1.0f) u = 1.0f;
+    float r = fmaf(u, 256.0f, LEANP_MAGIC);
     uint32_t bits;
     memcpy(&bits, &r, 4);
     return (uint8_t)(bits & 0xFF);
@@ -169,7 +179,7 @@ void leanp_attention_row(const float* s, int S_k, int tile, const double* v, int
         for (int j = 0; j < n; ++j) {
             int key = t * tile + j;
             if (key >= S_k || codes[j] == 0) continue;
-            double w = leanp_e4m3_decode(codes[j]) * ldexp(1.0, -(8 + ks[j / 64]));
+            double w = leanp_e4m3_decode(codes[j]) * ldexp(1.0, -(7 + ks[j / 64]));
             l += w;
             for (int d = 0; d < dv; ++d) acc[d] += w * v[(size_t)key * dv + d];
         }

@@ -41,8 +41,8 @@ def test_fmaf_single_rounding():
 
 
 def test_closed_form_block_max_code():
-    # with a power-of-two slope a*s is exact, so a score equal to the running max (in byte
-    # units) codes to 120 = 8*(7+8), i.e. 2^8, and the scale 2^-(8+0) gives weight 1
+    # with a power-of-two slope a*s is exact, so a score equal to the reference max (in
+    # code units) codes to 112 = 8*(7+7), i.e. 2^7, and the scale 2^-(7+0) gives weight 1
     checked = 0
     for a in (np.float32(0.25), np.float32(2.0), leanp.slope(128, 1.0, 1.0)):
         for m in (-40, 0, 7, 333):
@@ -52,13 +52,18 @@ def test_closed_form_block_max_code():
             kb = leanp.kshift(s, a, m)
             assert kb == 0
             c = leanp.code(s, a, m, kb)
-            assert c == 120 == 8 * (7 + 8)
-            assert e4m3.e4m3_decode(np.array([c]))[0] * 2.0 ** -(8 + kb) == 1.0
-            # one block below: k = 1 keeps the code in range and the weight 2^-1
+            assert c == 112 == 8 * (7 + 7)
+            assert e4m3.e4m3_decode(np.array([c]))[0] * 2.0 ** -(7 + kb) == 1.0
+            # one block (8 codes) below: k = 1 keeps the code at 112 and the weight 2^-1
             s2 = np.float32((m - 8) / float(a))
             if float(a) * float(s2) == m - 8:
                 assert leanp.kshift(s2, a, m) == 1
-                assert leanp.code(s2, a, m, 1) == 120
+                assert leanp.code(s2, a, m, 1) == 112
+            # up to the headroom above the reference: codes 113..126, never NaN (127)
+            for up in range(1, 15):
+                s3 = np.float32((m + up) / float(a))
+                if float(a) * float(s3) == m + up:
+                    assert leanp.code(s3, a, m, 0) == 112 + up
             checked += 1
     assert checked >= 8
 
@@ -74,13 +79,13 @@ def test_codes_follow_log_linear_rule_within_mitchell_bound():
             idx = t * 128 + j
             c = int(codes[idx])
             kb = int(ks[idx // 64])
-            y = (float(a) * float(s[idx]) - m) / 8.0 + 8 + kb     # wanted log2 of the value
+            y = (float(a) * float(s[idx]) - m) / 8.0 + 7 + kb     # wanted log2 of the value
             if c >= 8:                                          # normal e4m3 codes
                 got = np.log2(e4m3.e4m3_decode(np.array([c]))[0])
                 assert abs(got - y) <= 0.0861 + 1.0 / 16 + 1e-6
             elif c == 0:
-                assert y < 0.5 / 8 - 6                          # below the smallest code
-            assert c <= 120
+                assert y < 0.5 / 8 - 6 + 1e-6                   # below the smallest code
+            assert c <= 126
 
 
 def test_block_shift_rule_and_monotonicity():
@@ -92,13 +97,12 @@ def test_block_shift_rule_and_monotonicity():
         m = mref[0]
         for b in range(2):
             blk = s[b * 64:(b + 1) * 64]
-            mu = blk.max()
             kb = int(ks[b])
             top = int(codes[b * 64 + int(np.argmax(blk))])
             if 0 < kb < leanp.KMAX:
-                assert 112 <= top <= 120
+                assert 104 <= top <= 112
             if kb == 0:
-                assert top <= 120
+                assert top <= 126
             # monotone within a block
             order = np.argsort(blk, kind="stable")
             assert np.all(np.diff(codes[b * 64:(b + 1) * 64][order].astype(int)) >= 0)
@@ -114,11 +118,17 @@ def test_masked_scores_code_zero_and_full_mask_shift():
     assert ks[1] == leanp.KMAX
 
 
-def test_running_max_rescale_sequence():
+def test_lazy_reference_max():
     a = leanp.slope(128, 1.0, 1.0)
-    s = np.concatenate([np.full(128, 1.0), np.full(128, 3.0), np.full(128, 2.0)]).astype(np.float32)
+    ca = lambda x: int(np.ceil(np.float32(a * np.float32(x))))
+    # a small rise stays within the headroom (no rescale); a large one raises m
+    s = np.concatenate([np.full(128, 1.0), np.full(128, 10.0), np.full(128, 40.0),
+                        np.full(128, 20.0)]).astype(np.float32)
     _, _, mref = leanp.encode_row(s, a)
-    assert list(mref) == [int(np.ceil(np.float32(a * 1))), int(np.ceil(np.float32(a * 3))), int(np.ceil(np.float32(a * 3)))]
+    assert ca(10.0) <= ca(1.0) + 14 < ca(40.0)
+    assert list(mref) == [ca(1.0), ca(1.0), ca(40.0), ca(40.0)]
+    codes, _, _ = leanp.encode_row(s, a)
+    assert codes.max() <= 126 and codes[128:256].min() > codes[:128].max()
 
 
 @pytest.mark.parametrize("dist", ["gaussian", "outlier"])
