@@ -279,19 +279,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // so tile 1's softmax of j overlaps PV_0(j) + S_0(j+1) and tile 0's softmax of j+1
       // overlaps PV_1(j) + S_1(j+1) (ping-pong).
       auto nt = [&](int t) { return t == 0 ? n_t0 : n_t1; };
-      const uint32_t ones_base = smem_addr(smem + C::OFF_ONES);
+      // Descriptors are built once; advancing an operand by `off` bytes adds off >> 4 to
+      // the start-address field (shared-memory addresses stay below 2^18, so the 14-bit
+      // field never carries into its neighbours).
+      const uint64_t dq0 = smem_desc_sw128(smem_addr(smem + C::OFF_Q), 16, 1024);
+      const uint64_t dk0 = smem_desc_sw128(smem_addr(smem + C::OFF_K), 16, 1024);
+      const uint64_t dv0 = smem_desc_sw128(smem_addr(smem + C::OFF_V), C::BOX_BYTES, 1024);
+      const uint64_t dones = smem_desc_sw128(smem_addr(smem + C::OFF_ONES), 16, 1024);
       auto issue_s = [&](int t, int j) {
         const int sk = j % C::NK;
-        const uint32_t q_base = smem_addr(smem + C::OFF_Q + t * C::Q_BYTES);
-        const uint32_t k_base = smem_addr(smem + C::OFF_K + sk * C::K_BYTES);
+        const uint64_t qd = dq0 + static_cast<uint32_t>((t * C::Q_BYTES) >> 4);
+        const uint64_t kd = dk0 + static_cast<uint32_t>((sk * C::K_BYTES) >> 4);
         const uint32_t tm_s = tmem + t * 128;
         if (elect_one()) {
 #pragma unroll
           for (int s = 0; s < C::QK_STEPS; ++s) {
-            const uint32_t off = (s / 4) * C::BOX_BYTES + (s % 4) * 32;
-            mma_ss<FP8 ? 1 : 0>(tm_s, smem_desc_sw128(q_base + off, 16, 1024),
-                                smem_desc_sw128(k_base + off, 16, 1024), C::IDESC_S,
-                                s > 0 ? 1u : 0u);
+            const uint32_t off = ((s / 4) * C::BOX_BYTES + (s % 4) * 32) >> 4;
+            mma_ss<FP8 ? 1 : 0>(tm_s, qd + off, kd + off, C::IDESC_S, s > 0 ? 1u : 0u);
           }
           tc_commit(s_full(t));
           // K(j) is free once its last S has run: tile 1's, or tile 0's if tile 1 skips j
@@ -301,7 +305,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       };
       auto issue_pv = [&](int t, int j) {
         const int sv = j % C::NV;
-        const uint32_t v_base = smem_addr(smem + C::OFF_V + sv * C::V_BYTES);
+        const uint64_t vd = dv0 + static_cast<uint32_t>((sv * C::V_BYTES) >> 4);
         const uint32_t tm_s = tmem + t * 128;
         const uint32_t tm_o = tmem + TM_O + t * 128;
         if (elect_one()) {
@@ -309,18 +313,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
             for (int s = 0; s < C::PV_STEPS; ++s) {
               // V is [keys x d] with d contiguous: B operand MN-major; 8-key groups 1 KB
-              // apart, 64-column atoms 16 KB apart
-              mma_ts_f16(tm_o, tm_s + s * 8,
-                         smem_desc_sw128(v_base + s * 2048, C::BOX_BYTES, 1024),
-                         C::IDESC_PV_BF16, (j > 0 || s > 0) ? 1u : 0u);
+              // apart (16 keys per step), 64-column atoms 16 KB apart (LBO)
+              mma_ts_f16(tm_o, tm_s + s * 8, vd + ((s * 2048) >> 4), C::IDESC_PV_BF16,
+                         (j > 0 || s > 0) ? 1u : 0u);
             }
           } else {
 #pragma unroll
             for (int s = 0; s < C::PV_STEPS; ++s) {
               const uint32_t sfa = (tm_s + TM_SFA_OFF) | (static_cast<uint32_t>(s) << 30);
               const uint32_t sfb = (tm_s + TM_SFB_OFF) | (static_cast<uint32_t>(s) << 30);
-              mma_ts_mxf8(tm_o, tm_s + s * 8,
-                          smem_desc_sw128(v_base + s * 4096, C::BOX_BYTES, 1024),
+              mma_ts_mxf8(tm_o, tm_s + s * 8, vd + ((s * 4096) >> 4),
                           idesc_mxf8(0, 1, BLOCK_M, DV, s, s), sfa, sfb,
                           (j > 0 || s > 0) ? 1u : 0u);
             }
@@ -329,8 +331,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               // row sum of the rounded probabilities: P x ones (16 x 128 keys, K-major)
               const uint32_t sfa = (tm_s + TM_SFA_OFF) | (static_cast<uint32_t>(s) << 30);
               const uint32_t sfb = (tm_s + TM_SFB_OFF) | (static_cast<uint32_t>(s) << 30);
-              mma_ts_mxf8(tm_s + TM_RS_OFF, tm_s + s * 8,
-                          smem_desc_sw128(ones_base + s * 32, 16, 1024),
+              mma_ts_mxf8(tm_s + TM_RS_OFF, tm_s + s * 8, dones + ((s * 32) >> 4),
                           idesc_mxf8(0, 0, BLOCK_M, 16, s, s), sfa, sfb, s > 0 ? 1u : 0u);
             }
           }
