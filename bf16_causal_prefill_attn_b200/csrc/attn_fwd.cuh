@@ -27,10 +27,16 @@
 //               order PV_0(j), S_0(j+1), PV_1(j), S_1(j+1): one tile's softmax overlaps
 //               the other tile's MMAs (ping-pong);
 //   warp 10     idle; warp 11 TMEM allocator.
-// TMEM (512 columns x 128 lanes): S_0 [0,128), S_1 [128,256), O_0 [256,384),
-// O_1 [384,512).  P_t overwrites the first columns of S_t (bf16: 64, e4m3: 32); for FP8
-// the scale factors of P_t sit at S_t + 32 (4 columns), those of B at S_t + 36 (4) and the
-// row-sum MMA writes S_t + 64 (16), read back by the softmax group before S_t(j+1).
+// TMEM (512 columns x 128 lanes, see TmemMap):
+//   BF16  S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512); P_t (bf16, 64
+//         columns) overwrites the first columns of S_t.
+//   FP8   O_0 [0,144), O_1 [160,304): the PV MMA has N = 144, V extended by a 16-column
+//         block of ones, so columns 128..143 accumulate the row sum of the rounded P with
+//         the same block scales (the "extra matrix instruction" costs no extra issue);
+//         S_0 [320,448), S_1 [384,512) overlap in [384,448), so an S MMA is issued only
+//         after the other tile's softmax group has read its S (s_read barriers); P_t (32
+//         columns) and its scale factors live in the part of S_t the other tile never
+//         writes (S_0: [320,384), S_1: [448,512)).
 //
 // Every wait is bounded (mbar_wait): on expiry the CTA records DEV_TIMEOUT and unwinds.
 #pragma once
@@ -51,8 +57,17 @@ constexpr int REGS_OTHER = 88;     // per thread of warps 8-11
 // registers per thread the launch must provide at least for that split
 constexpr int REGS_NEEDED_AT_LAUNCH =
     (2 * 128 * REGS_SOFTMAX + 128 * REGS_OTHER + NUM_THREADS - 1) / NUM_THREADS;
-constexpr uint32_t TM_O = 256;
-constexpr uint32_t TM_SFA_OFF = 32, TM_SFB_OFF = 36, TM_RS_OFF = 64;
+// TMEM column map per precision (see the layout above)
+template <bool FP8>
+struct TmemMap {
+  __host__ __device__ static constexpr uint32_t S(int t) { return FP8 ? 320u + 64u * t : 128u * t; }
+  __host__ __device__ static constexpr uint32_t O(int t) { return FP8 ? 160u * t : 256u + 128u * t; }
+  __host__ __device__ static constexpr uint32_t P(int t) { return FP8 ? (t ? 448u : 320u) : 128u * t; }
+  __host__ __device__ static constexpr uint32_t SFA(int t) { return P(t) + 32; }  // 4 columns
+  __host__ __device__ static constexpr uint32_t SFB(int t) { return P(t) + 40; }  // 8 columns
+  static constexpr uint32_t RS = 128;                          // row-sum column of O(t)
+  static constexpr uint32_t PV_N = FP8 ? 144 : 128;
+};
 constexpr float LEANP_MAGIC = 12582912.0f;  // 1.5 * 2^23
 constexpr int LEANP_KMAX = 16;
 constexpr int LEANP_TOP = 112;       // code of a block maximum at the reference
@@ -96,22 +111,23 @@ struct FwdCfg {
   static constexpr int K_BYTES = Q_BYTES;
   static constexpr int V_BYTES = V_BOXES * BOX_BYTES;
   static constexpr int NK = FP8 ? (DQK == 128 ? 4 : 3) : 2;     // K ring depth
-  static constexpr int NV = FP8 ? (DQK == 128 ? 4 : 3) : (DQK == 128 ? 2 : 1);
+  static constexpr int NV = FP8 ? (DQK == 128 ? 4 : 2) : (DQK == 128 ? 2 : 1);
   static constexpr int KSTEP = FP8 ? 32 : 16;                   // MMA K per instruction
   static constexpr int QK_STEPS = DQK / KSTEP;
   static constexpr int PV_STEPS = BLOCK_N / KSTEP;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
   static constexpr int OFF_V = OFF_K + NK * K_BYTES;
-  static constexpr int OFF_ONES = OFF_V + NV * V_BYTES;         // FP8: 16 x 128 B of 1.0
-  static constexpr int OFF_BAR = OFF_ONES + (FP8 ? 2048 : 0);
+  static constexpr int OFF_ONES = OFF_V + NV * V_BYTES;  // FP8: 128 keys x 128 B of 1.0
+  static constexpr int OFF_BAR = OFF_ONES + (FP8 ? BOX_BYTES : 0);
   // barriers: q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], and per tile:
-  //           s_full, p_full, pv_done, s_free, sf_bar, mma_done
+  //           s_full, p_full, pv_done, s_read, sf_bar, mma_done
   static constexpr int NUM_BARS = 1 + 2 * NK + 2 * NV + 2 * 6;
   static constexpr int OFF_TMEMPTR = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_SF = (OFF_TMEMPTR + 4 + 15) / 16 * 16;  // [2 tiles][2][128] u32
   static constexpr int SMEM_BYTES = OFF_SF + (FP8 ? 2 * 2 * 128 * 4 : 0);
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;           // 1024-B alignment slack
+  static_assert(SMEM_ALLOC <= 232448, "shared memory per block exceeded");
   static constexpr uint32_t IDESC_S =
       idesc_dense(FP8 ? 0u : 1u, FP8 ? 0u : 1u, 0u, 0u, BLOCK_M, BLOCK_N);
   static constexpr uint32_t IDESC_PV_BF16 = idesc_dense(1u, 1u, 0u, 1u, BLOCK_M, DV);
@@ -164,7 +180,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   auto s_full = [&](int t) { return tbar + 6 * t + 0; };
   auto p_full = [&](int t) { return tbar + 6 * t + 1; };
   auto pv_done = [&](int t) { return tbar + 6 * t + 2; };
-  auto s_free = [&](int t) { return tbar + 6 * t + 3; };
+  auto s_read = [&](int t) { return tbar + 6 * t + 3; };
   auto sf_bar = [&](int t) { return tbar + 6 * t + 4; };
   auto mma_done = [&](int t) { return tbar + 6 * t + 5; };
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEMPTR);
@@ -202,7 +218,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(s_full(t), 1);
       mbar_init(p_full(t), 128);
       mbar_init(pv_done(t), 1);
-      mbar_init(s_free(t), 128);
+      mbar_init(s_read(t), 128);
       mbar_init(sf_bar(t), 128);
       mbar_init(mma_done(t), 1);
     }
@@ -218,9 +234,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&tm_v);
   }
   if constexpr (FP8) {
-    // ones matrix (e4m3 1.0 = 0x38) for the row-sum MMA, visible to the async proxy
+    // the ones block (e4m3 1.0 = 0x38) that extends every V tile to N = 144 for the row
+    // sum; written once, visible to the async proxy
     uint32_t* ones = reinterpret_cast<uint32_t*>(smem + C::OFF_ONES);
-    for (int i = tid; i < 512; i += NUM_THREADS) ones[i] = 0x38383838u;
+    for (int i = tid; i < C::BOX_BYTES / 4; i += NUM_THREADS) ones[i] = 0x38383838u;
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   __syncthreads();
@@ -278,19 +295,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       //   PV_0(j), S_0(j+1), PV_1(j), S_1(j+1)
       // so tile 1's softmax of j overlaps PV_0(j) + S_0(j+1) and tile 0's softmax of j+1
       // overlaps PV_1(j) + S_1(j+1) (ping-pong).
+      using TM = TmemMap<FP8>;
       auto nt = [&](int t) { return t == 0 ? n_t0 : n_t1; };
       // Descriptors are built once; advancing an operand by `off` bytes adds off >> 4 to
       // the start-address field (shared-memory addresses stay below 2^18, so the 14-bit
       // field never carries into its neighbours).
       const uint64_t dq0 = smem_desc_sw128(smem_addr(smem + C::OFF_Q), 16, 1024);
       const uint64_t dk0 = smem_desc_sw128(smem_addr(smem + C::OFF_K), 16, 1024);
-      const uint64_t dv0 = smem_desc_sw128(smem_addr(smem + C::OFF_V), C::BOX_BYTES, 1024);
-      const uint64_t dones = smem_desc_sw128(smem_addr(smem + C::OFF_ONES), 16, 1024);
+      auto v_desc = [&](int sv) -> uint64_t {
+        const uint32_t va = smem_addr(smem + C::OFF_V + sv * C::V_BYTES);
+        if constexpr (FP8) {
+          // N = 144: the 128 d-columns of V, then the ones block one leading offset away
+          return smem_desc_sw128(va, smem_addr(smem + C::OFF_ONES) - va, 1024);
+        } else {
+          return smem_desc_sw128(va, C::BOX_BYTES, 1024);  // two 64-column atoms of V
+        }
+      };
       auto issue_s = [&](int t, int j) {
         const int sk = j % C::NK;
         const uint64_t qd = dq0 + static_cast<uint32_t>((t * C::Q_BYTES) >> 4);
         const uint64_t kd = dk0 + static_cast<uint32_t>((sk * C::K_BYTES) >> 4);
-        const uint32_t tm_s = tmem + t * 128;
+        const uint32_t tm_s = tmem + TM::S(t);
         if (elect_one()) {
 #pragma unroll
           for (int s = 0; s < C::QK_STEPS; ++s) {
@@ -305,34 +330,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       };
       auto issue_pv = [&](int t, int j) {
         const int sv = j % C::NV;
-        const uint64_t vd = dv0 + static_cast<uint32_t>((sv * C::V_BYTES) >> 4);
-        const uint32_t tm_s = tmem + t * 128;
-        const uint32_t tm_o = tmem + TM_O + t * 128;
+        const uint64_t vd = v_desc(sv);
+        const uint32_t tm_p = tmem + TM::P(t);
+        const uint32_t tm_o = tmem + TM::O(t);
         if (elect_one()) {
           if constexpr (!FP8) {
 #pragma unroll
             for (int s = 0; s < C::PV_STEPS; ++s) {
               // V is [keys x d] with d contiguous: B operand MN-major; 8-key groups 1 KB
               // apart (16 keys per step), 64-column atoms 16 KB apart (LBO)
-              mma_ts_f16(tm_o, tm_s + s * 8, vd + ((s * 2048) >> 4), C::IDESC_PV_BF16,
+              mma_ts_f16(tm_o, tm_p + s * 8, vd + ((s * 2048) >> 4), C::IDESC_PV_BF16,
                          (j > 0 || s > 0) ? 1u : 0u);
             }
           } else {
 #pragma unroll
             for (int s = 0; s < C::PV_STEPS; ++s) {
-              const uint32_t sfa = (tm_s + TM_SFA_OFF) | (static_cast<uint32_t>(s) << 30);
-              const uint32_t sfb = (tm_s + TM_SFB_OFF) | (static_cast<uint32_t>(s) << 30);
-              mma_ts_mxf8(tm_o, tm_s + s * 8, vd + ((s * 4096) >> 4),
-                          idesc_mxf8(0, 1, BLOCK_M, DV, s, s), sfa, sfb,
+              // [O | row sum] += (P * 2^-(7+k)) x [V | 1]; 32 keys per step
+              const uint32_t sfa = (tmem + TM::SFA(t)) | (static_cast<uint32_t>(s) << 30);
+              const uint32_t sfb = (tmem + TM::SFB(t)) | (static_cast<uint32_t>(s) << 30);
+              mma_ts_mxf8(tm_o, tm_p + s * 8, vd + ((s * 4096) >> 4),
+                          idesc_mxf8(0, 1, BLOCK_M, TM::PV_N, s, s), sfa, sfb,
                           (j > 0 || s > 0) ? 1u : 0u);
-            }
-#pragma unroll
-            for (int s = 0; s < C::PV_STEPS; ++s) {
-              // row sum of the rounded probabilities: P x ones (16 x 128 keys, K-major)
-              const uint32_t sfa = (tm_s + TM_SFA_OFF) | (static_cast<uint32_t>(s) << 30);
-              const uint32_t sfb = (tm_s + TM_SFB_OFF) | (static_cast<uint32_t>(s) << 30);
-              mma_ts_mxf8(tm_s + TM_RS_OFF, tm_s + s * 8, dones + ((s * 32) >> 4),
-                          idesc_mxf8(0, 0, BLOCK_M, 16, s, s), sfa, sfb, s > 0 ? 1u : 0u);
             }
           }
           tc_commit(pv_done(t));
@@ -340,31 +358,46 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         __syncwarp();
       };
+      // FP8: S_0 and S_1 share 64 TMEM columns; before writing S_t, the other tile's
+      // softmax group must have read its latest S (the index of that S is passed)
+      auto wait_other_read = [&](int t, int jo) -> bool {
+        if constexpr (!FP8) return true;
+        if (jo < 0) return true;
+        return mbar_wait(s_read(1 - t), jo & 1, p.err, p.timeout_ns);
+      };
       bool ok = mbar_wait(q_full, 0, p.err, p.timeout_ns);
       if (__all_sync(0xffffffffu, ok)) {
         ok = mbar_wait(k_full, 0, p.err, p.timeout_ns);
         if (__all_sync(0xffffffffu, ok)) {
           tc_fence_after();
           if (n_t0 > 0) issue_s(0, 0);
-          if (n_t1 > 0) issue_s(1, 0);
+          if (n_t1 > 0) {
+            ok = wait_other_read(1, n_t0 > 0 ? 0 : -1);
+            if (__all_sync(0xffffffffu, ok)) {
+              tc_fence_after();
+              issue_s(1, 0);
+            }
+          }
         }
       }
       for (int j = 0; j < n_max && __all_sync(0xffffffffu, ok); ++j) {
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
           if (j >= nt(t)) continue;
-          ok = mbar_wait(p_full(t), j & 1, p.err, p.timeout_ns);
+          const bool next = j + 1 < nt(t);
+          if (next) {
+            // prerequisites of S_t(j+1), normally met long before P_t(j) is ready: K(j+1)
+            // landed, and the other tile's softmax read its latest S (S_1(j) or S_0(j+1))
+            const int jo = t == 0 ? min(j, n_t1 - 1) : min(j + 1, n_t0 - 1);
+            ok = wait_other_read(t, jo);
+            if (ok) ok = mbar_wait(k_full + (j + 1) % C::NK, ((j + 1) / C::NK) & 1, p.err, p.timeout_ns);
+          }
+          if (ok) ok = mbar_wait(p_full(t), j & 1, p.err, p.timeout_ns);
           if (ok) ok = mbar_wait(v_full + j % C::NV, (j / C::NV) & 1, p.err, p.timeout_ns);
           if (!__all_sync(0xffffffffu, ok)) break;
           tc_fence_after();
           issue_pv(t, j);
-          if (j + 1 < nt(t)) {
-            if (FP8) ok = mbar_wait(s_free(t), j & 1, p.err, p.timeout_ns);
-            if (ok) ok = mbar_wait(k_full + (j + 1) % C::NK, ((j + 1) / C::NK) & 1, p.err, p.timeout_ns);
-            if (!__all_sync(0xffffffffu, ok)) break;
-            tc_fence_after();
-            issue_s(t, j + 1);
-          }
+          if (next) issue_s(t, j + 1);
         }
       }
       // every MMA issued by this warp completes before TMEM is released
@@ -381,8 +414,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int r = tid & 127;                      // row within the tile == TMEM lane
     const int q_pos = qt * BLOCK_M + r;           // query position in the sequence
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const uint32_t ts = lane_base + t * 128;      // S_t / P_t columns of this lane
-    const uint32_t to = lane_base + TM_O + t * 128;
+    using TM = TmemMap<FP8>;
+    const uint32_t ts = lane_base + TM::S(t);     // S_t columns of this lane
+    const uint32_t tp = lane_base + TM::P(t);     // P_t columns
+    const uint32_t to = lane_base + TM::O(t);     // O_t (FP8: and the row sum) columns
     float a = 0.0f, a256 = 0.0f;  // FP8 slope in code units per raw score (and / 256)
     if constexpr (FP8) {
       a = static_cast<float>(p.leanp_c * static_cast<double>(*p.descale_q) *
@@ -401,6 +436,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(ts + c * 32, sraw + c * 32);
       tmem_wait_ld();
+      if constexpr (FP8) {
+        // S_t is in registers: the other tile may now overwrite the shared columns
+        tc_fence_before();
+        mbar_arrive(s_read(t));
+      }
       float s[BLOCK_N];
 #pragma unroll
       for (int c = 0; c < BLOCK_N; ++c) s[c] = __uint_as_float(sraw[c]);
@@ -410,17 +450,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int c = 0; c < BLOCK_N; ++c)
           if (c > r) s[c] = -INFINITY;
       }
-      float mu0 = s[0], mu1 = s[64];
+      // block maxima with two independent chains per 64-key block
+      float mx[4];
 #pragma unroll
-      for (int c = 1; c < 63; c += 2) {
-        mu0 = fmax3(mu0, s[c], s[c + 1]);
-        mu1 = fmax3(mu1, s[64 + c], s[64 + c + 1]);
+      for (int i = 0; i < 4; ++i) mx[i] = s[i * 32];
+#pragma unroll
+      for (int c = 1; c < 31; c += 2) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) mx[i] = fmax3(mx[i], s[i * 32 + c], s[i * 32 + c + 1]);
       }
-      mu0 = fmaxf(mu0, s[63]);
-      mu1 = fmaxf(mu1, s[127]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) mx[i] = fmaxf(mx[i], s[i * 32 + 31]);
+      const float mu0 = fmaxf(mx[0], mx[1]);
+      const float mu1 = fmaxf(mx[2], mx[3]);
 
       uint32_t pw[FP8 ? 32 : 64];
       float alpha = 1.0f;
+      uint32_t sf_w = 0;
       if constexpr (!FP8) {
         const float cand = fmaxf(mu0, mu1) * p.c1;
         const float ms_new = (j == 0 || cand > ms + BF16_HEADROOM) ? cand : ms;
@@ -457,7 +503,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int m_new = (j == 0 || cand > m_i + LEANP_HEADROOM) ? cand : m_i;
         if (j > 0) alpha = ex2_approx(static_cast<float>(m_i - m_new) * 0.125f);
         m_i = m_new;
-        l *= alpha;
         const int k0 = leanp_kshift(mu0, a, m_new);
         const int k1 = leanp_kshift(mu1, a, m_new);
         const float cb0 = __int2float_rn(LEANP_TOP + 8 * k0 - m_new) * 0.00390625f;
@@ -484,14 +529,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           dk[0] = static_cast<uint8_t>(k0);
           dk[1] = static_cast<uint8_t>(k1);
         }
-        // scale factors of P: the word for row R lives in column SFA + R/32 at lane R%32
-        // of every 32-lane quadrant (byte k = 32-key block k of the tile), so each warp
-        // writes the words of all 128 rows for its own quadrant: exchange through smem
-        sf_x[(t * 2 + (j & 1)) * 128 + r] = sf_word;
-        mbar_arrive(sf_bar(t));
+        sf_w = sf_word;
       }
-      // the previous PV of this tile is complete here (BF16: S_t(j) completed after it;
-      // FP8: the row sum was read back before S_t(j) was issued), so O_t may be rescaled
+      // the previous PV of this tile is complete here (S_t(j) was issued after it and
+      // has completed), so O_t (and the FP8 row sum) may be rescaled
       if (__any_sync(0xffffffffu, alpha != 1.0f)) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -502,42 +543,43 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
           tmem_st32(to + c * 32, o);
         }
+        if constexpr (FP8) {
+          uint32_t rs;
+          tmem_ld1(to + TM::RS, rs);
+          tmem_wait_ld();
+          tmem_st1(to + TM::RS, __float_as_uint(__uint_as_float(rs) * alpha));
+        }
       }
       if constexpr (!FP8) {
-        tmem_st32(ts, pw);
-        tmem_st32(ts + 32, pw + 32);
+        tmem_st32(tp, pw);
+        tmem_st32(tp + 32, pw + 32);
       } else {
-        tmem_st32(ts, pw);
-        tmem_st4(ts + TM_SFB_OFF, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
-        ok = mbar_wait(sf_bar(t), j & 1, p.err, p.timeout_ns);
-        if (!ok) break;
-        const uint32_t* x = sf_x + (t * 2 + (j & 1)) * 128;
-        tmem_st4(ts + TM_SFA_OFF, x[lane], x[32 + lane], x[64 + lane], x[96 + lane]);
+        tmem_st32(tp, pw);
+        const uint32_t sfb = lane_base + TM::SFB(t);
+        tmem_st4(sfb, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+        tmem_st4(sfb + 4, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+        // scale factors of P: row R's word (byte k = 32-key block k of the tile) at lane R,
+        // column SFA + R/32 -- the quadrant of the MMA datapath that computes row R
+        tmem_st1(lane_base + TM::SFA(t) + (warp & 3), sf_w);
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(p_full(t));
-      if constexpr (FP8) {
-        // the row sum of this tile's rounded probabilities, read back before S_t(j+1)
-        ok = mbar_wait(pv_done(t), j & 1, p.err, p.timeout_ns);
-        if (!ok) break;
-        tc_fence_after();
-        uint32_t rs;
-        tmem_ld1(ts + TM_RS_OFF, rs);
-        tmem_wait_ld();
-        l += __uint_as_float(rs);
-        tc_fence_before();
-        mbar_arrive(s_free(t));
-      }
     }
     tmem_wait_st();  // nothing of this thread may still be writing TMEM on any exit path
     // ------------------------------------------------------------- epilogue
-    if (ok && n_t > 0 && !FP8) ok = mbar_wait(pv_done(t), (n_t - 1) & 1, p.err, p.timeout_ns);
+    if (ok && n_t > 0) ok = mbar_wait(pv_done(t), (n_t - 1) & 1, p.err, p.timeout_ns);
     if (ok && n_t > 0) {
       tc_fence_after();
       uint32_t oraw[DV];
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(to + c * 32, oraw + c * 32);
+      if constexpr (FP8) {
+        uint32_t rs;
+        tmem_ld1(to + TM::RS, rs);
+        tmem_wait_ld();
+        l = __uint_as_float(rs);  // sum of the rounded probabilities, 2^-(7+k) scaled
+      }
       tmem_wait_ld();
       float o[DV];
 #pragma unroll
