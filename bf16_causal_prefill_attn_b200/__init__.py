@@ -58,6 +58,8 @@ def lib():
         L.attn_device_status.restype = i32
         L.attn_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
         L.attn_set_wait_timeout_ns.restype = None
+        L.attn_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
+        L.attn_selftest_wait_timeout.restype = i32
         L.attn_status_string.argtypes = [i32]
         L.attn_status_string.restype = ctypes.c_char_p
         L.attn_version.argtypes = []
@@ -173,3 +175,9 @@ def attn_device_status(stream=None):
 
 def attn_set_wait_timeout_ns(ns):
     lib().attn_set_wait_timeout_ns(int(ns))
+
+
+def attn_selftest_wait_timeout(timeout_ns, stream=None):
+    """Launch the test-only kernel whose bounded wait is never satisfied."""
+    _check(lib().attn_selftest_wait_timeout(int(timeout_ns), _stream(stream)),
+           "attn_selftest_wait_timeout")

@@ -150,6 +150,15 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, flo
   return launch_fwd<true, 192, false>(q, k, v, prm, st);
 }
 
+// A wait that nothing ever satisfies: one thread waits (bounded) on an mbarrier no one
+// arrives at, records DEV_TIMEOUT and returns.
+__global__ void selftest_wait_kernel(uint32_t* err, uint64_t timeout_ns) {
+  __shared__ uint64_t bar;
+  attn::mbar_init(&bar, 1);
+  attn::fence_barrier_init();
+  attn::mbar_wait(&bar, 0, err, timeout_ns);
+}
+
 int num_sms() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
@@ -250,6 +259,14 @@ attn_status_t attn_device_status(void* stream) {
 }
 
 void attn_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns = ns ? ns : kDefaultTimeoutNs; }
+
+attn_status_t attn_selftest_wait_timeout(uint64_t timeout_ns, void* stream) {
+  if (timeout_ns == 0 || timeout_ns > 10000000000ull) return ATTN_ERR_INVALID_ARG;
+  uint32_t* err = nullptr;
+  if (!dev_err_ptr(&err)) return ATTN_ERR_CUDA;
+  selftest_wait_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(err, timeout_ns);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
 
 const char* attn_status_string(attn_status_t s) {
   switch (s) {

@@ -139,6 +139,14 @@ attn_status_t attn_device_status(void* stream);
 /* Test-only: sets the bounded-wait limit in nanoseconds (0 restores the default, 2 s). */
 void attn_set_wait_timeout_ns(uint64_t ns);
 
+/*
+ * Test-only: launches one thread that waits, with the bounded wait the kernels use, on an
+ * mbarrier that nothing completes.  The wait gives up after timeout_ns (1 ns .. 10 s) and
+ * records the timeout in the device error word, so attn_device_status() then reports
+ * ATTN_ERR_TIMEOUT and the context stays usable.
+ */
+attn_status_t attn_selftest_wait_timeout(uint64_t timeout_ns, void* stream);
+
 const char* attn_status_string(attn_status_t status);
 int attn_version(void);
 
