@@ -20,23 +20,30 @@
 //   warps 0-3   softmax of tile 0, warps 4-7 softmax of tile 1: thread r of the group owns
 //               query row r (TMEM lane r); reads S, updates the reference max (lazily:
 //               only when the tile max exceeds it by more than the headroom), rescales O
-//               in TMEM when it does, writes P (and the FP8 scale factors) into the S
-//               columns it has consumed, and finally writes O and lse;
+//               in TMEM when it does, writes P (BF16: into the S columns it has consumed;
+//               FP8: into shared memory, with its scale factors in TMEM), and finally
+//               writes O and lse;
 //   warp 8      TMA producer: both Q tiles once, then K and V through NK / NV stages;
-//   warp 9      MMA issuer (warp-wide control flow, one elected lane issues), in the fixed
-//               order PV_0(j), S_0(j+1), PV_1(j), S_1(j+1): one tile's softmax overlaps
-//               the other tile's MMAs (ping-pong);
-//   warp 10     idle; warp 11 TMEM allocator.
+//   warp 9      MMA issuer (warp-wide control flow, one elected lane issues).  One tile's
+//               softmax overlaps the other tile's MMAs (ping-pong).  Order per key tile j:
+//                 BF16  PV_0(j), S_0(j+1), PV_1(j), S_1(j+1)  (P_t aliases S_t, so
+//                       S_t(j+1) must follow PV_t(j));
+//                 FP8   S_0(j+1), PV_0(j), S_1(j+1), PV_1(j)  (S_t(j+1) only needs S_t(j)
+//                       read into registers, so it runs during the softmax of S_t(j): each
+//                       softmax group then has a whole period, not half, for its tile);
+//   warp 10     FP8: PV MMA issuer (warp 9 then issues only the S MMAs); BF16: idle;
+//   warp 11     TMEM allocator.
 // TMEM (512 columns x 128 lanes, see TmemMap):
 //   BF16  S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512); P_t (bf16, 64
 //         columns) overwrites the first columns of S_t.
 //   FP8   O_0 [0,144), O_1 [160,304): the PV MMA has N = 144, V extended by a 16-column
 //         block of ones, so columns 128..143 accumulate the row sum of the rounded P with
 //         the same block scales (the "extra matrix instruction" costs no extra issue);
-//         S_0 [320,448), S_1 [384,512) overlap in [384,448), so an S MMA is issued only
-//         after the other tile's softmax group has read its S (s_read barriers); P_t (32
-//         columns) and its scale factors live in the part of S_t the other tile never
-//         writes (S_0: [320,384), S_1: [448,512)).
+//         scale factors of P_0, P_1 at [144,148), [148,152), the constant scale factors
+//         of V at [152,160); S_0 [320,448), S_1 [384,512) overlap in [384,448), so an S
+//         MMA is issued only after both softmax groups have read their latest S (s_read
+//         barriers).  P_t (128 x 128 e4m3) is in shared memory in the K-major 128-byte
+//         swizzled layout of an MMA A operand.
 //
 // Every wait is bounded (mbar_wait): on expiry the CTA records DEV_TIMEOUT and unwinds.
 #pragma once
@@ -62,9 +69,9 @@ template <bool FP8>
 struct TmemMap {
   __host__ __device__ static constexpr uint32_t S(int t) { return FP8 ? 320u + 64u * t : 128u * t; }
   __host__ __device__ static constexpr uint32_t O(int t) { return FP8 ? 160u * t : 256u + 128u * t; }
-  __host__ __device__ static constexpr uint32_t P(int t) { return FP8 ? (t ? 448u : 320u) : 128u * t; }
-  __host__ __device__ static constexpr uint32_t SFA(int t) { return P(t) + 32; }  // 4 columns
-  __host__ __device__ static constexpr uint32_t SFB(int t) { return P(t) + 40; }  // 8 columns
+  __host__ __device__ static constexpr uint32_t P(int t) { return 128u * t; }     // BF16 only
+  __host__ __device__ static constexpr uint32_t SFA(int t) { return 144u + 4u * t; }  // FP8, 4 columns
+  static constexpr uint32_t SFB = 152;                         // FP8, 8 columns
   static constexpr uint32_t RS = 128;                          // row-sum column of O(t)
   static constexpr uint32_t PV_N = FP8 ? 144 : 128;
 };
@@ -110,7 +117,7 @@ struct FwdCfg {
   static constexpr int Q_BYTES = Q_BOXES * BOX_BYTES;
   static constexpr int K_BYTES = Q_BYTES;
   static constexpr int V_BYTES = V_BOXES * BOX_BYTES;
-  static constexpr int NK = FP8 ? (DQK == 128 ? 4 : 3) : 2;     // K ring depth
+  static constexpr int NK = FP8 ? (DQK == 128 ? 4 : 2) : 2;     // K ring depth
   static constexpr int NV = FP8 ? (DQK == 128 ? 4 : 2) : (DQK == 128 ? 2 : 1);
   static constexpr int KSTEP = FP8 ? 32 : 16;                   // MMA K per instruction
   static constexpr int QK_STEPS = DQK / KSTEP;
@@ -119,13 +126,13 @@ struct FwdCfg {
   static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
   static constexpr int OFF_V = OFF_K + NK * K_BYTES;
   static constexpr int OFF_ONES = OFF_V + NV * V_BYTES;  // FP8: 128 keys x 128 B of 1.0
-  static constexpr int OFF_BAR = OFF_ONES + (FP8 ? BOX_BYTES : 0);
+  static constexpr int OFF_P = OFF_ONES + (FP8 ? BOX_BYTES : 0);  // FP8: P_0, P_1
+  static constexpr int OFF_BAR = OFF_P + (FP8 ? 2 * BOX_BYTES : 0);
   // barriers: q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], and per tile:
-  //           s_full, p_full, pv_done, s_read, sf_bar, mma_done
-  static constexpr int NUM_BARS = 1 + 2 * NK + 2 * NV + 2 * 6;
+  //           s_full, p_full, pv_done, s_read, mma_done
+  static constexpr int NUM_BARS = 1 + 2 * NK + 2 * NV + 2 * 5;
   static constexpr int OFF_TMEMPTR = OFF_BAR + NUM_BARS * 8;
-  static constexpr int OFF_SF = (OFF_TMEMPTR + 4 + 15) / 16 * 16;  // [2 tiles][2][128] u32
-  static constexpr int SMEM_BYTES = OFF_SF + (FP8 ? 2 * 2 * 128 * 4 : 0);
+  static constexpr int SMEM_BYTES = OFF_TMEMPTR + 16;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;           // 1024-B alignment slack
   static_assert(SMEM_ALLOC <= 232448, "shared memory per block exceeded");
   static constexpr uint32_t IDESC_S =
@@ -176,15 +183,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* k_empty = k_full + C::NK;
   uint64_t* v_full = k_empty + C::NK;
   uint64_t* v_empty = v_full + C::NV;
-  uint64_t* tbar = v_empty + C::NV;  // per tile: 6 barriers
-  auto s_full = [&](int t) { return tbar + 6 * t + 0; };
-  auto p_full = [&](int t) { return tbar + 6 * t + 1; };
-  auto pv_done = [&](int t) { return tbar + 6 * t + 2; };
-  auto s_read = [&](int t) { return tbar + 6 * t + 3; };
-  auto sf_bar = [&](int t) { return tbar + 6 * t + 4; };
-  auto mma_done = [&](int t) { return tbar + 6 * t + 5; };
+  uint64_t* tbar = v_empty + C::NV;  // per tile: 5 barriers
+  auto s_full = [&](int t) { return tbar + 5 * t + 0; };
+  auto p_full = [&](int t) { return tbar + 5 * t + 1; };
+  auto pv_done = [&](int t) { return tbar + 5 * t + 2; };
+  auto s_read = [&](int t) { return tbar + 5 * t + 3; };
+  auto mma_done = [&](int t) { return tbar + 5 * t + 4; };
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEMPTR);
-  uint32_t* sf_x = reinterpret_cast<uint32_t*>(smem + C::OFF_SF);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -219,7 +224,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(p_full(t), 128);
       mbar_init(pv_done(t), 1);
       mbar_init(s_read(t), 128);
-      mbar_init(sf_bar(t), 128);
       mbar_init(mma_done(t), 1);
     }
     fence_barrier_init();
@@ -289,12 +293,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mbar_wait(k_full + jj % C::NK, (jj / C::NK) & 1, p.err, DRAIN_TIMEOUT_NS, false);
       for (int jj = (jv > C::NV ? jv - C::NV : 0); jj < jv; ++jj)
         mbar_wait(v_full + jj % C::NV, (jj / C::NV) & 1, p.err, DRAIN_TIMEOUT_NS, false);
-    } else if (warp == 9) {
-      // ----------------------------------------------------------- MMA issuer (warp-wide
-      // control flow, one elected lane issues).  Fixed order per key tile j:
-      //   PV_0(j), S_0(j+1), PV_1(j), S_1(j+1)
-      // so tile 1's softmax of j overlaps PV_0(j) + S_0(j+1) and tile 0's softmax of j+1
-      // overlaps PV_1(j) + S_1(j+1) (ping-pong).
+    } else if (warp == 9 || (FP8 && warp == 10)) {
+      // ----------------------------------------------------------- MMA issuers (warp-wide
+      // control flow, one elected lane issues); the order per key tile is in the header.
+      // FP8: warp 9 issues the S MMAs, warp 10 the PV MMAs (they touch disjoint TMEM
+      // columns and P is in shared memory, so only mbarriers order them), so that one
+      // warp's waits and control flow overlap the other warp's issue.  BF16: warp 9 issues
+      // both (P_t aliases S_t, so S_t(j+1) must follow PV_t(j) in one issue stream).
       using TM = TmemMap<FP8>;
       auto nt = [&](int t) { return t == 0 ? n_t0 : n_t1; };
       // Descriptors are built once; advancing an operand by `off` bytes adds off >> 4 to
@@ -302,6 +307,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // field never carries into its neighbours).
       const uint64_t dq0 = smem_desc_sw128(smem_addr(smem + C::OFF_Q), 16, 1024);
       const uint64_t dk0 = smem_desc_sw128(smem_addr(smem + C::OFF_K), 16, 1024);
+      const uint64_t dp0 = smem_desc_sw128(smem_addr(smem + C::OFF_P), 16, 1024);  // FP8
       auto v_desc = [&](int sv) -> uint64_t {
         const uint32_t va = smem_addr(smem + C::OFF_V + sv * C::V_BYTES);
         if constexpr (FP8) {
@@ -331,10 +337,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       auto issue_pv = [&](int t, int j) {
         const int sv = j % C::NV;
         const uint64_t vd = v_desc(sv);
-        const uint32_t tm_p = tmem + TM::P(t);
         const uint32_t tm_o = tmem + TM::O(t);
         if (elect_one()) {
           if constexpr (!FP8) {
+            const uint32_t tm_p = tmem + TM::P(t);
 #pragma unroll
             for (int s = 0; s < C::PV_STEPS; ++s) {
               // V is [keys x d] with d contiguous: B operand MN-major; 8-key groups 1 KB
@@ -343,12 +349,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                          (j > 0 || s > 0) ? 1u : 0u);
             }
           } else {
+            const uint64_t pd = dp0 + static_cast<uint32_t>((t * C::BOX_BYTES) >> 4);
 #pragma unroll
             for (int s = 0; s < C::PV_STEPS; ++s) {
-              // [O | row sum] += (P * 2^-(7+k)) x [V | 1]; 32 keys per step
+              // [O | row sum] += (P * 2^-(7+k)) x [V | 1]; 32 keys (32 B of P) per step
               const uint32_t sfa = (tmem + TM::SFA(t)) | (static_cast<uint32_t>(s) << 30);
-              const uint32_t sfb = (tmem + TM::SFB(t)) | (static_cast<uint32_t>(s) << 30);
-              mma_ts_mxf8(tm_o, tm_p + s * 8, vd + ((s * 4096) >> 4),
+              const uint32_t sfb = (tmem + TM::SFB) | (static_cast<uint32_t>(s) << 30);
+              mma_ss_mxf8(tm_o, pd + ((s * 32) >> 4), vd + ((s * 4096) >> 4),
                           idesc_mxf8(0, 1, BLOCK_M, TM::PV_N, s, s), sfa, sfb,
                           (j > 0 || s > 0) ? 1u : 0u);
             }
@@ -365,17 +372,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (jo < 0) return true;
         return mbar_wait(s_read(1 - t), jo & 1, p.err, p.timeout_ns);
       };
-      bool ok = mbar_wait(q_full, 0, p.err, p.timeout_ns);
-      if (__all_sync(0xffffffffu, ok)) {
-        ok = mbar_wait(k_full, 0, p.err, p.timeout_ns);
+      const bool s_issuer = warp == 9;  // FP8: S MMAs; BF16: all MMAs
+      bool ok = true;
+      if (s_issuer) {
+        ok = mbar_wait(q_full, 0, p.err, p.timeout_ns);
         if (__all_sync(0xffffffffu, ok)) {
-          tc_fence_after();
-          if (n_t0 > 0) issue_s(0, 0);
-          if (n_t1 > 0) {
-            ok = wait_other_read(1, n_t0 > 0 ? 0 : -1);
-            if (__all_sync(0xffffffffu, ok)) {
-              tc_fence_after();
-              issue_s(1, 0);
+          ok = mbar_wait(k_full, 0, p.err, p.timeout_ns);
+          if (__all_sync(0xffffffffu, ok)) {
+            tc_fence_after();
+            if (n_t0 > 0) issue_s(0, 0);
+            if (n_t1 > 0) {
+              ok = wait_other_read(1, n_t0 > 0 ? 0 : -1);
+              if (__all_sync(0xffffffffu, ok)) {
+                tc_fence_after();
+                issue_s(1, 0);
+              }
             }
           }
         }
@@ -385,25 +396,46 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int t = 0; t < 2; ++t) {
           if (j >= nt(t)) continue;
           const bool next = j + 1 < nt(t);
-          if (next) {
-            // prerequisites of S_t(j+1), normally met long before P_t(j) is ready: K(j+1)
-            // landed, and the other tile's softmax read its latest S (S_1(j) or S_0(j+1))
-            const int jo = t == 0 ? min(j, n_t1 - 1) : min(j + 1, n_t0 - 1);
-            ok = wait_other_read(t, jo);
-            if (ok) ok = mbar_wait(k_full + (j + 1) % C::NK, ((j + 1) / C::NK) & 1, p.err, p.timeout_ns);
+          if constexpr (FP8) {
+            if (s_issuer) {
+              // S_t(j+1) once S_t(j) and the other tile's latest S (S_1(j) or S_0(j+1))
+              // have been read into registers and K(j+1) has landed
+              if (next) {
+                const int jo = t == 0 ? min(j, n_t1 - 1) : min(j + 1, n_t0 - 1);
+                ok = mbar_wait(s_read(t), j & 1, p.err, p.timeout_ns);
+                if (ok) ok = wait_other_read(t, jo);
+                if (ok) ok = mbar_wait(k_full + (j + 1) % C::NK, ((j + 1) / C::NK) & 1, p.err, p.timeout_ns);
+                if (!__all_sync(0xffffffffu, ok)) break;
+                tc_fence_after();
+                issue_s(t, j + 1);
+              }
+            } else {
+              // PV_t(j) once P_t(j) is in shared memory and V(j) has landed
+              ok = mbar_wait(p_full(t), j & 1, p.err, p.timeout_ns);
+              if (ok) ok = mbar_wait(v_full + j % C::NV, (j / C::NV) & 1, p.err, p.timeout_ns);
+              if (!__all_sync(0xffffffffu, ok)) break;
+              tc_fence_after();
+              issue_pv(t, j);
+            }
+          } else {
+            if (next) {
+              // prerequisites of S_t(j+1), normally met long before P_t(j) is ready
+              ok = mbar_wait(k_full + (j + 1) % C::NK, ((j + 1) / C::NK) & 1, p.err, p.timeout_ns);
+            }
+            if (ok) ok = mbar_wait(p_full(t), j & 1, p.err, p.timeout_ns);
+            if (ok) ok = mbar_wait(v_full + j % C::NV, (j / C::NV) & 1, p.err, p.timeout_ns);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            issue_pv(t, j);
+            if (next) issue_s(t, j + 1);
           }
-          if (ok) ok = mbar_wait(p_full(t), j & 1, p.err, p.timeout_ns);
-          if (ok) ok = mbar_wait(v_full + j % C::NV, (j / C::NV) & 1, p.err, p.timeout_ns);
-          if (!__all_sync(0xffffffffu, ok)) break;
-          tc_fence_after();
-          issue_pv(t, j);
-          if (next) issue_s(t, j + 1);
         }
       }
       // every MMA issued by this warp completes before TMEM is released
-      if (elect_one()) tc_commit(mma_done(0));
+      const int mine = s_issuer ? 0 : 1;
+      if (elect_one()) tc_commit(mma_done(mine));
       __syncwarp();
-      mbar_wait(mma_done(0), 0, p.err, DRAIN_TIMEOUT_NS, false);
+      mbar_wait(mma_done(mine), 0, p.err, DRAIN_TIMEOUT_NS, false);
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_SOFTMAX));
@@ -416,7 +448,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     using TM = TmemMap<FP8>;
     const uint32_t ts = lane_base + TM::S(t);     // S_t columns of this lane
-    const uint32_t tp = lane_base + TM::P(t);     // P_t columns
+    const uint32_t tp = lane_base + TM::P(t);     // BF16: P_t columns
     const uint32_t to = lane_base + TM::O(t);     // O_t (FP8: and the row sum) columns
     float a = 0.0f, a256 = 0.0f;  // FP8 slope in code units per raw score (and / 256)
     if constexpr (FP8) {
@@ -427,10 +459,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     float ms = -INFINITY;  // BF16 reference max, scaled to log2 units
     int m_i = 0;           // FP8 reference max, code units
     float l = 0.0f;        // running row sum
+    if constexpr (FP8) {
+      // scale factors of the B operand [V | 1]: 2^0, for every PV of this CTA
+      const uint32_t sfb = lane_base + TM::SFB;
+      tmem_st4(sfb, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+      tmem_st4(sfb + 4, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+    }
     bool ok = true;
     for (int j = 0; j < n_t; ++j) {
       ok = mbar_wait(s_full(t), j & 1, p.err, p.timeout_ns);
-      if (!ok) break;
+      if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       uint32_t sraw[BLOCK_N];
 #pragma unroll
@@ -531,8 +569,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         sf_w = sf_word;
       }
-      // the previous PV of this tile is complete here (S_t(j) was issued after it and
-      // has completed), so O_t (and the FP8 row sum) may be rescaled
+      if constexpr (FP8) {
+        // S_t(j) may have been issued before PV_t(j-1): that PV must be complete before
+        // O_t is rescaled and before P_t and its scale factors are overwritten
+        if (j > 0) {
+          ok = mbar_wait(pv_done(t), (j - 1) & 1, p.err, p.timeout_ns);
+          if (!__all_sync(0xffffffffu, ok)) break;
+          tc_fence_after();
+        }
+      }
+      // BF16: the previous PV of this tile is complete here (S_t(j) was issued after it
+      // and has completed).  O_t (and the FP8 row sum) may be rescaled.
       if (__any_sync(0xffffffffu, alpha != 1.0f)) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -554,10 +601,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_st32(tp, pw);
         tmem_st32(tp + 32, pw + 32);
       } else {
-        tmem_st32(tp, pw);
-        const uint32_t sfb = lane_base + TM::SFB(t);
-        tmem_st4(sfb, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
-        tmem_st4(sfb + 4, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+        // row r of P_t: 128 codes = 8 chunks of 16 B; chunk c sits at chunk position
+        // c ^ (r mod 8) of the row (128-byte swizzle, rows 128 B apart)
+        const uint32_t prow = smem_addr(smem + C::OFF_P + t * C::BOX_BYTES) + r * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          st_shared_v4(prow + ((c ^ (r & 7)) << 4), pw[4 * c], pw[4 * c + 1], pw[4 * c + 2],
+                       pw[4 * c + 3]);
+        fence_proxy_async_smem();
         // scale factors of P: row R's word (byte k = 32-key block k of the tile) at lane R,
         // column SFA + R/32 -- the quadrant of the MMA datapath that computes row R
         tmem_st1(lane_base + TM::SFA(t) + (warp & 3), sf_w);
