@@ -79,7 +79,7 @@ constexpr float LEANP_MAGIC = 12582912.0f;  // 1.5 * 2^23
 constexpr int LEANP_KMAX = 16;
 constexpr int LEANP_TOP = 112;       // code of a block maximum at the reference
 constexpr int LEANP_HEADROOM = 14;   // 126 - LEANP_TOP
-constexpr float BF16_HEADROOM = 8.0f;  // log2 units the reference max may lag the true max
+constexpr float BF16_HEADROOM = 24.0f;  // log2 units the reference max may lag the true max
 
 // 2^f on [-0.5, 0.5], degree 3, coefficients fitted here to minimise the relative error
 // (max 7.5e-5, well under the bf16 rounding of P)
@@ -154,7 +154,7 @@ __device__ __forceinline__ float fma_sat(float a, float b, float c) {
   return d;
 }
 
-// 2^x for x <= 8 on the FMA pipe: x = n + f, f in [-0.5, 0.5], 2^f by the polynomial,
+// 2^x for x <= BF16_HEADROOM on the FMA pipe: x = n + f, f in [-0.5, 0.5], 2^f by the polynomial,
 // 2^n added to the exponent field.  Inputs below -125 give 2^-125.
 __device__ __forceinline__ float exp2_poly(float x) {
   x = fmaxf(x, -125.0f);
