@@ -187,3 +187,20 @@ void leanp_attention_row(const float* s, int S_k, int tile, const double* v, int
     for (int d = 0; d < dv; ++d) o_out[d] = acc[d] / l;
     *lse_out = log(2.0) * ((double)m / 8.0 + log2(l));
 }
+
+/*
+ * Exact-P ablation ([ZYFA-mb] "Como o motor de atenção FP8 da Zyphra funciona" contrasts
+ * lean P with "exact P", the probabilities formed with an exponential and then rounded to
+ * FP8).  Reading: same reference max m and block shifts k_b as lean P; the value written
+ * is e4m3_rn(2^x) with the float32 exponent
+ *     x = fmaf(s, a / 8, (8 (7 + k_b) - m) / 8)      (a / 8 and the constant are exact)
+ * so that 2^x = 2^((a s - m)/8) 2^(7 + k_b), the quantity lean P approximates.  This
+ * function forms x for n scores; the exponential and the e4m3 rounding are done by the
+ * caller (oracle/leanp.py) in float64 and with the table codec.
+ */
+void leanp_exact_arg(const float* s, int n, float a, int m, int kb, float* x) {
+    const float a8 = a * 0.125f;
+    const float c = (float)(8 * (7 + kb) - m) * 0.125f;
+    for (int i = 0; i < n; ++i) x[i] = fmaf(s[i], a8, c);
+}
+

@@ -56,6 +56,8 @@ def lib():
                                           ctypes.POINTER(ctypes.c_int)]
         _lib.leanp_attention_row.restype = None
         _lib.leanp_attention_row.argtypes = [fp, i32, i32, dp, i32, f32, i32, dp, dp]
+        _lib.leanp_exact_arg.restype = None
+        _lib.leanp_exact_arg.argtypes = [fp, i32, f32, i32, i32, fp]
     return _lib
 
 
@@ -139,3 +141,89 @@ def attention_rows(q_codes, k_codes, v_codes, dq, dk, dv, rows, heads, batch=0,
             o[hi, ri] = orow
             lse[hi, ri] = lrow[0]
     return o, lse
+
+
+# ----------------------------------------------------------------------------- exact P
+# The ablation the pages contrast with lean P: the same reference max and 64-key block
+# shifts, but each probability formed by an exponential and rounded to e4m3 (round to
+# nearest even, saturating).  See leanp_exact_arg in leanp.c for the reading.
+
+def exact_arg(s, a, m, kb):
+    """float32 exponent x = fmaf(s, a/8, (8 (7 + kb) - m)/8) for an array of scores."""
+    s = np.ascontiguousarray(s, dtype=np.float32).ravel()
+    x = np.zeros_like(s)
+    lib().leanp_exact_arg(_ptr(s, ctypes.c_float), s.size, float(a), int(m), int(kb),
+                          _ptr(x, ctypes.c_float))
+    return x
+
+
+def exact_codes(s, a, m, kb):
+    """e4m3 codes of float32(2^x), x = exact_arg(s, a, m, kb); -inf scores give code 0."""
+    x = exact_arg(s, a, m, kb)
+    with np.errstate(over="ignore"):
+        v = np.exp2(x.astype(np.float64)).astype(np.float32)
+    return _e4m3.e4m3_encode(v)
+
+
+def encode_row_exact(s_row, a, tile=TILE, kmax=KMAX):
+    """Exact-P codes of one row: the lean-P state machine (encode_row) fixes the reference
+    max per tile and the shift per 64-key block; the codes are then exact_codes.
+    Returns (codes uint8 [n], kshift uint8 [n/64], mref int32 [n/tile])."""
+    s = np.ascontiguousarray(s_row, dtype=np.float32)
+    _, ks, mref = encode_row(s, a, tile, kmax)
+    codes = np.zeros(s.shape[0], dtype=np.uint8)
+    for b in range(s.shape[0] // 64):
+        t = (b * 64) // tile
+        blk = s[b * 64:(b + 1) * 64]
+        if np.all(np.isneginf(blk)):
+            continue
+        codes[b * 64:(b + 1) * 64] = exact_codes(blk, a, mref[t], int(ks[b]))
+    return codes, ks, mref
+
+
+def combine_row(codes, ks, mref, n_vis, vd, tile=TILE):
+    """Normalised output row and lse from the codes of one row, in float64: weight of key j
+    = decode(code_j) 2^-(7 + k_b(j)) 2^((m_t(j) - m_final)/8), o = sum w_j v_j / sum w_j,
+    lse = ln 2 (m_final/8 + log2 sum w_j) with the weights taken relative to m_final.  This
+    is the tile-by-tile online combination with its rescales written out."""
+    ntiles = (n_vis + tile - 1) // tile
+    m_final = int(mref[ntiles - 1])  # any common reference cancels in o; lse adds it back
+    j = np.arange(n_vis)
+    w = (_e4m3.e4m3_decode(codes[:n_vis]) * np.exp2(-(7.0 + ks[j // 64].astype(np.float64)))
+         * np.exp2((mref[j // tile].astype(np.float64) - m_final) / 8.0))
+    l = w.sum()
+    o = (w[:, None] * vd[:n_vis]).sum(axis=0) / l
+    return o, np.log(2.0) * (m_final / 8.0 + np.log2(l))
+
+
+def attention_rows_exact(q_codes, k_codes, v_codes, dq, dk, dv, rows, heads, batch=0,
+                         causal=True, tile=TILE, kmax=KMAX, lean=False):
+    """End-to-end exact-P prediction for selected rows/heads (layout as attention_rows).
+    With lean=True the same driver combines lean-P codes instead (used to pin the driver
+    against the C tile driver)."""
+    Hq = q_codes.shape[2]
+    Hkv = k_codes.shape[2]
+    G = Hq // Hkv
+    d_qk = q_codes.shape[3]
+    d_v = v_codes.shape[3]
+    a = slope(d_qk, dq, dk)
+    o = np.zeros((len(heads), len(rows), d_v))
+    lse = np.zeros((len(heads), len(rows)))
+    for hi, h in enumerate(heads):
+        g = h // G
+        kd = _e4m3.e4m3_decode(k_codes[batch, :, g, :])
+        vd = _e4m3.e4m3_decode(v_codes[batch, :, g, :]) * np.float64(dv)
+        S = kd.shape[0]
+        for ri, i in enumerate(rows):
+            n_vis = i + 1 if causal else S
+            qd = _e4m3.e4m3_decode(q_codes[batch, i, h, :])
+            n_pad = (n_vis + tile - 1) // tile * tile
+            s = np.full(n_pad, -np.inf, dtype=np.float32)
+            s[:n_vis] = (kd[:n_vis] @ qd).astype(np.float32)
+            if lean:
+                codes, ks, mref = encode_row(s, a, tile, kmax)
+            else:
+                codes, ks, mref = encode_row_exact(s, a, tile, kmax)
+            o[hi, ri], lse[hi, ri] = combine_row(codes, ks, mref, n_vis, vd, tile)
+    return o, lse
+
