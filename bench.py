@@ -177,7 +177,7 @@ def gpu_bench(args, rank, world, local_rank):
         if ev_a is not None:
             ev_a.record(stream)
         pkg.attn_fwd(q8, k8, v8, descale_q=ds[0], descale_k=ds[1], descale_v=ds[2], out=o, lse=lse,
-                     unrotate=args.hadamard)
+                     unrotate=args.hadamard, exact_p=args.exact_p)
         if ev_b is not None:
             ev_b.record(stream)
 
@@ -240,7 +240,8 @@ def gpu_bench(args, rank, world, local_rank):
     fp8_peak = 2.0 * bf16_peak  # measured bf16 peak x the nominal fp8/bf16 ratio (2)
     fp8_kern_tf = flops / (fp8_kern * 1e-3) / 1e12
     bf16_kern_tf = flops / (bf16_kern * 1e-3) / 1e12
-    traffic = load_traffic(args.workload)
+    # counters were taken for the lean-P kernel only
+    traffic = {} if args.exact_p else load_traffic(args.workload)
     result = {
         "metric": METRIC,
         "value": round(job_tflops(flops, world, fp8_ms), 2),
@@ -256,7 +257,8 @@ def gpu_bench(args, rank, world, local_rank):
         "data": "synthetic",
         "config": {"workload": desc, "name": args.workload, "B": B, "S": S, "Hq": Hq, "Hkv": Hkv,
                    "d_qk": dqk, "d_v": dv, "hadamard": bool(args.hadamard),
-                   "step": "e4m3 quantisation of Q, K, V + lean-P attention",
+                   "step": "e4m3 quantisation of Q, K, V + "
+                           + ("exact-P attention (ablation)" if args.exact_p else "lean-P attention"),
                    "l2": "256 MiB L2 flush written between steps, outside the timed step",
                    "parallelism": f"replicas x{world} (independent problems per GPU)"},
         "roofline": {"bound": "tensor", "achieved": round(fp8_kern_tf, 2),
@@ -264,7 +266,7 @@ def gpu_bench(args, rank, world, local_rank):
                      "frac": round(fp8_kern_tf / fp8_peak, 4),
                      "peak_source": f"{peak_src} bf16 cuBLAS burst x2 (fp8/bf16 nominal ratio)",
                      "frac_of_nominal_4500": round(fp8_kern_tf / NOMINAL_FP8_TFLOPS, 4),
-                     "kernel": "attn_fwd_kernel<fp8>", "kernel_ms": round(fp8_kern, 4),
+                     "kernel": "attn_fwd_kernel<fp8, exact P>" if args.exact_p else "attn_fwd_kernel<fp8>", "kernel_ms": round(fp8_kern, 4),
                      "traffic": traffic.get("fp8")},
         "bf16": {"value": round(job_tflops(flops, world, bf16_ms), 2), "unit": UNIT,
                  "ms_per_step": round(bf16_ms, 4), "dtype": "bf16",
@@ -394,6 +396,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="gqa16k_outlier", choices=sorted(WORKLOADS))
     ap.add_argument("--hadamard", action="store_true")
+    ap.add_argument("--exact-p", action="store_true",
+                    help="FP8 probabilities by exponential + e4m3 rounding (the ablation of lean P)")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

@@ -21,6 +21,7 @@ ATTN_ERR_TIMEOUT = 5
 ATTN_BF16 = 0
 ATTN_FP8_E4M3 = 1
 ATTN_FLAG_UNROTATE_O = 1
+ATTN_FLAG_EXACT_P = 2
 
 _lib = None
 
@@ -47,7 +48,7 @@ def lib():
         L.attn_fwd_ex.argtypes = fwd_args + [u32, vp]
         L.attn_fwd_ex.restype = i32
         L.attn_fwd_fp8_dump.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
-                                        vp, vp, vp, i32, vp, vp, vp, vp]
+                                        vp, vp, vp, i32, u32, vp, vp, vp, vp]
         L.attn_fwd_fp8_dump.restype = i32
         L.attn_quantize_e4m3.argtypes = [vp, vp, vp, ctypes.c_int64, i32, i32, i32, vp,
                                          ctypes.c_size_t, vp]
@@ -97,9 +98,10 @@ def _codes(t):
 
 
 def attn_fwd(q, k, v, causal=True, descale_q=None, descale_k=None, descale_v=None, out=None,
-             lse=None, return_lse=True, unrotate=False, stream=None):
+             lse=None, return_lse=True, unrotate=False, exact_p=False, stream=None):
     """Causal prefill attention.  q [B,S,Hq,d_qk], k [B,S,Hkv,d_qk], v [B,S,Hkv,d_v] on the
     GPU: bf16, or e4m3 codes (uint8 / float8_e4m3fn) with fp32 descale tensors.
+    exact_p (FP8): the exact-P ablation instead of lean P (ATTN_FLAG_EXACT_P).
     Returns (o bf16 [B,S,Hq,d_v], lse fp32 [B,Hq,S] or None)."""
     fp8 = q.dtype in (torch.uint8, torch.float8_e4m3fn)
     q, k, v = (_codes(x) for x in (q, k, v)) if fp8 else (q, k, v)
@@ -113,7 +115,7 @@ def attn_fwd(q, k, v, causal=True, descale_q=None, descale_k=None, descale_v=Non
         out = torch.empty((B, S, Hq, d_v), dtype=torch.bfloat16, device=q.device)
     if lse is None and return_lse:
         lse = torch.empty((B, Hq, S), dtype=torch.float32, device=q.device)
-    flags = ATTN_FLAG_UNROTATE_O if unrotate else 0
+    flags = (ATTN_FLAG_UNROTATE_O if unrotate else 0) | (ATTN_FLAG_EXACT_P if exact_p else 0)
     st = lib().attn_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, S,
                            d_qk, d_v, ATTN_FP8_E4M3 if fp8 else ATTN_BF16, _ptr(descale_q),
                            _ptr(descale_k), _ptr(descale_v), 1 if causal else 0, flags,
@@ -122,8 +124,10 @@ def attn_fwd(q, k, v, causal=True, descale_q=None, descale_k=None, descale_v=Non
     return out, lse
 
 
-def attn_fwd_fp8_dump(q, k, v, descale_q, descale_k, descale_v, causal=True, stream=None):
-    """Test-only FP8 forward that also returns the raw scores, lean-P codes and shifts."""
+def attn_fwd_fp8_dump(q, k, v, descale_q, descale_k, descale_v, causal=True, exact_p=False,
+                      stream=None):
+    """Test-only FP8 forward that also returns the raw scores, P codes (lean, or exact with
+    exact_p) and shifts."""
     q, k, v = (_codes(x) for x in (q, k, v))
     B, S, Hq, d_qk = q.shape
     Hkv = k.shape[2]
@@ -136,7 +140,8 @@ def attn_fwd_fp8_dump(q, k, v, descale_q, descale_k, descale_v, causal=True, str
     dk = torch.full((B, Hq, S, S // 64), 255, dtype=torch.uint8, device=dev)
     st = lib().attn_fwd_fp8_dump(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv,
                                  S, d_qk, d_v, _ptr(descale_q), _ptr(descale_k),
-                                 _ptr(descale_v), 1 if causal else 0, _ptr(ds), _ptr(dc),
+                                 _ptr(descale_v), 1 if causal else 0,
+                                 ATTN_FLAG_EXACT_P if exact_p else 0, _ptr(ds), _ptr(dc),
                                  _ptr(dk), _stream(stream))
     _check(st, "attn_fwd_fp8_dump")
     return out, lse, ds, dc, dk

@@ -61,7 +61,7 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esiz
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-template <bool FP8, int DQK, bool DUMP>
+template <bool FP8, int DQK, bool DUMP, bool EXACT = false>
 attn_status_t launch_fwd(const void* q, const void* k, const void* v, attn::FwdParams& prm,
                          cudaStream_t stream) {
   using C = attn::FwdCfg<FP8, DQK>;
@@ -73,7 +73,7 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, attn::FwdP
       !make_map(&mk, k, dt, C::E, DQK, prm.Hkv, T, C::BOX_COLS) ||
       !make_map(&mv, v, dt, C::E, attn::DV, prm.Hkv, T, C::BOX_COLS))
     return ATTN_ERR_CUDA;
-  auto kern = attn::attn_fwd_kernel<FP8, DQK, DUMP>;
+  auto kern = attn::attn_fwd_kernel<FP8, DQK, DUMP, EXACT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC) !=
       cudaSuccess)
     return ATTN_ERR_CUDA;
@@ -97,8 +97,10 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, flo
                        uint8_t* dump_kshift, bool dump, void* stream) {
   if (B < 0 || S < 0 || Hq <= 0 || Hkv <= 0 || (Hq % Hkv) != 0) return ATTN_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
-  if ((flags & ~static_cast<unsigned>(ATTN_FLAG_UNROTATE_O)) != 0) return ATTN_ERR_INVALID_ARG;
+  if ((flags & ~static_cast<unsigned>(ATTN_FLAG_UNROTATE_O | ATTN_FLAG_EXACT_P)) != 0)
+    return ATTN_ERR_INVALID_ARG;
   if (dtype != ATTN_BF16 && dtype != ATTN_FP8_E4M3) return ATTN_ERR_INVALID_ARG;
+  if ((flags & ATTN_FLAG_EXACT_P) && dtype != ATTN_FP8_E4M3) return ATTN_ERR_INVALID_ARG;
   if ((d_qk != 128 && d_qk != 192) || d_v != 128) return ATTN_ERR_UNSUPPORTED;
   if (B == 0 || S == 0) return ATTN_OK;
   if (!q || !k || !v || !o) return ATTN_ERR_INVALID_ARG;
@@ -142,9 +144,18 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, flo
     if (d_qk == 128) return launch_fwd<false, 128, false>(q, k, v, prm, st);
     return launch_fwd<false, 192, false>(q, k, v, prm, st);
   }
+  const bool exact = (flags & ATTN_FLAG_EXACT_P) != 0;
   if (dump) {
+    if (exact) {
+      if (d_qk == 128) return launch_fwd<true, 128, true, true>(q, k, v, prm, st);
+      return launch_fwd<true, 192, true, true>(q, k, v, prm, st);
+    }
     if (d_qk == 128) return launch_fwd<true, 128, true>(q, k, v, prm, st);
     return launch_fwd<true, 192, true>(q, k, v, prm, st);
+  }
+  if (exact) {
+    if (d_qk == 128) return launch_fwd<true, 128, false, true>(q, k, v, prm, st);
+    return launch_fwd<true, 192, false, true>(q, k, v, prm, st);
   }
   if (d_qk == 128) return launch_fwd<true, 128, false>(q, k, v, prm, st);
   return launch_fwd<true, 192, false>(q, k, v, prm, st);
@@ -189,10 +200,11 @@ attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v, void* o, 
 attn_status_t attn_fwd_fp8_dump(const void* q, const void* k, const void* v, void* o, float* lse,
                                 int B, int Hq, int Hkv, int S, int d_qk, int d_v,
                                 const float* descale_q, const float* descale_k,
-                                const float* descale_v, int causal, float* dump_s,
-                                uint8_t* dump_codes, uint8_t* dump_kshift, void* stream) {
+                                const float* descale_v, int causal, unsigned flags,
+                                float* dump_s, uint8_t* dump_codes, uint8_t* dump_kshift,
+                                void* stream) {
   return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, S, d_qk, d_v, ATTN_FP8_E4M3, descale_q, descale_k,
-                  descale_v, causal, 0u, dump_s, dump_codes, dump_kshift, true, stream);
+                  descale_v, causal, flags, dump_s, dump_codes, dump_kshift, true, stream);
 }
 
 size_t attn_quantize_workspace_size(int64_t tokens, int H, int d) {

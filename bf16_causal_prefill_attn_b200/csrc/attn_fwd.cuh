@@ -168,7 +168,11 @@ __device__ __forceinline__ float exp2_poly(float x) {
   return __int_as_float(__float_as_int(j) * (1 << 23) + __float_as_int(p));
 }
 
-template <bool FP8, int DQK, bool DUMP>
+// EXACT (FP8 only): the exact-P ablation -- P = e4m3_rn(2^((a s - m)/8 + 7 + k_b)) by the
+// MUFU exponential and the hardware e4m3 conversion, instead of the lean-P multiply-add and
+// integer conversion; everything else (reference max, block shifts, block-scaled PV, row
+// sum) is shared.
+template <bool FP8, int DQK, bool DUMP, bool EXACT = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
@@ -543,17 +547,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         m_i = m_new;
         const int k0 = leanp_kshift(mu0, a, m_new);
         const int k1 = leanp_kshift(mu1, a, m_new);
-        const float cb0 = __int2float_rn(LEANP_TOP + 8 * k0 - m_new) * 0.00390625f;
-        const float cb1 = __int2float_rn(LEANP_TOP + 8 * k1 - m_new) * 0.00390625f;
+        if constexpr (EXACT) {
+          // x = fmaf(s, a/8, (8 (7 + k_b) - m)/8); P code = e4m3_rn(2^x)
+          const float a8 = a * 0.125f;
+          const float cx0 = __int2float_rn(8 * (7 + k0) - m_new) * 0.125f;
+          const float cx1 = __int2float_rn(8 * (7 + k1) - m_new) * 0.125f;
 #pragma unroll
-        for (int c = 0; c < BLOCK_N; c += 4) {
-          const float cb = c < 64 ? cb0 : cb1;
-          // multiply-add (saturating to [0,1]) and the integer conversion by a magic fma
-          const uint32_t b0 = __float_as_uint(__fmaf_rn(fma_sat(s[c + 0], a256, cb), 256.0f, LEANP_MAGIC));
-          const uint32_t b1 = __float_as_uint(__fmaf_rn(fma_sat(s[c + 1], a256, cb), 256.0f, LEANP_MAGIC));
-          const uint32_t b2 = __float_as_uint(__fmaf_rn(fma_sat(s[c + 2], a256, cb), 256.0f, LEANP_MAGIC));
-          const uint32_t b3 = __float_as_uint(__fmaf_rn(fma_sat(s[c + 3], a256, cb), 256.0f, LEANP_MAGIC));
-          pw[c >> 2] = pack_low_bytes(b0, b1, b2, b3);
+          for (int c = 0; c < BLOCK_N; c += 4) {
+            const float cx = c < 64 ? cx0 : cx1;
+            const float p0 = ex2_approx(__fmaf_rn(s[c + 0], a8, cx));
+            const float p1 = ex2_approx(__fmaf_rn(s[c + 1], a8, cx));
+            const float p2 = ex2_approx(__fmaf_rn(s[c + 2], a8, cx));
+            const float p3 = ex2_approx(__fmaf_rn(s[c + 3], a8, cx));
+            pw[c >> 2] = f32_to_e4m3x2(p0, p1) | (f32_to_e4m3x2(p2, p3) << 16);
+          }
+        } else {
+          const float cb0 = __int2float_rn(LEANP_TOP + 8 * k0 - m_new) * 0.00390625f;
+          const float cb1 = __int2float_rn(LEANP_TOP + 8 * k1 - m_new) * 0.00390625f;
+#pragma unroll
+          for (int c = 0; c < BLOCK_N; c += 4) {
+            const float cb = c < 64 ? cb0 : cb1;
+            // multiply-add (saturating to [0,1]) and the integer conversion by a magic fma
+            const uint32_t b0 = __float_as_uint(__fmaf_rn(fma_sat(s[c + 0], a256, cb), 256.0f, LEANP_MAGIC));
+            const uint32_t b1 = __float_as_uint(__fmaf_rn(fma_sat(s[c + 1], a256, cb), 256.0f, LEANP_MAGIC));
+            const uint32_t b2 = __float_as_uint(__fmaf_rn(fma_sat(s[c + 2], a256, cb), 256.0f, LEANP_MAGIC));
+            const uint32_t b3 = __float_as_uint(__fmaf_rn(fma_sat(s[c + 3], a256, cb), 256.0f, LEANP_MAGIC));
+            pw[c >> 2] = pack_low_bytes(b0, b1, b2, b3);
+          }
         }
         const uint32_t e0 = static_cast<uint32_t>(120 - k0), e1 = static_cast<uint32_t>(120 - k1);
         const uint32_t sf_word = e0 | (e0 << 8) | (e1 << 16) | (e1 << 24);  // UE8M0 2^-(7+k)

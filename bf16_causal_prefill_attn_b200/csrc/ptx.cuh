@@ -287,6 +287,12 @@ __host__ __device__ constexpr uint32_t idesc_mxf8(uint32_t a_mn, uint32_t b_mn, 
 }
 
 // ------------------------------------------------------------------ misc math
+// two float32 -> e4m3 codes (round to nearest even, saturating to +-448), lo in bits 0-7
+__device__ __forceinline__ uint32_t f32_to_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

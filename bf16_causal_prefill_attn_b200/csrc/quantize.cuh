@@ -17,15 +17,11 @@
 
 #include <cstdint>
 
+#include "ptx.cuh"
+
 namespace attn {
 
 constexpr float HAD_R = 0.08838834764831845f;  // float32(1/sqrt(128))
-
-__device__ __forceinline__ uint32_t f32_to_e4m3x2(float lo, float hi) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-  return r;
-}
 
 // ---- rotated rows: one warp per 128-element row, 4 consecutive elements per lane
 __device__ __forceinline__ void load_row4(const __nv_bfloat16* x, int64_t row, int lane,

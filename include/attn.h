@@ -50,6 +50,17 @@ typedef enum attn_dtype { ATTN_BF16 = 0, ATTN_FP8_E4M3 = 1 } attn_dtype_t;
 
 /* flags of attn_fwd_ex */
 #define ATTN_FLAG_UNROTATE_O 1u /* V was Hadamard-rotated: apply x H/sqrt(128) to O rows */
+/*
+ * FP8 only (else ATTN_ERR_INVALID_ARG): the exact-P ablation that [ZYFA-mb] ("Como o motor
+ * de atenção FP8 da Zyphra funciona") contrasts with lean P.  Each probability is formed
+ * by an exponential, P = e4m3_rn(2^x) with x = fmaf(s, a/8, (8 (7 + k_b) - m)/8), instead
+ * of the lean-P multiply-add and integer conversion; the reference max m, the 64-key block
+ * shifts k_b, the block-scaled PV and the row sum are the same.  2^x is evaluated by the
+ * hardware approximate exponential (relative error below 2^-21), so codes can differ by
+ * one from the correctly rounded e4m3 of 2^x where 2^x lies that close to a rounding
+ * midpoint.
+ */
+#define ATTN_FLAG_EXACT_P 2u
 
 /*
  * attn_fwd: forward causal prefill attention.
@@ -117,8 +128,9 @@ attn_status_t attn_quantize_e4m3_static(const void* x_bf16, void* x_e4m3, float*
                                         void* stream);
 
 /*
- * Test-only: FP8 attn_fwd that also dumps, for every (query row, visible key tile), the
- * raw fp32 scores after masking, the lean-P e4m3 codes and the per-64-key shifts:
+ * Test-only: FP8 attn_fwd_ex that also dumps, for every (query row, visible key tile), the
+ * raw fp32 scores after masking, the P e4m3 codes (lean P, or exact P with
+ * ATTN_FLAG_EXACT_P in flags) and the per-64-key shifts:
  *   dump_s      [B, Hq, S, S] fp32      dump_codes [B, Hq, S, S] uint8
  *   dump_kshift [B, Hq, S, S/64] uint8  (entries of key tiles that are not visible are
  *   left untouched).  d_qk must be 128 or 192; slow; for small S only.
@@ -126,8 +138,9 @@ attn_status_t attn_quantize_e4m3_static(const void* x_bf16, void* x_e4m3, float*
 attn_status_t attn_fwd_fp8_dump(const void* q, const void* k, const void* v, void* o, float* lse,
                                 int B, int Hq, int Hkv, int S, int d_qk, int d_v,
                                 const float* descale_q, const float* descale_k,
-                                const float* descale_v, int causal, float* dump_s,
-                                uint8_t* dump_codes, uint8_t* dump_kshift, void* stream);
+                                const float* descale_v, int causal, unsigned flags,
+                                float* dump_s, uint8_t* dump_codes, uint8_t* dump_kshift,
+                                void* stream);
 
 /*
  * Synchronises `stream` and reports (then clears) the device error word of the current

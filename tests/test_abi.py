@@ -52,6 +52,7 @@ def test_fwd_argument_validation(L):
     assert _fwd(L, B=-1) == pkg.ATTN_ERR_INVALID_ARG
     assert _fwd(L, causal=2) == pkg.ATTN_ERR_INVALID_ARG
     assert _fwd(L, flags=8) == pkg.ATTN_ERR_INVALID_ARG
+    assert _fwd(L, flags=pkg.ATTN_FLAG_EXACT_P) == pkg.ATTN_ERR_INVALID_ARG  # BF16 + exact P
     assert _fwd(L, dtype=7) == pkg.ATTN_ERR_INVALID_ARG
     assert _fwd(L, dqk=64) == pkg.ATTN_ERR_UNSUPPORTED
     assert _fwd(L, dv=192) == pkg.ATTN_ERR_UNSUPPORTED
