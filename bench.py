@@ -83,6 +83,52 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def gpu_selector(dev_index):
+    """The GPU as nvidia-smi / NVML name it: its UUID (they ignore CUDA_VISIBLE_DEVICES, so
+    a CUDA ordinal can name another GPU), else the ordinal."""
+    try:
+        import torch
+        u = str(torch.cuda.get_device_properties(dev_index).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(dev_index)
+
+
+# ----------------------------------------------------------------------------- energy
+def energy_summary(flops_per_call, calls, mj_start, mj_end, seconds):
+    """TFLOP/J and mean power from two readings of the NVML cumulative energy counter
+    (millijoules) around `calls` back-to-back launches of `flops_per_call` each."""
+    joules = (mj_end - mj_start) / 1000.0
+    if joules <= 0 or seconds <= 0:
+        return {"tflop_per_j": None, "joules": joules, "avg_w": None, "calls": calls,
+                "seconds": round(seconds, 3)}
+    return {"tflop_per_j": round(flops_per_call * calls / joules / 1e12, 4),
+            "joules": round(joules, 3), "avg_w": round(joules / seconds, 1), "calls": calls,
+            "seconds": round(seconds, 3)}
+
+
+def measure_energy(nvml, handle, fn, flops_per_call, sync, seconds=3.0):
+    """Run fn back to back for about `seconds` (after a warm-up of the same length, so that
+    clocks and power have settled) and read the energy counter around the measured window."""
+    t0 = time.perf_counter()
+    n = 0
+    while time.perf_counter() - t0 < seconds or n < 3:  # warm-up; also sizes the window
+        fn()
+        n += 1
+        if n % 8 == 0:
+            sync()
+    sync()
+    calls = max(3, int(n * seconds / max(time.perf_counter() - t0, 1e-6)))
+    e0 = nvml.nvmlDeviceGetTotalEnergyConsumption(handle)
+    t1 = time.perf_counter()
+    for _ in range(calls):
+        fn()
+    sync()
+    t2 = time.perf_counter()
+    e1 = nvml.nvmlDeviceGetTotalEnergyConsumption(handle)
+    return energy_summary(flops_per_call, calls, e0, e1, t2 - t1)
+
+
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled every 50 ms while active."""
@@ -214,7 +260,7 @@ def gpu_bench(args, rank, world, local_rank):
         return step_ms, kern_ms
 
     peaks, peak_src = load_peaks()
-    with ClockSampler(local_rank) as clk:
+    with ClockSampler(gpu_selector(local_rank)) as clk:
         fp8_step_ms, fp8_kern_ms = timed(fp8_step, args.steps, args.warmup)
         bf16_step_ms, bf16_kern_ms = timed(bf16_step, args.steps, args.warmup)
     clocks = clk.summary()
@@ -228,6 +274,28 @@ def gpu_bench(args, rank, world, local_rank):
         o_h.copy_(o, non_blocking=True)
 
     e2e_ms, _ = timed(e2e_step, max(3, args.steps // 4), max(1, args.warmup // 2))
+
+    # energy of the attention kernels at sustained clocks (NVML cumulative counter)
+    energy = None
+    if not args.no_energy:
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            sel = gpu_selector(local_rank)
+            handle = (pynvml.nvmlDeviceGetHandleByUUID(sel) if sel.startswith("GPU-")
+                      else pynvml.nvmlDeviceGetHandleByIndex(int(sel)))
+            sync = lambda: torch.cuda.synchronize(dev)
+            with ClockSampler(gpu_selector(local_rank)) as eclk:
+                e_fp8 = measure_energy(pynvml, handle, lambda: pkg.attn_fwd(
+                    q8, k8, v8, descale_q=ds[0], descale_k=ds[1], descale_v=ds[2], out=o, lse=lse,
+                    unrotate=args.hadamard, exact_p=args.exact_p), flops, sync)
+                e_bf16 = measure_energy(pynvml, handle, lambda: pkg.attn_fwd(q, k, v, out=o, lse=lse),
+                                        flops, sync)
+            energy = {"fp8": e_fp8, "bf16": e_bf16, "clocks": eclk.summary(),
+                      "source": "nvmlDeviceGetTotalEnergyConsumption around back-to-back "
+                                "attention launches (whole-board energy, this GPU)"}
+        except Exception as exc:  # NVML missing or not permitted: report why, keep the run
+            energy = {"unavailable": f"{type(exc).__name__}: {exc}"}
     h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h))
     d2h = o_h.numel() * o_h.element_size()
 
@@ -282,6 +350,8 @@ def gpu_bench(args, rank, world, local_rank):
         "gpu_launches": args.steps * 7 + args.steps,
         "clocks": clocks,
     }
+    if energy is not None:
+        result["energy"] = energy
     return result
 
 
@@ -396,6 +466,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="gqa16k_outlier", choices=sorted(WORKLOADS))
     ap.add_argument("--hadamard", action="store_true")
+    ap.add_argument("--no-energy", action="store_true",
+                    help="skip the NVML energy windows (about 12 s of extra GPU time)")
     ap.add_argument("--exact-p", action="store_true",
                     help="FP8 probabilities by exponential + e4m3 rounding (the ablation of lean P)")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])

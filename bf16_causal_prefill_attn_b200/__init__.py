@@ -47,6 +47,9 @@ def lib():
         L.attn_fwd.restype = i32
         L.attn_fwd_ex.argtypes = fwd_args + [u32, vp]
         L.attn_fwd_ex.restype = i32
+        L.attn_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, ctypes.c_int64, i32,
+                                      i32, i32, i32, i32, vp, vp, vp, i32, u32, vp]
+        L.attn_fwd_varlen.restype = i32
         L.attn_fwd_fp8_dump.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                         vp, vp, vp, i32, u32, vp, vp, vp, vp]
         L.attn_fwd_fp8_dump.restype = i32
@@ -121,6 +124,37 @@ def attn_fwd(q, k, v, causal=True, descale_q=None, descale_k=None, descale_v=Non
                            _ptr(descale_k), _ptr(descale_v), 1 if causal else 0, flags,
                            _stream(stream))
     _check(st, "attn_fwd")
+    return out, lse
+
+
+def attn_fwd_varlen(q, k, v, cu_seqlens, max_seqlen, causal=True, descale_q=None,
+                    descale_k=None, descale_v=None, out=None, lse=None, return_lse=True,
+                    unrotate=False, stream=None):
+    """Packed variable-length batch: q [T,Hq,d_qk], k/v [T,Hkv,d], cu_seqlens int32 [B+1] on
+    the GPU (sequence b = tokens cu_seqlens[b] .. cu_seqlens[b+1]-1).  Returns (o bf16
+    [T,Hq,d_v], lse fp32 [Hq,T] or None); tokens outside every sequence are left as
+    allocated."""
+    fp8 = q.dtype in (torch.uint8, torch.float8_e4m3fn)
+    q, k, v = (_codes(x) for x in (q, k, v)) if fp8 else (q, k, v)
+    for x in (q, k, v):
+        if not x.is_contiguous():
+            raise ValueError("q, k, v must be contiguous [T, H, d]")
+    if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_contiguous():
+        raise ValueError("cu_seqlens must be a contiguous int32 tensor")
+    T, Hq, d_qk = q.shape
+    Hkv = k.shape[1]
+    d_v = v.shape[2]
+    B = cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty((T, Hq, d_v), dtype=torch.bfloat16, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((Hq, T), dtype=torch.float32, device=q.device)
+    st = lib().attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(cu_seqlens),
+                               B, int(max_seqlen), T, Hq, Hkv, d_qk, d_v,
+                               ATTN_FP8_E4M3 if fp8 else ATTN_BF16, _ptr(descale_q),
+                               _ptr(descale_k), _ptr(descale_v), 1 if causal else 0,
+                               ATTN_FLAG_UNROTATE_O if unrotate else 0, _stream(stream))
+    _check(st, "attn_fwd_varlen")
     return out, lse
 
 

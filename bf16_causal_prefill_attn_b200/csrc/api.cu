@@ -61,19 +61,19 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esiz
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-template <bool FP8, int DQK, bool DUMP, bool EXACT = false>
+template <bool FP8, int DQK, bool DUMP, bool EXACT = false, bool VARLEN = false>
 attn_status_t launch_fwd(const void* q, const void* k, const void* v, attn::FwdParams& prm,
                          cudaStream_t stream) {
   using C = attn::FwdCfg<FP8, DQK>;
   const CUtensorMapDataType dt =
       FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  const uint64_t T = static_cast<uint64_t>(prm.B) * prm.S;
+  const uint64_t T = static_cast<uint64_t>(prm.total_tokens);
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, q, dt, C::E, DQK, prm.Hq, T, C::BOX_COLS) ||
       !make_map(&mk, k, dt, C::E, DQK, prm.Hkv, T, C::BOX_COLS) ||
       !make_map(&mv, v, dt, C::E, attn::DV, prm.Hkv, T, C::BOX_COLS))
     return ATTN_ERR_CUDA;
-  auto kern = attn::attn_fwd_kernel<FP8, DQK, DUMP, EXACT>;
+  auto kern = attn::attn_fwd_kernel<FP8, DQK, DUMP, EXACT, VARLEN>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC) !=
       cudaSuccess)
     return ATTN_ERR_CUDA;
@@ -90,61 +90,67 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, attn::FwdP
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                       int Hq, int Hkv, int S, int d_qk, int d_v, attn_dtype_t dtype,
-                       const float* dq, const float* dk, const float* dv, int causal,
-                       unsigned flags, float* dump_s, uint8_t* dump_codes,
-                       uint8_t* dump_kshift, bool dump, void* stream) {
-  if (B < 0 || S < 0 || Hq <= 0 || Hkv <= 0 || (Hq % Hkv) != 0) return ATTN_ERR_INVALID_ARG;
+// Checks shared by the fixed-length and packed entry points; fills the parameters that
+// do not depend on the sequence layout.
+attn_status_t common_args(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int Hq, int Hkv, int d_qk, int d_v, attn_dtype_t dtype,
+                          const float* dq, const float* dk, const float* dv, int causal,
+                          unsigned flags, attn::FwdParams* prm) {
+  if (Hq <= 0 || Hkv <= 0 || (Hq % Hkv) != 0) return ATTN_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
   if ((flags & ~static_cast<unsigned>(ATTN_FLAG_UNROTATE_O | ATTN_FLAG_EXACT_P)) != 0)
     return ATTN_ERR_INVALID_ARG;
   if (dtype != ATTN_BF16 && dtype != ATTN_FP8_E4M3) return ATTN_ERR_INVALID_ARG;
   if ((flags & ATTN_FLAG_EXACT_P) && dtype != ATTN_FP8_E4M3) return ATTN_ERR_INVALID_ARG;
   if ((d_qk != 128 && d_qk != 192) || d_v != 128) return ATTN_ERR_UNSUPPORTED;
-  if (B == 0 || S == 0) return ATTN_OK;
-  if (!q || !k || !v || !o) return ATTN_ERR_INVALID_ARG;
-  if (dtype == ATTN_FP8_E4M3 && (!dq || !dk || !dv)) return ATTN_ERR_INVALID_ARG;
-  if (dump && (dtype != ATTN_FP8_E4M3 || !dump_s || !dump_codes || !dump_kshift))
-    return ATTN_ERR_INVALID_ARG;
-  if (S % 128 != 0) return ATTN_ERR_UNSUPPORTED;
-  if (static_cast<int64_t>(B) * S > INT32_MAX ||
-      static_cast<int64_t>((S / 128 + 1) / 2) * B * Hq > INT32_MAX)
-    return ATTN_ERR_UNSUPPORTED;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_ALIGNMENT;
-  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATTN_ERR_ALIGNMENT;
-
-  attn::FwdParams prm{};
-  prm.B = B;
-  prm.S = S;
-  prm.Hq = Hq;
-  prm.Hkv = Hkv;
-  prm.G = Hq / Hkv;
-  prm.n_q_tiles = S / 128;
-  prm.n_pairs = (prm.n_q_tiles + 1) / 2;
-  prm.causal = causal;
-  prm.o = static_cast<__nv_bfloat16*>(o);
-  prm.lse = lse;
+  (void)q; (void)k; (void)v; (void)o; (void)lse;
+  prm->Hq = Hq;
+  prm->Hkv = Hkv;
+  prm->G = Hq / Hkv;
+  prm->causal = causal;
+  prm->o = static_cast<__nv_bfloat16*>(o);
+  prm->lse = lse;
   const double scale = 1.0 / std::sqrt(static_cast<double>(d_qk));
   const double log2e = 1.4426950408889634;
-  prm.c1 = static_cast<float>(scale * log2e);
-  prm.leanp_c = 8.0 * log2e * scale;
-  prm.descale_q = dq;
-  prm.descale_k = dk;
-  prm.descale_v = dv;
-  prm.unrotate = (flags & ATTN_FLAG_UNROTATE_O) ? 1 : 0;
-  prm.timeout_ns = g_timeout_ns;
-  prm.dump_s = dump_s;
-  prm.dump_codes = dump_codes;
-  prm.dump_kshift = dump_kshift;
-  if (!dev_err_ptr(&prm.err)) return ATTN_ERR_CUDA;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  prm->c1 = static_cast<float>(scale * log2e);
+  prm->leanp_c = 8.0 * log2e * scale;
+  prm->descale_q = dq;
+  prm->descale_k = dk;
+  prm->descale_v = dv;
+  prm->unrotate = (flags & ATTN_FLAG_UNROTATE_O) ? 1 : 0;
+  prm->timeout_ns = g_timeout_ns;
+  return ATTN_OK;
+}
 
+attn_status_t pointer_args(const void* q, const void* k, const void* v, void* o, float* lse,
+                           attn_dtype_t dtype, const float* dq, const float* dk,
+                           const float* dv) {
+  if (!q || !k || !v || !o) return ATTN_ERR_INVALID_ARG;
+  if (dtype == ATTN_FP8_E4M3 && (!dq || !dk || !dv)) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_ALIGNMENT;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATTN_ERR_ALIGNMENT;
+  return ATTN_OK;
+}
+
+attn_status_t dispatch(const void* q, const void* k, const void* v, int d_qk, attn_dtype_t dtype,
+                       unsigned flags, bool dump, bool varlen, attn::FwdParams& prm,
+                       cudaStream_t st) {
+  const bool exact = (flags & ATTN_FLAG_EXACT_P) != 0;
+  if (varlen) {
+    // sequences of any length: lean-P FP8 and BF16 (not the exact-P ablation, not the
+    // test-only dump)
+    if (exact || dump) return ATTN_ERR_UNSUPPORTED;
+    if (dtype == ATTN_BF16) {
+      if (d_qk == 128) return launch_fwd<false, 128, false, false, true>(q, k, v, prm, st);
+      return launch_fwd<false, 192, false, false, true>(q, k, v, prm, st);
+    }
+    if (d_qk == 128) return launch_fwd<true, 128, false, false, true>(q, k, v, prm, st);
+    return launch_fwd<true, 192, false, false, true>(q, k, v, prm, st);
+  }
   if (dtype == ATTN_BF16) {
     if (d_qk == 128) return launch_fwd<false, 128, false>(q, k, v, prm, st);
     return launch_fwd<false, 192, false>(q, k, v, prm, st);
   }
-  const bool exact = (flags & ATTN_FLAG_EXACT_P) != 0;
   if (dump) {
     if (exact) {
       if (d_qk == 128) return launch_fwd<true, 128, true, true>(q, k, v, prm, st);
@@ -159,6 +165,74 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, flo
   }
   if (d_qk == 128) return launch_fwd<true, 128, false>(q, k, v, prm, st);
   return launch_fwd<true, 192, false>(q, k, v, prm, st);
+}
+
+attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                       int Hq, int Hkv, int S, int d_qk, int d_v, attn_dtype_t dtype,
+                       const float* dq, const float* dk, const float* dv, int causal,
+                       unsigned flags, float* dump_s, uint8_t* dump_codes,
+                       uint8_t* dump_kshift, bool dump, void* stream) {
+  attn::FwdParams prm{};
+  if (B < 0 || S < 0) return ATTN_ERR_INVALID_ARG;
+  attn_status_t e = common_args(q, k, v, o, lse, Hq, Hkv, d_qk, d_v, dtype, dq, dk, dv, causal,
+                                flags, &prm);
+  if (e != ATTN_OK) return e;
+  if (B == 0 || S == 0) return ATTN_OK;
+  if (dump && (dtype != ATTN_FP8_E4M3 || !dump_s || !dump_codes || !dump_kshift))
+    return ATTN_ERR_INVALID_ARG;
+  // the tail-masking variant covers lean-P FP8 and BF16 only
+  if ((S % 128) != 0 && (dump || (flags & ATTN_FLAG_EXACT_P))) return ATTN_ERR_UNSUPPORTED;
+  const int n_q_tiles = (S + 127) / 128;
+  if (static_cast<int64_t>(B) * S > INT32_MAX ||
+      static_cast<int64_t>((n_q_tiles + 1) / 2) * B * Hq > INT32_MAX)
+    return ATTN_ERR_UNSUPPORTED;
+  e = pointer_args(q, k, v, o, lse, dtype, dq, dk, dv);
+  if (e != ATTN_OK) return e;
+  prm.B = B;
+  prm.S = S;
+  prm.n_q_tiles = n_q_tiles;
+  prm.n_pairs = (n_q_tiles + 1) / 2;
+  prm.cu_seqlens = nullptr;
+  prm.max_seqlen = S;
+  prm.total_tokens = static_cast<int64_t>(B) * S;
+  prm.dump_s = dump_s;
+  prm.dump_codes = dump_codes;
+  prm.dump_kshift = dump_kshift;
+  if (!dev_err_ptr(&prm.err)) return ATTN_ERR_CUDA;
+  // S not a multiple of 128: the kernel variant that masks the tail of each sequence
+  return dispatch(q, k, v, d_qk, dtype, flags, dump, (S % 128) != 0, prm,
+                  static_cast<cudaStream_t>(stream));
+}
+
+attn_status_t varlen_impl(const void* q, const void* k, const void* v, void* o, float* lse,
+                          const int32_t* cu_seqlens, int B, int max_seqlen,
+                          int64_t total_tokens, int Hq, int Hkv, int d_qk, int d_v,
+                          attn_dtype_t dtype, const float* dq, const float* dk,
+                          const float* dv, int causal, unsigned flags, void* stream) {
+  attn::FwdParams prm{};
+  if (B < 0 || max_seqlen < 0 || total_tokens < 0) return ATTN_ERR_INVALID_ARG;
+  attn_status_t e = common_args(q, k, v, o, lse, Hq, Hkv, d_qk, d_v, dtype, dq, dk, dv, causal,
+                                flags, &prm);
+  if (e != ATTN_OK) return e;
+  if (B == 0 || max_seqlen == 0 || total_tokens == 0) return ATTN_OK;
+  if (flags & ATTN_FLAG_EXACT_P) return ATTN_ERR_UNSUPPORTED;
+  if (!cu_seqlens) return ATTN_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) return ATTN_ERR_ALIGNMENT;
+  const int n_q_tiles = (max_seqlen + 127) / 128;
+  if (total_tokens > INT32_MAX || max_seqlen > total_tokens ||
+      static_cast<int64_t>((n_q_tiles + 1) / 2) * B * Hq > INT32_MAX)
+    return ATTN_ERR_UNSUPPORTED;
+  e = pointer_args(q, k, v, o, lse, dtype, dq, dk, dv);
+  if (e != ATTN_OK) return e;
+  prm.B = B;
+  prm.S = 0;  // unused with cu_seqlens
+  prm.n_q_tiles = n_q_tiles;
+  prm.n_pairs = (n_q_tiles + 1) / 2;
+  prm.cu_seqlens = cu_seqlens;
+  prm.max_seqlen = max_seqlen;
+  prm.total_tokens = total_tokens;
+  if (!dev_err_ptr(&prm.err)) return ATTN_ERR_CUDA;
+  return dispatch(q, k, v, d_qk, dtype, flags, false, true, prm, static_cast<cudaStream_t>(stream));
 }
 
 // A wait that nothing ever satisfies: one thread waits (bounded) on an mbarrier no one
@@ -195,6 +269,15 @@ attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v, void* o, 
                           const float* descale_v, int causal, unsigned flags, void* stream) {
   return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, S, d_qk, d_v, dtype, descale_q, descale_k,
                   descale_v, causal, flags, nullptr, nullptr, nullptr, false, stream);
+}
+
+attn_status_t attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                              const int32_t* cu_seqlens, int B, int max_seqlen,
+                              int64_t total_tokens, int Hq, int Hkv, int d_qk, int d_v,
+                              attn_dtype_t dtype, const float* descale_q, const float* descale_k,
+                              const float* descale_v, int causal, unsigned flags, void* stream) {
+  return varlen_impl(q, k, v, o, lse, cu_seqlens, B, max_seqlen, total_tokens, Hq, Hkv, d_qk,
+                     d_v, dtype, descale_q, descale_k, descale_v, causal, flags, stream);
 }
 
 attn_status_t attn_fwd_fp8_dump(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -265,7 +348,7 @@ attn_status_t attn_device_status(void* stream) {
   if (host != attn::DEV_OK) {
     const uint32_t zero = 0;
     if (cudaMemcpyToSymbol(g_dev_err, &zero, sizeof(zero)) != cudaSuccess) return ATTN_ERR_CUDA;
-    return ATTN_ERR_TIMEOUT;
+    return host == attn::DEV_BAD_SEQLENS ? ATTN_ERR_INVALID_ARG : ATTN_ERR_TIMEOUT;
   }
   return ATTN_OK;
 }

@@ -90,8 +90,14 @@ constexpr float EXP2_C3 = 0.05517097562551498f;
 
 struct FwdParams {
   int B, S, Hq, Hkv, G;
-  int n_q_tiles, n_pairs;
+  int n_q_tiles, n_pairs;  // VARLEN: of the longest sequence (max_seqlen)
   int causal;
+  // VARLEN: sequence b is tokens [cu_seqlens[b], cu_seqlens[b+1]) of the packed tensors
+  // (null: every sequence has S tokens, sequence b starting at token b S), at most
+  // max_seqlen long; total_tokens bounds every token index written
+  const int* cu_seqlens;
+  int max_seqlen;
+  int64_t total_tokens;
   __nv_bfloat16* o;   // [B, S, Hq, DV]
   float* lse;         // [B, Hq, S] or null
   float c1;           // BF16: scale * log2(e)
@@ -172,7 +178,9 @@ __device__ __forceinline__ float exp2_poly(float x) {
 // MUFU exponential and the hardware e4m3 conversion, instead of the lean-P multiply-add and
 // integer conversion; everything else (reference max, block shifts, block-scaled PV, row
 // sum) is shared.
-template <bool FP8, int DQK, bool DUMP, bool EXACT = false>
+// VARLEN: sequences of any length (packed, or a fixed S not a multiple of 128): keys past
+// the end of the sequence are masked, rows past it are not written.
+template <bool FP8, int DQK, bool DUMP, bool EXACT = false, bool VARLEN = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
@@ -206,12 +214,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int b = bh / p.Hq;
   const int h = bh % p.Hq;
   const int g = h / p.G;
+  int tok0 = b * p.S;       // first token of this sequence
+  int seq_len = p.S;        // its length
+  int n_q_tiles = p.n_q_tiles;
+  if constexpr (VARLEN) {
+    if (p.cu_seqlens != nullptr) {
+      const int c0 = p.cu_seqlens[b], c1 = p.cu_seqlens[b + 1];
+      if (c0 < 0 || c1 < c0 || static_cast<int64_t>(c1) > p.total_tokens ||
+          c1 - c0 > p.max_seqlen) {
+        if (threadIdx.x == 0) atomicCAS(p.err, DEV_OK, DEV_BAD_SEQLENS);
+        return;  // the whole CTA, before any barrier or allocation
+      }
+      tok0 = c0;
+      seq_len = c1 - c0;
+    }
+    n_q_tiles = (seq_len + BLOCK_M - 1) / BLOCK_M;
+    if (2 * pr >= n_q_tiles) return;  // this sequence has fewer query-tile pairs
+  }
   const int qt0 = 2 * pr;                               // query tile of t = 0
-  const bool has1 = qt0 + 1 < p.n_q_tiles;              // t = 1 exists
-  const int n_t0 = p.causal ? qt0 + 1 : p.n_q_tiles;     // key tiles of each query tile
-  const int n_t1 = has1 ? (p.causal ? qt0 + 2 : p.n_q_tiles) : 0;
+  const bool has1 = qt0 + 1 < n_q_tiles;                // t = 1 exists
+  const int n_t0 = p.causal ? qt0 + 1 : n_q_tiles;      // key tiles of each query tile
+  const int n_t1 = has1 ? (p.causal ? qt0 + 2 : n_q_tiles) : 0;
   const int n_max = n_t1 > n_t0 ? n_t1 : n_t0;
-  const int tok0 = b * p.S;  // first token of this batch entry
 
   if (tid == 0) {
     mbar_init(q_full, 1);
@@ -492,6 +516,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int c = 0; c < BLOCK_N; ++c)
           if (c > r) s[c] = -INFINITY;
       }
+      if constexpr (VARLEN) {
+        // keys past the end of the sequence (the next sequence's, or zero fill)
+        const int kvalid = seq_len - j * BLOCK_N;
+        if (kvalid < BLOCK_N) {
+#pragma unroll
+          for (int c = 0; c < BLOCK_N; ++c)
+            if (c >= kvalid) s[c] = -INFINITY;
+        }
+      }
       // block maxima with two independent chains per 64-key block
       float mx[4];
 #pragma unroll
@@ -672,6 +705,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         inv *= 0.08838834764831845f;
       }
+      // VARLEN: rows past the end of the sequence hold another sequence's queries (or zero
+      // fill) and are not written
+      const bool row_in = !VARLEN || q_pos < seq_len;
       __nv_bfloat16* orow = p.o + ((static_cast<size_t>(tok0) + q_pos) * p.Hq + h) * DV;
 #pragma unroll
       for (int c = 0; c < DV; c += 8) {
@@ -680,15 +716,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         v.y = pack_bf16x2(o[c + 2] * inv, o[c + 3] * inv);
         v.z = pack_bf16x2(o[c + 4] * inv, o[c + 5] * inv);
         v.w = pack_bf16x2(o[c + 6] * inv, o[c + 7] * inv);
-        *reinterpret_cast<uint4*>(orow + c) = v;
+        if (row_in) *reinterpret_cast<uint4*>(orow + c) = v;
       }
-      if (p.lse != nullptr) {
+      if (p.lse != nullptr && row_in) {
         float lse_v;
         if constexpr (FP8)
           lse_v = 0.69314718055994531f * (static_cast<float>(m_i) * 0.125f + __log2f(l));
         else
           lse_v = 0.69314718055994531f * (ms + __log2f(l));
-        p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.S + q_pos] = lse_v;
+        // lse [B, Hq, S], or [Hq, total tokens] for packed sequences
+        const size_t li = (VARLEN && p.cu_seqlens != nullptr)
+                              ? static_cast<size_t>(h) * p.total_tokens + tok0 + q_pos
+                              : (static_cast<size_t>(b) * p.Hq + h) * p.S + q_pos;
+        p.lse[li] = lse_v;
       }
     }
   }

@@ -16,6 +16,7 @@ namespace attn {
 enum : uint32_t {
   DEV_OK = 0,
   DEV_TIMEOUT = 1,
+  DEV_BAD_SEQLENS = 2,  // cu_seqlens not non-decreasing within [0, total tokens]
 };
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {

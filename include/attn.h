@@ -40,7 +40,8 @@ extern "C" {
 typedef enum attn_status {
   ATTN_OK = 0,
   ATTN_ERR_INVALID_ARG = 1, /* null pointer, negative size, Hq % Hkv != 0, bad flag */
-  ATTN_ERR_UNSUPPORTED = 2, /* head dims other than 128/192 (qk) and 128 (v); S % 128 != 0 */
+  ATTN_ERR_UNSUPPORTED = 2, /* head dims other than 128/192 (qk) and 128 (v); a flag or
+                               the dump combined with sequences not a multiple of 128 */
   ATTN_ERR_ALIGNMENT = 3,   /* a tensor pointer not 16-byte aligned */
   ATTN_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed */
   ATTN_ERR_TIMEOUT = 5      /* a device-side bounded wait expired (see attn_device_status) */
@@ -74,8 +75,10 @@ typedef enum attn_dtype { ATTN_BF16 = 0, ATTN_FP8_E4M3 = 1 } attn_dtype_t;
  *   descale_q/k/v  DEVICE pointers to one fp32 each (x = code * descale), as written by
  *             attn_quantize_e4m3; required for FP8, ignored (may be NULL) for BF16
  *   causal    1 = causal mask (the contract), 0 = full attention
- * Requirements: S % 128 == 0, Hq % Hkv == 0, pointers 16-byte aligned.
- * B == 0 or S == 0 is a no-op.
+ * Requirements: Hq % Hkv == 0, pointers 16-byte aligned.  Any S >= 0: when S % 128 != 0
+ * the kernel variant that masks the keys past the end of each sequence and does not write
+ * the rows past it runs (then ATTN_FLAG_EXACT_P is not supported).  B == 0 or S == 0 is a
+ * no-op.
  */
 attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                        int Hq, int Hkv, int S, int d_qk, int d_v, attn_dtype_t dtype,
@@ -87,6 +90,29 @@ attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v, void* o, 
                           int B, int Hq, int Hkv, int S, int d_qk, int d_v, attn_dtype_t dtype,
                           const float* descale_q, const float* descale_k,
                           const float* descale_v, int causal, unsigned flags, void* stream);
+
+/*
+ * attn_fwd_varlen: attn_fwd over a batch of sequences of different lengths packed along
+ * the token axis (variable-length batches, which [ZYFA-fr] "Ce que couvrent les noyaux"
+ * lists as not yet supported by the pages' kernels).
+ *   q [T, Hq, d_qk], k [T, Hkv, d_qk], v [T, Hkv, d_v], o [T, Hq, d_v] (T = total_tokens),
+ *   same types and head rules as attn_fwd; lse [Hq, T] fp32 or NULL.
+ *   cu_seqlens  DEVICE int32 [B + 1]: sequence b is tokens [cu_seqlens[b], cu_seqlens[b+1]);
+ *               non-decreasing, cu_seqlens[0] >= 0, cu_seqlens[B] <= T, each length at
+ *               most max_seqlen.  Read by the kernel (no host synchronisation): a sequence
+ *               that breaks these rules is skipped (its outputs are not written) and
+ *               attn_device_status() then reports ATTN_ERR_INVALID_ARG.
+ *   max_seqlen  the longest sequence (sizes the grid), <= T.
+ *   causal      1: key j of a sequence is visible from its query i iff j <= i.
+ *   flags       ATTN_FLAG_UNROTATE_O only (ATTN_FLAG_EXACT_P: ATTN_ERR_UNSUPPORTED).
+ * Tokens not covered by any sequence are not written.  B == 0, max_seqlen == 0 or T == 0 is
+ * a no-op.  Requirements: pointers 16-byte aligned (cu_seqlens 4-byte), T <= 2^31 - 1.
+ */
+attn_status_t attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                              const int32_t* cu_seqlens, int B, int max_seqlen,
+                              int64_t total_tokens, int Hq, int Hkv, int d_qk, int d_v,
+                              attn_dtype_t dtype, const float* descale_q, const float* descale_k,
+                              const float* descale_v, int causal, unsigned flags, void* stream);
 
 /*
  * attn_quantize_e4m3: per-tensor e4m3 quantisation of a bf16 tensor [tokens, H, d]

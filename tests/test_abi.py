@@ -56,7 +56,8 @@ def test_fwd_argument_validation(L):
     assert _fwd(L, dtype=7) == pkg.ATTN_ERR_INVALID_ARG
     assert _fwd(L, dqk=64) == pkg.ATTN_ERR_UNSUPPORTED
     assert _fwd(L, dv=192) == pkg.ATTN_ERR_UNSUPPORTED
-    assert _fwd(L, S=100) == pkg.ATTN_ERR_UNSUPPORTED
+    # S % 128 != 0 runs the tail-masking variant, which has no exact-P form
+    assert _fwd(L, S=100, dtype=1, ds=(1, 1, 1), flags=pkg.ATTN_FLAG_EXACT_P) == pkg.ATTN_ERR_UNSUPPORTED
     assert _fwd(L, q=0) == pkg.ATTN_ERR_INVALID_ARG
     assert _fwd(L, o=0) == pkg.ATTN_ERR_INVALID_ARG
     assert _fwd(L, dtype=1) == pkg.ATTN_ERR_INVALID_ARG      # FP8 without descales
@@ -90,3 +91,29 @@ def test_binding_raises_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(pkg, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="not built"):
         pkg.lib()
+
+
+def _varlen(L, q=1, k=1, v=1, o=1, cu=1, B=2, max_s=100, T=150, Hq=2, Hkv=1, dtype=0,
+            causal=1, flags=0, cu_off=0):
+    vp = ctypes.c_void_p
+    p = lambda x: vp(x * 256) if x else None  # fake, aligned, never dereferenced
+    cu_p = vp(cu * 256 + cu_off) if cu else None
+    return L.attn_fwd_varlen(p(q), p(k), p(v), p(o), None, cu_p, B, max_s, T, Hq, Hkv, 128, 128,
+                             dtype, None, None, None, causal, flags, None)
+
+
+def test_varlen_argument_validation(L):
+    assert _varlen(L, B=-1) == pkg.ATTN_ERR_INVALID_ARG
+    assert _varlen(L, max_s=-1) == pkg.ATTN_ERR_INVALID_ARG
+    assert _varlen(L, Hq=3, Hkv=2) == pkg.ATTN_ERR_INVALID_ARG
+    assert _varlen(L, cu=0) == pkg.ATTN_ERR_INVALID_ARG
+    assert _varlen(L, q=0) == pkg.ATTN_ERR_INVALID_ARG
+    assert _varlen(L, cu_off=2) == pkg.ATTN_ERR_ALIGNMENT
+    assert _varlen(L, max_s=200, T=150) == pkg.ATTN_ERR_UNSUPPORTED   # longer than the tensor
+    assert _varlen(L, T=2 ** 31) == pkg.ATTN_ERR_UNSUPPORTED
+    assert _varlen(L, dtype=1, flags=pkg.ATTN_FLAG_EXACT_P) == pkg.ATTN_ERR_UNSUPPORTED
+    assert _varlen(L, flags=4) == pkg.ATTN_ERR_INVALID_ARG
+    # empty problems are no-ops that never touch the device
+    assert _varlen(L, B=0, q=0, k=0, v=0, o=0, cu=0) == pkg.ATTN_OK
+    assert _varlen(L, T=0, max_s=0, q=0, k=0, v=0, o=0, cu=0) == pkg.ATTN_OK
+

@@ -59,3 +59,29 @@ def test_reference_arm_prints_one_line():
     assert d["impl"] == "reference" and d["unit"] == "TFLOP/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+class _FakeNVML:
+    """Stands in for pynvml: a cumulative energy counter (millijoules) that grows by a fixed
+    amount per reading."""
+
+    def __init__(self, step_mj):
+        self.mj = 1_000_000
+        self.step = step_mj
+
+    def nvmlDeviceGetTotalEnergyConsumption(self, handle):
+        self.mj += self.step
+        return self.mj
+
+
+def test_energy_summary_and_window_with_fake_nvml():
+    e = bench.energy_summary(1e12, 10, 5000, 7000, 0.5)    # 2 J for 10 TFLOP
+    assert e["tflop_per_j"] == 5.0 and e["avg_w"] == 4.0 and e["joules"] == 2.0
+    assert bench.energy_summary(1e12, 10, 7000, 7000, 0.5)["tflop_per_j"] is None
+    calls = []
+    nv = _FakeNVML(step_mj=250)
+    r = bench.measure_energy(nv, None, lambda: calls.append(1), 2e11, lambda: None, seconds=0.05)
+    # one counter step between the two readings: 0.25 J for r["calls"] launches
+    assert r["joules"] == 0.25 and r["calls"] >= 3
+    assert abs(r["tflop_per_j"] - 2e11 * r["calls"] / 0.25 / 1e12) < 1e-3
+    assert len(calls) > r["calls"]   # the warm-up ran first
