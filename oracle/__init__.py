@@ -20,7 +20,9 @@ Modules
   e4m3       OCP e4m3fn codec (decode, round-to-nearest-even saturating encode)
   hadamard   Sylvester-Hadamard rotation along the head dimension
   quantize   per-tensor e4m3 quantisation (+ optional rotation)
-  leanp      bit-level lean-P / power-of-two block-scale emulator (plain C, via ctypes)
+  leanp      bit-level lean-P / power-of-two block-scale emulator (plain C, via ctypes),
+             and the exact-P ablation (exponential then e4m3 rounding)
+  decode     fp64 decode attention over a paged KV cache (one query token per sequence)
 
 Pins (what each function is checked against, in ``tests/test_oracle_*.py``):
   attention  brute force on tiny inputs, 2x2 hand-computed case, Q=0 prefix mean,
@@ -32,5 +34,9 @@ Pins (what each function is checked against, in ``tests/test_oracle_*.py``):
   quantize   codes and descale recomputed from the e4m3 value table by brute force.
   leanp      closed forms (s = max gives byte 8*(7+k)), Mitchell error bound,
              monotonicity, exact fma against rational arithmetic, and the end-to-end
-             tile driver against fp64 attention within the FP8 tolerance.
+             tile driver against fp64 attention within the FP8 tolerance; exact P:
+             power-of-two closed forms, e4m3 rounding bound, driver pinned to the C one.
+  decode     equals the last row of the (pinned) prefill oracle on the gathered
+             sequence, page-permutation invariance, length 1 gives v_0, Q = 0 gives the
+             mean of V, an empty sequence gives zeros.
 """
