@@ -50,6 +50,12 @@ def lib():
         L.attn_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, ctypes.c_int64, i32,
                                       i32, i32, i32, i32, vp, vp, vp, i32, u32, vp]
         L.attn_fwd_varlen.restype = i32
+        L.attn_decode_paged.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
+                                        i32, i32, i32, i32, i32, vp, vp, vp, vp, ctypes.c_size_t,
+                                        vp]
+        L.attn_decode_paged.restype = i32
+        L.attn_decode_workspace_size.argtypes = [i32, i32, i32, i32]
+        L.attn_decode_workspace_size.restype = ctypes.c_size_t
         L.attn_fwd_fp8_dump.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                         vp, vp, vp, i32, u32, vp, vp, vp, vp]
         L.attn_fwd_fp8_dump.restype = i32
@@ -155,6 +161,43 @@ def attn_fwd_varlen(q, k, v, cu_seqlens, max_seqlen, causal=True, descale_q=None
                                _ptr(descale_k), _ptr(descale_v), 1 if causal else 0,
                                ATTN_FLAG_UNROTATE_O if unrotate else 0, _stream(stream))
     _check(st, "attn_fwd_varlen")
+    return out, lse
+
+
+def attn_decode_workspace_size(B, Hq, Hkv, max_seqlen):
+    return lib().attn_decode_workspace_size(int(B), int(Hq), int(Hkv), int(max_seqlen))
+
+
+def attn_decode_paged(q, k_cache, v_cache, block_table, seq_lens, max_seqlen, descale_q=None,
+                      descale_k=None, descale_v=None, out=None, lse=None, return_lse=True,
+                      workspace=None, stream=None):
+    """Decode over a paged cache: q [B,Hq,128], caches [P,page,Hkv,128] (bf16, or e4m3 codes
+    with fp32 descale tensors), block_table int32 [B,max_blocks], seq_lens int32 [B], all on
+    the GPU.  Returns (o bf16 [B,Hq,128], lse fp32 [B,Hq] or None)."""
+    fp8 = q.dtype in (torch.uint8, torch.float8_e4m3fn)
+    q, k_cache, v_cache = ((_codes(x) for x in (q, k_cache, v_cache)) if fp8
+                           else (q, k_cache, v_cache))
+    for x in (q, k_cache, v_cache, block_table, seq_lens):
+        if not x.is_contiguous():
+            raise ValueError("all tensors must be contiguous")
+    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise ValueError("block_table and seq_lens must be int32")
+    B, Hq, d = q.shape
+    P, page, Hkv, _ = k_cache.shape
+    if out is None:
+        out = torch.empty((B, Hq, v_cache.shape[3]), dtype=torch.bfloat16, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    ws_bytes = attn_decode_workspace_size(B, Hq, Hkv, max(int(max_seqlen), 1))
+    if workspace is None:
+        workspace = torch.empty((ws_bytes + 15) // 16 * 4, dtype=torch.float32, device=q.device)
+    st = lib().attn_decode_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse),
+                                 _ptr(block_table), _ptr(seq_lens), B, Hq, Hkv, d,
+                                 v_cache.shape[3], P, page, block_table.shape[1], int(max_seqlen),
+                                 ATTN_FP8_E4M3 if fp8 else ATTN_BF16, _ptr(descale_q),
+                                 _ptr(descale_k), _ptr(descale_v), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "attn_decode_paged")
     return out, lse
 
 

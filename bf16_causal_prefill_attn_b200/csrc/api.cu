@@ -11,6 +11,7 @@
 
 #include "../../include/attn.h"
 #include "attn_fwd.cuh"
+#include "decode.cuh"
 #include "quantize.cuh"
 
 namespace {
@@ -235,6 +236,32 @@ attn_status_t varlen_impl(const void* q, const void* k, const void* v, void* o, 
   return dispatch(q, k, v, d_qk, dtype, flags, false, true, prm, static_cast<cudaStream_t>(stream));
 }
 
+template <bool FP8, int G>
+attn_status_t launch_decode(attn::DecodeParams& prm, cudaStream_t st) {
+  auto k1 = attn::decode_split_kernel<FP8, G>;
+  constexpr int smem = attn::dec_smem_bytes<FP8, G>();
+  if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  const dim3 grid(static_cast<unsigned>(prm.n_splits), static_cast<unsigned>(prm.Hkv),
+                  static_cast<unsigned>(prm.B));
+  k1<<<grid, attn::DEC_THREADS, smem, st>>>(prm);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  attn::decode_combine_kernel<FP8><<<static_cast<unsigned>(prm.B) * prm.Hq, attn::DEC_D, 0, st>>>(prm);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <bool FP8>
+attn_status_t dispatch_decode(attn::DecodeParams& prm, cudaStream_t st) {
+  switch (prm.G) {
+    case 1: return launch_decode<FP8, 1>(prm, st);
+    case 2: return launch_decode<FP8, 2>(prm, st);
+    case 4: return launch_decode<FP8, 4>(prm, st);
+    case 8: return launch_decode<FP8, 8>(prm, st);
+    case 16: return launch_decode<FP8, 16>(prm, st);
+    default: return ATTN_ERR_UNSUPPORTED;
+  }
+}
+
 // A wait that nothing ever satisfies: one thread waits (bounded) on an mbarrier no one
 // arrives at, records DEV_TIMEOUT and returns.
 __global__ void selftest_wait_kernel(uint32_t* err, uint64_t timeout_ns) {
@@ -278,6 +305,79 @@ attn_status_t attn_fwd_varlen(const void* q, const void* k, const void* v, void*
                               const float* descale_v, int causal, unsigned flags, void* stream) {
   return varlen_impl(q, k, v, o, lse, cu_seqlens, B, max_seqlen, total_tokens, Hq, Hkv, d_qk,
                      d_v, dtype, descale_q, descale_k, descale_v, causal, flags, stream);
+}
+
+size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int max_seqlen) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || max_seqlen <= 0) return 0;
+  const int ns = attn::dec_n_splits(B, Hkv, max_seqlen);
+  return static_cast<size_t>(B) * Hq * ns * (attn::DEC_D + 2) * sizeof(float);
+}
+
+attn_status_t attn_decode_paged(const void* q, const void* k_cache, const void* v_cache, void* o,
+                                float* lse, const int32_t* block_table, const int32_t* seq_lens,
+                                int B, int Hq, int Hkv, int d_qk, int d_v, int num_pages,
+                                int page_size, int max_blocks_per_seq, int max_seqlen,
+                                attn_dtype_t dtype, const float* descale_q,
+                                const float* descale_k, const float* descale_v, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || (Hq % Hkv) != 0 || max_seqlen < 0 || num_pages < 0 ||
+      max_blocks_per_seq < 0 || page_size <= 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (dtype != ATTN_BF16 && dtype != ATTN_FP8_E4M3) return ATTN_ERR_INVALID_ARG;
+  if ((page_size & (page_size - 1)) != 0 || page_size > 65536) return ATTN_ERR_UNSUPPORTED;
+  const int G = Hq / Hkv;
+  if (d_qk != 128 || d_v != 128 || (G != 1 && G != 2 && G != 4 && G != 8 && G != 16))
+    return ATTN_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(max_blocks_per_seq) * page_size > INT32_MAX || B > 65535 ||
+      Hkv > 65535)
+    return ATTN_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(max_seqlen) > static_cast<int64_t>(max_blocks_per_seq) * page_size)
+    return ATTN_ERR_INVALID_ARG;
+  if (B == 0) return ATTN_OK;
+  if (!q || !o || !seq_lens) return ATTN_ERR_INVALID_ARG;
+  if (dtype == ATTN_FP8_E4M3 && (!descale_q || !descale_k || !descale_v))
+    return ATTN_ERR_INVALID_ARG;
+  if (!workspace) return ATTN_ERR_INVALID_ARG;  // the partial results always go there
+  if (max_seqlen > 0 && (!k_cache || !v_cache || !block_table || num_pages == 0 ||
+                         max_blocks_per_seq == 0))
+    return ATTN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(q) & 1u) || (reinterpret_cast<uintptr_t>(o) & 1u) ||
+      (reinterpret_cast<uintptr_t>(seq_lens) & 3u) ||
+      (reinterpret_cast<uintptr_t>(block_table) & 3u) || !aligned16(k_cache) ||
+      !aligned16(v_cache) || !aligned16(workspace) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return ATTN_ERR_ALIGNMENT;
+  const int msl = max_seqlen > 0 ? max_seqlen : 1;
+  if (workspace_bytes < attn_decode_workspace_size(B, Hq, Hkv, msl)) return ATTN_ERR_INVALID_ARG;
+  attn::DecodeParams prm{};
+  prm.q = q;
+  prm.k_cache = static_cast<const uint8_t*>(k_cache);
+  prm.v_cache = static_cast<const uint8_t*>(v_cache);
+  prm.block_table = block_table;
+  prm.seq_lens = seq_lens;
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.G = G;
+  prm.num_pages = num_pages;
+  int shift = 0;
+  while ((1 << shift) < page_size) ++shift;
+  prm.page_shift = shift;
+  prm.max_blocks = max_blocks_per_seq;
+  prm.max_seqlen = max_seqlen;
+  prm.n_splits = attn::dec_n_splits(B, Hkv, msl);
+  prm.split_tokens = attn::dec_split_tokens(msl, prm.n_splits);
+  prm.qk_scale = static_cast<float>((1.0 / std::sqrt(128.0)) * 1.4426950408889634);
+  prm.descale_q = descale_q;
+  prm.descale_k = descale_k;
+  prm.descale_v = descale_v;
+  prm.part_o = static_cast<float*>(workspace);
+  prm.part_ml = prm.part_o + static_cast<size_t>(B) * Hq * prm.n_splits * attn::DEC_D;
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.lse = lse;
+  if (!dev_err_ptr(&prm.err)) return ATTN_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return dtype == ATTN_FP8_E4M3 ? dispatch_decode<true>(prm, st) : dispatch_decode<false>(prm, st);
 }
 
 attn_status_t attn_fwd_fp8_dump(const void* q, const void* k, const void* v, void* o, float* lse,

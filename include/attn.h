@@ -115,6 +115,39 @@ attn_status_t attn_fwd_varlen(const void* q, const void* k, const void* v, void*
                               const float* descale_v, int causal, unsigned flags, void* stream);
 
 /*
+ * attn_decode_paged: decode attention over a paged KV cache -- one new query token per
+ * sequence against every cached token of its sequence, the cache holding the token itself
+ * (decode and paged KV caches are listed as not yet supported by the pages' kernels,
+ * [ZYFA-fr] "Ce que couvrent les noyaux").
+ *   q          [B, Hq, 128]  bf16, or e4m3 codes (ATTN_FP8_E4M3) with descale_q
+ *   k_cache    [num_pages, page_size, Hkv, 128]  same type as q (FP8: descale_k)
+ *   v_cache    [num_pages, page_size, Hkv, 128]  same type (FP8: descale_v)
+ *   o          [B, Hq, 128] bf16;  lse [B, Hq] fp32 natural log, or NULL
+ *   block_table DEVICE int32 [B, max_blocks_per_seq]: token j of sequence b is slot
+ *              j % page_size of page block_table[b][j / page_size]
+ *   seq_lens   DEVICE int32 [B]: cached tokens of each sequence, <= max_seqlen
+ *   max_seqlen the longest sequence (sizes the split of the work), <= max_blocks_per_seq *
+ *              page_size
+ *   workspace  DEVICE scratch of at least attn_decode_workspace_size(B, Hq, Hkv, max_seqlen)
+ *              bytes (16-byte aligned), owned by the caller; not shared by concurrent calls
+ * o = softmax(q K^T / sqrt(128)) V over the sequence's tokens; query head h reads kv head
+ * h / (Hq / Hkv).  A sequence of length 0 gives o = 0, lse = -inf.  Lengths and page ids
+ * are read on the device: a length above max_seqlen or a page id outside [0, num_pages)
+ * skips that (sequence, kv head) range and attn_device_status() reports
+ * ATTN_ERR_INVALID_ARG; nothing outside the cache is read.  Computed in fp32.
+ * Requirements: d_qk = d_v = 128; Hq / Hkv in {1, 2, 4, 8, 16}; page_size a power of two
+ * <= 65536; caches and workspace 16-byte aligned.  B == 0 is a no-op.
+ */
+attn_status_t attn_decode_paged(const void* q, const void* k_cache, const void* v_cache, void* o,
+                                float* lse, const int32_t* block_table, const int32_t* seq_lens,
+                                int B, int Hq, int Hkv, int d_qk, int d_v, int num_pages,
+                                int page_size, int max_blocks_per_seq, int max_seqlen,
+                                attn_dtype_t dtype, const float* descale_q,
+                                const float* descale_k, const float* descale_v, void* workspace,
+                                size_t workspace_bytes, void* stream);
+size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int max_seqlen);
+
+/*
  * attn_quantize_e4m3: per-tensor e4m3 quantisation of a bf16 tensor [tokens, H, d]
  * ([ZYFA-mb], "Precisão, estabilidade e efeito na prática").
  *   y = x, or with hadamard = 1, y = (x H_128) * float32(1/sqrt(128)) along d (d must be

@@ -117,3 +117,32 @@ def test_varlen_argument_validation(L):
     assert _varlen(L, B=0, q=0, k=0, v=0, o=0, cu=0) == pkg.ATTN_OK
     assert _varlen(L, T=0, max_s=0, q=0, k=0, v=0, o=0, cu=0) == pkg.ATTN_OK
 
+
+
+def _decode(L, B=2, Hq=8, Hkv=2, dqk=128, dv=128, P=4, page=16, mb=4, msl=64, dtype=0, ws=1,
+            ws_bytes=None, cache_off=0, q=1, o=1, table=1, lens=1):
+    vp = ctypes.c_void_p
+    p = lambda x: vp(x * 256) if x else None  # fake, aligned, never dereferenced
+    need = L.attn_decode_workspace_size(B, Hq, Hkv, max(msl, 1))
+    return L.attn_decode_paged(p(q), vp(256 + cache_off), vp(512), p(o), None, p(table), p(lens),
+                               B, Hq, Hkv, dqk, dv, P, page, mb, msl, dtype, None, None, None,
+                               p(ws), need if ws_bytes is None else ws_bytes, None)
+
+
+def test_decode_argument_validation(L):
+    assert L.attn_decode_workspace_size(0, 8, 2, 64) == 0
+    assert L.attn_decode_workspace_size(2, 8, 2, 64) > 0
+    assert _decode(L, Hq=6, Hkv=4) == pkg.ATTN_ERR_INVALID_ARG
+    assert _decode(L, B=-1) == pkg.ATTN_ERR_INVALID_ARG
+    assert _decode(L, page=0) == pkg.ATTN_ERR_INVALID_ARG
+    assert _decode(L, dtype=5) == pkg.ATTN_ERR_INVALID_ARG
+    assert _decode(L, page=24) == pkg.ATTN_ERR_UNSUPPORTED       # not a power of two
+    assert _decode(L, dqk=192) == pkg.ATTN_ERR_UNSUPPORTED
+    assert _decode(L, Hq=6, Hkv=2) == pkg.ATTN_ERR_UNSUPPORTED   # 3 query heads per kv head
+    assert _decode(L, msl=100, mb=4, page=16) == pkg.ATTN_ERR_INVALID_ARG  # beyond the table
+    assert _decode(L, ws=0) == pkg.ATTN_ERR_INVALID_ARG
+    assert _decode(L, ws_bytes=16) == pkg.ATTN_ERR_INVALID_ARG
+    assert _decode(L, dtype=1) == pkg.ATTN_ERR_INVALID_ARG       # FP8 without descales
+    assert _decode(L, q=0) == pkg.ATTN_ERR_INVALID_ARG
+    assert _decode(L, cache_off=8) == pkg.ATTN_ERR_ALIGNMENT
+    assert _decode(L, B=0, q=0, o=0, table=0, lens=0, ws=0) == pkg.ATTN_OK
