@@ -50,6 +50,17 @@ WORKLOADS = {
     "mla32k_outlier": (1, 32768, 16, 16, 192, 128, "outlier",
                        "MLA-shaped causal prefill B=1 H=16 S=32768 d_qk=192 d_v=128, outlier inputs"),
 }
+# decode over a paged KV cache: name -> (B, L, Hq, Hkv, page_size, description)
+DECODE_WORKLOADS = {
+    "decode_gqa_b64_s4k": (64, 4096, 32, 8, 64,
+                           "paged decode B=64 sequences x 4096 cached tokens, Hq=32 Hkv=8 d=128, "
+                           "pages of 64 tokens in shuffled order"),
+    "decode_gqa_b16_s32k": (16, 32768, 32, 8, 64,
+                            "paged decode B=16 sequences x 32768 cached tokens, Hq=32 Hkv=8 "
+                            "d=128, pages of 64 tokens in shuffled order"),
+}
+DECODE_METRIC = "paged decode attention KV-cache read GB/s (FP8 e4m3, BF16); % of B200 HBM"
+
 for _s in (1024, 2048, 4096, 8192, 16384, 32768):
     WORKLOADS[f"sweep_s{_s // 1024}k"] = (
         32768 // _s, _s, 32, 8, 128, 128, "gaussian",
@@ -190,6 +201,126 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(loaded) if loaded else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
                 "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- decode leg
+def gpu_bench_decode(args, rank, world, local_rank):
+    """Decode over a paged KV cache: K timed calls (split + combine kernels) per precision,
+    CUDA events around each call; the caches (> L2) are read once per call."""
+    import torch
+    import torch.distributed as dist
+
+    import bf16_causal_prefill_attn_b200 as pkg
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    B, L, Hq, Hkv, page, desc = DECODE_WORKLOADS[args.workload]
+    P = B * L // page
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1000 + rank)
+    kc = torch.randn((P, page, Hkv, 128), generator=gen, device=dev).to(torch.bfloat16)
+    vc = torch.randn((P, page, Hkv, 128), generator=gen, device=dev).to(torch.bfloat16)
+    q = torch.randn((B, Hq, 128), generator=gen, device=dev).to(torch.bfloat16)
+    table = torch.randperm(P, generator=gen, device=dev).to(torch.int32).reshape(B, L // page)
+    lens = torch.full((B,), L, dtype=torch.int32, device=dev)
+    (q8, dq), (k8, dk), (v8, dv) = [pkg.attn_quantize_e4m3(t.reshape(-1, t.shape[-2], 128))
+                                    for t in (q, kc, vc)]
+    k8, v8, q8 = k8.reshape(kc.shape), v8.reshape(vc.shape), q8.reshape(q.shape)
+    o = torch.empty((B, Hq, 128), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    ws_bytes = pkg.attn_decode_workspace_size(B, Hq, Hkv, L)
+    ws = torch.empty((ws_bytes + 15) // 16 * 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def call_fp8():
+        pkg.attn_decode_paged(q8, k8, v8, table, lens, L, descale_q=dq, descale_k=dk,
+                              descale_v=dv, out=o, lse=lse, workspace=ws)
+
+    def call_bf16():
+        pkg.attn_decode_paged(q, kc, vc, table, lens, L, out=o, lse=lse, workspace=ws)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    def timed(fn, K, W):
+        for _ in range(W):
+            fn()
+        barrier()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(K)]
+        for a, b_ in evs:
+            a.record(stream)
+            fn()
+            b_.record(stream)
+        barrier()
+        st = pkg.attn_device_status()
+        if st != pkg.ATTN_OK:
+            raise RuntimeError(f"device status {pkg.status_string(st)}")
+        return statistics.mean(a.elapsed_time(b_) for a, b_ in evs)
+
+    peaks, peak_src = load_peaks()
+    with ClockSampler(gpu_selector(local_rank)) as clk:
+        fp8_ms = max_over_ranks(timed(call_fp8, args.steps, args.warmup), world, dev)
+        bf16_ms = max_over_ranks(timed(call_bf16, args.steps, args.warmup), world, dev)
+    clocks = clk.summary()
+
+    # e2e: the query uploaded from pinned host memory and the output read back every call
+    q_h = q8.cpu().pin_memory()
+    o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+
+    def call_e2e():
+        q8.copy_(q_h, non_blocking=True)
+        call_fp8()
+        o_h.copy_(o, non_blocking=True)
+
+    e2e_ms = max_over_ranks(timed(call_e2e, args.steps, args.warmup), world, dev)
+
+    def kv_bytes(e):
+        return 2.0 * B * L * Hkv * 128 * e
+    io_bytes = B * Hq * 128 * 2 + B * Hq * 4       # o (bf16) and lse written
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    flops = 2.0 * B * Hq * L * 256
+    fp8_gbs = (kv_bytes(1) + B * Hq * 128 + io_bytes) / (fp8_ms * 1e-3) / 1e9
+    bf16_gbs = (kv_bytes(2) + B * Hq * 256 + io_bytes) / (bf16_ms * 1e-3) / 1e9
+    return {
+        "metric": DECODE_METRIC,
+        "value": round(fp8_gbs * world, 1),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(fp8_ms, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e4m3",
+        "data": "synthetic",
+        "config": {"workload": desc, "name": args.workload, "B": B, "L": L, "Hq": Hq, "Hkv": Hkv,
+                   "d": 128, "page_size": page,
+                   "step": "one decode call (split-KV kernel + combine kernel)",
+                   "l2": f"no flush: the caches ({kv_bytes(1) / 1e9:.2f} GB FP8, "
+                         f"{kv_bytes(2) / 1e9:.2f} GB BF16) exceed the 126 MB L2",
+                   "parallelism": f"replicas x{world} (independent problems per GPU)"},
+        "roofline": {"bound": "hbm", "achieved": round(fp8_gbs, 1), "peak": hbm,
+                     "unit": "GB/s", "frac": round(fp8_gbs / hbm, 4),
+                     "peak_source": f"{peak_src} copy bandwidth",
+                     "kernel": "decode_split_kernel<fp8> + decode_combine_kernel",
+                     "tflops": round(flops / (fp8_ms * 1e-3) / 1e12, 2), "traffic": None},
+        "bf16": {"value": round(bf16_gbs * world, 1), "unit": "GB/s",
+                 "ms_per_step": round(bf16_ms, 4),
+                 "roofline": {"bound": "hbm", "achieved": round(bf16_gbs, 1), "peak": hbm,
+                              "unit": "GB/s", "frac": round(bf16_gbs / hbm, 4),
+                              "tflops": round(flops / (bf16_ms * 1e-3) / 1e12, 2),
+                              "traffic": None}},
+        "e2e": {"value": round((kv_bytes(1) + B * Hq * 128 + io_bytes) / (e2e_ms * 1e-3) / 1e9
+                               * world, 1),
+                "unit": "GB/s", "h2d_bytes_per_step": B * Hq * 128, "d2h_bytes_per_step":
+                B * Hq * 128 * 2, "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": args.steps * 2,
+        "clocks": clocks,
+    }
 
 
 # ----------------------------------------------------------------------------- GPU leg
@@ -536,7 +667,8 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="gqa16k_outlier", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="gqa16k_outlier",
+                    choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS))
     ap.add_argument("--hadamard", action="store_true")
     ap.add_argument("--no-energy", action="store_true",
                     help="skip the NVML energy windows (about 12 s of extra GPU time)")
@@ -552,10 +684,15 @@ def main(argv=None):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
+        if args.workload in DECODE_WORKLOADS:
+            if rank == 0:
+                print(json.dumps({"impl": "reference", "unavailable":
+                                  "the oracle reference arm covers the prefill workloads"}))
+            return 0
         return reference_main(args, rank, world)
     # the oracle baseline is measured before any CUDA call (no fork after CUDA init)
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload in WORKLOADS:
         cpu = cpu_reference(args.workload, args.cpu_seconds)
         cpu.pop("seconds", None)
     if world > 1:
@@ -566,7 +703,10 @@ def main(argv=None):
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     try:
-        res = gpu_bench(args, rank, world, local_rank)
+        if args.workload in DECODE_WORKLOADS:
+            res = gpu_bench_decode(args, rank, world, local_rank)
+        else:
+            res = gpu_bench(args, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

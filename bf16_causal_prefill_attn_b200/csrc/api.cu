@@ -242,7 +242,7 @@ attn_status_t launch_decode(attn::DecodeParams& prm, cudaStream_t st) {
   constexpr int smem = attn::dec_smem_bytes<FP8, G>();
   if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return ATTN_ERR_CUDA;
-  const dim3 grid(static_cast<unsigned>(prm.n_splits), static_cast<unsigned>(prm.Hkv),
+  const dim3 grid(static_cast<unsigned>(prm.Hkv), static_cast<unsigned>(prm.n_splits),
                   static_cast<unsigned>(prm.B));
   k1<<<grid, attn::DEC_THREADS, smem, st>>>(prm);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
@@ -329,7 +329,7 @@ attn_status_t attn_decode_paged(const void* q, const void* k_cache, const void* 
   if (d_qk != 128 || d_v != 128 || (G != 1 && G != 2 && G != 4 && G != 8 && G != 16))
     return ATTN_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(max_blocks_per_seq) * page_size > INT32_MAX || B > 65535 ||
-      Hkv > 65535)
+      attn::dec_n_splits(B, Hkv, max_seqlen > 0 ? max_seqlen : 1) > 65535)
     return ATTN_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(max_seqlen) > static_cast<int64_t>(max_blocks_per_seq) * page_size)
     return ATTN_ERR_INVALID_ARG;

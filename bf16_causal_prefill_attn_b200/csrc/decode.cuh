@@ -10,16 +10,19 @@
 // Hq / Hkv query heads share a kv head): HBM-bound, so it runs on the CUDA cores, with the
 // cache streamed through shared memory by 16-byte asynchronous copies; no tensor cores.
 //
-// Split-KV: CTA (split, g, b) takes one kv head g of sequence b, all G query heads that read
+// Split-KV: CTA (g, split, b) takes one kv head g of sequence b, all G query heads that read
 // it, and a contiguous range of its tokens; it writes the unnormalised partial output and
 // the (max, sum) of its range, and decode_combine_kernel merges the ranges.  Per 64-token
 // tile (double-buffered):
 //   A  scores: TPT threads per token, each with a DPT-element slice of the G queries in
-//      registers (already scaled by scale * log2 e, and for FP8 by the Q and K descales),
-//      reduce their partial dot products by shuffles;
+//      registers as 16-bit pairs, multiply the cached keys by mixed-precision fma (16-bit
+//      operands, exact products, fp32 accumulation), reduce their partial dot products by
+//      shuffles and scale them by scale * log2 e (FP8: times the Q and K descales);
 //   B  per head: the tile max, the running max, alpha = 2^(m_old - m_new), p = 2^(s - m_new)
 //      and the running sum (one warp per head, shuffles);
-//   C  O += p V: each thread owns two value columns of all G heads.
+//   C  O += p V with p rounded to 16 bits (f16 for FP8 caches, bf16 for BF16 ones; the
+//      running sum adds the same rounded values): each thread owns four value columns of
+//      all G heads and a quarter of the tokens, by mixed-precision fma.
 // Page ids and sequence lengths are read on the device: entries outside the cache make the
 // CTA record DEV_BAD_SEQLENS and write an empty partial instead of reading out of bounds.
 #pragma once
@@ -69,15 +72,17 @@ struct DecCfg {
 // the queries, the scores / probabilities, per-head state and the half-sum exchange
 template <bool FP8, int G>
 constexpr int dec_smem_bytes() {
-  return 4 * DecCfg<FP8>::TILE_BYTES + (G * DEC_D + DEC_TT * G + 3 * G + G * DEC_D) * 4;
+  return 4 * DecCfg<FP8>::TILE_BYTES + (G * DEC_D + DEC_TT * G + 3 * G + G * DEC_D) * 4 +
+         DEC_TT * G * 2;
 }
 
-// split-KV policy: about four CTAs per SM of a 148-SM B200 over B x Hkv (sequence, kv head)
+// split-KV policy: about sixteen CTAs per SM of a 148-SM B200 (several full waves at the
+// kernel's occupancy, so the last wave's tail is small) over B x Hkv (sequence, kv head)
 // pairs, each split at least two tiles; tokens per split a multiple of the tile
 inline int dec_n_splits(int B, int Hkv, int max_seqlen) {
   const int tiles = (max_seqlen + DEC_TT - 1) / DEC_TT;
   const long long pairs = static_cast<long long>(B) * Hkv;
-  long long want = pairs > 0 ? (4 * 148 + pairs - 1) / pairs : 1;
+  long long want = pairs > 0 ? (16 * 148 + pairs - 1) / pairs : 1;
   const long long cap = tiles / 2 > 1 ? tiles / 2 : 1;
   if (want > cap) want = cap;
   return static_cast<int>(want < 1 ? 1 : want);
@@ -104,6 +109,46 @@ __device__ __forceinline__ void cp_async_commit() {
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// acc + a.lo * b.lo + a.hi * b.hi for two pairs of 16-bit floats (f16, or bf16 with BF),
+// each product exact in fp32 and each step rounded once (mixed-precision fma of sm_100)
+template <bool BF>
+__device__ __forceinline__ float fma2_mixed(uint32_t a, uint32_t b, float acc) {
+  float d;
+  if constexpr (BF) {
+    asm("{.reg .b16 al, ah, bl, bh; .reg .f32 t; mov.b32 {al, ah}, %1; mov.b32 {bl, bh}, %2;"
+        " fma.rn.f32.bf16 t, al, bl, %3; fma.rn.f32.bf16 %0, ah, bh, t;}"
+        : "=f"(d) : "r"(a), "r"(b), "f"(acc));
+  } else {
+    asm("{.reg .b16 al, ah, bl, bh; .reg .f32 t; mov.b32 {al, ah}, %1; mov.b32 {bl, bh}, %2;"
+        " fma.rn.f32.f16 t, al, bl, %3; fma.rn.f32.f16 %0, ah, bh, t;}"
+        : "=f"(d) : "r"(a), "r"(b), "f"(acc));
+  }
+  return d;
+}
+
+// a[c] += p * v_c for the four 16-bit values of v01, v23 (f16, or bf16 with BF); p 16-bit
+template <bool BF>
+__device__ __forceinline__ void pv4_mixed(uint16_t p, uint32_t v01, uint32_t v23, float* a) {
+  if constexpr (BF) {
+    asm("{.reg .b16 x0, x1, x2, x3; mov.b32 {x0, x1}, %4; mov.b32 {x2, x3}, %5;"
+        " fma.rn.f32.bf16 %0, %6, x0, %0; fma.rn.f32.bf16 %1, %6, x1, %1;"
+        " fma.rn.f32.bf16 %2, %6, x2, %2; fma.rn.f32.bf16 %3, %6, x3, %3;}"
+        : "+f"(a[0]), "+f"(a[1]), "+f"(a[2]), "+f"(a[3]) : "r"(v01), "r"(v23), "h"(p));
+  } else {
+    asm("{.reg .b16 x0, x1, x2, x3; mov.b32 {x0, x1}, %4; mov.b32 {x2, x3}, %5;"
+        " fma.rn.f32.f16 %0, %6, x0, %0; fma.rn.f32.f16 %1, %6, x1, %1;"
+        " fma.rn.f32.f16 %2, %6, x2, %2; fma.rn.f32.f16 %3, %6, x3, %3;}"
+        : "+f"(a[0]), "+f"(a[1]), "+f"(a[2]), "+f"(a[3]) : "r"(v01), "r"(v23), "h"(p));
+  }
+}
+
+// two e4m3 codes (low 16 bits) -> f16x2, exact
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t pair) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<uint16_t>(pair)));
+  return h2;
 }
 
 // 8 elements of a 16-byte chunk (bf16 x8, or the low 8 bytes as e4m3 x8) to float
@@ -154,9 +199,12 @@ __global__ void __launch_bounds__(DEC_THREADS)
   float* hm = s_s + DEC_TT * G;                          // [G] running max (log2 units)
   float* hl = hm + G;                                    // [G] running sum
   float* ha = hl + G;                                    // [G] alpha of this tile
-  float* ored = ha + G;                                  // [G][128] half-sum exchange
+  float* ored = ha + G;                                  // [G][128] token-group exchange
+  uint16_t* p16 = reinterpret_cast<uint16_t*>(ored + G * DEC_D);  // [DEC_TT][G] p, 16-bit
 
-  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  // kv head fastest: the CTAs of one (sequence, split) read the same pages (their head's
+  // slice of every token row) at about the same time, which keeps DRAM rows open
+  const int g = blockIdx.x, split = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int len = p.seq_lens[b];
   const int t_begin = split * p.split_tokens;
@@ -187,21 +235,20 @@ __global__ void __launch_bounds__(DEC_THREADS)
     return;
   }
 
-  // ---- queries of the G heads, scaled into log2 units
+  // ---- queries of the G heads as 16-bit pairs (FP8: the e4m3 values in f16, exact; BF16:
+  // the inputs); the scale into log2 units is applied to each finished dot product
   float qs = p.qk_scale;
   if constexpr (FP8) qs *= *p.descale_q * *p.descale_k;
-  for (int i = tid; i < G * DEC_D; i += DEC_THREADS) {
-    const size_t qi = (static_cast<size_t>(b) * p.Hq + g * G) * DEC_D + i;
-    float x;
+  uint32_t* q_w = reinterpret_cast<uint32_t*>(q_s);  // [G][64] pairs
+  for (int i = tid; i < G * DEC_D / 2; i += DEC_THREADS) {
+    const size_t qi = (static_cast<size_t>(b) * p.Hq + g * G) * DEC_D + 2 * i;
     if constexpr (FP8) {
-      uint32_t h2;
-      const uint16_t pair = static_cast<const uint8_t*>(p.q)[qi];
-      asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(pair));
-      x = __low2float(*reinterpret_cast<const __half2*>(&h2));
+      const uint8_t* qc = static_cast<const uint8_t*>(p.q) + qi;
+      q_w[i] = e4m3x2_to_f16x2(static_cast<uint32_t>(qc[0]) | (static_cast<uint32_t>(qc[1]) << 8));
     } else {
-      x = __bfloat162float(static_cast<const __nv_bfloat16*>(p.q)[qi]);
+      const uint16_t* qb = static_cast<const uint16_t*>(p.q) + qi;
+      q_w[i] = static_cast<uint32_t>(qb[0]) | (static_cast<uint32_t>(qb[1]) << 16);
     }
-    q_s[i] = x * qs;
   }
   if (tid < G) {
     hm[tid] = -INFINITY;
@@ -231,18 +278,17 @@ __global__ void __launch_bounds__(DEC_THREADS)
   load_tile(t_begin, 0);
   __syncthreads();  // q_s, hm, hl
 
-  // phase A mapping and the query slice in registers
+  // phase A mapping and the query slice in registers (16-bit pairs)
   const int a_tok = tid / TPT, a_part = tid % TPT;
-  float qr[G][DPT];
+  uint32_t qr[G][DPT / 2];
 #pragma unroll
   for (int h = 0; h < G; ++h)
 #pragma unroll
-    for (int e = 0; e < DPT; ++e) qr[h][e] = q_s[h * DEC_D + a_part * DPT + e];
-  // phase C mapping: value columns 2 ce, 2 ce + 1, tokens of parity cpar
-  const int ce = tid & 63, cpar = tid >> 6;
-  float acc[G][2];
+    for (int e = 0; e < DPT / 2; ++e) qr[h][e] = q_w[h * (DEC_D / 2) + a_part * (DPT / 2) + e];
+  // phase C mapping: value columns 4 lane .. 4 lane + 3, tokens j = warp (mod 4)
+  float acc[G][4];
 #pragma unroll
-  for (int h = 0; h < G; ++h) acc[h][0] = acc[h][1] = 0.0f;
+  for (int h = 0; h < G; ++h) acc[h][0] = acc[h][1] = acc[h][2] = acc[h][3] = 0.0f;
 
   for (int it = 0; it < n_tiles; ++it) {
     const int buf = it & 1;
@@ -269,24 +315,35 @@ __global__ void __launch_bounds__(DEC_THREADS)
         // bytes [a_part * SLICE_BYTES + lb, + LOAD_BYTES) of row j
         const int byte = a_part * SLICE_BYTES + lb;
         const uint8_t* src = kt + dec_chunk_off<FP8>(j, byte >> 4) + (byte & 15);
-        float kf[16];
+        // the loaded elements as 16-bit pairs (FP8: converted to f16, exact)
+        uint32_t kw[8];
         if constexpr (LOAD_BYTES == 16) {
           const uint4 w = *reinterpret_cast<const uint4*>(src);
           if constexpr (FP8) {
-            dec_unpack8<true>(w, kf);
-            dec_unpack8<true>(make_uint4(w.z, w.w, 0, 0), kf + 8);
+            const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              kw[2 * i] = e4m3x2_to_f16x2(u[i]);
+              kw[2 * i + 1] = e4m3x2_to_f16x2(u[i] >> 16);
+            }
           } else {
-            dec_unpack8<false>(w, kf);
+            kw[0] = w.x;
+            kw[1] = w.y;
+            kw[2] = w.z;
+            kw[3] = w.w;
           }
         } else {
           const uint2 w = *reinterpret_cast<const uint2*>(src);  // FP8, 8 elements
-          dec_unpack8<true>(make_uint4(w.x, w.y, 0, 0), kf);
+          kw[0] = e4m3x2_to_f16x2(w.x);
+          kw[1] = e4m3x2_to_f16x2(w.x >> 16);
+          kw[2] = e4m3x2_to_f16x2(w.y);
+          kw[3] = e4m3x2_to_f16x2(w.y >> 16);
         }
 #pragma unroll
-        for (int e = 0; e < LOAD_ELEMS; ++e)
+        for (int e = 0; e < LOAD_ELEMS / 2; ++e)
 #pragma unroll
           for (int h = 0; h < G; ++h)
-            part[h] = __fmaf_rn(qr[h][lb / C::E + e], kf[e], part[h]);
+            part[h] = fma2_mixed<!FP8>(qr[h][lb / (2 * C::E) + e], kw[e], part[h]);
       }
 #pragma unroll
       for (int off = 1; off < TPT; off <<= 1)
@@ -295,7 +352,7 @@ __global__ void __launch_bounds__(DEC_THREADS)
       if (a_part == 0) {
         const bool in = t0 + j < t_end;
 #pragma unroll
-        for (int h = 0; h < G; ++h) s_s[j * G + h] = in ? part[h] : -INFINITY;
+        for (int h = 0; h < G; ++h) s_s[j * G + h] = in ? part[h] * qs : -INFINITY;
       }
     }
     __syncthreads();
@@ -308,9 +365,23 @@ __global__ void __launch_bounds__(DEC_THREADS)
       for (int off = 16; off > 0; off >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
       const float m_old = hm[h];
       const float m_new = fmaxf(m_old, mt);
-      const float p0 = ex2_approx(s0 - m_new), p1 = ex2_approx(s1 - m_new);
-      s_s[lane * G + h] = p0;
-      s_s[(lane + 32) * G + h] = p1;
+      // p rounded to the 16-bit type of the cached values (FP8: f16, BF16: bf16), the
+      // form O += p V multiplies; the row sum adds the same rounded values
+      float p0 = ex2_approx(s0 - m_new), p1 = ex2_approx(s1 - m_new);
+      uint16_t r0, r1;
+      if constexpr (FP8) {
+        r0 = __half_as_ushort(__float2half_rn(p0));
+        r1 = __half_as_ushort(__float2half_rn(p1));
+        p0 = __half2float(__ushort_as_half(r0));
+        p1 = __half2float(__ushort_as_half(r1));
+      } else {
+        r0 = __bfloat16_as_ushort(__float2bfloat16_rn(p0));
+        r1 = __bfloat16_as_ushort(__float2bfloat16_rn(p1));
+        p0 = __bfloat162float(__ushort_as_bfloat16(r0));
+        p1 = __bfloat162float(__ushort_as_bfloat16(r1));
+      }
+      p16[lane * G + h] = r0;
+      p16[(lane + 32) * G + h] = r1;
       float ls = p0 + p1;
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, off);
@@ -324,55 +395,66 @@ __global__ void __launch_bounds__(DEC_THREADS)
     }
     __syncthreads();
 
-    // ---- C: O += p V over the tokens of this thread's parity
+    // ---- C: O += p V; 4 value columns x G heads per thread, tokens j = warp (mod 4), by
+    // mixed-precision fma (16-bit p and v, fp32 accumulators)
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       const float a = ha[h];
-      acc[h][0] *= a;
-      acc[h][1] *= a;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[h][c] *= a;
     }
 #pragma unroll 4
-    for (int j = cpar; j < DEC_TT; j += 2) {
-      float v0, v1;
+    for (int j = warp; j < DEC_TT; j += 4) {
+      uint32_t v01, v23;
       if constexpr (FP8) {
-        const uint16_t pair = *reinterpret_cast<const uint16_t*>(
-            vt + dec_chunk_off<true>(j, (2 * ce) >> 4) + ((2 * ce) & 15));
-        uint32_t h2;
-        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(pair));
-        const __half2 hv = *reinterpret_cast<const __half2*>(&h2);
-        v0 = __low2float(hv);
-        v1 = __high2float(hv);
+        const uint32_t codes = *reinterpret_cast<const uint32_t*>(
+            vt + dec_chunk_off<true>(j, (4 * lane) >> 4) + ((4 * lane) & 15));
+        v01 = e4m3x2_to_f16x2(codes);
+        v23 = e4m3x2_to_f16x2(codes >> 16);
       } else {
-        const uint32_t w = *reinterpret_cast<const uint32_t*>(
-            vt + dec_chunk_off<false>(j, (4 * ce) >> 4) + ((4 * ce) & 15));
-        v0 = __uint_as_float(w << 16);
-        v1 = __uint_as_float(w & 0xffff0000u);
+        const uint2 w = *reinterpret_cast<const uint2*>(
+            vt + dec_chunk_off<false>(j, (8 * lane) >> 4) + ((8 * lane) & 15));
+        v01 = w.x;
+        v23 = w.y;
+      }
+      uint32_t pw[(G + 1) / 2];
+      if constexpr (G == 1) {
+        pw[0] = p16[j];
+      } else {
+#pragma unroll
+        for (int i = 0; i < G / 2; ++i) pw[i] = reinterpret_cast<const uint32_t*>(p16 + j * G)[i];
       }
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float pj = s_s[j * G + h];
-        acc[h][0] = __fmaf_rn(pj, v0, acc[h][0]);
-        acc[h][1] = __fmaf_rn(pj, v1, acc[h][1]);
-      }
+      for (int h = 0; h < G; ++h)
+        pv4_mixed<!FP8>(static_cast<uint16_t>(pw[h / 2] >> (16 * (h & 1))), v01, v23, acc[h]);
     }
     __syncthreads();  // this buffer is refilled two tiles later; s_s is rewritten
   }
 
-  // ---- the two token parities, then the partial output of this range
-  if (cpar == 1) {
+  // ---- the four token groups (warps), then the partial output of this range
+#pragma unroll 1
+  for (int w = 1; w < 4; ++w) {
+    if (warp == w) {
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      ored[h * DEC_D + 2 * ce] = acc[h][0];
-      ored[h * DEC_D + 2 * ce + 1] = acc[h][1];
+      for (int h = 0; h < G; ++h)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float* dst = ored + h * DEC_D + 4 * lane + c;
+          *dst = (w == 1 ? 0.0f : *dst) + acc[h][c];
+        }
     }
+    __syncthreads();
   }
-  __syncthreads();
-  if (cpar == 0) {
+  if (warp == 0) {
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      float* po = p.part_o + (pidx + static_cast<size_t>(h) * p.n_splits) * DEC_D + 2 * ce;
-      po[0] = acc[h][0] + ored[h * DEC_D + 2 * ce];
-      po[1] = acc[h][1] + ored[h * DEC_D + 2 * ce + 1];
+      float* po = p.part_o + (pidx + static_cast<size_t>(h) * p.n_splits) * DEC_D + 4 * lane;
+      float4 r;
+      r.x = acc[h][0] + ored[h * DEC_D + 4 * lane + 0];
+      r.y = acc[h][1] + ored[h * DEC_D + 4 * lane + 1];
+      r.z = acc[h][2] + ored[h * DEC_D + 4 * lane + 2];
+      r.w = acc[h][3] + ored[h * DEC_D + 4 * lane + 3];
+      *reinterpret_cast<float4*>(po) = r;
     }
   }
   if (tid < G) {
