@@ -93,10 +93,9 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, attn::FwdP
 
 // Checks shared by the fixed-length and packed entry points; fills the parameters that
 // do not depend on the sequence layout.
-attn_status_t common_args(const void* q, const void* k, const void* v, void* o, float* lse,
-                          int Hq, int Hkv, int d_qk, int d_v, attn_dtype_t dtype,
-                          const float* dq, const float* dk, const float* dv, int causal,
-                          unsigned flags, attn::FwdParams* prm) {
+attn_status_t common_args(void* o, float* lse, int Hq, int Hkv, int d_qk, int d_v,
+                          attn_dtype_t dtype, const float* dq, const float* dk,
+                          const float* dv, int causal, unsigned flags, attn::FwdParams* prm) {
   if (Hq <= 0 || Hkv <= 0 || (Hq % Hkv) != 0) return ATTN_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
   if ((flags & ~static_cast<unsigned>(ATTN_FLAG_UNROTATE_O | ATTN_FLAG_EXACT_P)) != 0)
@@ -104,7 +103,6 @@ attn_status_t common_args(const void* q, const void* k, const void* v, void* o, 
   if (dtype != ATTN_BF16 && dtype != ATTN_FP8_E4M3) return ATTN_ERR_INVALID_ARG;
   if ((flags & ATTN_FLAG_EXACT_P) && dtype != ATTN_FP8_E4M3) return ATTN_ERR_INVALID_ARG;
   if ((d_qk != 128 && d_qk != 192) || d_v != 128) return ATTN_ERR_UNSUPPORTED;
-  (void)q; (void)k; (void)v; (void)o; (void)lse;
   prm->Hq = Hq;
   prm->Hkv = Hkv;
   prm->G = Hq / Hkv;
@@ -175,8 +173,8 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, flo
                        uint8_t* dump_kshift, bool dump, void* stream) {
   attn::FwdParams prm{};
   if (B < 0 || S < 0) return ATTN_ERR_INVALID_ARG;
-  attn_status_t e = common_args(q, k, v, o, lse, Hq, Hkv, d_qk, d_v, dtype, dq, dk, dv, causal,
-                                flags, &prm);
+  attn_status_t e = common_args(o, lse, Hq, Hkv, d_qk, d_v, dtype, dq, dk, dv, causal, flags,
+                                &prm);
   if (e != ATTN_OK) return e;
   if (B == 0 || S == 0) return ATTN_OK;
   if (dump && (dtype != ATTN_FP8_E4M3 || !dump_s || !dump_codes || !dump_kshift))
@@ -212,8 +210,8 @@ attn_status_t varlen_impl(const void* q, const void* k, const void* v, void* o, 
                           const float* dv, int causal, unsigned flags, void* stream) {
   attn::FwdParams prm{};
   if (B < 0 || max_seqlen < 0 || total_tokens < 0) return ATTN_ERR_INVALID_ARG;
-  attn_status_t e = common_args(q, k, v, o, lse, Hq, Hkv, d_qk, d_v, dtype, dq, dk, dv, causal,
-                                flags, &prm);
+  attn_status_t e = common_args(o, lse, Hq, Hkv, d_qk, d_v, dtype, dq, dk, dv, causal, flags,
+                                &prm);
   if (e != ATTN_OK) return e;
   if (B == 0 || max_seqlen == 0 || total_tokens == 0) return ATTN_OK;
   if (flags & ATTN_FLAG_EXACT_P) return ATTN_ERR_UNSUPPORTED;
