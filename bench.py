@@ -635,6 +635,41 @@ def cpu_reference(workload, budget_s, rank=0):
             "seconds": dt}
 
 
+def cpu_reference_decode(workload, budget_s):
+    """The decode oracle (fp64, paged gather + softmax per head), as it stands, on a bounded
+    sample: sequences of the workload's length and heads, each with its own query, over one
+    synthetic cache (made before the timing); value in GB/s of the FP8 KV bytes it stands
+    for, like the GPU line."""
+    import numpy as np
+
+    from oracle import decode
+
+    B, L, Hq, Hkv, page, desc = DECODE_WORKLOADS[workload]
+    rng = np.random.default_rng(0)
+    P = L // page
+    kc = rng.standard_normal((P, page, Hkv, 128))
+    vc = rng.standard_normal((P, page, Hkv, 128))
+    table = rng.permutation(P).astype(np.int32)[None]
+    lens = np.array([L], dtype=np.int32)
+    n = 0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < budget_s or n == 0:
+        q = rng.standard_normal((1, Hq, 128))
+        decode.decode_attention(q, kc, vc, table, lens, page)
+        n += 1
+    dt = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    return {"value": n * 2.0 * L * Hkv * 128 / dt / 1e9, "unit": "GB/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"{n} sequences of {L} cached tokens (all {Hq} query heads each) of "
+                      f"{desc}; {dt:.1f} s; cache generation not timed",
+            "seconds": dt}
+
+
 def reference_main(args, rank, world):
     if rank != 0:
         return 0
@@ -686,14 +721,28 @@ def main(argv=None):
     if args.impl == "reference":
         if args.workload in DECODE_WORKLOADS:
             if rank == 0:
-                print(json.dumps({"impl": "reference", "unavailable":
-                                  "the oracle reference arm covers the prefill workloads"}))
+                c = cpu_reference_decode(args.workload, min(args.cpu_seconds, 20.0))
+                c.pop("seconds", None)
+                B, L, Hq, Hkv, page, desc = DECODE_WORKLOADS[args.workload]
+                print(json.dumps({"impl": "reference", "metric": DECODE_METRIC,
+                                  "value": c["value"], "unit": "GB/s", "n_gpus": world,
+                                  "steps": args.steps, "warmup": args.warmup,
+                                  "higher_is_better": True, "scaling": "weak",
+                                  "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                                  "config": {"workload": desc, "name": args.workload},
+                                  "cpu_baseline": c,
+                                  "e2e": {"value": c["value"], "unit": "GB/s",
+                                          "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+                      flush=True)
             return 0
         return reference_main(args, rank, world)
     # the oracle baseline is measured before any CUDA call (no fork after CUDA init)
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload in WORKLOADS:
-        cpu = cpu_reference(args.workload, args.cpu_seconds)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        if args.workload in WORKLOADS:
+            cpu = cpu_reference(args.workload, args.cpu_seconds)
+        else:
+            cpu = cpu_reference_decode(args.workload, min(args.cpu_seconds, 10.0))
         cpu.pop("seconds", None)
     if world > 1:
         import datetime

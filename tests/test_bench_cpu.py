@@ -85,3 +85,16 @@ def test_energy_summary_and_window_with_fake_nvml():
     assert r["joules"] == 0.25 and r["calls"] >= 3
     assert abs(r["tflop_per_j"] - 2e11 * r["calls"] / 0.25 / 1e12) < 1e-3
     assert len(calls) > r["calls"]   # the warm-up ran first
+
+
+def test_decode_reference_arm_prints_one_line():
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+           "--workload", "decode_gqa_b64_s4k", "--steps", "1", "--warmup", "3",
+           "--cpu-seconds", "0.5"]
+    res = subprocess.run(cmd, capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert res.returncode == 0, res.stderr
+    lines = [l for l in res.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["d2h_bytes_per_step"] == 0
