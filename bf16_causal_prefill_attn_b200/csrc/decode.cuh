@@ -13,7 +13,7 @@
 // Split-KV: CTA (g, split, b) takes one kv head g of sequence b, all G query heads that read
 // it, and a contiguous range of its tokens; it writes the unnormalised partial output and
 // the (max, sum) of its range, and decode_combine_kernel merges the ranges.  Per 64-token
-// tile (double-buffered):
+// tile (NST tiles in flight):
 //   A  scores: TPT threads per token, each with a DPT-element slice of the G queries in
 //      registers as 16-bit pairs, multiply the cached keys by mixed-precision fma (16-bit
 //      operands, exact products, fp32 accumulation), reduce their partial dot products by
@@ -66,13 +66,16 @@ struct DecCfg {
   static constexpr int ROW = DEC_D * E;          // bytes of one token's K (or V) row
   static constexpr int CHUNKS = ROW / 16;        // 16-byte chunks per row
   static constexpr int TILE_BYTES = DEC_TT * ROW;
+  // tiles in flight per CTA: e4m3 tiles are half the size, so three fit at four CTAs per SM
+  static constexpr int NST = FP8 ? 3 : 2;
 };
 
 // dynamic shared memory of decode_split_kernel<FP8, G>: K and V tiles (double-buffered),
 // the queries, the scores / probabilities, per-head state and the half-sum exchange
 template <bool FP8, int G>
 constexpr int dec_smem_bytes() {
-  return 4 * DecCfg<FP8>::TILE_BYTES + (G * DEC_D + DEC_TT * G + 3 * G + G * DEC_D) * 4 +
+  return 2 * DecCfg<FP8>::NST * DecCfg<FP8>::TILE_BYTES +
+         (G * DEC_D + DEC_TT * G + 3 * G + G * DEC_D) * 4 +
          DEC_TT * G * 2;
 }
 
@@ -192,9 +195,9 @@ __global__ void __launch_bounds__(DEC_THREADS)
   constexpr int LOAD_ELEMS = LOAD_BYTES / C::E;
 
   extern __shared__ __align__(16) uint8_t dsm[];
-  uint8_t* kbuf = dsm;                                   // [2][TILE_BYTES]
-  uint8_t* vbuf = dsm + 2 * C::TILE_BYTES;               // [2][TILE_BYTES]
-  float* q_s = reinterpret_cast<float*>(dsm + 4 * C::TILE_BYTES);   // [G][128]
+  uint8_t* kbuf = dsm;                                   // [NST][TILE_BYTES]
+  uint8_t* vbuf = dsm + C::NST * C::TILE_BYTES;          // [NST][TILE_BYTES]
+  float* q_s = reinterpret_cast<float*>(dsm + 2 * C::NST * C::TILE_BYTES);  // [G][128]
   float* s_s = q_s + G * DEC_D;                          // [DEC_TT][G] scores, then p
   float* hm = s_s + DEC_TT * G;                          // [G] running max (log2 units)
   float* hl = hm + G;                                    // [G] running sum
@@ -275,7 +278,13 @@ __global__ void __launch_bounds__(DEC_THREADS)
   };
 
   const int n_tiles = (t_end - t_begin + DEC_TT - 1) / DEC_TT;
-  load_tile(t_begin, 0);
+  // prologue: the first NST - 1 tiles (an empty group where there is no tile keeps the
+  // count of committed groups uniform)
+#pragma unroll
+  for (int st = 0; st < C::NST - 1; ++st) {
+    if (st < n_tiles) load_tile(t_begin + st * DEC_TT, st);
+    else cp_async_commit();
+  }
   __syncthreads();  // q_s, hm, hl
 
   // phase A mapping and the query slice in registers (16-bit pairs)
@@ -291,14 +300,12 @@ __global__ void __launch_bounds__(DEC_THREADS)
   for (int h = 0; h < G; ++h) acc[h][0] = acc[h][1] = acc[h][2] = acc[h][3] = 0.0f;
 
   for (int it = 0; it < n_tiles; ++it) {
-    const int buf = it & 1;
+    const int buf = it % C::NST;
     const int t0 = t_begin + it * DEC_TT;
-    if (it + 1 < n_tiles) {
-      load_tile(t0 + DEC_TT, buf ^ 1);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
+    // tile it + NST - 1 into the buffer tile it - 1 used (every thread is past it)
+    if (it + C::NST - 1 < n_tiles) load_tile(t0 + (C::NST - 1) * DEC_TT, (it + C::NST - 1) % C::NST);
+    else cp_async_commit();
+    cp_async_wait<C::NST - 1>();  // tile it has landed
     __syncthreads();
     const uint8_t* kt = kbuf + buf * C::TILE_BYTES;
     const uint8_t* vt = vbuf + buf * C::TILE_BYTES;
@@ -428,7 +435,7 @@ __global__ void __launch_bounds__(DEC_THREADS)
       for (int h = 0; h < G; ++h)
         pv4_mixed<!FP8>(static_cast<uint16_t>(pw[h / 2] >> (16 * (h & 1))), v01, v23, acc[h]);
     }
-    __syncthreads();  // this buffer is refilled two tiles later; s_s is rewritten
+    __syncthreads();  // this buffer is refilled next iteration; s_s is rewritten
   }
 
   // ---- the four token groups (warps), then the partial output of this range
