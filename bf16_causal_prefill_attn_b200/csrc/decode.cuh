@@ -66,8 +66,9 @@ struct DecCfg {
   static constexpr int ROW = DEC_D * E;          // bytes of one token's K (or V) row
   static constexpr int CHUNKS = ROW / 16;        // 16-byte chunks per row
   static constexpr int TILE_BYTES = DEC_TT * ROW;
-  // tiles in flight per CTA: e4m3 tiles are half the size, so three fit at four CTAs per SM
-  static constexpr int NST = FP8 ? 3 : 2;
+  // tiles in flight per CTA (a third did not change the time: the kernel is issue-bound
+  // with e4m3 caches and near the copy bandwidth with bf16 ones)
+  static constexpr int NST = 2;
 };
 
 // dynamic shared memory of decode_split_kernel<FP8, G>: K and V tiles (double-buffered),
