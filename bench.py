@@ -118,7 +118,8 @@ def energy_summary(flops_per_call, calls, mj_start, mj_end, seconds):
                 "seconds": round(seconds, 3)}
     return {"tflop_per_j": round(flops_per_call * calls / joules / 1e12, 4),
             "joules": round(joules, 3), "avg_w": round(joules / seconds, 1), "calls": calls,
-            "seconds": round(seconds, 3)}
+            "seconds": round(seconds, 3),
+            "sustained_tflops": round(flops_per_call * calls / seconds / 1e12, 2)}
 
 
 def measure_energy(nvml, handle, fn, flops_per_call, sync, seconds=3.0):
@@ -533,6 +534,8 @@ def gpu_bench(args, rank, world, local_rank):
                      "peak_source": f"{peak_src} bf16 cuBLAS burst x2 (fp8/bf16 nominal ratio)",
                      "frac_of_nominal_4500": round(fp8_kern_tf / NOMINAL_FP8_TFLOPS, 4),
                      "kernel": "attn_fwd_kernel<fp8, exact P>" if args.exact_p else "attn_fwd_kernel<fp8>", "kernel_ms": round(fp8_kern, 4),
+                     "kernel_ms_median": round(statistics.median(fp8_kern_ms), 4),
+                     "kernel_ms_min": round(min(fp8_kern_ms), 4),
                      "traffic": traffic.get("fp8")},
         "bf16": {"value": round(job_tflops(flops, world, bf16_ms), 2), "unit": UNIT,
                  "ms_per_step": round(bf16_ms, 4), "dtype": "bf16",
@@ -541,6 +544,9 @@ def gpu_bench(args, rank, world, local_rank):
                               "frac": round(bf16_kern_tf / bf16_peak, 4),
                               "peak_source": f"{peak_src} bf16 cuBLAS burst",
                               "frac_of_nominal_2250": round(bf16_kern_tf / NOMINAL_BF16_TFLOPS, 4),
+                              "kernel_ms": round(bf16_kern, 4),
+                              "kernel_ms_median": round(statistics.median(bf16_kern_ms), 4),
+                              "kernel_ms_min": round(min(bf16_kern_ms), 4),
                               "traffic": traffic.get("bf16")}},
         "e2e": {"value": round(job_tflops(flops, world, e2e_pipe), 2), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

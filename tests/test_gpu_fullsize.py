@@ -94,3 +94,29 @@ def test_fp8_fullsize(name, rotate):
         got = o[b][rows][:, heads, :].transpose(1, 0, 2)
         assert rel_rms(got, emu) <= 5e-3
         assert rel_rms(got, ref) <= 3e-2
+
+
+@pytest.mark.parametrize("name", ["gqa16k_outlier", "mha32k_gaussian"])
+def test_fullsize_bitwise_deterministic_1000_launches(name):
+    """1000 launches per precision at the full workload size, every output and lse bitwise
+    equal to the first launch's (no atomics or order-dependent reductions in the kernels)."""
+    B, S, Hq, Hkv, dqk, dist = CONFIGS[name]
+    q, k, v = [t.cuda() for t in synth.make_qkv(B, S, Hq, Hkv, dqk, 128, seed=21, dist=dist)]
+    (q8, dq), (k8, dk), (v8, dv) = [pkg.attn_quantize_e4m3(t) for t in (q, k, v)]
+    runs = [
+        (lambda o, l: pkg.attn_fwd(q, k, v, out=o, lse=l)),
+        (lambda o, l: pkg.attn_fwd(q8, k8, v8, descale_q=dq, descale_k=dk, descale_v=dv,
+                                   out=o, lse=l)),
+    ]
+    for run in runs:
+        o0, l0 = (torch.empty((B, S, Hq, 128), dtype=torch.bfloat16, device="cuda"),
+                  torch.empty((B, Hq, S), dtype=torch.float32, device="cuda"))
+        run(o0, l0)
+        o, l = torch.empty_like(o0), torch.empty_like(l0)
+        diff = torch.zeros((), dtype=torch.int64, device="cuda")
+        for _ in range(1000):
+            run(o, l)
+            diff += (o.view(torch.int16) != o0.view(torch.int16)).sum()
+            diff += (l.view(torch.int32) != l0.view(torch.int32)).sum()
+        assert int(diff) == 0
+        assert pkg.attn_device_status() == pkg.ATTN_OK
