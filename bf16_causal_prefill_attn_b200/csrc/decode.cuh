@@ -155,33 +155,6 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t pair) {
   return h2;
 }
 
-// 8 elements of a 16-byte chunk (bf16 x8, or the low 8 bytes as e4m3 x8) to float
-template <bool FP8>
-__device__ __forceinline__ void dec_unpack8(const uint4& w, float* f) {
-  if constexpr (!FP8) {
-    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      f[2 * i] = __uint_as_float(u[i] << 16);
-      f[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
-    }
-  } else {
-    const uint32_t u[2] = {w.x, w.y};
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-#pragma unroll
-      for (int hlf = 0; hlf < 2; ++hlf) {
-        const uint16_t pair = static_cast<uint16_t>(u[i] >> (16 * hlf));
-        uint32_t h2;
-        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(pair));
-        const __half2 hv = *reinterpret_cast<const __half2*>(&h2);
-        f[4 * i + 2 * hlf] = __low2float(hv);
-        f[4 * i + 2 * hlf + 1] = __high2float(hv);
-      }
-    }
-  }
-}
-
 // G query heads per kv head; DPT elements of d per thread in phase A
 template <bool FP8, int G>
 __global__ void __launch_bounds__(DEC_THREADS)
