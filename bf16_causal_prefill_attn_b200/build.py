@@ -6,7 +6,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libattn_b200.so")
-SOURCES = ["api.cu", "attn_fwd.cuh", "quantize.cuh", "ptx.cuh"]
+SOURCES = ["api.cu", "attn_fwd.cuh", "quantize.cuh", "ptx.cuh", "decode.cuh"]
 HEADER = os.path.join(ROOT, "include", "attn.h")
 
 

@@ -7,22 +7,31 @@
 //   k_cache / v_cache [num_pages, page_size, Hkv, 128]; query head h reads kv head h / G.
 //
 // The operation reads every cached K and V byte once and does ~2 G flops per byte (G =
-// Hq / Hkv query heads share a kv head): HBM-bound, so it runs on the CUDA cores, with the
-// cache streamed through shared memory by 16-byte asynchronous copies; no tensor cores.
+// Hq / Hkv query heads share a kv head): HBM-bound, with the cache streamed through shared
+// memory by 16-byte asynchronous copies.  What has to keep up with the copies is the
+// instruction issue of the contractions: with e4m3 caches a CUDA-core loop (convert, then
+// one fma per product) issues ~4x more instructions per cached byte than with bf16 ones,
+// so the FP8 kernel hands both contractions to warp-level tensor-core MMAs
+// (mma.sync m16n8k32 e4m3 for the scores, m16n8k16 f16 for PV: each replaces 128 or 64
+// fma instructions of a warp); the MMA shapes are not the point here, the issue slots are.
 //
 // Split-KV: CTA (g, split, b) takes one kv head g of sequence b, all G query heads that read
 // it, and a contiguous range of its tokens; it writes the unnormalised partial output and
 // the (max, sum) of its range, and decode_combine_kernel merges the ranges.  Per 64-token
 // tile (NST tiles in flight):
-//   A  scores: TPT threads per token, each with a DPT-element slice of the G queries in
-//      registers as 16-bit pairs, multiply the cached keys by mixed-precision fma (16-bit
-//      operands, exact products, fp32 accumulation), reduce their partial dot products by
-//      shuffles and scale them by scale * log2 e (FP8: times the Q and K descales);
+//   A  scores, scaled by scale * log2 e (FP8: times the Q and K descales).  FP8: warp w
+//      multiplies tokens 16 w .. 16 w + 15 (the MMA's 16 rows) by the G queries (its
+//      8-wide columns) over four 32-element steps of d, fp32 accumulators.  BF16: TPT
+//      threads per token, each with a DPT-element slice of the G queries in registers,
+//      by mixed-precision fma (bf16 operands, exact products, fp32 accumulation), partial
+//      dot products reduced by shuffles;
 //   B  per head: the tile max, the running max, alpha = 2^(m_old - m_new), p = 2^(s - m_new)
 //      and the running sum (one warp per head, shuffles);
 //   C  O += p V with p rounded to 16 bits (f16 for FP8 caches, bf16 for BF16 ones; the
-//      running sum adds the same rounded values): each thread owns four value columns of
-//      all G heads and a quarter of the tokens, by mixed-precision fma.
+//      running sum adds the same rounded values).  FP8: warp w owns value columns
+//      32 w .. 32 w + 31 of all G heads (the MMA's rows) and all 64 tokens; V is
+//      converted to f16 (exact) in registers.  BF16: each thread owns four value columns
+//      of all G heads and a quarter of the tokens, by mixed-precision fma.
 // Page ids and sequence lengths are read on the device: entries outside the cache make the
 // CTA record DEV_BAD_SEQLENS and write an empty partial instead of reading out of bounds.
 #pragma once
@@ -71,13 +80,17 @@ struct DecCfg {
   static constexpr int NST = 2;
 };
 
+// row stride (16-bit elements) of the FP8 kernel's p [G][DEC_TT]: padded so that the eight
+// heads of one MMA fragment load fall in different banks
+constexpr int DEC_PST = DEC_TT + 8;
+
 // dynamic shared memory of decode_split_kernel<FP8, G>: K and V tiles (double-buffered),
-// the queries, the scores / probabilities, per-head state and the half-sum exchange
+// the scores, per-head state, p in 16 bits, and (BF16 only) the queries and the exchange
+// of the four token groups' partial outputs
 template <bool FP8, int G>
 constexpr int dec_smem_bytes() {
-  return 2 * DecCfg<FP8>::NST * DecCfg<FP8>::TILE_BYTES +
-         (G * DEC_D + DEC_TT * G + 3 * G + G * DEC_D) * 4 +
-         DEC_TT * G * 2;
+  return 2 * DecCfg<FP8>::NST * DecCfg<FP8>::TILE_BYTES + (DEC_TT * G + 3 * G) * 4 +
+         (FP8 ? G * DEC_PST * 2 : 2 * G * DEC_D * 4 + DEC_TT * G * 2);
 }
 
 // split-KV policy: about sixteen CTAs per SM of a 148-SM B200 (several full waves at the
@@ -155,34 +168,60 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t pair) {
   return h2;
 }
 
-// G query heads per kv head; DPT elements of d per thread in phase A
+// d += a b for one warp: a 16 x 32 e4m3 (row-major fragments), b 32 x 8 e4m3 (column-major),
+// d 16 x 8 fp32.  Fragments (r = lane / 4, c = lane % 4): a[0] row r, elements 4c .. 4c+3;
+// a[1] row r + 8, same; a[2], a[3] the same rows, elements 16 + 4c ..; b0 column r,
+// elements 4c .. 4c+3, b1 column r, 16 + 4c ..; d[0], d[1] row r, columns 2c, 2c+1;
+// d[2], d[3] row r + 8
+__device__ __forceinline__ void mma_16832_e4m3(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7},"
+      " {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// d += a b for one warp: a 16 x 16 f16 (a[0] row r, elements 2c, 2c+1; a[1] row r + 8;
+// a[2], a[3] the same rows, elements 2c + 8, 2c + 9), b 16 x 8 f16 (b0 column r, elements
+// 2c, 2c+1; b1 elements 2c + 8, 2c + 9), d as for mma_16832_e4m3
+__device__ __forceinline__ void mma_16816_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                              uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7},"
+      " {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// G query heads per kv head; BF16: DPT elements of d per thread in phase A
 template <bool FP8, int G>
 __global__ void __launch_bounds__(DEC_THREADS)
     decode_split_kernel(const DecodeParams p) {
   using C = DecCfg<FP8>;
   constexpr int DPT = G <= 4 ? 32 : (G == 8 ? 16 : 8);
-  constexpr int TPT = DEC_D / DPT;               // threads per token in phase A
+  constexpr int TPT = DEC_D / DPT;               // threads per token in phase A (BF16)
   constexpr int TOK_PER_PASS = DEC_THREADS / TPT;
   constexpr int PASSES = DEC_TT / TOK_PER_PASS;
   constexpr int SLICE_BYTES = DPT * C::E;        // bytes of a token row per thread in phase A
-  constexpr int LOAD_BYTES = SLICE_BYTES < 16 ? SLICE_BYTES : 16;
-  constexpr int LOAD_ELEMS = LOAD_BYTES / C::E;
+  constexpr int QNT = (G + 7) / 8;               // FP8: 8-wide MMA column tiles of heads
+  static_assert(DEC_THREADS == 128 && DEC_TT == 64, "FP8 phases A and C: four warps of 16 tokens / 32 columns");
 
   extern __shared__ __align__(16) uint8_t dsm[];
   uint8_t* kbuf = dsm;                                   // [NST][TILE_BYTES]
   uint8_t* vbuf = dsm + C::NST * C::TILE_BYTES;          // [NST][TILE_BYTES]
-  float* q_s = reinterpret_cast<float*>(dsm + 2 * C::NST * C::TILE_BYTES);  // [G][128]
-  float* s_s = q_s + G * DEC_D;                          // [DEC_TT][G] scores, then p
+  float* s_s = reinterpret_cast<float*>(dsm + 2 * C::NST * C::TILE_BYTES);  // [DEC_TT][G]
   float* hm = s_s + DEC_TT * G;                          // [G] running max (log2 units)
   float* hl = hm + G;                                    // [G] running sum
   float* ha = hl + G;                                    // [G] alpha of this tile
-  float* ored = ha + G;                                  // [G][128] token-group exchange
-  uint16_t* p16 = reinterpret_cast<uint16_t*>(ored + G * DEC_D);  // [DEC_TT][G] p, 16-bit
+  float* q_s = ha + G;                                   // BF16: [G][128] queries
+  float* ored = q_s + G * DEC_D;                         // BF16: [G][128] token-group exchange
+  // p in 16 bits: FP8 [G][DEC_PST] (head rows, the MMA's A operand), BF16 [DEC_TT][G]
+  uint16_t* p16 = FP8 ? reinterpret_cast<uint16_t*>(q_s) : reinterpret_cast<uint16_t*>(ored + G * DEC_D);
 
   // kv head fastest: the CTAs of one (sequence, split) read the same pages (their head's
   // slice of every token row) at about the same time, which keeps DRAM rows open
   const int g = blockIdx.x, split = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int fr = lane >> 2, fc = lane & 3;  // FP8: MMA fragment row group and column pair
   const int len = p.seq_lens[b];
   const int t_begin = split * p.split_tokens;
   const int t_end = min(len, t_begin + p.split_tokens);
@@ -212,19 +251,36 @@ __global__ void __launch_bounds__(DEC_THREADS)
     return;
   }
 
-  // ---- queries of the G heads as 16-bit pairs (FP8: the e4m3 values in f16, exact; BF16:
-  // the inputs); the scale into log2 units is applied to each finished dot product
+  // ---- queries; the scale into log2 units is applied to each finished dot product.
+  // FP8: the MMA's column fragments of the e4m3 codes in registers (head 8 nt + fr, elements
+  // 32 ks + 4 fc .. + 3 and 32 ks + 16 + 4 fc .. + 3; zero for heads >= G).  BF16: the
+  // bf16 pairs through shared memory.
   float qs = p.qk_scale;
   if constexpr (FP8) qs *= *p.descale_q * *p.descale_k;
-  uint32_t* q_w = reinterpret_cast<uint32_t*>(q_s);  // [G][64] pairs
-  for (int i = tid; i < G * DEC_D / 2; i += DEC_THREADS) {
-    const size_t qi = (static_cast<size_t>(b) * p.Hq + g * G) * DEC_D + 2 * i;
-    if constexpr (FP8) {
-      const uint8_t* qc = static_cast<const uint8_t*>(p.q) + qi;
-      q_w[i] = e4m3x2_to_f16x2(static_cast<uint32_t>(qc[0]) | (static_cast<uint32_t>(qc[1]) << 8));
-    } else {
-      const uint16_t* qb = static_cast<const uint16_t*>(p.q) + qi;
-      q_w[i] = static_cast<uint32_t>(qb[0]) | (static_cast<uint32_t>(qb[1]) << 16);
+  uint32_t qb[QNT][4][2];
+  if constexpr (FP8) {
+    const uint8_t* qc = static_cast<const uint8_t*>(p.q) + (static_cast<size_t>(b) * p.Hq + g * G) * DEC_D;
+#pragma unroll
+    for (int nt = 0; nt < QNT; ++nt) {
+      const int h = 8 * nt + fr;
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t w = 0;
+          if (h < G) {
+            const uint8_t* src = qc + h * DEC_D + 32 * ks + 16 * hf + 4 * fc;
+            w = static_cast<uint32_t>(src[0]) | (static_cast<uint32_t>(src[1]) << 8) |
+                (static_cast<uint32_t>(src[2]) << 16) | (static_cast<uint32_t>(src[3]) << 24);
+          }
+          qb[nt][ks][hf] = w;
+        }
+    }
+  } else {
+    uint32_t* q_w = reinterpret_cast<uint32_t*>(q_s);  // [G][64] pairs
+    for (int i = tid; i < G * DEC_D / 2; i += DEC_THREADS) {
+      const uint16_t* qb16 = static_cast<const uint16_t*>(p.q) + (static_cast<size_t>(b) * p.Hq + g * G) * DEC_D + 2 * i;
+      q_w[i] = static_cast<uint32_t>(qb16[0]) | (static_cast<uint32_t>(qb16[1]) << 16);
     }
   }
   if (tid < G) {
@@ -261,17 +317,22 @@ __global__ void __launch_bounds__(DEC_THREADS)
   }
   __syncthreads();  // q_s, hm, hl
 
-  // phase A mapping and the query slice in registers (16-bit pairs)
+  // BF16 phase A mapping and the query slice in registers (bf16 pairs)
   const int a_tok = tid / TPT, a_part = tid % TPT;
-  uint32_t qr[G][DPT / 2];
+  uint32_t qr[FP8 ? 1 : G][FP8 ? 1 : DPT / 2];
+  if constexpr (!FP8) {
+    const uint32_t* q_w = reinterpret_cast<const uint32_t*>(q_s);
 #pragma unroll
-  for (int h = 0; h < G; ++h)
+    for (int h = 0; h < G; ++h)
 #pragma unroll
-    for (int e = 0; e < DPT / 2; ++e) qr[h][e] = q_w[h * (DEC_D / 2) + a_part * (DPT / 2) + e];
-  // phase C mapping: value columns 4 lane .. 4 lane + 3, tokens j = warp (mod 4)
-  float acc[G][4];
+      for (int e = 0; e < DPT / 2; ++e) qr[h][e] = q_w[h * (DEC_D / 2) + a_part * (DPT / 2) + e];
+  }
+  // phase C accumulators.  FP8: MMA tile i (of four) of warp w, fragment element e: head
+  // fr + 8 (e >> 1), value column 32 w + 8 fc + 4 (e & 1) + i.  BF16: value columns
+  // 4 lane .. 4 lane + 3 of head h, tokens j = warp (mod 4).
+  float acc[FP8 ? 4 : G][4];
 #pragma unroll
-  for (int h = 0; h < G; ++h) acc[h][0] = acc[h][1] = acc[h][2] = acc[h][3] = 0.0f;
+  for (int h = 0; h < (FP8 ? 4 : G); ++h) acc[h][0] = acc[h][1] = acc[h][2] = acc[h][3] = 0.0f;
 
   for (int it = 0; it < n_tiles; ++it) {
     const int buf = it % C::NST;
@@ -285,55 +346,57 @@ __global__ void __launch_bounds__(DEC_THREADS)
     const uint8_t* vt = vbuf + buf * C::TILE_BYTES;
 
     // ---- A: scores of the tile
+    if constexpr (FP8) {
+      // warp w: tokens 16 w .. 16 w + 15 as the MMA's rows, the heads as its columns
+      const int j0 = 16 * warp;
+      float sc[QNT][4];
 #pragma unroll
-    for (int ps = 0; ps < PASSES; ++ps) {
-      const int j = ps * TOK_PER_PASS + a_tok;
-      float part[G];
+      for (int nt = 0; nt < QNT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.0f;
 #pragma unroll
-      for (int h = 0; h < G; ++h) part[h] = 0.0f;
+      for (int ks = 0; ks < 4; ++ks) {
+        // elements 32 ks + 4 fc (chunk 2 ks) and 32 ks + 16 + 4 fc (chunk 2 ks + 1)
+        uint32_t af[4];
+        af[0] = *reinterpret_cast<const uint32_t*>(kt + dec_chunk_off<true>(j0 + fr, 2 * ks) + 4 * fc);
+        af[1] = *reinterpret_cast<const uint32_t*>(kt + dec_chunk_off<true>(j0 + fr + 8, 2 * ks) + 4 * fc);
+        af[2] = *reinterpret_cast<const uint32_t*>(kt + dec_chunk_off<true>(j0 + fr, 2 * ks + 1) + 4 * fc);
+        af[3] = *reinterpret_cast<const uint32_t*>(kt + dec_chunk_off<true>(j0 + fr + 8, 2 * ks + 1) + 4 * fc);
 #pragma unroll
-      for (int lb = 0; lb < SLICE_BYTES; lb += LOAD_BYTES) {
-        // bytes [a_part * SLICE_BYTES + lb, + LOAD_BYTES) of row j
-        const int byte = a_part * SLICE_BYTES + lb;
-        const uint8_t* src = kt + dec_chunk_off<FP8>(j, byte >> 4) + (byte & 15);
-        // the loaded elements as 16-bit pairs (FP8: converted to f16, exact)
-        uint32_t kw[8];
-        if constexpr (LOAD_BYTES == 16) {
-          const uint4 w = *reinterpret_cast<const uint4*>(src);
-          if constexpr (FP8) {
-            const uint32_t u[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              kw[2 * i] = e4m3x2_to_f16x2(u[i]);
-              kw[2 * i + 1] = e4m3x2_to_f16x2(u[i] >> 16);
-            }
-          } else {
-            kw[0] = w.x;
-            kw[1] = w.y;
-            kw[2] = w.z;
-            kw[3] = w.w;
-          }
-        } else {
-          const uint2 w = *reinterpret_cast<const uint2*>(src);  // FP8, 8 elements
-          kw[0] = e4m3x2_to_f16x2(w.x);
-          kw[1] = e4m3x2_to_f16x2(w.x >> 16);
-          kw[2] = e4m3x2_to_f16x2(w.y);
-          kw[3] = e4m3x2_to_f16x2(w.y >> 16);
-        }
-#pragma unroll
-        for (int e = 0; e < LOAD_ELEMS / 2; ++e)
-#pragma unroll
-          for (int h = 0; h < G; ++h)
-            part[h] = fma2_mixed<!FP8>(qr[h][lb / (2 * C::E) + e], kw[e], part[h]);
+        for (int nt = 0; nt < QNT; ++nt) mma_16832_e4m3(sc[nt], af, qb[nt][ks][0], qb[nt][ks][1]);
       }
 #pragma unroll
-      for (int off = 1; off < TPT; off <<= 1)
+      for (int nt = 0; nt < QNT; ++nt)
 #pragma unroll
-        for (int h = 0; h < G; ++h) part[h] += __shfl_xor_sync(0xffffffffu, part[h], off);
-      if (a_part == 0) {
-        const bool in = t0 + j < t_end;
+        for (int e = 0; e < 4; ++e) {
+          const int j = j0 + fr + 8 * (e >> 1), h = 8 * nt + 2 * fc + (e & 1);
+          if (h < G) s_s[j * G + h] = t0 + j < t_end ? sc[nt][e] * qs : -INFINITY;
+        }
+    } else {
 #pragma unroll
-        for (int h = 0; h < G; ++h) s_s[j * G + h] = in ? part[h] * qs : -INFINITY;
+      for (int ps = 0; ps < PASSES; ++ps) {
+        const int j = ps * TOK_PER_PASS + a_tok;
+        float part[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) part[h] = 0.0f;
+#pragma unroll
+        for (int lb = 0; lb < SLICE_BYTES; lb += 16) {
+          // bytes [a_part * SLICE_BYTES + lb, + 16) of row j: eight bf16 as pairs
+          const int byte = a_part * SLICE_BYTES + lb;
+          const uint4 w = *reinterpret_cast<const uint4*>(kt + dec_chunk_off<false>(j, byte >> 4));
+          const uint32_t kw[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+#pragma unroll
+            for (int h = 0; h < G; ++h) part[h] = fma2_mixed<true>(qr[h][lb / 4 + e], kw[e], part[h]);
+        }
+#pragma unroll
+        for (int off = 1; off < TPT; off <<= 1)
+#pragma unroll
+          for (int h = 0; h < G; ++h) part[h] += __shfl_xor_sync(0xffffffffu, part[h], off);
+        if (a_part == 0) {
+          const bool in = t0 + j < t_end;
+#pragma unroll
+          for (int h = 0; h < G; ++h) s_s[j * G + h] = in ? part[h] * qs : -INFINITY;
+        }
       }
     }
     __syncthreads();
@@ -355,14 +418,16 @@ __global__ void __launch_bounds__(DEC_THREADS)
         r1 = __half_as_ushort(__float2half_rn(p1));
         p0 = __half2float(__ushort_as_half(r0));
         p1 = __half2float(__ushort_as_half(r1));
+        p16[h * DEC_PST + lane] = r0;
+        p16[h * DEC_PST + lane + 32] = r1;
       } else {
         r0 = __bfloat16_as_ushort(__float2bfloat16_rn(p0));
         r1 = __bfloat16_as_ushort(__float2bfloat16_rn(p1));
         p0 = __bfloat162float(__ushort_as_bfloat16(r0));
         p1 = __bfloat162float(__ushort_as_bfloat16(r1));
+        p16[lane * G + h] = r0;
+        p16[(lane + 32) * G + h] = r1;
       }
-      p16[lane * G + h] = r0;
-      p16[(lane + 32) * G + h] = r1;
       float ls = p0 + p1;
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, off);
@@ -376,66 +441,108 @@ __global__ void __launch_bounds__(DEC_THREADS)
     }
     __syncthreads();
 
-    // ---- C: O += p V; 4 value columns x G heads per thread, tokens j = warp (mod 4), by
-    // mixed-precision fma (16-bit p and v, fp32 accumulators)
+    // ---- C: O += p V
+    if constexpr (FP8) {
+      // warp w: value columns 32 w .. 32 w + 31 as four 8-wide MMA tiles (column n of tile
+      // i = value column 32 w + 4 n + i, so each lane's 32-bit read of a token row feeds
+      // all four), the heads as the MMA's rows, the tile's tokens in four 16-token steps
+      const float a_lo = fr < G ? ha[fr] : 1.0f, a_hi = fr + 8 < G ? ha[fr + 8] : 1.0f;
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const float a = ha[h];
+      for (int i = 0; i < 4; ++i) {
+        acc[i][0] *= a_lo;
+        acc[i][1] *= a_lo;
+        acc[i][2] *= a_hi;
+        acc[i][3] *= a_hi;
+      }
+      const int vb = 32 * warp + 4 * fr;  // byte (= column) of this lane's value read
+      const uint32_t* pw = reinterpret_cast<const uint32_t*>(p16);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) acc[h][c] *= a;
-    }
+      for (int ks = 0; ks < 4; ++ks) {
+        const int k0 = 16 * ks + 2 * fc;  // this lane's tokens k0, k0 + 1, k0 + 8, k0 + 9
+        uint32_t af[4];
+        af[0] = fr < G ? pw[(fr * DEC_PST + k0) >> 1] : 0u;
+        af[1] = fr + 8 < G ? pw[((fr + 8) * DEC_PST + k0) >> 1] : 0u;
+        af[2] = fr < G ? pw[(fr * DEC_PST + k0 + 8) >> 1] : 0u;
+        af[3] = fr + 8 < G ? pw[((fr + 8) * DEC_PST + k0 + 8) >> 1] : 0u;
+        const uint32_t w0 = *reinterpret_cast<const uint32_t*>(vt + dec_chunk_off<true>(k0, vb >> 4) + (vb & 15));
+        const uint32_t w1 = *reinterpret_cast<const uint32_t*>(vt + dec_chunk_off<true>(k0 + 1, vb >> 4) + (vb & 15));
+        const uint32_t w2 = *reinterpret_cast<const uint32_t*>(vt + dec_chunk_off<true>(k0 + 8, vb >> 4) + (vb & 15));
+        const uint32_t w3 = *reinterpret_cast<const uint32_t*>(vt + dec_chunk_off<true>(k0 + 9, vb >> 4) + (vb & 15));
+        // byte i of the two tokens of a pair, side by side: (k0, k0 + 1) and (k0 + 8, k0 + 9)
+        const uint32_t lo01 = __byte_perm(w0, w1, 0x5140), hi01 = __byte_perm(w0, w1, 0x7362);
+        const uint32_t lo89 = __byte_perm(w2, w3, 0x5140), hi89 = __byte_perm(w2, w3, 0x7362);
+        mma_16816_f16(acc[0], af, e4m3x2_to_f16x2(lo01), e4m3x2_to_f16x2(lo89));
+        mma_16816_f16(acc[1], af, e4m3x2_to_f16x2(lo01 >> 16), e4m3x2_to_f16x2(lo89 >> 16));
+        mma_16816_f16(acc[2], af, e4m3x2_to_f16x2(hi01), e4m3x2_to_f16x2(hi89));
+        mma_16816_f16(acc[3], af, e4m3x2_to_f16x2(hi01 >> 16), e4m3x2_to_f16x2(hi89 >> 16));
+      }
+    } else {
+      // 4 value columns x G heads per thread, tokens j = warp (mod 4), by mixed-precision
+      // fma (bf16 p and v, fp32 accumulators)
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float a = ha[h];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[h][c] *= a;
+      }
 #pragma unroll 4
-    for (int j = warp; j < DEC_TT; j += 4) {
-      uint32_t v01, v23;
-      if constexpr (FP8) {
-        const uint32_t codes = *reinterpret_cast<const uint32_t*>(
-            vt + dec_chunk_off<true>(j, (4 * lane) >> 4) + ((4 * lane) & 15));
-        v01 = e4m3x2_to_f16x2(codes);
-        v23 = e4m3x2_to_f16x2(codes >> 16);
-      } else {
+      for (int j = warp; j < DEC_TT; j += 4) {
         const uint2 w = *reinterpret_cast<const uint2*>(
             vt + dec_chunk_off<false>(j, (8 * lane) >> 4) + ((8 * lane) & 15));
-        v01 = w.x;
-        v23 = w.y;
-      }
-      uint32_t pw[(G + 1) / 2];
-      if constexpr (G == 1) {
-        pw[0] = p16[j];
-      } else {
+        uint32_t pw[(G + 1) / 2];
+        if constexpr (G == 1) {
+          pw[0] = p16[j];
+        } else {
 #pragma unroll
-        for (int i = 0; i < G / 2; ++i) pw[i] = reinterpret_cast<const uint32_t*>(p16 + j * G)[i];
-      }
+          for (int i = 0; i < G / 2; ++i) pw[i] = reinterpret_cast<const uint32_t*>(p16 + j * G)[i];
+        }
 #pragma unroll
-      for (int h = 0; h < G; ++h)
-        pv4_mixed<!FP8>(static_cast<uint16_t>(pw[h / 2] >> (16 * (h & 1))), v01, v23, acc[h]);
+        for (int h = 0; h < G; ++h)
+          pv4_mixed<true>(static_cast<uint16_t>(pw[h / 2] >> (16 * (h & 1))), w.x, w.y, acc[h]);
+      }
     }
     __syncthreads();  // this buffer is refilled next iteration; s_s is rewritten
   }
 
-  // ---- the four token groups (warps), then the partial output of this range
-#pragma unroll 1
-  for (int w = 1; w < 4; ++w) {
-    if (warp == w) {
+  // ---- the partial output of this range
+  if constexpr (FP8) {
+    // lane (fr, fc) of warp w holds columns 32 w + 8 fc .. + 7 of heads fr and fr + 8
 #pragma unroll
-      for (int h = 0; h < G; ++h)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float* dst = ored + h * DEC_D + 4 * lane + c;
-          *dst = (w == 1 ? 0.0f : *dst) + acc[h][c];
-        }
+    for (int hh = 0; hh < 2; ++hh) {
+      const int h = fr + 8 * hh;
+      if (h < G) {
+        float* po = p.part_o + (pidx + static_cast<size_t>(h) * p.n_splits) * DEC_D + 32 * warp + 8 * fc;
+        *reinterpret_cast<float4*>(po) = make_float4(acc[0][2 * hh], acc[1][2 * hh], acc[2][2 * hh], acc[3][2 * hh]);
+        *reinterpret_cast<float4*>(po + 4) =
+            make_float4(acc[0][2 * hh + 1], acc[1][2 * hh + 1], acc[2][2 * hh + 1], acc[3][2 * hh + 1]);
+      }
     }
-    __syncthreads();
-  }
-  if (warp == 0) {
+  } else {
+    // the four token groups (warps) first
+#pragma unroll 1
+    for (int w = 1; w < 4; ++w) {
+      if (warp == w) {
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      float* po = p.part_o + (pidx + static_cast<size_t>(h) * p.n_splits) * DEC_D + 4 * lane;
-      float4 r;
-      r.x = acc[h][0] + ored[h * DEC_D + 4 * lane + 0];
-      r.y = acc[h][1] + ored[h * DEC_D + 4 * lane + 1];
-      r.z = acc[h][2] + ored[h * DEC_D + 4 * lane + 2];
-      r.w = acc[h][3] + ored[h * DEC_D + 4 * lane + 3];
-      *reinterpret_cast<float4*>(po) = r;
+        for (int h = 0; h < G; ++h)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            float* dst = ored + h * DEC_D + 4 * lane + c;
+            *dst = (w == 1 ? 0.0f : *dst) + acc[h][c];
+          }
+      }
+      __syncthreads();
+    }
+    if (warp == 0) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float* po = p.part_o + (pidx + static_cast<size_t>(h) * p.n_splits) * DEC_D + 4 * lane;
+        float4 r;
+        r.x = acc[h][0] + ored[h * DEC_D + 4 * lane + 0];
+        r.y = acc[h][1] + ored[h * DEC_D + 4 * lane + 1];
+        r.z = acc[h][2] + ored[h * DEC_D + 4 * lane + 2];
+        r.w = acc[h][3] + ored[h * DEC_D + 4 * lane + 3];
+        *reinterpret_cast<float4*>(po) = r;
+      }
     }
   }
   if (tid < G) {
