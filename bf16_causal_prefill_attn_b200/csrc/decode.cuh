@@ -9,29 +9,26 @@
 // The operation reads every cached K and V byte once and does ~2 G flops per byte (G =
 // Hq / Hkv query heads share a kv head): HBM-bound, with the cache streamed through shared
 // memory by 16-byte asynchronous copies.  What has to keep up with the copies is the
-// instruction issue of the contractions: with e4m3 caches a CUDA-core loop (convert, then
-// one fma per product) issues ~4x more instructions per cached byte than with bf16 ones,
-// so the FP8 kernel hands both contractions to warp-level tensor-core MMAs
-// (mma.sync m16n8k32 e4m3 for the scores, m16n8k16 f16 for PV: each replaces 128 or 64
-// fma instructions of a warp); the MMA shapes are not the point here, the issue slots are.
+// instruction issue of the two contractions: a CUDA-core loop needs one fma per product
+// (plus conversions for e4m3), which held e4m3 caches to ~3 TB/s, so both contractions are
+// warp-level tensor-core MMAs (mma.sync: scores m16n8k32 e4m3 or m16n8k16 bf16, PV
+// m16n8k16 f16 or bf16; each replaces 64-128 fma instructions of a warp).  The tiles are
+// thin (the G heads are the MMA's 8 or 16 rows or columns): issue slots are the point,
+// not the tensor throughput.
 //
 // Split-KV: CTA (g, split, b) takes one kv head g of sequence b, all G query heads that read
 // it, and a contiguous range of its tokens; it writes the unnormalised partial output and
 // the (max, sum) of its range, and decode_combine_kernel merges the ranges.  Per 64-token
 // tile (NST tiles in flight):
-//   A  scores, scaled by scale * log2 e (FP8: times the Q and K descales).  FP8: warp w
-//      multiplies tokens 16 w .. 16 w + 15 (the MMA's 16 rows) by the G queries (its
-//      8-wide columns) over four 32-element steps of d, fp32 accumulators.  BF16: TPT
-//      threads per token, each with a DPT-element slice of the G queries in registers,
-//      by mixed-precision fma (bf16 operands, exact products, fp32 accumulation), partial
-//      dot products reduced by shuffles;
+//   A  scores: warp w multiplies tokens 16 w .. 16 w + 15 (the MMA's rows) by the G
+//      queries (its 8-wide columns, query fragments in registers), fp32 accumulators,
+//      scaled by scale * log2 e (FP8: times the Q and K descales);
 //   B  per head: the tile max, the running max, alpha = 2^(m_old - m_new), p = 2^(s - m_new)
 //      and the running sum (one warp per head, shuffles);
 //   C  O += p V with p rounded to 16 bits (f16 for FP8 caches, bf16 for BF16 ones; the
-//      running sum adds the same rounded values).  FP8: warp w owns value columns
-//      32 w .. 32 w + 31 of all G heads (the MMA's rows) and all 64 tokens; V is
-//      converted to f16 (exact) in registers.  BF16: each thread owns four value columns
-//      of all G heads and a quarter of the tokens, by mixed-precision fma.
+//      running sum adds the same rounded values): warp w owns value columns 32 w .. 32 w +
+//      31 of all G heads (the heads are the MMA's rows) and all 64 tokens; e4m3 values are
+//      converted to f16 (exact) in registers.
 // Page ids and sequence lengths are read on the device: entries outside the cache make the
 // CTA record DEV_BAD_SEQLENS and write an empty partial instead of reading out of bounds.
 #pragma once
@@ -85,12 +82,10 @@ struct DecCfg {
 constexpr int DEC_PST = DEC_TT + 8;
 
 // dynamic shared memory of decode_split_kernel<FP8, G>: K and V tiles (double-buffered),
-// the scores, per-head state, p in 16 bits, and (BF16 only) the queries and the exchange
-// of the four token groups' partial outputs
+// the scores, per-head state and p in 16 bits
 template <bool FP8, int G>
 constexpr int dec_smem_bytes() {
-  return 2 * DecCfg<FP8>::NST * DecCfg<FP8>::TILE_BYTES + (DEC_TT * G + 3 * G) * 4 +
-         (FP8 ? G * DEC_PST * 2 : 2 * G * DEC_D * 4 + DEC_TT * G * 2);
+  return 2 * DecCfg<FP8>::NST * DecCfg<FP8>::TILE_BYTES + (DEC_TT * G + 3 * G) * 4 + G * DEC_PST * 2;
 }
 
 // split-KV policy: about sixteen CTAs per SM of a 148-SM B200 (several full waves at the
@@ -109,8 +104,9 @@ inline int dec_split_tokens(int max_seqlen, int n_splits) {
   return ((tiles + n_splits - 1) / n_splits) * DEC_TT;
 }
 
-// 16-byte chunk c of token row j of a tile, XOR-swizzled so that the reads of phase A (8 or
-// more tokens x consecutive chunks) and C (one row, consecutive words) spread over banks
+// 16-byte chunk c of token row j of a tile, XOR-swizzled so that the MMA fragment reads
+// spread over the banks: phase A reads one chunk of eight consecutive rows, phase C the same
+// one or two chunks of four rows two apart
 template <bool FP8>
 __device__ __forceinline__ int dec_chunk_off(int j, int c) {
   using C = DecCfg<FP8>;
@@ -126,39 +122,6 @@ __device__ __forceinline__ void cp_async_commit() {
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-// acc + a.lo * b.lo + a.hi * b.hi for two pairs of 16-bit floats (f16, or bf16 with BF),
-// each product exact in fp32 and each step rounded once (mixed-precision fma of sm_100)
-template <bool BF>
-__device__ __forceinline__ float fma2_mixed(uint32_t a, uint32_t b, float acc) {
-  float d;
-  if constexpr (BF) {
-    asm("{.reg .b16 al, ah, bl, bh; .reg .f32 t; mov.b32 {al, ah}, %1; mov.b32 {bl, bh}, %2;"
-        " fma.rn.f32.bf16 t, al, bl, %3; fma.rn.f32.bf16 %0, ah, bh, t;}"
-        : "=f"(d) : "r"(a), "r"(b), "f"(acc));
-  } else {
-    asm("{.reg .b16 al, ah, bl, bh; .reg .f32 t; mov.b32 {al, ah}, %1; mov.b32 {bl, bh}, %2;"
-        " fma.rn.f32.f16 t, al, bl, %3; fma.rn.f32.f16 %0, ah, bh, t;}"
-        : "=f"(d) : "r"(a), "r"(b), "f"(acc));
-  }
-  return d;
-}
-
-// a[c] += p * v_c for the four 16-bit values of v01, v23 (f16, or bf16 with BF); p 16-bit
-template <bool BF>
-__device__ __forceinline__ void pv4_mixed(uint16_t p, uint32_t v01, uint32_t v23, float* a) {
-  if constexpr (BF) {
-    asm("{.reg .b16 x0, x1, x2, x3; mov.b32 {x0, x1}, %4; mov.b32 {x2, x3}, %5;"
-        " fma.rn.f32.bf16 %0, %6, x0, %0; fma.rn.f32.bf16 %1, %6, x1, %1;"
-        " fma.rn.f32.bf16 %2, %6, x2, %2; fma.rn.f32.bf16 %3, %6, x3, %3;}"
-        : "+f"(a[0]), "+f"(a[1]), "+f"(a[2]), "+f"(a[3]) : "r"(v01), "r"(v23), "h"(p));
-  } else {
-    asm("{.reg .b16 x0, x1, x2, x3; mov.b32 {x0, x1}, %4; mov.b32 {x2, x3}, %5;"
-        " fma.rn.f32.f16 %0, %6, x0, %0; fma.rn.f32.f16 %1, %6, x1, %1;"
-        " fma.rn.f32.f16 %2, %6, x2, %2; fma.rn.f32.f16 %3, %6, x3, %3;}"
-        : "+f"(a[0]), "+f"(a[1]), "+f"(a[2]), "+f"(a[3]) : "r"(v01), "r"(v23), "h"(p));
-  }
 }
 
 // two e4m3 codes (low 16 bits) -> f16x2, exact
@@ -181,29 +144,33 @@ __device__ __forceinline__ void mma_16832_e4m3(float (&d)[4], const uint32_t (&a
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// d += a b for one warp: a 16 x 16 f16 (a[0] row r, elements 2c, 2c+1; a[1] row r + 8;
-// a[2], a[3] the same rows, elements 2c + 8, 2c + 9), b 16 x 8 f16 (b0 column r, elements
-// 2c, 2c+1; b1 elements 2c + 8, 2c + 9), d as for mma_16832_e4m3
-__device__ __forceinline__ void mma_16816_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                              uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7},"
-      " {%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+// d += a b for one warp: a 16 x 16 f16, or bf16 with BF (a[0] row r, elements 2c, 2c+1;
+// a[1] row r + 8; a[2], a[3] the same rows, elements 2c + 8, 2c + 9), b 16 x 8 of the same
+// type (b0 column r, elements 2c, 2c+1; b1 elements 2c + 8, 2c + 9), d as for
+// mma_16832_e4m3
+template <bool BF>
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  if constexpr (BF) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7},"
+        " {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  } else {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7},"
+        " {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
 }
 
-// G query heads per kv head; BF16: DPT elements of d per thread in phase A
+// G query heads per kv head
 template <bool FP8, int G>
 __global__ void __launch_bounds__(DEC_THREADS)
     decode_split_kernel(const DecodeParams p) {
   using C = DecCfg<FP8>;
-  constexpr int DPT = G <= 4 ? 32 : (G == 8 ? 16 : 8);
-  constexpr int TPT = DEC_D / DPT;               // threads per token in phase A (BF16)
-  constexpr int TOK_PER_PASS = DEC_THREADS / TPT;
-  constexpr int PASSES = DEC_TT / TOK_PER_PASS;
-  constexpr int SLICE_BYTES = DPT * C::E;        // bytes of a token row per thread in phase A
-  constexpr int QNT = (G + 7) / 8;               // FP8: 8-wide MMA column tiles of heads
-  static_assert(DEC_THREADS == 128 && DEC_TT == 64, "FP8 phases A and C: four warps of 16 tokens / 32 columns");
+  constexpr int QNT = (G + 7) / 8;   // 8-wide MMA column tiles of heads in phase A
+  constexpr int KS = FP8 ? 4 : 8;    // phase A steps of d: 32 e4m3 or 16 bf16 elements (32 bytes)
+  static_assert(DEC_THREADS == 128 && DEC_TT == 64, "phases A and C: four warps of 16 tokens / 32 columns");
 
   extern __shared__ __align__(16) uint8_t dsm[];
   uint8_t* kbuf = dsm;                                   // [NST][TILE_BYTES]
@@ -212,16 +179,13 @@ __global__ void __launch_bounds__(DEC_THREADS)
   float* hm = s_s + DEC_TT * G;                          // [G] running max (log2 units)
   float* hl = hm + G;                                    // [G] running sum
   float* ha = hl + G;                                    // [G] alpha of this tile
-  float* q_s = ha + G;                                   // BF16: [G][128] queries
-  float* ored = q_s + G * DEC_D;                         // BF16: [G][128] token-group exchange
-  // p in 16 bits: FP8 [G][DEC_PST] (head rows, the MMA's A operand), BF16 [DEC_TT][G]
-  uint16_t* p16 = FP8 ? reinterpret_cast<uint16_t*>(q_s) : reinterpret_cast<uint16_t*>(ored + G * DEC_D);
+  uint16_t* p16 = reinterpret_cast<uint16_t*>(ha + G);   // [G][DEC_PST] p, 16-bit
 
   // kv head fastest: the CTAs of one (sequence, split) read the same pages (their head's
   // slice of every token row) at about the same time, which keeps DRAM rows open
   const int g = blockIdx.x, split = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int fr = lane >> 2, fc = lane & 3;  // FP8: MMA fragment row group and column pair
+  const int fr = lane >> 2, fc = lane & 3;  // MMA fragment row group and column pair
   const int len = p.seq_lens[b];
   const int t_begin = split * p.split_tokens;
   const int t_end = min(len, t_begin + p.split_tokens);
@@ -251,36 +215,29 @@ __global__ void __launch_bounds__(DEC_THREADS)
     return;
   }
 
-  // ---- queries; the scale into log2 units is applied to each finished dot product.
-  // FP8: the MMA's column fragments of the e4m3 codes in registers (head 8 nt + fr, elements
-  // 32 ks + 4 fc .. + 3 and 32 ks + 16 + 4 fc .. + 3; zero for heads >= G).  BF16: the
-  // bf16 pairs through shared memory.
+  // ---- the queries as the score MMA's column fragments, in registers: head 8 nt + fr,
+  // bytes 32 ks + 4 fc .. + 3 and 32 ks + 16 + 4 fc .. + 3 of its row (zero for heads >= G).
+  // The scale into log2 units is applied to each finished dot product.
   float qs = p.qk_scale;
   if constexpr (FP8) qs *= *p.descale_q * *p.descale_k;
-  uint32_t qb[QNT][4][2];
-  if constexpr (FP8) {
-    const uint8_t* qc = static_cast<const uint8_t*>(p.q) + (static_cast<size_t>(b) * p.Hq + g * G) * DEC_D;
+  uint32_t qb[QNT][KS][2];
+  {
+    const uint8_t* qrow = static_cast<const uint8_t*>(p.q) + (static_cast<size_t>(b) * p.Hq + g * G) * C::ROW;
 #pragma unroll
     for (int nt = 0; nt < QNT; ++nt) {
       const int h = 8 * nt + fr;
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks)
+      for (int ks = 0; ks < KS; ++ks)
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
           uint32_t w = 0;
           if (h < G) {
-            const uint8_t* src = qc + h * DEC_D + 32 * ks + 16 * hf + 4 * fc;
+            const uint8_t* src = qrow + h * C::ROW + 32 * ks + 16 * hf + 4 * fc;
             w = static_cast<uint32_t>(src[0]) | (static_cast<uint32_t>(src[1]) << 8) |
                 (static_cast<uint32_t>(src[2]) << 16) | (static_cast<uint32_t>(src[3]) << 24);
           }
           qb[nt][ks][hf] = w;
         }
-    }
-  } else {
-    uint32_t* q_w = reinterpret_cast<uint32_t*>(q_s);  // [G][64] pairs
-    for (int i = tid; i < G * DEC_D / 2; i += DEC_THREADS) {
-      const uint16_t* qb16 = static_cast<const uint16_t*>(p.q) + (static_cast<size_t>(b) * p.Hq + g * G) * DEC_D + 2 * i;
-      q_w[i] = static_cast<uint32_t>(qb16[0]) | (static_cast<uint32_t>(qb16[1]) << 16);
     }
   }
   if (tid < G) {
@@ -315,24 +272,13 @@ __global__ void __launch_bounds__(DEC_THREADS)
     if (st < n_tiles) load_tile(t_begin + st * DEC_TT, st);
     else cp_async_commit();
   }
-  __syncthreads();  // q_s, hm, hl
+  __syncthreads();  // hm, hl
 
-  // BF16 phase A mapping and the query slice in registers (bf16 pairs)
-  const int a_tok = tid / TPT, a_part = tid % TPT;
-  uint32_t qr[FP8 ? 1 : G][FP8 ? 1 : DPT / 2];
-  if constexpr (!FP8) {
-    const uint32_t* q_w = reinterpret_cast<const uint32_t*>(q_s);
+  // phase C accumulators: MMA tile i (of four) of warp w, fragment element e: head
+  // fr + 8 (e >> 1), value column 32 w + 8 fc + 4 (e & 1) + i
+  float acc[4][4];
 #pragma unroll
-    for (int h = 0; h < G; ++h)
-#pragma unroll
-      for (int e = 0; e < DPT / 2; ++e) qr[h][e] = q_w[h * (DEC_D / 2) + a_part * (DPT / 2) + e];
-  }
-  // phase C accumulators.  FP8: MMA tile i (of four) of warp w, fragment element e: head
-  // fr + 8 (e >> 1), value column 32 w + 8 fc + 4 (e & 1) + i.  BF16: value columns
-  // 4 lane .. 4 lane + 3 of head h, tokens j = warp (mod 4).
-  float acc[FP8 ? 4 : G][4];
-#pragma unroll
-  for (int h = 0; h < (FP8 ? 4 : G); ++h) acc[h][0] = acc[h][1] = acc[h][2] = acc[h][3] = 0.0f;
+  for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.0f;
 
   for (int it = 0; it < n_tiles; ++it) {
     const int buf = it % C::NST;
@@ -345,23 +291,25 @@ __global__ void __launch_bounds__(DEC_THREADS)
     const uint8_t* kt = kbuf + buf * C::TILE_BYTES;
     const uint8_t* vt = vbuf + buf * C::TILE_BYTES;
 
-    // ---- A: scores of the tile
-    if constexpr (FP8) {
-      // warp w: tokens 16 w .. 16 w + 15 as the MMA's rows, the heads as its columns
+    // ---- A: scores of the tile; warp w: tokens 16 w .. 16 w + 15 as the MMA's rows, the
+    // heads as its columns; step ks covers bytes 32 ks .. 32 ks + 31 of the rows
+    {
       const int j0 = 16 * warp;
       float sc[QNT][4];
 #pragma unroll
       for (int nt = 0; nt < QNT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.0f;
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
-        // elements 32 ks + 4 fc (chunk 2 ks) and 32 ks + 16 + 4 fc (chunk 2 ks + 1)
+      for (int ks = 0; ks < KS; ++ks) {
         uint32_t af[4];
-        af[0] = *reinterpret_cast<const uint32_t*>(kt + dec_chunk_off<true>(j0 + fr, 2 * ks) + 4 * fc);
-        af[1] = *reinterpret_cast<const uint32_t*>(kt + dec_chunk_off<true>(j0 + fr + 8, 2 * ks) + 4 * fc);
-        af[2] = *reinterpret_cast<const uint32_t*>(kt + dec_chunk_off<true>(j0 + fr, 2 * ks + 1) + 4 * fc);
-        af[3] = *reinterpret_cast<const uint32_t*>(kt + dec_chunk_off<true>(j0 + fr + 8, 2 * ks + 1) + 4 * fc);
+        af[0] = *reinterpret_cast<const uint32_t*>(kt + dec_chunk_off<FP8>(j0 + fr, 2 * ks) + 4 * fc);
+        af[1] = *reinterpret_cast<const uint32_t*>(kt + dec_chunk_off<FP8>(j0 + fr + 8, 2 * ks) + 4 * fc);
+        af[2] = *reinterpret_cast<const uint32_t*>(kt + dec_chunk_off<FP8>(j0 + fr, 2 * ks + 1) + 4 * fc);
+        af[3] = *reinterpret_cast<const uint32_t*>(kt + dec_chunk_off<FP8>(j0 + fr + 8, 2 * ks + 1) + 4 * fc);
 #pragma unroll
-        for (int nt = 0; nt < QNT; ++nt) mma_16832_e4m3(sc[nt], af, qb[nt][ks][0], qb[nt][ks][1]);
+        for (int nt = 0; nt < QNT; ++nt) {
+          if constexpr (FP8) mma_16832_e4m3(sc[nt], af, qb[nt][ks][0], qb[nt][ks][1]);
+          else mma_16816<true>(sc[nt], af, qb[nt][ks][0], qb[nt][ks][1]);
+        }
       }
 #pragma unroll
       for (int nt = 0; nt < QNT; ++nt)
@@ -370,34 +318,6 @@ __global__ void __launch_bounds__(DEC_THREADS)
           const int j = j0 + fr + 8 * (e >> 1), h = 8 * nt + 2 * fc + (e & 1);
           if (h < G) s_s[j * G + h] = t0 + j < t_end ? sc[nt][e] * qs : -INFINITY;
         }
-    } else {
-#pragma unroll
-      for (int ps = 0; ps < PASSES; ++ps) {
-        const int j = ps * TOK_PER_PASS + a_tok;
-        float part[G];
-#pragma unroll
-        for (int h = 0; h < G; ++h) part[h] = 0.0f;
-#pragma unroll
-        for (int lb = 0; lb < SLICE_BYTES; lb += 16) {
-          // bytes [a_part * SLICE_BYTES + lb, + 16) of row j: eight bf16 as pairs
-          const int byte = a_part * SLICE_BYTES + lb;
-          const uint4 w = *reinterpret_cast<const uint4*>(kt + dec_chunk_off<false>(j, byte >> 4));
-          const uint32_t kw[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-#pragma unroll
-            for (int h = 0; h < G; ++h) part[h] = fma2_mixed<true>(qr[h][lb / 4 + e], kw[e], part[h]);
-        }
-#pragma unroll
-        for (int off = 1; off < TPT; off <<= 1)
-#pragma unroll
-          for (int h = 0; h < G; ++h) part[h] += __shfl_xor_sync(0xffffffffu, part[h], off);
-        if (a_part == 0) {
-          const bool in = t0 + j < t_end;
-#pragma unroll
-          for (int h = 0; h < G; ++h) s_s[j * G + h] = in ? part[h] * qs : -INFINITY;
-        }
-      }
     }
     __syncthreads();
 
@@ -418,16 +338,14 @@ __global__ void __launch_bounds__(DEC_THREADS)
         r1 = __half_as_ushort(__float2half_rn(p1));
         p0 = __half2float(__ushort_as_half(r0));
         p1 = __half2float(__ushort_as_half(r1));
-        p16[h * DEC_PST + lane] = r0;
-        p16[h * DEC_PST + lane + 32] = r1;
       } else {
         r0 = __bfloat16_as_ushort(__float2bfloat16_rn(p0));
         r1 = __bfloat16_as_ushort(__float2bfloat16_rn(p1));
         p0 = __bfloat162float(__ushort_as_bfloat16(r0));
         p1 = __bfloat162float(__ushort_as_bfloat16(r1));
-        p16[lane * G + h] = r0;
-        p16[(lane + 32) * G + h] = r1;
       }
+      p16[h * DEC_PST + lane] = r0;
+      p16[h * DEC_PST + lane + 32] = r1;
       float ls = p0 + p1;
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, off);
@@ -441,11 +359,11 @@ __global__ void __launch_bounds__(DEC_THREADS)
     }
     __syncthreads();
 
-    // ---- C: O += p V
-    if constexpr (FP8) {
-      // warp w: value columns 32 w .. 32 w + 31 as four 8-wide MMA tiles (column n of tile
-      // i = value column 32 w + 4 n + i, so each lane's 32-bit read of a token row feeds
-      // all four), the heads as the MMA's rows, the tile's tokens in four 16-token steps
+    // ---- C: O += p V.  Warp w: value columns 32 w .. 32 w + 31 as four 8-wide MMA tiles
+    // (column n of tile i = value column 32 w + 4 n + i, so one read of four columns of a
+    // token row feeds all four tiles), the heads as the MMA's rows, the tile's tokens in
+    // four 16-token steps
+    {
       const float a_lo = fr < G ? ha[fr] : 1.0f, a_hi = fr + 8 < G ? ha[fr + 8] : 1.0f;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -454,7 +372,8 @@ __global__ void __launch_bounds__(DEC_THREADS)
         acc[i][2] *= a_hi;
         acc[i][3] *= a_hi;
       }
-      const int vb = 32 * warp + 4 * fr;  // byte (= column) of this lane's value read
+      const int vb = (32 * warp + 4 * fr) * C::E;  // byte of this lane's four value columns
+      const uint8_t* vcol = vt + (vb & 15);
       const uint32_t* pw = reinterpret_cast<const uint32_t*>(p16);
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks) {
@@ -464,85 +383,56 @@ __global__ void __launch_bounds__(DEC_THREADS)
         af[1] = fr + 8 < G ? pw[((fr + 8) * DEC_PST + k0) >> 1] : 0u;
         af[2] = fr < G ? pw[(fr * DEC_PST + k0 + 8) >> 1] : 0u;
         af[3] = fr + 8 < G ? pw[((fr + 8) * DEC_PST + k0 + 8) >> 1] : 0u;
-        const uint32_t w0 = *reinterpret_cast<const uint32_t*>(vt + dec_chunk_off<true>(k0, vb >> 4) + (vb & 15));
-        const uint32_t w1 = *reinterpret_cast<const uint32_t*>(vt + dec_chunk_off<true>(k0 + 1, vb >> 4) + (vb & 15));
-        const uint32_t w2 = *reinterpret_cast<const uint32_t*>(vt + dec_chunk_off<true>(k0 + 8, vb >> 4) + (vb & 15));
-        const uint32_t w3 = *reinterpret_cast<const uint32_t*>(vt + dec_chunk_off<true>(k0 + 9, vb >> 4) + (vb & 15));
-        // byte i of the two tokens of a pair, side by side: (k0, k0 + 1) and (k0 + 8, k0 + 9)
-        const uint32_t lo01 = __byte_perm(w0, w1, 0x5140), hi01 = __byte_perm(w0, w1, 0x7362);
-        const uint32_t lo89 = __byte_perm(w2, w3, 0x5140), hi89 = __byte_perm(w2, w3, 0x7362);
-        mma_16816_f16(acc[0], af, e4m3x2_to_f16x2(lo01), e4m3x2_to_f16x2(lo89));
-        mma_16816_f16(acc[1], af, e4m3x2_to_f16x2(lo01 >> 16), e4m3x2_to_f16x2(lo89 >> 16));
-        mma_16816_f16(acc[2], af, e4m3x2_to_f16x2(hi01), e4m3x2_to_f16x2(hi89));
-        mma_16816_f16(acc[3], af, e4m3x2_to_f16x2(hi01 >> 16), e4m3x2_to_f16x2(hi89 >> 16));
-      }
-    } else {
-      // 4 value columns x G heads per thread, tokens j = warp (mod 4), by mixed-precision
-      // fma (bf16 p and v, fp32 accumulators)
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float a = ha[h];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) acc[h][c] *= a;
-      }
-#pragma unroll 4
-      for (int j = warp; j < DEC_TT; j += 4) {
-        const uint2 w = *reinterpret_cast<const uint2*>(
-            vt + dec_chunk_off<false>(j, (8 * lane) >> 4) + ((8 * lane) & 15));
-        uint32_t pw[(G + 1) / 2];
-        if constexpr (G == 1) {
-          pw[0] = p16[j];
+        // bf[i][0]: column i of tokens (k0, k0 + 1), bf[i][1]: of tokens (k0 + 8, k0 + 9)
+        uint32_t bf[4][2];
+        if constexpr (FP8) {
+          const uint32_t w0 = *reinterpret_cast<const uint32_t*>(vcol + dec_chunk_off<true>(k0, vb >> 4));
+          const uint32_t w1 = *reinterpret_cast<const uint32_t*>(vcol + dec_chunk_off<true>(k0 + 1, vb >> 4));
+          const uint32_t w2 = *reinterpret_cast<const uint32_t*>(vcol + dec_chunk_off<true>(k0 + 8, vb >> 4));
+          const uint32_t w3 = *reinterpret_cast<const uint32_t*>(vcol + dec_chunk_off<true>(k0 + 9, vb >> 4));
+          // byte i of the two tokens of a pair side by side, then e4m3 -> f16 (exact)
+          const uint32_t lo01 = __byte_perm(w0, w1, 0x5140), hi01 = __byte_perm(w0, w1, 0x7362);
+          const uint32_t lo89 = __byte_perm(w2, w3, 0x5140), hi89 = __byte_perm(w2, w3, 0x7362);
+          bf[0][0] = e4m3x2_to_f16x2(lo01);
+          bf[1][0] = e4m3x2_to_f16x2(lo01 >> 16);
+          bf[2][0] = e4m3x2_to_f16x2(hi01);
+          bf[3][0] = e4m3x2_to_f16x2(hi01 >> 16);
+          bf[0][1] = e4m3x2_to_f16x2(lo89);
+          bf[1][1] = e4m3x2_to_f16x2(lo89 >> 16);
+          bf[2][1] = e4m3x2_to_f16x2(hi89);
+          bf[3][1] = e4m3x2_to_f16x2(hi89 >> 16);
         } else {
-#pragma unroll
-          for (int i = 0; i < G / 2; ++i) pw[i] = reinterpret_cast<const uint32_t*>(p16 + j * G)[i];
+          const uint2 w0 = *reinterpret_cast<const uint2*>(vcol + dec_chunk_off<false>(k0, vb >> 4));
+          const uint2 w1 = *reinterpret_cast<const uint2*>(vcol + dec_chunk_off<false>(k0 + 1, vb >> 4));
+          const uint2 w2 = *reinterpret_cast<const uint2*>(vcol + dec_chunk_off<false>(k0 + 8, vb >> 4));
+          const uint2 w3 = *reinterpret_cast<const uint2*>(vcol + dec_chunk_off<false>(k0 + 9, vb >> 4));
+          // bf16 column i of the two tokens of a pair side by side
+          bf[0][0] = __byte_perm(w0.x, w1.x, 0x5410);
+          bf[1][0] = __byte_perm(w0.x, w1.x, 0x7632);
+          bf[2][0] = __byte_perm(w0.y, w1.y, 0x5410);
+          bf[3][0] = __byte_perm(w0.y, w1.y, 0x7632);
+          bf[0][1] = __byte_perm(w2.x, w3.x, 0x5410);
+          bf[1][1] = __byte_perm(w2.x, w3.x, 0x7632);
+          bf[2][1] = __byte_perm(w2.y, w3.y, 0x5410);
+          bf[3][1] = __byte_perm(w2.y, w3.y, 0x7632);
         }
 #pragma unroll
-        for (int h = 0; h < G; ++h)
-          pv4_mixed<true>(static_cast<uint16_t>(pw[h / 2] >> (16 * (h & 1))), w.x, w.y, acc[h]);
+        for (int i = 0; i < 4; ++i) mma_16816<!FP8>(acc[i], af, bf[i][0], bf[i][1]);
       }
     }
-    __syncthreads();  // this buffer is refilled next iteration; s_s is rewritten
+    __syncthreads();  // this buffer is refilled next iteration; s_s and p16 are rewritten
   }
 
-  // ---- the partial output of this range
-  if constexpr (FP8) {
-    // lane (fr, fc) of warp w holds columns 32 w + 8 fc .. + 7 of heads fr and fr + 8
+  // ---- the partial output of this range: lane (fr, fc) of warp w holds value columns
+  // 32 w + 8 fc .. + 7 of heads fr and fr + 8
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int h = fr + 8 * hh;
-      if (h < G) {
-        float* po = p.part_o + (pidx + static_cast<size_t>(h) * p.n_splits) * DEC_D + 32 * warp + 8 * fc;
-        *reinterpret_cast<float4*>(po) = make_float4(acc[0][2 * hh], acc[1][2 * hh], acc[2][2 * hh], acc[3][2 * hh]);
-        *reinterpret_cast<float4*>(po + 4) =
-            make_float4(acc[0][2 * hh + 1], acc[1][2 * hh + 1], acc[2][2 * hh + 1], acc[3][2 * hh + 1]);
-      }
-    }
-  } else {
-    // the four token groups (warps) first
-#pragma unroll 1
-    for (int w = 1; w < 4; ++w) {
-      if (warp == w) {
-#pragma unroll
-        for (int h = 0; h < G; ++h)
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            float* dst = ored + h * DEC_D + 4 * lane + c;
-            *dst = (w == 1 ? 0.0f : *dst) + acc[h][c];
-          }
-      }
-      __syncthreads();
-    }
-    if (warp == 0) {
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        float* po = p.part_o + (pidx + static_cast<size_t>(h) * p.n_splits) * DEC_D + 4 * lane;
-        float4 r;
-        r.x = acc[h][0] + ored[h * DEC_D + 4 * lane + 0];
-        r.y = acc[h][1] + ored[h * DEC_D + 4 * lane + 1];
-        r.z = acc[h][2] + ored[h * DEC_D + 4 * lane + 2];
-        r.w = acc[h][3] + ored[h * DEC_D + 4 * lane + 3];
-        *reinterpret_cast<float4*>(po) = r;
-      }
+  for (int hh = 0; hh < 2; ++hh) {
+    const int h = fr + 8 * hh;
+    if (h < G) {
+      float* po = p.part_o + (pidx + static_cast<size_t>(h) * p.n_splits) * DEC_D + 32 * warp + 8 * fc;
+      *reinterpret_cast<float4*>(po) = make_float4(acc[0][2 * hh], acc[1][2 * hh], acc[2][2 * hh], acc[3][2 * hh]);
+      *reinterpret_cast<float4*>(po + 4) =
+          make_float4(acc[0][2 * hh + 1], acc[1][2 * hh + 1], acc[2][2 * hh + 1], acc[3][2 * hh + 1]);
     }
   }
   if (tid < G) {
