@@ -364,7 +364,8 @@ attn_status_t attn_decode_paged(const void* q, const void* k_cache, const void* 
   prm.max_blocks = max_blocks_per_seq;
   prm.max_seqlen = max_seqlen;
   prm.n_splits = attn::dec_n_splits(B, Hkv, msl);
-  prm.split_tokens = attn::dec_split_tokens(msl, prm.n_splits);
+  prm.split_tokens = dtype == ATTN_FP8_E4M3 ? attn::dec_split_tokens<true>(msl, prm.n_splits)
+                                          : attn::dec_split_tokens<false>(msl, prm.n_splits);
   prm.qk_scale = static_cast<float>((1.0 / std::sqrt(128.0)) * 1.4426950408889634);
   prm.descale_q = descale_q;
   prm.descale_k = descale_k;

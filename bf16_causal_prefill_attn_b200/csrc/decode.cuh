@@ -18,16 +18,16 @@
 //
 // Split-KV: CTA (g, split, b) takes one kv head g of sequence b, all G query heads that read
 // it, and a contiguous range of its tokens; it writes the unnormalised partial output and
-// the (max, sum) of its range, and decode_combine_kernel merges the ranges.  Per 64-token
-// tile (NST tiles in flight):
-//   A  scores: warp w multiplies tokens 16 w .. 16 w + 15 (the MMA's rows) by the G
+// the (max, sum) of its range, and decode_combine_kernel merges the ranges.  Per tile of TT
+// tokens (NST tiles in flight):
+//   A  scores: warp w multiplies tokens 64 m + 16 w .. + 15 (the MMA's rows) by the G
 //      queries (its 8-wide columns, query fragments in registers), fp32 accumulators,
 //      scaled by scale * log2 e (FP8: times the Q and K descales);
 //   B  per head: the tile max, the running max, alpha = 2^(m_old - m_new), p = 2^(s - m_new)
 //      and the running sum (one warp per head, shuffles);
 //   C  O += p V with p rounded to 16 bits (f16 for FP8 caches, bf16 for BF16 ones; the
 //      running sum adds the same rounded values): warp w owns value columns 32 w .. 32 w +
-//      31 of all G heads (the heads are the MMA's rows) and all 64 tokens; e4m3 values are
+//      31 of all G heads (the heads are the MMA's rows) and all TT tokens; e4m3 values are
 //      converted to f16 (exact) in registers.
 // Page ids and sequence lengths are read on the device: entries outside the cache make the
 // CTA record DEV_BAD_SEQLENS and write an empty partial instead of reading out of bounds.
@@ -43,7 +43,7 @@
 namespace attn {
 
 constexpr int DEC_D = 128;        // head dim of q, k and v
-constexpr int DEC_TT = 64;        // tokens per tile
+constexpr int DEC_TT = 64;        // split unit (tokens); the kernels' tiles are multiples of it
 constexpr int DEC_THREADS = 128;
 
 struct DecodeParams {
@@ -54,7 +54,7 @@ struct DecodeParams {
   const int* seq_lens;      // [B]
   int B, Hq, Hkv, G;
   int num_pages, page_shift, max_blocks, max_seqlen;
-  int n_splits, split_tokens;  // tokens per split: a multiple of DEC_TT
+  int n_splits, split_tokens;  // tokens per split: a multiple of the kernel's tile
   float qk_scale;              // scale * log2(e) (FP8: times the Q and K descales later)
   const float* descale_q;
   const float* descale_k;
@@ -69,23 +69,24 @@ struct DecodeParams {
 template <bool FP8>
 struct DecCfg {
   static constexpr int E = FP8 ? 1 : 2;
+  static constexpr int TT = DEC_TT;              // tokens per tile
+  static constexpr int PST = TT + 8;             // row stride (16-bit elements) of p [G][PST]
   static constexpr int ROW = DEC_D * E;          // bytes of one token's K (or V) row
   static constexpr int CHUNKS = ROW / 16;        // 16-byte chunks per row
-  static constexpr int TILE_BYTES = DEC_TT * ROW;
+  static constexpr int TILE_BYTES = TT * ROW;
   // tiles in flight per CTA (a third did not change the time: the kernel is issue-bound
   // with e4m3 caches and near the copy bandwidth with bf16 ones)
   static constexpr int NST = 2;
 };
 
-// row stride (16-bit elements) of the FP8 kernel's p [G][DEC_TT]: padded so that the eight
-// heads of one MMA fragment load fall in different banks
-constexpr int DEC_PST = DEC_TT + 8;
-
 // dynamic shared memory of decode_split_kernel<FP8, G>: K and V tiles (double-buffered),
 // the scores, per-head state and p in 16 bits
+// (the row stride of p is padded so that the eight heads of one MMA fragment read fall in
+// different banks)
 template <bool FP8, int G>
 constexpr int dec_smem_bytes() {
-  return 2 * DecCfg<FP8>::NST * DecCfg<FP8>::TILE_BYTES + (DEC_TT * G + 3 * G) * 4 + G * DEC_PST * 2;
+  using C = DecCfg<FP8>;
+  return 2 * C::NST * C::TILE_BYTES + (C::TT * G + 3 * G) * 4 + G * C::PST * 2;
 }
 
 // split-KV policy: about sixteen CTAs per SM of a 148-SM B200 (several full waves at the
@@ -99,9 +100,13 @@ inline int dec_n_splits(int B, int Hkv, int max_seqlen) {
   if (want > cap) want = cap;
   return static_cast<int>(want < 1 ? 1 : want);
 }
+// tokens per split: the split of max_seqlen into n_splits ranges of whole 64-token units,
+// rounded up to whole kernel tiles (trailing splits may then be empty)
+template <bool FP8>
 inline int dec_split_tokens(int max_seqlen, int n_splits) {
   const int tiles = (max_seqlen + DEC_TT - 1) / DEC_TT;
-  return ((tiles + n_splits - 1) / n_splits) * DEC_TT;
+  const int tok = ((tiles + n_splits - 1) / n_splits) * DEC_TT;
+  return (tok + DecCfg<FP8>::TT - 1) / DecCfg<FP8>::TT * DecCfg<FP8>::TT;
 }
 
 // 16-byte chunk c of token row j of a tile, XOR-swizzled so that the MMA fragment reads
@@ -170,16 +175,17 @@ __global__ void __launch_bounds__(DEC_THREADS)
   using C = DecCfg<FP8>;
   constexpr int QNT = (G + 7) / 8;   // 8-wide MMA column tiles of heads in phase A
   constexpr int KS = FP8 ? 4 : 8;    // phase A steps of d: 32 e4m3 or 16 bf16 elements (32 bytes)
-  static_assert(DEC_THREADS == 128 && DEC_TT == 64, "phases A and C: four warps of 16 tokens / 32 columns");
+  constexpr int TT = C::TT, PST = C::PST;
+  static_assert(DEC_THREADS == 128 && TT % 64 == 0, "phases A and C: four warps of 16-token MMA rows / 32 columns");
 
   extern __shared__ __align__(16) uint8_t dsm[];
   uint8_t* kbuf = dsm;                                   // [NST][TILE_BYTES]
   uint8_t* vbuf = dsm + C::NST * C::TILE_BYTES;          // [NST][TILE_BYTES]
-  float* s_s = reinterpret_cast<float*>(dsm + 2 * C::NST * C::TILE_BYTES);  // [DEC_TT][G]
-  float* hm = s_s + DEC_TT * G;                          // [G] running max (log2 units)
+  float* s_s = reinterpret_cast<float*>(dsm + 2 * C::NST * C::TILE_BYTES);  // [TT][G]
+  float* hm = s_s + TT * G;                          // [G] running max (log2 units)
   float* hl = hm + G;                                    // [G] running sum
   float* ha = hl + G;                                    // [G] alpha of this tile
-  uint16_t* p16 = reinterpret_cast<uint16_t*>(ha + G);   // [G][DEC_PST] p, 16-bit
+  uint16_t* p16 = reinterpret_cast<uint16_t*>(ha + G);   // [G][PST] p, 16-bit
 
   // kv head fastest: the CTAs of one (sequence, split) read the same pages (their head's
   // slice of every token row) at about the same time, which keeps DRAM rows open
@@ -245,13 +251,13 @@ __global__ void __launch_bounds__(DEC_THREADS)
     hl[tid] = 0.0f;
   }
 
-  // ---- tile loader: rows of tokens [t0, t0 + 64) of kv head g, 16-byte chunks
+  // ---- tile loader: rows of tokens [t0, t0 + TT) of kv head g, 16-byte chunks
   const uint32_t kbuf_a = smem_addr(kbuf), vbuf_a = smem_addr(vbuf);
   const size_t head_off = static_cast<size_t>(g) * C::ROW;
   const size_t tok_stride = static_cast<size_t>(p.Hkv) * C::ROW;
   const int pmask = (1 << p.page_shift) - 1;
   auto load_tile = [&](int t0, int buf) {
-    for (int i = tid; i < DEC_TT * C::CHUNKS; i += DEC_THREADS) {
+    for (int i = tid; i < TT * C::CHUNKS; i += DEC_THREADS) {
       const int j = i / C::CHUNKS, c = i % C::CHUNKS;
       int t = t0 + j;
       if (t >= t_end) t = t_end - 1;  // tail rows: a valid row, masked in phase A
@@ -264,12 +270,12 @@ __global__ void __launch_bounds__(DEC_THREADS)
     cp_async_commit();
   };
 
-  const int n_tiles = (t_end - t_begin + DEC_TT - 1) / DEC_TT;
+  const int n_tiles = (t_end - t_begin + TT - 1) / TT;
   // prologue: the first NST - 1 tiles (an empty group where there is no tile keeps the
   // count of committed groups uniform)
 #pragma unroll
   for (int st = 0; st < C::NST - 1; ++st) {
-    if (st < n_tiles) load_tile(t_begin + st * DEC_TT, st);
+    if (st < n_tiles) load_tile(t_begin + st * TT, st);
     else cp_async_commit();
   }
   __syncthreads();  // hm, hl
@@ -282,19 +288,20 @@ __global__ void __launch_bounds__(DEC_THREADS)
 
   for (int it = 0; it < n_tiles; ++it) {
     const int buf = it % C::NST;
-    const int t0 = t_begin + it * DEC_TT;
+    const int t0 = t_begin + it * TT;
     // tile it + NST - 1 into the buffer tile it - 1 used (every thread is past it)
-    if (it + C::NST - 1 < n_tiles) load_tile(t0 + (C::NST - 1) * DEC_TT, (it + C::NST - 1) % C::NST);
+    if (it + C::NST - 1 < n_tiles) load_tile(t0 + (C::NST - 1) * TT, (it + C::NST - 1) % C::NST);
     else cp_async_commit();
     cp_async_wait<C::NST - 1>();  // tile it has landed
     __syncthreads();
     const uint8_t* kt = kbuf + buf * C::TILE_BYTES;
     const uint8_t* vt = vbuf + buf * C::TILE_BYTES;
 
-    // ---- A: scores of the tile; warp w: tokens 16 w .. 16 w + 15 as the MMA's rows, the
-    // heads as its columns; step ks covers bytes 32 ks .. 32 ks + 31 of the rows
-    {
-      const int j0 = 16 * warp;
+    // ---- A: scores of the tile; warp w: tokens 64 mt + 16 w .. + 15 as the MMA's rows,
+    // the heads as its columns; step ks covers bytes 32 ks .. 32 ks + 31 of the rows
+#pragma unroll
+    for (int mt = 0; mt < TT / 64; ++mt) {
+      const int j0 = 64 * mt + 16 * warp;
       float sc[QNT][4];
 #pragma unroll
       for (int nt = 0; nt < QNT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.0f;
@@ -323,30 +330,36 @@ __global__ void __launch_bounds__(DEC_THREADS)
 
     // ---- B: per-head tile softmax in log2 units
     for (int h = warp; h < G; h += DEC_THREADS / 32) {
-      const float s0 = s_s[lane * G + h], s1 = s_s[(lane + 32) * G + h];
-      float mt = fmaxf(s0, s1);
+      constexpr int U = TT / 32;  // tokens lane + 32 u of the tile
+      float sv[U];
+      float mx = -INFINITY;
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
+      for (int u = 0; u < U; ++u) {
+        sv[u] = s_s[(lane + 32 * u) * G + h];
+        mx = fmaxf(mx, sv[u]);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
       const float m_old = hm[h];
-      const float m_new = fmaxf(m_old, mt);
+      const float m_new = fmaxf(m_old, mx);
       // p rounded to the 16-bit type of the cached values (FP8: f16, BF16: bf16), the
       // form O += p V multiplies; the row sum adds the same rounded values
-      float p0 = ex2_approx(s0 - m_new), p1 = ex2_approx(s1 - m_new);
-      uint16_t r0, r1;
-      if constexpr (FP8) {
-        r0 = __half_as_ushort(__float2half_rn(p0));
-        r1 = __half_as_ushort(__float2half_rn(p1));
-        p0 = __half2float(__ushort_as_half(r0));
-        p1 = __half2float(__ushort_as_half(r1));
-      } else {
-        r0 = __bfloat16_as_ushort(__float2bfloat16_rn(p0));
-        r1 = __bfloat16_as_ushort(__float2bfloat16_rn(p1));
-        p0 = __bfloat162float(__ushort_as_bfloat16(r0));
-        p1 = __bfloat162float(__ushort_as_bfloat16(r1));
+      float ls = 0.0f;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const float pf = ex2_approx(sv[u] - m_new);
+        uint16_t r;
+        float pr;
+        if constexpr (FP8) {
+          r = __half_as_ushort(__float2half_rn(pf));
+          pr = __half2float(__ushort_as_half(r));
+        } else {
+          r = __bfloat16_as_ushort(__float2bfloat16_rn(pf));
+          pr = __bfloat162float(__ushort_as_bfloat16(r));
+        }
+        p16[h * PST + lane + 32 * u] = r;
+        ls += pr;
       }
-      p16[h * DEC_PST + lane] = r0;
-      p16[h * DEC_PST + lane + 32] = r1;
-      float ls = p0 + p1;
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, off);
       __syncwarp();
@@ -362,7 +375,7 @@ __global__ void __launch_bounds__(DEC_THREADS)
     // ---- C: O += p V.  Warp w: value columns 32 w .. 32 w + 31 as four 8-wide MMA tiles
     // (column n of tile i = value column 32 w + 4 n + i, so one read of four columns of a
     // token row feeds all four tiles), the heads as the MMA's rows, the tile's tokens in
-    // four 16-token steps
+    // 16-token steps
     {
       const float a_lo = fr < G ? ha[fr] : 1.0f, a_hi = fr + 8 < G ? ha[fr + 8] : 1.0f;
 #pragma unroll
@@ -376,13 +389,13 @@ __global__ void __launch_bounds__(DEC_THREADS)
       const uint8_t* vcol = vt + (vb & 15);
       const uint32_t* pw = reinterpret_cast<const uint32_t*>(p16);
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
+      for (int ks = 0; ks < TT / 16; ++ks) {
         const int k0 = 16 * ks + 2 * fc;  // this lane's tokens k0, k0 + 1, k0 + 8, k0 + 9
         uint32_t af[4];
-        af[0] = fr < G ? pw[(fr * DEC_PST + k0) >> 1] : 0u;
-        af[1] = fr + 8 < G ? pw[((fr + 8) * DEC_PST + k0) >> 1] : 0u;
-        af[2] = fr < G ? pw[(fr * DEC_PST + k0 + 8) >> 1] : 0u;
-        af[3] = fr + 8 < G ? pw[((fr + 8) * DEC_PST + k0 + 8) >> 1] : 0u;
+        af[0] = fr < G ? pw[(fr * PST + k0) >> 1] : 0u;
+        af[1] = fr + 8 < G ? pw[((fr + 8) * PST + k0) >> 1] : 0u;
+        af[2] = fr < G ? pw[(fr * PST + k0 + 8) >> 1] : 0u;
+        af[3] = fr + 8 < G ? pw[((fr + 8) * PST + k0 + 8) >> 1] : 0u;
         // bf[i][0]: column i of tokens (k0, k0 + 1), bf[i][1]: of tokens (k0 + 8, k0 + 9)
         uint32_t bf[4][2];
         if constexpr (FP8) {
