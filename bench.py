@@ -283,6 +283,7 @@ def gpu_bench_decode(args, rank, world, local_rank):
     io_bytes = B * Hq * 128 * 2 + B * Hq * 4       # o (bf16) and lse written
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     flops = 2.0 * B * Hq * L * 256
+    traffic = load_traffic(args.workload, "traffic_decode.json", DECODE_SOURCES)
     fp8_gbs = (kv_bytes(1) + B * Hq * 128 + io_bytes) / (fp8_ms * 1e-3) / 1e9
     bf16_gbs = (kv_bytes(2) + B * Hq * 256 + io_bytes) / (bf16_ms * 1e-3) / 1e9
     return {
@@ -308,13 +309,16 @@ def gpu_bench_decode(args, rank, world, local_rank):
                      "unit": "GB/s", "frac": round(fp8_gbs / hbm, 4),
                      "peak_source": f"{peak_src} copy bandwidth",
                      "kernel": "decode_split_kernel<fp8> + decode_combine_kernel",
-                     "tflops": round(flops / (fp8_ms * 1e-3) / 1e12, 2), "traffic": None},
+                     "tflops": round(flops / (fp8_ms * 1e-3) / 1e12, 2),
+                     "traffic": traffic.get("fp8"),
+                     "traffic_of": "decode_split_kernel (the combine kernel reads its partials "
+                                   "from L2)"},
         "bf16": {"value": round(bf16_gbs * world, 1), "unit": "GB/s",
                  "ms_per_step": round(bf16_ms, 4),
                  "roofline": {"bound": "hbm", "achieved": round(bf16_gbs, 1), "peak": hbm,
                               "unit": "GB/s", "frac": round(bf16_gbs / hbm, 4),
                               "tflops": round(flops / (bf16_ms * 1e-3) / 1e12, 2),
-                              "traffic": None}},
+                              "traffic": traffic.get("bf16")}},
         "e2e": {"value": round((kv_bytes(1) + B * Hq * 128 + io_bytes) / (e2e_ms * 1e-3) / 1e9
                                * world, 1),
                 "unit": "GB/s", "h2d_bytes_per_step": B * Hq * 128, "d2h_bytes_per_step":
@@ -564,26 +568,30 @@ def gpu_bench(args, rank, world, local_rank):
     return result
 
 
-def kernel_source_hash():
-    """Hash of the attention kernel's sources, to tie ncu counters to the code measured."""
+PREFILL_SOURCES = ("attn_fwd.cuh", "ptx.cuh")
+DECODE_SOURCES = ("decode.cuh", "ptx.cuh")
+
+
+def kernel_source_hash(names=PREFILL_SOURCES):
+    """Hash of a kernel's sources, to tie ncu counters to the code measured."""
     import hashlib
     h = hashlib.sha256()
-    for name in ("attn_fwd.cuh", "ptx.cuh"):
+    for name in names:
         with open(os.path.join(ROOT, "bf16_causal_prefill_attn_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def load_traffic(workload):
+def load_traffic(workload, fname="traffic.json", names=PREFILL_SOURCES):
     """DRAM bytes (read + write) per launch from the committed ncu summary, if it covers
     this workload and the current kernel source; otherwise null."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
+    p = os.path.join(ROOT, "profiles", fname)
     try:
         with open(p) as f:
             d = json.load(f)
     except (OSError, ValueError):
         return {}
-    if d.get("kernel_source_hash") != kernel_source_hash():
+    if d.get("kernel_source_hash") != kernel_source_hash(names):
         return {}
     return d.get("workloads", {}).get(workload, {})
 

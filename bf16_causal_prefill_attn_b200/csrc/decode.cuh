@@ -251,21 +251,43 @@ __global__ void __launch_bounds__(DEC_THREADS)
     hl[tid] = 0.0f;
   }
 
-  // ---- tile loader: rows of tokens [t0, t0 + TT) of kv head g, 16-byte chunks
+  // ---- tile loader: rows of tokens [t0, t0 + TT) of kv head g, 16-byte chunks; thread tid
+  // copies chunk lc = tid % CHUNKS of rows lj + k RSTEP.  Rows past the end of the range
+  // repeat its last row (a valid one; phase A masks them).  Tiles start at multiples of TT,
+  // so with pages of TT tokens or more a tile lies in one page: one page-table read per tile
+  // instead of one per row.
+  constexpr int RSTEP = DEC_THREADS / C::CHUNKS;
+  constexpr int LK = TT / RSTEP;
+  const int lc = tid % C::CHUNKS, lj = tid / C::CHUNKS;
   const uint32_t kbuf_a = smem_addr(kbuf), vbuf_a = smem_addr(vbuf);
-  const size_t head_off = static_cast<size_t>(g) * C::ROW;
+  const size_t col_off = static_cast<size_t>(g) * C::ROW + lc * 16;
   const size_t tok_stride = static_cast<size_t>(p.Hkv) * C::ROW;
   const int pmask = (1 << p.page_shift) - 1;
+  const bool one_page = (1 << p.page_shift) >= TT;
   auto load_tile = [&](int t0, int buf) {
-    for (int i = tid; i < TT * C::CHUNKS; i += DEC_THREADS) {
-      const int j = i / C::CHUNKS, c = i % C::CHUNKS;
-      int t = t0 + j;
-      if (t >= t_end) t = t_end - 1;  // tail rows: a valid row, masked in phase A
-      const size_t row = (static_cast<size_t>(table[t >> p.page_shift]) << p.page_shift) + (t & pmask);
-      const size_t go = row * tok_stride + head_off + c * 16;
-      const uint32_t so = buf * C::TILE_BYTES + dec_chunk_off<FP8>(j, c);
-      cp_async16(kbuf_a + so, p.k_cache + go);
-      cp_async16(vbuf_a + so, p.v_cache + go);
+    const int last = t_end - 1 - t0;
+    if (one_page) {
+      const size_t row0 = (static_cast<size_t>(table[t0 >> p.page_shift]) << p.page_shift) + (t0 & pmask);
+      const uint8_t* kg = p.k_cache + row0 * tok_stride + col_off;
+      const uint8_t* vg = p.v_cache + row0 * tok_stride + col_off;
+#pragma unroll
+      for (int k = 0; k < LK; ++k) {
+        const int j = lj + k * RSTEP;
+        const size_t off = static_cast<size_t>(min(j, last)) * tok_stride;
+        const uint32_t so = buf * C::TILE_BYTES + dec_chunk_off<FP8>(j, lc);
+        cp_async16(kbuf_a + so, kg + off);
+        cp_async16(vbuf_a + so, vg + off);
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < LK; ++k) {
+        const int j = lj + k * RSTEP;
+        const int t = t0 + min(j, last);
+        const size_t go = ((static_cast<size_t>(table[t >> p.page_shift]) << p.page_shift) + (t & pmask)) * tok_stride + col_off;
+        const uint32_t so = buf * C::TILE_BYTES + dec_chunk_off<FP8>(j, lc);
+        cp_async16(kbuf_a + so, p.k_cache + go);
+        cp_async16(vbuf_a + so, p.v_cache + go);
+      }
     }
     cp_async_commit();
   };

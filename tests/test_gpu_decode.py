@@ -41,6 +41,8 @@ CASES = [
     (3, 16, 16, [3000, 0, 129], 64),     # G = 1, several splits, an empty sequence
     (2, 16, 2, [2048, 700], 128),        # G = 8
     (2, 16, 1, [513, 1], 16),            # G = 16
+    (2, 32, 8, [777, 1500], 256),        # G = 4, tiles inside large pages, ragged tails
+    (3, 16, 8, [64, 200, 1], 64),        # G = 2, pages of exactly one tile
 ]
 
 
