@@ -98,3 +98,19 @@ def test_decode_reference_arm_prints_one_line():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_reference_arm_under_two_ranks_prints_once():
+    """Launched like the multi-GPU bench (torchrun, 2 ranks): rank 0 alone runs the oracle
+    and prints one line for the whole job; rank 1 exits 0 without work."""
+    port = 29700 + os.getpid() % 200
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port),
+           os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "small_s256",
+           "--gpus", "2", "--steps", "1", "--warmup", "3"]
+    res = subprocess.run(cmd, capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [l for l in res.stdout.splitlines() if l.strip().startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
