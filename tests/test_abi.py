@@ -129,6 +129,19 @@ def _decode(L, B=2, Hq=8, Hkv=2, dqk=128, dv=128, P=4, page=16, mb=4, msl=64, dt
                                p(ws), need if ws_bytes is None else ws_bytes, None)
 
 
+def test_decode_workspace_follows_the_split_policy(L):
+    """Partials of B x Hq heads x n_splits ranges (128 floats + max and sum each); the split
+    count aims at ~16 CTAs per SM of 148 over the B x Hkv pairs, each split at least two
+    64-token tiles."""
+    def want(B, Hq, Hkv, msl):
+        tiles = -(-msl // 64)
+        ns = min(-(-(16 * 148) // (B * Hkv)), max(1, tiles // 2))
+        return B * Hq * max(ns, 1) * 130 * 4
+    for B, Hq, Hkv, msl in [(64, 32, 8, 4096), (16, 32, 8, 32768), (1, 8, 1, 64), (1, 32, 8, 1),
+                            (3, 16, 16, 3000), (256, 64, 8, 128), (1, 16, 1, 1 << 20)]:
+        assert L.attn_decode_workspace_size(B, Hq, Hkv, msl) == want(B, Hq, Hkv, msl)
+
+
 def test_decode_argument_validation(L):
     assert L.attn_decode_workspace_size(0, 8, 2, 64) == 0
     assert L.attn_decode_workspace_size(2, 8, 2, 64) > 0
