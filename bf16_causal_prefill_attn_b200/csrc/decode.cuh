@@ -74,8 +74,7 @@ struct DecCfg {
   static constexpr int ROW = DEC_D * E;          // bytes of one token's K (or V) row
   static constexpr int CHUNKS = ROW / 16;        // 16-byte chunks per row
   static constexpr int TILE_BYTES = TT * ROW;
-  // tiles in flight per CTA (a third did not change the time: the kernel is issue-bound
-  // with e4m3 caches and near the copy bandwidth with bf16 ones)
+  // tiles in flight per CTA (a third cost the e4m3 kernel 7%: fewer CTAs fit on an SM)
   static constexpr int NST = 2;
 };
 
