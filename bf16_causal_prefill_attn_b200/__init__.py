@@ -68,6 +68,8 @@ def lib():
         L.attn_device_status.restype = i32
         L.attn_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
         L.attn_set_wait_timeout_ns.restype = None
+        L.attn_selftest_stall_tile.argtypes = [i32]
+        L.attn_selftest_stall_tile.restype = None
         L.attn_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
         L.attn_selftest_wait_timeout.restype = i32
         L.attn_status_string.argtypes = [i32]
@@ -257,6 +259,11 @@ def attn_device_status(stream=None):
 
 def attn_set_wait_timeout_ns(ns):
     lib().attn_set_wait_timeout_ns(int(ns))
+
+
+def attn_selftest_stall_tile(tile):
+    """Test-only: prefill calls stop loading before key tile `tile` (negative: normal)."""
+    lib().attn_selftest_stall_tile(int(tile))
 
 
 def attn_selftest_wait_timeout(timeout_ns, stream=None):

@@ -23,6 +23,7 @@ constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s per bounded wait
 __device__ uint32_t g_dev_err = 0;
 
 uint64_t g_timeout_ns = kDefaultTimeoutNs;
+int g_stall_tile = -1;  // test-only (attn_selftest_stall_tile)
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -118,6 +119,7 @@ attn_status_t common_args(void* o, float* lse, int Hq, int Hkv, int d_qk, int d_
   prm->descale_v = dv;
   prm->unrotate = (flags & ATTN_FLAG_UNROTATE_O) ? 1 : 0;
   prm->timeout_ns = g_timeout_ns;
+  prm->stall_tile = g_stall_tile;
   return ATTN_OK;
 }
 
@@ -411,11 +413,8 @@ attn_status_t attn_quantize_e4m3(const void* x_bf16, void* x_e4m3, float* descal
   const int64_t rows = tokens * H;
   uint32_t* amax = static_cast<uint32_t*>(workspace);
   if (rows == 0) {
-    const float one = 1.0f;
-    return cudaMemcpyAsync(descale_out, &one, sizeof(float), cudaMemcpyHostToDevice, st) ==
-                   cudaSuccess
-               ? ATTN_OK
-               : ATTN_ERR_CUDA;
+    attn::descale_one_kernel<<<1, 1, 0, st>>>(descale_out);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
   }
   if (!x_bf16 || !x_e4m3) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(x_bf16) || !aligned16(x_e4m3)) return ATTN_ERR_ALIGNMENT;
@@ -453,6 +452,8 @@ attn_status_t attn_device_status(void* stream) {
 }
 
 void attn_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns = ns ? ns : kDefaultTimeoutNs; }
+
+void attn_selftest_stall_tile(int tile) { g_stall_tile = tile < 0 ? -1 : tile; }
 
 attn_status_t attn_selftest_wait_timeout(uint64_t timeout_ns, void* stream) {
   if (timeout_ns == 0 || timeout_ns > 10000000000ull) return ATTN_ERR_INVALID_ARG;
@@ -492,25 +493,17 @@ namespace {
 constexpr size_t kStaticScratchBytes = 256;  // maximum scratch this entry point can use
 static __device__ __align__(256) uint32_t g_static_scratch[kStaticScratchBytes / 4];
 
-constexpr int kMaxDevices = 128;
-std::mutex g_static_mu;
-uint32_t* g_static_ptr[kMaxDevices] = {};
-
-// Device address of g_static_scratch on the current device.  In host code the array's
-// name only stands in for the symbol; the address is looked up once per device, with that
-// device current, on the first call made on it.
+// Device address of g_static_scratch in the current context.  In host code the array's
+// name only stands in for the symbol; the runtime translates it for the device (and
+// context) current at the call.  It is looked up on every call -- a lookup allocates
+// nothing -- so the address stays right after cudaDeviceReset or in another context.  The
+// first call on a device loads this library's device code there if it is not yet loaded,
+// which must not happen during a stream capture.
 attn_status_t static_scratch(uint32_t** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_static_mu);
-  if (g_static_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr)
-      return ATTN_ERR_CUDA;
-    g_static_ptr[dev] = static_cast<uint32_t*>(p);
-  }
-  *out = g_static_ptr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr)
+    return ATTN_ERR_CUDA;
+  *out = static_cast<uint32_t*>(p);
   return ATTN_OK;
 }
 

@@ -108,6 +108,7 @@ struct FwdParams {
   int unrotate;       // apply x H / sqrt(128) to each output row (Hadamard-rotated V)
   uint32_t* err;
   uint64_t timeout_ns;
+  int stall_tile;        // test-only: the producer stops before this key tile (-1: never)
   float* dump_s;         // FP8 debug: raw scores [B, Hq, S, S]
   uint8_t* dump_codes;   // FP8 debug: P codes   [B, Hq, S, S]
   uint8_t* dump_kshift;  // FP8 debug: shifts    [B, Hq, S, S/64]
@@ -292,6 +293,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       __syncwarp();
       int jk = 0, jv = 0;  // K and V tiles issued
       for (int j = 0; j < n_max && ok; ++j) {
+        if (j == p.stall_tile) break;  // test-only: the waits on this tile must run out
         const int sk = j % C::NK;
         if (j >= C::NK) ok = mbar_wait(k_empty + sk, ((j / C::NK) - 1) & 1, p.err, p.timeout_ns);
         if (!__all_sync(0xffffffffu, ok)) break;

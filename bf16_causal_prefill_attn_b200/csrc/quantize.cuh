@@ -107,6 +107,10 @@ __device__ __forceinline__ float quant_scale(uint32_t amax_bits) {
   return amax > 0.0f ? __fdiv_rn(448.0f, amax) : 1.0f;
 }
 
+// descale of an empty tensor (amax 0): 1, written on the device so the call stays
+// stream-ordered and capturable (no host-to-device copy)
+__global__ void descale_one_kernel(float* descale_out) { *descale_out = 1.0f; }
+
 __device__ __forceinline__ void write_descale(uint32_t amax_bits, float* descale_out) {
   if (blockIdx.x == 0 && threadIdx.x == 0) {
     const float amax = __uint_as_float(amax_bits);

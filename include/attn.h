@@ -176,10 +176,12 @@ size_t attn_quantize_workspace_size(int64_t tokens, int H, int d);
  *   scratch is a fixed 256-byte array compiled into the library, held on every GPU that
  *   loads it until the process exits.  A problem whose scratch need
  *   (attn_quantize_workspace_size) exceeds 256 bytes returns ATTN_ERR_UNSUPPORTED.
- *   The first call on a device looks up the array's device address (with that device
- *   current); make that first call before any stream capture.  All calls share the array
- *   (it keeps the last call's contents; the amax word is cleared at the start of each call),
- *   so calls that may overlap on the GPU -- on different streams, or from different host
+ *   Every call looks up the array's device address in the current context (a lookup that
+ *   allocates nothing), so the address stays valid after cudaDeviceReset or with a
+ *   non-primary context.  The first call on a device may load the library's device code on
+ *   it: make that first call before any stream capture.  All calls share the array (it
+ *   keeps the last call's contents; the amax word is cleared at the start of each call), so
+ *   calls that may overlap on the GPU -- on different streams, or from different host
  *   threads -- race and must be serialised by the caller.  Allocates nothing.
  */
 attn_status_t attn_quantize_e4m3_static(const void* x_bf16, void* x_e4m3, float* descale_out,
@@ -210,6 +212,15 @@ attn_status_t attn_device_status(void* stream);
 
 /* Test-only: sets the bounded-wait limit in nanoseconds (0 restores the default, 2 s). */
 void attn_set_wait_timeout_ns(uint64_t ns);
+
+/*
+ * Test-only: the prefill kernels' load warp stops before key tile `tile` (a negative value
+ * restores normal operation), so the waits on that tile are never satisfied: they run out
+ * after the bounded-wait limit, the kernel records ATTN_ERR_TIMEOUT in the device error word
+ * and every warp unwinds (no copy or MMA is left in flight), leaving the context usable.
+ * Applies to the attn_fwd* calls made while it is set.
+ */
+void attn_selftest_stall_tile(int tile);
 
 /*
  * Test-only: launches one thread that waits, with the bounded wait the kernels use, on an

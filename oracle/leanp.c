@@ -25,23 +25,31 @@
  *     m      reference max in code units, an integer, raised lazily:
  *            cand = ceil(float32(a * mu_tile)) (mu_tile = tile max of the raw scores);
  *            m = cand on the first tile, afterwards m = cand only if cand > m + H
- *            (H = 14, the headroom between the block-max code 112 and the largest
+ *            (H = 14, the headroom between the block-max code T = 112 and the largest
  *            finite code 126); otherwise m is kept
  *     k_b    per 64-key block b with block max mu_b:
- *            t = fmaf(mu_b, a, -m);  k_b = clamp(floor(-t / 8), 0, KMAX)
- *            (a block whose max sits below m by 8 k_b or more is lifted by 2^k_b)
+ *            t = fmaf(mu_b, a, -m);  k_b = clamp(floor(-t / 8), KMIN, KMAX), KMIN = 0,
+ *            KMAX = 16 (a block whose max sits below m by 8 k_b or more is lifted by
+ *            2^k_b, so its maximum codes into (T - 8, T])
  *     code   the multiply-add, saturating to [0, 1] (negative codes clamp to 0):
- *              u = sat(fmaf(s, a / 256, (112 + 8 k_b - m) / 256))
+ *              u = sat(fmaf(s, a / 256, (T + 8 k_b - m) / 256))
  *            and the integer conversion, one fma whose rounding at magnitude 2^23 is the
  *            round-to-nearest-even integer:  r = fmaf(u, 256, 1.5 * 2^23);
- *            byte = low 8 bits of r  (at most 126: never the NaN code 127)
- *     value  decode(byte) ~ 2^((a s - m)/8) * 2^(7 + k_b); the matrix instruction
- *            applies 2^-(7 + k_b) per (row, 64-key block) through UE8M0 scale factors
- *     l      l <- alpha l + sum_j decode(byte_j) 2^-(7+k_b(j));   O likewise with v_j
+ *            byte = low 8 bits of r  (at most T + H = 126: never the NaN code 127)
+ *     value  decode(byte) ~ 2^((a s - m)/8) * 2^(T/8 - 7 + k_b); the matrix instruction
+ *            applies 2^-(T/8 - 7 + k_b) per (row, 64-key block) through UE8M0 scale
+ *            factors, so a score at the reference weighs 1
+ *     l      l <- alpha l + sum_j decode(byte_j) 2^-(T/8-7+k_b(j));   O likewise with v_j
  *     alpha  2^((m_old - m_new)/8) when m is raised (0 on the first tile)
  *   final:   o = O * dv / l,  lse = ln 2 * (m / 8 + log2 l)
  * Masked scores are -inf: their code is 0.  A fully masked block gets k_b = KMAX (its
  * codes are all 0, so its scale multiplies zeros).
+ *
+ * The eager reading (the reference follows the running maximum on every tile, H = 0, with
+ * block maxima at T = 120 as first proposed for this method) is the other plain reading of
+ * the pages; every function taking (top, headroom, kmin) accepts any reading (T, H, KMIN)
+ * with T + H <= 126, and the functions without those arguments use the one above.  The
+ * tests compare the two readings' accuracy.
  *
  * Build: gcc -O2 -ffp-contract=off -fno-fast-math -shared -fPIC (every a*b+c here is
  * written as the operation it is; the compiler must not fuse or reorder them).
@@ -51,8 +59,14 @@
 #include <string.h>
 
 #define LEANP_MAGIC 12582912.0f /* 1.5 * 2^23 */
-#define LEANP_TOP 112          /* code of a block maximum at the reference */
-#define LEANP_HEADROOM 14      /* 126 - LEANP_TOP */
+#define LEANP_TOP 112          /* T: a block maximum codes into (T - 8, T] */
+#define LEANP_HEADROOM 14      /* H: codes the tile max may exceed the reference by */
+#define LEANP_KMIN 0           /* blocks above the reference keep k_b = 0 */
+
+/* the reading the functions without reading arguments use */
+int leanp_reading_top(void) { return LEANP_TOP; }
+int leanp_reading_headroom(void) { return LEANP_HEADROOM; }
+int leanp_reading_kmin(void) { return LEANP_KMIN; }
 
 /* ---- e4m3fn decode by the format definition (independent of the Python codec) ---- */
 double leanp_e4m3_decode(uint8_t c) {
@@ -67,30 +81,42 @@ double leanp_e4m3_decode(uint8_t c) {
 /* exposed for the tests' exact-rounding pin */
 float leanp_fmaf(float x, float y, float z) { return fmaf(x, y, z); }
 
-/* reference max in code units after seeing a tile whose raw-score maximum is mu_tile */
-int leanp_update_max(float mu_tile, float a, int m_old, int m_valid) {
+/* reference max in code units after seeing a tile whose raw-score maximum is mu_tile.
+ * headroom: how far (in codes) the tile maximum may rise above the reference before the
+ * reference is raised -- LEANP_HEADROOM for the lazy reading, 0 for the eager one (the
+ * reference follows the running maximum on every tile). */
+int leanp_update_max_ex(float mu_tile, float a, int m_old, int m_valid, int headroom) {
     if (isinf(mu_tile) && mu_tile < 0) return m_old;  /* no visible key in the tile */
     float prod = a * mu_tile;                          /* one float32 rounding */
     int cand = (int)ceilf(prod);
     if (!m_valid) return cand;
-    return cand > m_old + LEANP_HEADROOM ? cand : m_old;
+    return cand > m_old + headroom ? cand : m_old;
 }
 
-/* power-of-two shift of one 64-key block */
-int leanp_kshift(float mu_b, float a, int m, int kmax) {
+int leanp_update_max(float mu_tile, float a, int m_old, int m_valid) {
+    return leanp_update_max_ex(mu_tile, a, m_old, m_valid, LEANP_HEADROOM);
+}
+
+/* power-of-two shift of one 64-key block: floor(-t/8) clamped to [kmin, kmax] */
+int leanp_kshift_ex(float mu_b, float a, int m, int kmin, int kmax) {
     if (isinf(mu_b) && mu_b < 0) return kmax;          /* fully masked block */
     float t = fmaf(mu_b, a, -(float)m);
     float g = -t * 0.125f;                             /* exact */
     if (g >= (float)kmax) return kmax;
     float f = floorf(g);
-    if (f <= 0.0f) return 0;
+    if (f <= (float)kmin) return kmin;
     return (int)f;
 }
 
-/* code of one score given the block shift */
-uint8_t leanp_code(float s, float a, int m, int kb) {
+int leanp_kshift(float mu_b, float a, int m, int kmax) {
+    return leanp_kshift_ex(mu_b, a, m, LEANP_KMIN, kmax);
+}
+
+/* code of one score given the block shift; top = code of a block maximum at the
+ * reference (LEANP_TOP in the lazy reading, 120 in the eager one) */
+uint8_t leanp_code_ex(float s, float a, int m, int kb, int top) {
     const float inv256 = 0.00390625f;
-    float c = (float)(LEANP_TOP + 8 * kb - m) * inv256; /* exact: small integer / 256 */
+    float c = (float)(top + 8 * kb - m) * inv256;      /* exact: small integer / 256 */
     float u = fmaf(s, a * inv256, c);                  /* a / 256 exact */
     if (!(u > 0.0f)) u = 0.0f;                         /* saturate (NaN, -inf, <= 0 -> 0) */
     if (u > 1.0f) u = 1.0f;
@@ -100,65 +126,86 @@ uint8_t leanp_code(float s, float a, int m, int kb) {
     return (uint8_t)(bits & 0xFF);
 }
 
+uint8_t leanp_code(float s, float a, int m, int kb) {
+    return leanp_code_ex(s, a, m, kb, LEANP_TOP);
+}
+
 /*
  * Encode one row of one key tile.  s: n raw scores (n a multiple of 64, -inf = masked),
  * m: the running max already updated with this tile.  Writes n codes and n/64 shifts.
  */
-void leanp_encode_row_tile(const float* s, int n, float a, int m, int kmax,
-                           uint8_t* codes, uint8_t* kshift) {
+/* kshift holds k_b as a signed byte */
+static void encode_row_tile_top(const float* s, int n, float a, int m, int kmin, int kmax,
+                                int top, uint8_t* codes, int8_t* kshift) {
     for (int b = 0; b < n / 64; ++b) {
         float mu = -INFINITY;
         for (int j = 0; j < 64; ++j) mu = fmaxf(mu, s[b * 64 + j]);
-        int kb = leanp_kshift(mu, a, m, kmax);
-        kshift[b] = (uint8_t)kb;
-        for (int j = 0; j < 64; ++j) codes[b * 64 + j] = leanp_code(s[b * 64 + j], a, m, kb);
+        int kb = leanp_kshift_ex(mu, a, m, kmin, kmax);
+        kshift[b] = (int8_t)kb;
+        for (int j = 0; j < 64; ++j) codes[b * 64 + j] = leanp_code_ex(s[b * 64 + j], a, m, kb, top);
     }
+}
+
+void leanp_encode_row_tile(const float* s, int n, float a, int m, int kmax,
+                           uint8_t* codes, int8_t* kshift) {
+    encode_row_tile_top(s, n, a, m, LEANP_KMIN, kmax, LEANP_TOP, codes, kshift);
 }
 
 /*
  * Replay the kernel's per-row state machine over a row of raw scores, tile by tile in
  * ascending key order, and return codes, shifts and the reference max used per tile.
  *   s       [ntiles * tile] raw scores of one query row (-inf where masked)
- *   codes   [ntiles * tile] out, kshift [ntiles * tile / 64] out, mref [ntiles] out
+ *   codes   [ntiles * tile] out, kshift [ntiles * tile / 64] out (signed), mref [ntiles] out
  * Tiles with no visible key are skipped (their codes are 0 and shifts KMAX).
  */
-void leanp_encode_row(const float* s, int ntiles, int tile, float a, int kmax,
-                      uint8_t* codes, uint8_t* kshift, int* mref) {
+void leanp_encode_row_ex(const float* s, int ntiles, int tile, float a, int kmax, int top,
+                         int headroom, int kmin, uint8_t* codes, int8_t* kshift, int* mref) {
     int m = 0, m_valid = 0;
     for (int t = 0; t < ntiles; ++t) {
         const float* st = s + (size_t)t * tile;
         float mu = -INFINITY;
         for (int j = 0; j < tile; ++j) mu = fmaxf(mu, st[j]);
-        m = leanp_update_max(mu, a, m, m_valid);
+        m = leanp_update_max_ex(mu, a, m, m_valid, headroom);
         if (!(isinf(mu) && mu < 0)) m_valid = 1;
         mref[t] = m_valid ? m : 0;
         if (!m_valid) {
             memset(codes + (size_t)t * tile, 0, tile);
-            for (int b = 0; b < tile / 64; ++b) kshift[(size_t)t * tile / 64 + b] = (uint8_t)kmax;
+            for (int b = 0; b < tile / 64; ++b) kshift[(size_t)t * tile / 64 + b] = (int8_t)kmax;
             continue;
         }
-        leanp_encode_row_tile(st, tile, a, m, kmax, codes + (size_t)t * tile,
-                              kshift + (size_t)t * tile / 64);
+        encode_row_tile_top(st, tile, a, m, kmin, kmax, top, codes + (size_t)t * tile,
+                            kshift + (size_t)t * tile / 64);
     }
+}
+
+void leanp_encode_row(const float* s, int ntiles, int tile, float a, int kmax,
+                      uint8_t* codes, int8_t* kshift, int* mref) {
+    leanp_encode_row_ex(s, ntiles, tile, a, kmax, LEANP_TOP, LEANP_HEADROOM, LEANP_KMIN, codes,
+                        kshift, mref);
 }
 
 /*
  * End-to-end tile driver for one query row: from the row's raw scores (float32) and the
- * value rows (float64, already dequantised), the lean-P output row and lse.
- *   s [S_k] raw scores (-inf masked), v [S_k * dv] dequantised values (row-major),
- *   scale_nat = softmax scale * dq * dk (natural units per raw score unit) for lse.
+ * value rows (float64, already dequantised), the lean-P output row and lse, under the
+ * reading (top, headroom, kmin) -- the one above is (120, 16, -2); the eager reading is
+ * (120, 0, 0).
+ *   s [S_k] raw scores (-inf masked), v [S_k * dv] dequantised values (row-major).
  * The products and sums of this step are formed in float64 (the tensor core's float32
  * accumulation order is not specified), so this predicts the kernel within float32
- * accumulation error, not bit for bit.
+ * accumulation error, not bit for bit.  The weight of a code is
+ * decode(byte) 2^-(top/8 - 7 + k_b), so a score at the reference weighs 1.
  */
-void leanp_attention_row(const float* s, int S_k, int tile, const double* v, int dv,
-                         float a, int kmax, double* o_out, double* lse_out) {
+void leanp_attention_row_ex(const float* s, int S_k, int tile, const double* v, int dv,
+                            float a, int kmax, int top, int headroom, int kmin,
+                            double* o_out, double* lse_out) {
     int ntiles = (S_k + tile - 1) / tile;
     double acc[1024];
     double l = 0.0;
     int m = 0, m_valid = 0;
     float buf[512];
-    uint8_t codes[512], ks[8];
+    uint8_t codes[512];
+    int8_t ks[8];
+    const double unit = ldexp(1.0, -(top / 8 - 7));
     for (int d = 0; d < dv; ++d) acc[d] = 0.0;
     for (int t = 0; t < ntiles; ++t) {
         int n = tile;
@@ -169,17 +216,17 @@ void leanp_attention_row(const float* s, int S_k, int tile, const double* v, int
         float mu = -INFINITY;
         for (int j = 0; j < n; ++j) mu = fmaxf(mu, buf[j]);
         if (isinf(mu) && mu < 0) continue;
-        int m_new = leanp_update_max(mu, a, m, m_valid);
+        int m_new = leanp_update_max_ex(mu, a, m, m_valid, headroom);
         double alpha = m_valid ? exp2((double)(m - m_new) / 8.0) : 0.0;
         m = m_new;
         m_valid = 1;
-        leanp_encode_row_tile(buf, n, a, m, kmax, codes, ks);
+        encode_row_tile_top(buf, n, a, m, kmin, kmax, top, codes, ks);
         l *= alpha;
         for (int d = 0; d < dv; ++d) acc[d] *= alpha;
         for (int j = 0; j < n; ++j) {
             int key = t * tile + j;
             if (key >= S_k || codes[j] == 0) continue;
-            double w = leanp_e4m3_decode(codes[j]) * ldexp(1.0, -(7 + ks[j / 64]));
+            double w = leanp_e4m3_decode(codes[j]) * unit * ldexp(1.0, -ks[j / 64]);
             l += w;
             for (int d = 0; d < dv; ++d) acc[d] += w * v[(size_t)key * dv + d];
         }
@@ -188,19 +235,25 @@ void leanp_attention_row(const float* s, int S_k, int tile, const double* v, int
     *lse_out = log(2.0) * ((double)m / 8.0 + log2(l));
 }
 
+void leanp_attention_row(const float* s, int S_k, int tile, const double* v, int dv,
+                         float a, int kmax, double* o_out, double* lse_out) {
+    leanp_attention_row_ex(s, S_k, tile, v, dv, a, kmax, LEANP_TOP, LEANP_HEADROOM, LEANP_KMIN,
+                           o_out, lse_out);
+}
+
 /*
  * Exact-P ablation ([ZYFA-mb] "Como o motor de atenção FP8 da Zyphra funciona" contrasts
  * lean P with "exact P", the probabilities formed with an exponential and then rounded to
  * FP8).  Reading: same reference max m and block shifts k_b as lean P; the value written
  * is e4m3_rn(2^x) with the float32 exponent
- *     x = fmaf(s, a / 8, (8 (7 + k_b) - m) / 8)      (a / 8 and the constant are exact)
- * so that 2^x = 2^((a s - m)/8) 2^(7 + k_b), the quantity lean P approximates.  This
- * function forms x for n scores; the exponential and the e4m3 rounding are done by the
- * caller (oracle/leanp.py) in float64 and with the table codec.
+ *     x = fmaf(s, a / 8, (T - 56 + 8 k_b - m) / 8)   (a / 8 and the constant are exact)
+ * so that 2^x = 2^((a s - m)/8) 2^(T/8 - 7 + k_b), the value whose log-linear code lean P
+ * writes (a score at the reference gives 2^(T/8 - 7) with k_b = 0).  This function forms
+ * x for n scores; the exponential and the e4m3 rounding are done by the caller
+ * (oracle/leanp.py) in float64 and with the table codec.
  */
 void leanp_exact_arg(const float* s, int n, float a, int m, int kb, float* x) {
     const float a8 = a * 0.125f;
-    const float c = (float)(8 * (7 + kb) - m) * 0.125f;
+    const float c = (float)(LEANP_TOP - 56 + 8 * kb - m) * 0.125f;
     for (int i = 0; i < n; ++i) x[i] = fmaf(s[i], a8, c);
 }
-

@@ -37,28 +37,47 @@ def lib():
     if _lib is None:
         _lib = ctypes.CDLL(build())
         f32, i32, u8p = ctypes.c_float, ctypes.c_int, ctypes.POINTER(ctypes.c_uint8)
+        i8p = ctypes.POINTER(ctypes.c_int8)
         fp = ctypes.POINTER(ctypes.c_float)
         dp = ctypes.POINTER(ctypes.c_double)
-        _lib.leanp_fmaf.restype = f32
-        _lib.leanp_fmaf.argtypes = [f32, f32, f32]
-        _lib.leanp_e4m3_decode.restype = ctypes.c_double
-        _lib.leanp_e4m3_decode.argtypes = [ctypes.c_uint8]
-        _lib.leanp_update_max.restype = i32
-        _lib.leanp_update_max.argtypes = [f32, f32, i32, i32]
-        _lib.leanp_kshift.restype = i32
-        _lib.leanp_kshift.argtypes = [f32, f32, i32, i32]
-        _lib.leanp_code.restype = ctypes.c_uint8
-        _lib.leanp_code.argtypes = [f32, f32, i32, i32]
-        _lib.leanp_encode_row_tile.restype = None
-        _lib.leanp_encode_row_tile.argtypes = [fp, i32, f32, i32, i32, u8p, u8p]
-        _lib.leanp_encode_row.restype = None
-        _lib.leanp_encode_row.argtypes = [fp, i32, i32, f32, i32, u8p, u8p,
-                                          ctypes.POINTER(ctypes.c_int)]
-        _lib.leanp_attention_row.restype = None
-        _lib.leanp_attention_row.argtypes = [fp, i32, i32, dp, i32, f32, i32, dp, dp]
-        _lib.leanp_exact_arg.restype = None
-        _lib.leanp_exact_arg.argtypes = [fp, i32, f32, i32, i32, fp]
+        ip = ctypes.POINTER(ctypes.c_int)
+        sigs = {
+            "leanp_fmaf": (f32, [f32, f32, f32]),
+            "leanp_e4m3_decode": (ctypes.c_double, [ctypes.c_uint8]),
+            "leanp_reading_top": (i32, []),
+            "leanp_reading_headroom": (i32, []),
+            "leanp_reading_kmin": (i32, []),
+            "leanp_update_max": (i32, [f32, f32, i32, i32]),
+            "leanp_update_max_ex": (i32, [f32, f32, i32, i32, i32]),
+            "leanp_kshift": (i32, [f32, f32, i32, i32]),
+            "leanp_kshift_ex": (i32, [f32, f32, i32, i32, i32]),
+            "leanp_code": (ctypes.c_uint8, [f32, f32, i32, i32]),
+            "leanp_code_ex": (ctypes.c_uint8, [f32, f32, i32, i32, i32]),
+            "leanp_encode_row_tile": (None, [fp, i32, f32, i32, i32, u8p, i8p]),
+            "leanp_encode_row": (None, [fp, i32, i32, f32, i32, u8p, i8p, ip]),
+            "leanp_encode_row_ex": (None, [fp, i32, i32, f32, i32, i32, i32, i32, u8p, i8p,
+                                           ip]),
+            "leanp_attention_row": (None, [fp, i32, i32, dp, i32, f32, i32, dp, dp]),
+            "leanp_attention_row_ex": (None, [fp, i32, i32, dp, i32, f32, i32, i32, i32, i32,
+                                              dp, dp]),
+            "leanp_exact_arg": (None, [fp, i32, f32, i32, i32, fp]),
+        }
+        for name, (res, args) in sigs.items():
+            fn = getattr(_lib, name)
+            fn.restype = res
+            fn.argtypes = args
     return _lib
+
+
+def reading():
+    """(T, H, KMIN) of the reading the kernel follows: block maxima code into (T - 8, T],
+    the reference max is raised once the tile max exceeds it by more than H codes, and a
+    block's shift k_b lies in [KMIN, KMAX]."""
+    L = lib()
+    return L.leanp_reading_top(), L.leanp_reading_headroom(), L.leanp_reading_kmin()
+
+
+EAGER = (120, 0, 0)  # the eager reading: reference raised on every tile, block max at 120
 
 
 def _ptr(a, ct):
@@ -84,38 +103,40 @@ def code(s, a, m, kb):
     return lib().leanp_code(float(s), float(a), int(m), int(kb))
 
 
+def unit_exponent():
+    """log2 of the weight of code T: weights are decode(code) 2^-(T/8 - 7 + k_b)."""
+    return reading()[0] // 8 - 7
+
+
 def update_max(mu_tile, a, m_old, m_valid):
     return lib().leanp_update_max(float(mu_tile), float(a), int(m_old), int(m_valid))
 
 
-def encode_row(s_row, a, tile=TILE, kmax=KMAX):
+def encode_row(s_row, a, tile=TILE, kmax=KMAX, rd=None):
     """Replay the per-row state machine over raw float32 scores ``s_row`` (length a
-    multiple of ``tile``; -inf where masked).  Returns (codes uint8 [n], kshift uint8
-    [n/64], mref int32 [n/tile])."""
+    multiple of ``tile``; -inf where masked) under the reading ``rd`` = (T, H, KMIN)
+    (default: the kernel's).  Returns (codes uint8 [n], kshift int8 [n/64],
+    mref int32 [n/tile])."""
     s = np.ascontiguousarray(s_row, dtype=np.float32)
     n = s.shape[0]
     assert n % tile == 0 and tile % 64 == 0
+    top, hr, kmin = reading() if rd is None else rd
     codes = np.zeros(n, dtype=np.uint8)
-    ks = np.zeros(n // 64, dtype=np.uint8)
+    ks = np.zeros(n // 64, dtype=np.int8)
     mref = np.zeros(n // tile, dtype=np.int32)
-    lib().leanp_encode_row(_ptr(s, ctypes.c_float), n // tile, tile, float(a), int(kmax),
-                           _ptr(codes, ctypes.c_uint8), _ptr(ks, ctypes.c_uint8),
-                           _ptr(mref, ctypes.c_int))
+    lib().leanp_encode_row_ex(_ptr(s, ctypes.c_float), n // tile, tile, float(a), int(kmax),
+                              int(top), int(hr), int(kmin), _ptr(codes, ctypes.c_uint8),
+                              _ptr(ks, ctypes.c_int8), _ptr(mref, ctypes.c_int))
     return codes, ks, mref
 
 
-def raw_scores(q_codes_row, k_codes):
-    """Raw scores of one query row: float32(exact sum of decoded e4m3 products)."""
-    qd = _e4m3.e4m3_decode(q_codes_row)
-    kd = _e4m3.e4m3_decode(k_codes)
-    return (kd @ qd).astype(np.float32)
-
-
 def attention_rows(q_codes, k_codes, v_codes, dq, dk, dv, rows, heads, batch=0,
-                   causal=True, tile=TILE, kmax=KMAX):
+                   causal=True, tile=TILE, kmax=KMAX, rd=None):
     """End-to-end lean-P prediction for selected rows/heads from e4m3 codes and descales.
-    Layout as in oracle.attention (BSHD).  Returns (o [len(heads), len(rows), d_v],
-    lse [len(heads), len(rows)])."""
+    Layout as in oracle.attention (BSHD).  rd = (T, H, KMIN) selects the reading (default:
+    the kernel's lazy one; EAGER for the reference raised on every tile).
+    Returns (o [len(heads), len(rows), d_v], lse [len(heads), len(rows)])."""
+    top, hr, kmin = reading() if rd is None else rd
     Hq = q_codes.shape[2]
     Hkv = k_codes.shape[2]
     G = Hq // Hkv
@@ -135,9 +156,10 @@ def attention_rows(q_codes, k_codes, v_codes, dq, dk, dv, rows, heads, batch=0,
             s = np.ascontiguousarray((kd[:n_vis] @ qd).astype(np.float32))
             orow = np.zeros(d_v)
             lrow = np.zeros(1)
-            L.leanp_attention_row(_ptr(s, ctypes.c_float), n_vis, tile,
-                                  _ptr(vd, ctypes.c_double), d_v, float(a), int(kmax),
-                                  _ptr(orow, ctypes.c_double), _ptr(lrow, ctypes.c_double))
+            L.leanp_attention_row_ex(_ptr(s, ctypes.c_float), n_vis, tile,
+                                     _ptr(vd, ctypes.c_double), d_v, float(a), int(kmax),
+                                     int(top), int(hr), int(kmin), _ptr(orow, ctypes.c_double),
+                                     _ptr(lrow, ctypes.c_double))
             o[hi, ri] = orow
             lse[hi, ri] = lrow[0]
     return o, lse
@@ -168,7 +190,7 @@ def exact_codes(s, a, m, kb):
 def encode_row_exact(s_row, a, tile=TILE, kmax=KMAX):
     """Exact-P codes of one row: the lean-P state machine (encode_row) fixes the reference
     max per tile and the shift per 64-key block; the codes are then exact_codes.
-    Returns (codes uint8 [n], kshift uint8 [n/64], mref int32 [n/tile])."""
+    Returns (codes uint8 [n], kshift int8 [n/64], mref int32 [n/tile])."""
     s = np.ascontiguousarray(s_row, dtype=np.float32)
     _, ks, mref = encode_row(s, a, tile, kmax)
     codes = np.zeros(s.shape[0], dtype=np.uint8)
@@ -183,13 +205,14 @@ def encode_row_exact(s_row, a, tile=TILE, kmax=KMAX):
 
 def combine_row(codes, ks, mref, n_vis, vd, tile=TILE):
     """Normalised output row and lse from the codes of one row, in float64: weight of key j
-    = decode(code_j) 2^-(7 + k_b(j)) 2^((m_t(j) - m_final)/8), o = sum w_j v_j / sum w_j,
+    = decode(code_j) 2^-(T/8 - 7 + k_b(j)) 2^((m_t(j) - m_final)/8), o = sum w_j v_j / sum w_j,
     lse = ln 2 (m_final/8 + log2 sum w_j) with the weights taken relative to m_final.  This
     is the tile-by-tile online combination with its rescales written out."""
     ntiles = (n_vis + tile - 1) // tile
     m_final = int(mref[ntiles - 1])  # any common reference cancels in o; lse adds it back
     j = np.arange(n_vis)
-    w = (_e4m3.e4m3_decode(codes[:n_vis]) * np.exp2(-(7.0 + ks[j // 64].astype(np.float64)))
+    w = (_e4m3.e4m3_decode(codes[:n_vis])
+         * np.exp2(-(unit_exponent() + ks[j // 64].astype(np.float64)))
          * np.exp2((mref[j // tile].astype(np.float64) - m_final) / 8.0))
     l = w.sum()
     o = (w[:, None] * vd[:n_vis]).sum(axis=0) / l

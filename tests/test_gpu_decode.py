@@ -85,9 +85,24 @@ def test_decode_fp8(B, Hq, Hkv, lengths, page):
     ref, lref = decode.decode_attention(deq(q8, dq), deq(k8, dk), deq(v8, dv), table, lens, page)
     got = o.float().cpu().numpy()
     ok = lens > 0
-    # fp32 arithmetic on exactly dequantised inputs: only the bf16 output rounding remains
+    # fp32 arithmetic on exactly dequantised inputs: only the 16-bit rounding of p and the
+    # bf16 output rounding remain
     assert rel_rms(got[ok], ref[ok]) <= 5e-3
     np.testing.assert_allclose(lse.cpu().numpy()[ok], lref[ok], rtol=0, atol=1e-3)
+    # elementwise: the rounding errors scale with sum_j p_j |v_j| (>= |o|), the attention of
+    # |V| -- 1e-2 of it, or 1e-2 absolute where that is below one (as for BF16 prefill)
+    mag, _ = decode.decode_attention(deq(q8, dq), deq(k8, dk), np.abs(deq(v8, dv)), table, lens,
+                                     page)
+    assert (np.abs(got[ok] - ref[ok]) / (1e-2 * np.maximum(1.0, mag[ok]))).max() <= 1.0
+    # one cached token: o is that token's dequantised value row, fp32(code * descale_v)
+    # rounded to bf16, exactly
+    G = Hq // Hkv
+    v8h = v8.cpu().numpy()
+    for b in np.nonzero(lens == 1)[0]:
+        codes = v8h[table[b, 0], 0, [h // G for h in range(Hq)]]
+        want = (quantize.dequantize(codes, 1.0).astype(np.float32) * np.float32(dv.item()))
+        want = torch.from_numpy(want.astype(np.float32)).to(torch.bfloat16)
+        assert torch.equal(o[b].cpu(), want)
 
 
 def test_bad_page_id_reported_not_faulted():

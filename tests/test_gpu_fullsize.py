@@ -56,6 +56,9 @@ def test_bf16_fullsize(name):
         got = o[b][rows][:, heads, :].transpose(1, 0, 2)
         err = np.abs(got - ref)
         assert (err / (1e-2 * np.maximum(1.0, mag))).max() <= 1.0
+        if dist == "gaussian":
+            # unit-scale inputs: the plain BF16 bar, max-abs 1e-2
+            assert err.max() <= 1e-2
         assert rel_rms(got, ref) <= 5e-3
         assert np.abs(lse[b][heads][:, rows] - lref).max() <= 2e-3
 

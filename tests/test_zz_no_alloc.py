@@ -51,3 +51,20 @@ def test_static_entry_rejects_bad_arguments():
     assert f(vp(256), vp(256), vp(256), 4, 2, 100, 0, None) == pkg.ATTN_ERR_INVALID_ARG
     assert f(vp(256), vp(256), vp(256), -1, 2, 128, 0, None) == pkg.ATTN_ERR_INVALID_ARG
     assert f(vp(256), vp(256), vp(256), 4, 2, 64, 1, None) == pkg.ATTN_ERR_UNSUPPORTED
+
+
+def test_static_entry_empty_tensor_sets_descale_one_and_writes_no_codes():
+    """tokens == 0: no element to quantise; descale is set to 1 on the device and the
+    output buffer is left as it was."""
+    f = _static_entry()
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    codes = torch.full((64,), 0xAB, dtype=torch.uint8, device="cuda")
+    ds = torch.full((1,), -1.0, dtype=torch.float32, device="cuda")
+    x = torch.zeros((64,), dtype=torch.bfloat16, device="cuda")
+    st = f(ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(codes.data_ptr()),
+           ctypes.c_void_p(ds.data_ptr()), 0, 4, 128, 0, stream)
+    assert st == pkg.ATTN_OK, pkg.status_string(st)
+    torch.cuda.synchronize()
+    assert ds.item() == 1.0
+    assert bool((codes == 0xAB).all())
+    assert pkg.attn_device_status() == pkg.ATTN_OK
