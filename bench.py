@@ -338,9 +338,22 @@ def gpu_bench(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
+    pkg.attn_select_prefill_kernel(pkg.ATTN_KERNEL_PAIR if args.kernel == "pair"
+                                   else pkg.ATTN_KERNEL_SINGLE)
     B, S, Hq, Hkv, dqk, dv, distn, desc = WORKLOADS[args.workload]
-    flops = causal_flops(B, Hq, S, dqk, dv)
-    q_h, k_h, v_h = synth.make_qkv(B, S, Hq, Hkv, dqk, dv, seed=rank, dist=distn)
+    if args.split == "heads":
+        # one problem shared by all ranks: rank r takes a contiguous range of kv heads and
+        # their query heads; no data-path collective
+        from bf16_causal_prefill_attn_b200 import shard
+        q_h, k_h, v_h = synth.make_qkv(B, S, Hq, Hkv, dqk, dv, seed=0, dist=distn)
+        q_h, k_h, v_h = shard.slice_heads(q_h, k_h, v_h, Hq, Hkv, world, rank)
+        job_flops = causal_flops(B, Hq, S, dqk, dv)
+        Hq, Hkv = q_h.shape[2], k_h.shape[2]
+        flops = causal_flops(B, Hq, S, dqk, dv)
+    else:
+        q_h, k_h, v_h = synth.make_qkv(B, S, Hq, Hkv, dqk, dv, seed=rank, dist=distn)
+        flops = causal_flops(B, Hq, S, dqk, dv)
+        job_flops = flops * world
     q_h, k_h, v_h = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
     q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
     stream = torch.cuda.current_stream(dev)
@@ -356,9 +369,8 @@ def gpu_bench(args, rank, world, local_rank):
     o_h = torch.empty(o.shape, dtype=torch.bfloat16).pin_memory()
 
     def fp8_step(ev_a=None, ev_b=None):
-        pkg.attn_quantize_e4m3(q, hadamard=args.hadamard, out=q8, descale=ds[0], workspace=ws[0])
-        pkg.attn_quantize_e4m3(k, hadamard=args.hadamard, out=k8, descale=ds[1], workspace=ws[1])
-        pkg.attn_quantize_e4m3(v, hadamard=args.hadamard, out=v8, descale=ds[2], workspace=ws[2])
+        pkg.attn_quantize_qkv_e4m3(q, k, v, hadamard=args.hadamard, out=(q8, k8, v8),
+                                   descales=ds, workspace=ws[0])
         if ev_a is not None:
             ev_a.record(stream)
         pkg.attn_fwd(q8, k8, v8, descale_q=ds[0], descale_k=ds[1], descale_v=ds[2], out=o, lse=lse,
@@ -445,9 +457,10 @@ def gpu_bench(args, rank, world, local_rank):
                     s_cmp.wait_event(bf["in"])
                     if bf["used"]:
                         s_cmp.wait_event(bf["out"])      # O of step i-2 has left the device
-                    for x, c, d_, w_ in zip(("q", "k", "v"), ("q8", "k8", "v8"), bf["ds"], bf["ws"]):
-                        pkg.attn_quantize_e4m3(bf[x], hadamard=args.hadamard, out=bf[c],
-                                               descale=d_, workspace=w_, stream=s_cmp)
+                    pkg.attn_quantize_qkv_e4m3(bf["q"], bf["k"], bf["v"], hadamard=args.hadamard,
+                                               out=(bf["q8"], bf["k8"], bf["v8"]),
+                                               descales=bf["ds"], workspace=bf["ws"][0],
+                                               stream=s_cmp)
                     pkg.attn_fwd(bf["q8"], bf["k8"], bf["v8"], descale_q=bf["ds"][0],
                                  descale_k=bf["ds"][1], descale_v=bf["ds"][2], out=bf["o"],
                                  lse=bf["lse"], unrotate=args.hadamard, exact_p=args.exact_p,
@@ -515,23 +528,28 @@ def gpu_bench(args, rank, world, local_rank):
     traffic = {} if args.exact_p else load_traffic(args.workload)
     result = {
         "metric": METRIC,
-        "value": round(job_tflops(flops, world, fp8_ms), 2),
+        "value": round(job_tflops(job_flops, 1, fp8_ms), 2),
         "unit": UNIT,
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": round(fp8_ms, 4),
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "strong" if args.split == "heads" else "weak",
         "vs_baseline": None,
         "dtype": "e4m3",
         "data": "synthetic",
-        "config": {"workload": desc, "name": args.workload, "B": B, "S": S, "Hq": Hq, "Hkv": Hkv,
+        "config": {"workload": desc, "name": args.workload, "B": B, "S": S,
+                   "Hq": WORKLOADS[args.workload][2], "Hkv": WORKLOADS[args.workload][3],
                    "d_qk": dqk, "d_v": dv, "hadamard": bool(args.hadamard),
+                   "kernel": args.kernel,
                    "step": "e4m3 quantisation of Q, K, V + "
                            + ("exact-P attention (ablation)" if args.exact_p else "lean-P attention"),
                    "l2": "256 MiB L2 flush written between steps, outside the timed step",
-                   "parallelism": f"replicas x{world} (independent problems per GPU)"},
+                   "parallelism": (f"heads split x{world} (one problem; each GPU {Hkv} kv heads "
+                                   f"and their {Hq} query heads; no data-path collective)"
+                                   if args.split == "heads" else
+                                   f"replicas x{world} (independent problems per GPU)")},
         "roofline": {"bound": "tensor", "achieved": round(fp8_kern_tf, 2),
                      "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
                      "frac": round(fp8_kern_tf / fp8_peak, 4),
@@ -541,7 +559,7 @@ def gpu_bench(args, rank, world, local_rank):
                      "kernel_ms_median": round(statistics.median(fp8_kern_ms), 4),
                      "kernel_ms_min": round(min(fp8_kern_ms), 4),
                      "traffic": traffic.get("fp8")},
-        "bf16": {"value": round(job_tflops(flops, world, bf16_ms), 2), "unit": UNIT,
+        "bf16": {"value": round(job_tflops(job_flops, 1, bf16_ms), 2), "unit": UNIT,
                  "ms_per_step": round(bf16_ms, 4), "dtype": "bf16",
                  "roofline": {"bound": "tensor", "achieved": round(bf16_kern_tf, 2),
                               "peak": round(bf16_peak, 1), "unit": "TFLOP/s",
@@ -552,15 +570,16 @@ def gpu_bench(args, rank, world, local_rank):
                               "kernel_ms_median": round(statistics.median(bf16_kern_ms), 4),
                               "kernel_ms_min": round(min(bf16_kern_ms), 4),
                               "traffic": traffic.get("bf16")}},
-        "e2e": {"value": round(job_tflops(flops, world, e2e_pipe), 2), "unit": UNIT,
+        "e2e": {"value": round(job_tflops(job_flops, 1, e2e_pipe), 2), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_pipe, 4),
                 "mode": "K steps pipelined over three streams (inputs in, compute, result out); "
                         "time of the whole region / K",
-                "serial": {"value": round(job_tflops(flops, world, e2e_mean), 2),
+                "serial": {"value": round(job_tflops(job_flops, 1, e2e_mean), 2),
                            "ms_per_step": round(e2e_mean, 4),
                            "mode": "each step: copies in, quantise + attention, copy out"}},
-        "gpu_launches": args.steps * 7 + args.steps,
+        # per FP8 step: 2 quantiser kernels + 1 attention kernel; per BF16 step: 1
+        "gpu_launches": args.steps * 3 + args.steps,
         "clocks": clocks,
     }
     if energy is not None:
@@ -723,12 +742,22 @@ def main(argv=None):
                     help="skip the NVML energy windows (about 12 s of extra GPU time)")
     ap.add_argument("--exact-p", action="store_true",
                     help="FP8 probabilities by exponential + e4m3 rounding (the ablation of lean P)")
+    ap.add_argument("--kernel", default="single", choices=["pair", "single"],
+                    help="prefill kernel family: CTA pairs with M = 256 MMAs (default) or "
+                         "single CTAs with M = 128 MMAs")
+    ap.add_argument("--split", default="replicas", choices=["replicas", "heads"],
+                    help="multi-GPU: an independent problem per GPU (weak scaling), or one "
+                         "problem divided by kv heads (strong scaling)")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
+    if args.split == "heads" and args.workload in WORKLOADS:
+        world_ = int(os.environ.get("WORLD_SIZE", "1"))
+        if world_ > WORKLOADS[args.workload][3]:
+            ap.error("--split heads needs at most Hkv GPUs")
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

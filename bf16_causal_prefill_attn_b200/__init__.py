@@ -22,6 +22,8 @@ ATTN_BF16 = 0
 ATTN_FP8_E4M3 = 1
 ATTN_FLAG_UNROTATE_O = 1
 ATTN_FLAG_EXACT_P = 2
+ATTN_KERNEL_SINGLE = 0
+ATTN_KERNEL_PAIR = 1
 
 _lib = None
 
@@ -62,12 +64,19 @@ def lib():
         L.attn_quantize_e4m3.argtypes = [vp, vp, vp, ctypes.c_int64, i32, i32, i32, vp,
                                          ctypes.c_size_t, vp]
         L.attn_quantize_e4m3.restype = i32
+        L.attn_quantize_qkv_e4m3.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int64,
+                                             i32, i32, i32, i32, i32, vp, ctypes.c_size_t, vp]
+        L.attn_quantize_qkv_e4m3.restype = i32
+        L.attn_quantize_qkv_workspace_size.argtypes = []
+        L.attn_quantize_qkv_workspace_size.restype = ctypes.c_size_t
         L.attn_quantize_workspace_size.argtypes = [ctypes.c_int64, i32, i32]
         L.attn_quantize_workspace_size.restype = ctypes.c_size_t
         L.attn_device_status.argtypes = [vp]
         L.attn_device_status.restype = i32
         L.attn_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
         L.attn_set_wait_timeout_ns.restype = None
+        L.attn_select_prefill_kernel.argtypes = [i32]
+        L.attn_select_prefill_kernel.restype = i32
         L.attn_selftest_stall_tile.argtypes = [i32]
         L.attn_selftest_stall_tile.restype = None
         L.attn_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
@@ -252,6 +261,35 @@ def attn_quantize_e4m3(x, hadamard=False, out=None, descale=None, workspace=None
     return out, descale
 
 
+def attn_quantize_qkv_e4m3(q, k, v, hadamard=False, out=None, descales=None, workspace=None,
+                           stream=None):
+    """Per-tensor e4m3 quantisation of Q, K and V (contiguous bf16 [.., H, d]) in two
+    launches.  out: optional (q8, k8, v8) uint8 tensors; descales: optional three fp32 [1]
+    tensors.  Returns ((q8, dq), (k8, dk), (v8, dv))."""
+    for x in (q, k, v):
+        if x.dtype != torch.bfloat16 or not x.is_contiguous():
+            raise ValueError("q, k, v must be contiguous bf16 tensors")
+    Hq, d_qk = q.shape[-2], q.shape[-1]
+    Hkv, d_v = v.shape[-2], v.shape[-1]
+    tokens = q.numel() // (Hq * d_qk) if q.numel() else 0
+    if k.numel() != tokens * Hkv * d_qk or v.numel() != tokens * Hkv * d_v:
+        raise ValueError("q, k, v token counts differ")
+    if out is None:
+        out = tuple(torch.empty(x.shape, dtype=torch.uint8, device=x.device) for x in (q, k, v))
+    if descales is None:
+        descales = tuple(torch.empty((1,), dtype=torch.float32, device=q.device) for _ in range(3))
+    ws_bytes = lib().attn_quantize_qkv_workspace_size()
+    if workspace is None:
+        workspace = torch.empty((ws_bytes + 3) // 4, dtype=torch.int32, device=q.device)
+    st = lib().attn_quantize_qkv_e4m3(_ptr(q), _ptr(k), _ptr(v), *(_ptr(t) for t in out),
+                                      *(_ptr(t) for t in descales), tokens, Hq, Hkv, d_qk, d_v,
+                                      1 if hadamard else 0, _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(),
+                                      _stream(stream))
+    _check(st, "attn_quantize_qkv_e4m3")
+    return tuple(zip(out, descales))
+
+
 def attn_device_status(stream=None):
     """Synchronise the stream and return the device status code (ATTN_OK, ATTN_ERR_*)."""
     return lib().attn_device_status(_stream(stream))
@@ -259,6 +297,12 @@ def attn_device_status(stream=None):
 
 def attn_set_wait_timeout_ns(ns):
     lib().attn_set_wait_timeout_ns(int(ns))
+
+
+def attn_select_prefill_kernel(kernel):
+    """Prefill kernel family for later calls: ATTN_KERNEL_PAIR (default, CTA pairs with
+    M = 256 MMAs) or ATTN_KERNEL_SINGLE (one CTA, M = 128)."""
+    _check(lib().attn_select_prefill_kernel(int(kernel)), "attn_select_prefill_kernel")
 
 
 def attn_selftest_stall_tile(tile):

@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -11,6 +13,7 @@
 
 #include "../../include/attn.h"
 #include "attn_fwd.cuh"
+#include "attn_pair.cuh"
 #include "decode.cuh"
 #include "quantize.cuh"
 
@@ -24,6 +27,7 @@ __device__ uint32_t g_dev_err = 0;
 
 uint64_t g_timeout_ns = kDefaultTimeoutNs;
 int g_stall_tile = -1;  // test-only (attn_selftest_stall_tile)
+int g_kernel = ATTN_KERNEL_SINGLE;  // prefill kernel family (attn_select_prefill_kernel)
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -46,19 +50,37 @@ bool dev_err_ptr(uint32_t** out) {
   return true;
 }
 
-// 3-D tiled map over [T, H, d] (d innermost), box = (box_cols, 1, 128), 128-B swizzle.
+// 3-D tiled map over [T, H, d] (d innermost), box = (box_cols, 1, box_rows).
 bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, uint64_t d,
-              uint64_t H, uint64_t T, uint32_t box_cols) {
+              uint64_t H, uint64_t T, uint32_t box_cols, uint32_t box_rows = 128,
+              CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {d, H, T};
   cuuint64_t strides[2] = {d * esize, H * d * esize};
-  cuuint32_t box[3] = {box_cols, 1, 128};
+  cuuint32_t box[3] = {box_cols, 1, box_rows};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// The prefill kernels move registers from their producer/MMA warps to their softmax warps
+// (setmaxnreg); the increase only succeeds if the block was launched with at least
+// REGS_NEEDED_AT_LAUNCH registers per thread, so never launch one with fewer.  The count
+// is a property of the compiled kernel: checked once per kernel, then remembered.
+template <typename K>
+attn_status_t register_split_ok(K kern) {
+  static std::atomic<int> known{0};  // 0 not yet checked, 1 ok, 2 too few registers
+  const int k = known.load(std::memory_order_relaxed);
+  if (k != 0) return k == 1 ? ATTN_OK : ATTN_ERR_UNSUPPORTED;
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return ATTN_ERR_CUDA;  // not cached
+  const bool ok = fa.numRegs >= attn::REGS_NEEDED_AT_LAUNCH &&
+                  fa.numRegs * attn::NUM_THREADS <= 65536;
+  known.store(ok ? 1 : 2, std::memory_order_relaxed);
+  return ok ? ATTN_OK : ATTN_ERR_UNSUPPORTED;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -79,17 +101,64 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, attn::FwdP
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC) !=
       cudaSuccess)
     return ATTN_ERR_CUDA;
-  // The kernel moves registers from its producer/MMA warps to its softmax warps
-  // (setmaxnreg); the increase only succeeds if the block was launched with at least
-  // REGS_NEEDED_AT_LAUNCH registers per thread, so never launch with fewer.
-  cudaFuncAttributes fa;
-  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return ATTN_ERR_CUDA;
-  if (fa.numRegs < attn::REGS_NEEDED_AT_LAUNCH ||
-      fa.numRegs * attn::NUM_THREADS > 65536)
-    return ATTN_ERR_UNSUPPORTED;
+  const attn_status_t rs = register_split_ok(kern);
+  if (rs != ATTN_OK) return rs;
   const unsigned grid = static_cast<unsigned>(prm.n_pairs) * prm.B * prm.Hq;
   kern<<<grid, attn::NUM_THREADS, C::SMEM_ALLOC, stream>>>(mq, mk, mv, prm);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// The pair kernel: clusters of two CTAs, M = 256 MMAs (attn_pair.cuh).  Units along the
+// queries: pairs of query tiles (heads mode, Hq / Hkv even) or quads (rows mode).
+template <bool FP8, int DQK, bool DUMP, bool EXACT = false, bool VARLEN = false>
+attn_status_t launch_pair(const void* q, const void* k, const void* v, attn::FwdParams& prm,
+                          cudaStream_t stream) {
+  using C = attn::PairCfg<FP8, DQK>;
+  const CUtensorMapDataType dt =
+      FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const uint64_t T = static_cast<uint64_t>(prm.total_tokens);
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, dt, C::E, DQK, prm.Hq, T, C::BOX_COLS) ||
+      !make_map(&mk, k, dt, C::E, DQK, prm.Hkv, T, C::BOX_COLS, 64) ||
+      !make_map(&mv, v, dt, C::E, attn::DV, prm.Hkv, T, 64, 128,
+                FP8 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B))
+    return ATTN_ERR_CUDA;
+  auto kern = attn::attn_pair_kernel<FP8, DQK, DUMP, EXACT, VARLEN>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC) !=
+      cudaSuccess)
+    return ATTN_ERR_CUDA;
+  const attn_status_t rs = register_split_ok(kern);
+  if (rs != ATTN_OK) return rs;
+  const bool heads_mode = (prm.G % 2) == 0;
+  attn::FwdParams pp = prm;
+  pp.n_pairs = heads_mode ? (prm.n_q_tiles + 1) / 2 : (prm.n_q_tiles + 3) / 4;
+  const int64_t units =
+      static_cast<int64_t>(pp.n_pairs) * prm.B * (heads_mode ? prm.Hq / 2 : prm.Hq);
+  if (units * 2 > INT32_MAX) return ATTN_ERR_UNSUPPORTED;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(units * 2));
+  cfg.blockDim = dim3(attn::NUM_THREADS);
+  cfg.dynamicSmemBytes = C::SMEM_ALLOC;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, pp) != cudaSuccess) return ATTN_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// Kernel family for one instantiation: the pair kernel unless the single-CTA one is
+// selected (attn_select_prefill_kernel).
+template <bool FP8, int DQK, bool DUMP, bool EXACT = false, bool VARLEN = false>
+attn_status_t launch_prefill(const void* q, const void* k, const void* v, attn::FwdParams& prm,
+                             cudaStream_t stream) {
+  if (g_kernel == ATTN_KERNEL_PAIR)
+    return launch_pair<FP8, DQK, DUMP, EXACT, VARLEN>(q, k, v, prm, stream);
+  return launch_fwd<FP8, DQK, DUMP, EXACT, VARLEN>(q, k, v, prm, stream);
 }
 
 // Checks shared by the fixed-length and packed entry points; fills the parameters that
@@ -142,30 +211,30 @@ attn_status_t dispatch(const void* q, const void* k, const void* v, int d_qk, at
     // test-only dump)
     if (exact || dump) return ATTN_ERR_UNSUPPORTED;
     if (dtype == ATTN_BF16) {
-      if (d_qk == 128) return launch_fwd<false, 128, false, false, true>(q, k, v, prm, st);
-      return launch_fwd<false, 192, false, false, true>(q, k, v, prm, st);
+      if (d_qk == 128) return launch_prefill<false, 128, false, false, true>(q, k, v, prm, st);
+      return launch_prefill<false, 192, false, false, true>(q, k, v, prm, st);
     }
-    if (d_qk == 128) return launch_fwd<true, 128, false, false, true>(q, k, v, prm, st);
-    return launch_fwd<true, 192, false, false, true>(q, k, v, prm, st);
+    if (d_qk == 128) return launch_prefill<true, 128, false, false, true>(q, k, v, prm, st);
+    return launch_prefill<true, 192, false, false, true>(q, k, v, prm, st);
   }
   if (dtype == ATTN_BF16) {
-    if (d_qk == 128) return launch_fwd<false, 128, false>(q, k, v, prm, st);
-    return launch_fwd<false, 192, false>(q, k, v, prm, st);
+    if (d_qk == 128) return launch_prefill<false, 128, false>(q, k, v, prm, st);
+    return launch_prefill<false, 192, false>(q, k, v, prm, st);
   }
   if (dump) {
     if (exact) {
-      if (d_qk == 128) return launch_fwd<true, 128, true, true>(q, k, v, prm, st);
-      return launch_fwd<true, 192, true, true>(q, k, v, prm, st);
+      if (d_qk == 128) return launch_prefill<true, 128, true, true>(q, k, v, prm, st);
+      return launch_prefill<true, 192, true, true>(q, k, v, prm, st);
     }
-    if (d_qk == 128) return launch_fwd<true, 128, true>(q, k, v, prm, st);
-    return launch_fwd<true, 192, true>(q, k, v, prm, st);
+    if (d_qk == 128) return launch_prefill<true, 128, true>(q, k, v, prm, st);
+    return launch_prefill<true, 192, true>(q, k, v, prm, st);
   }
   if (exact) {
-    if (d_qk == 128) return launch_fwd<true, 128, false, true>(q, k, v, prm, st);
-    return launch_fwd<true, 192, false, true>(q, k, v, prm, st);
+    if (d_qk == 128) return launch_prefill<true, 128, false, true>(q, k, v, prm, st);
+    return launch_prefill<true, 192, false, true>(q, k, v, prm, st);
   }
-  if (d_qk == 128) return launch_fwd<true, 128, false>(q, k, v, prm, st);
-  return launch_fwd<true, 192, false>(q, k, v, prm, st);
+  if (d_qk == 128) return launch_prefill<true, 128, false>(q, k, v, prm, st);
+  return launch_prefill<true, 192, false>(q, k, v, prm, st);
 }
 
 attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B,
@@ -438,6 +507,85 @@ attn_status_t attn_quantize_e4m3(const void* x_bf16, void* x_e4m3, float* descal
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+size_t attn_quantize_qkv_workspace_size(void) { return 16; }
+
+attn_status_t attn_quantize_qkv_e4m3(const void* q, const void* k, const void* v, void* q8,
+                                     void* k8, void* v8, float* descale_q, float* descale_k,
+                                     float* descale_v, int64_t tokens, int Hq, int Hkv, int d_qk,
+                                     int d_v, int hadamard, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  if (tokens < 0 || Hq <= 0 || Hkv <= 0 || d_qk <= 0 || d_v <= 0 || (d_qk % 8) != 0 ||
+      (d_v % 8) != 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (hadamard != 0 && hadamard != 1) return ATTN_ERR_INVALID_ARG;
+  if (hadamard && (d_qk != 128 || d_v != 128)) return ATTN_ERR_UNSUPPORTED;
+  if (!descale_q || !descale_k || !descale_v || !workspace) return ATTN_ERR_INVALID_ARG;
+  if (workspace_bytes < attn_quantize_qkv_workspace_size()) return ATTN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 3u) ||
+      (reinterpret_cast<uintptr_t>(descale_q) & 3u) ||
+      (reinterpret_cast<uintptr_t>(descale_k) & 3u) ||
+      (reinterpret_cast<uintptr_t>(descale_v) & 3u))
+    return ATTN_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (tokens == 0) {
+    for (float* d : {descale_q, descale_k, descale_v}) {
+      attn::descale_one_kernel<<<1, 1, 0, st>>>(d);
+      if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    }
+    return ATTN_OK;
+  }
+  if (!q || !k || !v || !q8 || !k8 || !v8) return ATTN_ERR_INVALID_ARG;
+  for (const void* p : {q, k, v, static_cast<const void*>(q8), static_cast<const void*>(k8),
+                        static_cast<const void*>(v8)})
+    if (!aligned16(p)) return ATTN_ERR_ALIGNMENT;
+  uint32_t* amax = static_cast<uint32_t*>(workspace);
+  if (cudaMemsetAsync(amax, 0, 3 * sizeof(uint32_t), st) != cudaSuccess) return ATTN_ERR_CUDA;
+  // jobs in the order Q, K, V for the amax pass and V, K, Q for the convert pass: the
+  // tensors read last by the first pass are the first re-read by the second, while they
+  // may still be in L2
+  const int64_t el[3] = {tokens * Hq * d_qk, tokens * Hkv * d_qk, tokens * Hkv * d_v};
+  const void* xs[3] = {q, k, v};
+  void* ys[3] = {q8, k8, v8};
+  float* ds[3] = {descale_q, descale_k, descale_v};
+  const int threads = 256;
+  const int64_t per_block_items = hadamard ? threads / 32 : threads;  // rows or chunks
+  const int sms = num_sms();
+  const int64_t budget = int64_t(sms) * 16;  // blocks per pass, split by size
+  int64_t total = 0;
+  for (int i = 0; i < 3; ++i) total += el[i];
+  attn::QuantBatch fwd{}, rev{};
+  fwd.njobs = rev.njobs = 3;
+  int end_f = 0, end_r = 0;
+  for (int o = 0; o < 3; ++o) {
+    for (int pass = 0; pass < 2; ++pass) {
+      const int i = pass == 0 ? o : 2 - o;
+      const int64_t n = hadamard ? el[i] / 128 : el[i] / 8;
+      const int64_t want = (n + per_block_items - 1) / per_block_items;
+      const int64_t share = std::max<int64_t>(1, (budget * el[i] + total - 1) / total);
+      const int nb = static_cast<int>(std::max<int64_t>(1, std::min(want, share)));
+      attn::QuantJob jb{static_cast<const __nv_bfloat16*>(xs[i]), static_cast<uint8_t*>(ys[i]),
+                        n, amax + i, ds[i]};
+      if (pass == 0) {
+        fwd.job[o] = jb;
+        end_f += nb;
+        fwd.block_end[o] = end_f;
+      } else {
+        rev.job[o] = jb;
+        end_r += nb;
+        rev.block_end[o] = end_r;
+      }
+    }
+  }
+  if (hadamard) {
+    attn::amax_batch_kernel<true><<<end_f, threads, 0, st>>>(fwd);
+    attn::convert_batch_kernel<true><<<end_r, threads, 0, st>>>(rev);
+  } else {
+    attn::amax_batch_kernel<false><<<end_f, threads, 0, st>>>(fwd);
+    attn::convert_batch_kernel<false><<<end_r, threads, 0, st>>>(rev);
+  }
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 attn_status_t attn_device_status(void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(st) != cudaSuccess) return ATTN_ERR_CUDA;
@@ -454,6 +602,12 @@ attn_status_t attn_device_status(void* stream) {
 void attn_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns = ns ? ns : kDefaultTimeoutNs; }
 
 void attn_selftest_stall_tile(int tile) { g_stall_tile = tile < 0 ? -1 : tile; }
+
+attn_status_t attn_select_prefill_kernel(int kernel) {
+  if (kernel != ATTN_KERNEL_SINGLE && kernel != ATTN_KERNEL_PAIR) return ATTN_ERR_INVALID_ARG;
+  g_kernel = kernel;
+  return ATTN_OK;
+}
 
 attn_status_t attn_selftest_wait_timeout(uint64_t timeout_ns, void* stream) {
   if (timeout_ns == 0 || timeout_ns > 10000000000ull) return ATTN_ERR_INVALID_ARG;

@@ -62,18 +62,33 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// the same with cluster-scope acquire: for barriers that the other CTA of a pair arrives on
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{.reg .pred p; mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2; "
+      "selp.u32 %0, 1, 0, p;}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait: returns false (and records DEV_TIMEOUT in *err) if the phase with the
 // given parity has not completed within timeout_ns.  A timeout never traps or spins
 // forever; callers unwind and the host reports the error word.  With abort_on_err the
 // wait also gives up as soon as another thread has recorded an error; drains of work
 // already in flight (copies, MMAs) pass false so they always run to their own limit.
+// CLUSTER: acquire at cluster scope (the barrier receives arrivals from the peer CTA).
+template <bool CLUSTER = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err,
                                           uint64_t timeout_ns, bool abort_on_err = true) {
-  if (mbar_try_wait(bar, parity)) return true;
+  auto probe = [&]() { return CLUSTER ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+  if (probe()) return true;
   uint64_t t0 = globaltimer_ns();
   uint32_t it = 0;
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (probe()) return true;
     if ((++it & 63u) == 0u) {
       if (abort_on_err && *reinterpret_cast<volatile uint32_t*>(err) != DEV_OK) return false;
       if (globaltimer_ns() - t0 > timeout_ns) {
@@ -278,7 +293,8 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
   return r;
 }
-// arrive (release, cluster scope) on an mbarrier given by its shared::cluster address
+// arrive (release, cluster scope) on an mbarrier given by its shared::cluster address (this
+// CTA's or the peer's)
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                : "memory");
@@ -380,6 +396,19 @@ __host__ __device__ constexpr uint32_t idesc_mxf8(uint32_t a_mn, uint32_t b_mn, 
                                                   uint32_t N, uint32_t a_sf_id, uint32_t b_sf_id) {
   return (b_sf_id << 4) | (0u << 7) | (0u << 10) | (a_mn << 15) | (b_mn << 16) |
          ((N >> 3) << 17) | (1u << 23) /* UE8M0 */ | ((M >> 4) << 24) | (a_sf_id << 29);
+}
+
+// Shared-memory matrix descriptor, SWIZZLE_64B (layout code 4), version 1: atoms of 8 rows
+// x 64 bytes.
+__device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t saddr, uint32_t lbo_bytes,
+                                                   uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1u << 46;  // version (sm_100)
+  d |= (uint64_t)4u << 61;  // SWIZZLE_64B
+  return d;
 }
 
 // ------------------------------------------------------------------ misc math

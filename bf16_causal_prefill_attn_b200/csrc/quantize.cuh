@@ -157,4 +157,103 @@ __global__ void convert_flat_kernel(const __nv_bfloat16* __restrict__ x, uint8_t
   }
 }
 
+// ---- several tensors in one launch per pass (Q, K and V of one attention call): block b
+// works on job j for block_end[j-1] <= b < block_end[j], grid-striding over that job's
+// range only, so each block reads one tensor and its own amax word.  Same arithmetic and
+// results as one launch per tensor.
+constexpr int QUANT_MAX_JOBS = 3;
+struct QuantJob {
+  const __nv_bfloat16* x;
+  uint8_t* y;
+  int64_t n;          // 16-byte chunks (flat) or 128-element rows (rotated)
+  uint32_t* amax;     // this tensor's amax word (cleared before the amax pass)
+  float* descale;
+};
+struct QuantBatch {
+  QuantJob job[QUANT_MAX_JOBS];
+  int block_end[QUANT_MAX_JOBS];
+  int njobs;
+};
+
+__device__ __forceinline__ int batch_job(const QuantBatch& b, int& first_block) {
+  int j = 0;
+  first_block = 0;
+  while (j + 1 < b.njobs && static_cast<int>(blockIdx.x) >= b.block_end[j]) {
+    first_block = b.block_end[j];
+    ++j;
+  }
+  return j;
+}
+
+template <bool ROT>
+__global__ void amax_batch_kernel(const QuantBatch b) {
+  int first = 0;
+  const int j = batch_job(b, first);
+  const QuantJob& jb = b.job[j];
+  const int nblk = b.block_end[j] - first;
+  const int64_t tid = static_cast<int64_t>(blockIdx.x - first) * blockDim.x + threadIdx.x;
+  float m = 0.0f;
+  if constexpr (ROT) {
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = (static_cast<int64_t>(nblk) * blockDim.x) >> 5;
+    for (int64_t row = tid >> 5; row < jb.n; row += nwarps) {
+      float v[4];
+      load_row4(jb.x, row, lane, v);
+      hadamard_row4(v, lane);
+      m = fmaxf(m, fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3]))));
+    }
+  } else {
+    const int64_t stride = static_cast<int64_t>(nblk) * blockDim.x;
+    for (int64_t i = tid; i < jb.n; i += stride) {
+      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(jb.x) + i);
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        m = fmaxf(m, fmaxf(fabsf(__low2float(h2[k])), fabsf(__high2float(h2[k]))));
+    }
+  }
+  block_amax_atomic(m, jb.amax);
+}
+
+template <bool ROT>
+__global__ void convert_batch_kernel(const QuantBatch b) {
+  int first = 0;
+  const int j = batch_job(b, first);
+  const QuantJob& jb = b.job[j];
+  const int nblk = b.block_end[j] - first;
+  const uint32_t ab = *jb.amax;
+  const float sc = quant_scale(ab);
+  if (blockIdx.x == first && threadIdx.x == 0) {
+    const float amax = __uint_as_float(ab);
+    *jb.descale = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+  }
+  const int64_t tid = static_cast<int64_t>(blockIdx.x - first) * blockDim.x + threadIdx.x;
+  if constexpr (ROT) {
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = (static_cast<int64_t>(nblk) * blockDim.x) >> 5;
+    for (int64_t row = tid >> 5; row < jb.n; row += nwarps) {
+      float v[4];
+      load_row4(jb.x, row, lane, v);
+      hadamard_row4(v, lane);
+      const uint32_t lo = f32_to_e4m3x2(__fmul_rn(v[0], sc), __fmul_rn(v[1], sc));
+      const uint32_t hi = f32_to_e4m3x2(__fmul_rn(v[2], sc), __fmul_rn(v[3], sc));
+      reinterpret_cast<uint32_t*>(jb.y + row * 128)[lane] = lo | (hi << 16);
+    }
+  } else {
+    const int64_t stride = static_cast<int64_t>(nblk) * blockDim.x;
+    for (int64_t i = tid; i < jb.n; i += stride) {
+      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(jb.x) + i);
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+      uint32_t w[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        w[k] = f32_to_e4m3x2(__fmul_rn(__low2float(h2[k]), sc), __fmul_rn(__high2float(h2[k]), sc));
+      uint2 out;
+      out.x = w[0] | (w[1] << 16);
+      out.y = w[2] | (w[3] << 16);
+      reinterpret_cast<uint2*>(jb.y)[i] = out;
+    }
+  }
+}
+
 }  // namespace attn

@@ -168,6 +168,25 @@ attn_status_t attn_quantize_e4m3(const void* x_bf16, void* x_e4m3, float* descal
 size_t attn_quantize_workspace_size(int64_t tokens, int H, int d);
 
 /*
+ * attn_quantize_qkv_e4m3: attn_quantize_e4m3 of Q, K and V of one attention call in two
+ * launches (one amax pass and one conversion pass over the three tensors) instead of six;
+ * codes and descales identical to three attn_quantize_e4m3 calls.
+ *   q, k, v      device bf16 [tokens, Hq, d_qk], [tokens, Hkv, d_qk], [tokens, Hkv, d_v]
+ *   q8, k8, v8   device uint8 outputs of the same shapes; descale_q/k/v one fp32 each
+ *   hadamard     0, or 1 to rotate all three (d_qk = d_v = 128)
+ *   workspace    device scratch of at least attn_quantize_qkv_workspace_size() bytes,
+ *                4-byte aligned, not shared by calls running concurrently
+ * Requirements: d_qk % 8 == d_v % 8 == 0, tensors 16-byte aligned.  tokens == 0 sets the
+ * three descales to 1.
+ */
+attn_status_t attn_quantize_qkv_e4m3(const void* q, const void* k, const void* v, void* q8,
+                                     void* k8, void* v8, float* descale_q, float* descale_k,
+                                     float* descale_v, int64_t tokens, int Hq, int Hkv, int d_qk,
+                                     int d_v, int hadamard, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+size_t attn_quantize_qkv_workspace_size(void);
+
+/*
  * attn_quantize_e4m3_static: attn_quantize_e4m3 for callers that cannot allocate device
  * memory (e.g. a plugin inside an engine that owns and pre-plans all device memory, or a
  * latency-critical loop where cudaMalloc's possible device synchronisation is not allowed).
@@ -209,6 +228,21 @@ attn_status_t attn_fwd_fp8_dump(const void* q, const void* k, const void* v, voi
  * reported an error, ATTN_OK otherwise.
  */
 attn_status_t attn_device_status(void* stream);
+
+/*
+ * Prefill kernel family used by attn_fwd, attn_fwd_ex, attn_fwd_varlen and the dump:
+ *   ATTN_KERNEL_PAIR    clusters of two CTAs on two SMs issuing M = 256 MMAs
+ *                       (tcgen05 cta_group::2): two query heads of one kv group, or four
+ *                       query tiles of one head, per cluster, each K/V tile split between
+ *                       the two CTAs;
+ *   ATTN_KERNEL_SINGLE  (default) one CTA per two query tiles of one head, M = 128 MMAs.
+ * Both compute the same function (bitwise the same lean-P codes; outputs equal up to the
+ * tensor cores' fp32 summation order).  A process-wide setting, for measurement and tests;
+ * returns ATTN_ERR_INVALID_ARG for another value.
+ */
+#define ATTN_KERNEL_SINGLE 0
+#define ATTN_KERNEL_PAIR 1
+attn_status_t attn_select_prefill_kernel(int kernel);
 
 /* Test-only: sets the bounded-wait limit in nanoseconds (0 restores the default, 2 s). */
 void attn_set_wait_timeout_ns(uint64_t ns);

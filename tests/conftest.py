@@ -24,3 +24,14 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(params=["pair", "single"])
+def prefill_kernel(request):
+    """Runs a test under each prefill kernel family (CTA pairs with M = 256 MMAs, and single
+    CTAs with M = 128 MMAs), restoring the default afterwards."""
+    import bf16_causal_prefill_attn_b200 as pkg
+    k = pkg.ATTN_KERNEL_PAIR if request.param == "pair" else pkg.ATTN_KERNEL_SINGLE
+    pkg.attn_select_prefill_kernel(k)
+    yield request.param
+    pkg.attn_select_prefill_kernel(pkg.ATTN_KERNEL_SINGLE)

@@ -114,3 +114,68 @@ def test_reference_arm_under_two_ranks_prints_once():
     assert len(lines) == 1
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
+
+
+def _shard_main(rank, world, port, out):
+    """Each rank computes its slice of one problem with the fp64 oracle; rank 0 gathers the
+    slices over gloo and checks them against the whole problem."""
+    import numpy as np
+    import torch
+
+    import synth
+    from bf16_causal_prefill_attn_b200 import shard
+    from oracle import attention
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        B, S, Hq, Hkv = 1, 96, 12, 3
+        q, k, v = synth.make_qkv(B, S, Hq, Hkv, 16, 16, seed=4)
+        kv_lo, kv_hi, q_lo, q_hi = shard.head_partition(Hq, Hkv, world, rank)
+        qs, ks, vs = shard.slice_heads(q, k, v, Hq, Hkv, world, rank)
+        o, _ = attention.causal_attention(qs.float().numpy(), ks.float().numpy(),
+                                          vs.float().numpy())
+        ranges = [None] * world
+        dist.all_gather_object(ranges, (q_lo, q_hi, kv_lo, kv_hi))
+        parts = [None] * world
+        dist.all_gather_object(parts, o)
+        if rank == 0:
+            heads = [h for lo, hi, _, _ in ranges for h in range(lo, hi)]
+            full, _ = attention.causal_attention(q.float().numpy(), k.float().numpy(),
+                                                 v.float().numpy())
+            got = np.concatenate([p_ for p_ in parts if p_.shape[2]], axis=2)
+            out["heads"] = heads
+            out["max_err"] = float(np.abs(got - full).max())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_head_split_gloo_world2_covers_every_head_once():
+    ctx = mp.get_context("spawn")
+    manager = ctx.Manager()
+    out = manager.dict()
+    port = 30500 + os.getpid() % 1000
+    procs = [ctx.Process(target=_shard_main, args=(r, 2, port, out)) for r in range(2)]
+    for p_ in procs:
+        p_.start()
+    for p_ in procs:
+        p_.join(timeout=180)
+        assert p_.exitcode == 0
+    assert out["heads"] == list(range(12))         # every query head once, in order
+    assert out["max_err"] == 0.0                   # slices reassemble the whole problem
+
+
+def test_head_partition_edge_cases():
+    from bf16_causal_prefill_attn_b200 import shard
+    for Hq, Hkv in ((32, 8), (32, 32), (16, 16), (12, 3)):
+        for world in (1, 2, 3, 4, 8, 9):
+            got = [shard.head_partition(Hq, Hkv, world, r) for r in range(world)]
+            kv = [h for lo, hi, _, _ in got for h in range(lo, hi)]
+            qh = [h for _, _, lo, hi in got for h in range(lo, hi)]
+            assert kv == list(range(Hkv)) and qh == list(range(Hq))
+            sizes = [hi - lo for lo, hi, _, _ in got]
+            assert max(sizes) - min(sizes) <= 1
+    with pytest.raises(ValueError):
+        shard.head_partition(6, 4, 2, 0)
+    with pytest.raises(ValueError):
+        shard.head_partition(8, 4, 2, 2)

@@ -9,7 +9,7 @@ import bf16_causal_prefill_attn_b200 as pkg
 import synth
 from oracle import attention, hadamard, leanp, quantize
 
-pytestmark = pytest.mark.gpu
+pytestmark = [pytest.mark.gpu, pytest.mark.usefixtures("prefill_kernel")]
 
 BF16_MAX_ABS = 1e-2
 BF16_REL_RMS = 5e-3
@@ -44,6 +44,8 @@ def quantize_dev(ts, rotate=False):
     (1, 384, 2, 2, 192, True, "gaussian"),      # MLA shape in BF16
     (1, 256, 2, 1, 128, False, "gaussian"),     # full (non-causal) attention
     (1, 128, 3, 3, 128, True, "outlier"),       # a single tile
+    (2, 384, 6, 2, 128, True, "gaussian"),      # odd group size (G = 3), odd tile count
+    (1, 640, 4, 4, 192, True, "outlier"),       # MLA heads, five tiles
 ])
 def test_bf16_matches_fp64(B, S, Hq, Hkv, dqk, causal, dist):
     q, k, v = synth.make_qkv(B, S, Hq, Hkv, dqk, 128, seed=S + Hq, dist=dist)
@@ -80,6 +82,8 @@ def _fp8_inputs(B, S, Hq, Hkv, dqk, seed, dist, rotate=False):
     (1, 384, 2, 2, 192, True, "outlier"),       # MLA shape
     (1, 256, 2, 2, 128, False, "gaussian"),
     (1, 1024, 1, 1, 128, True, "gaussian"),
+    (2, 384, 6, 2, 128, True, "outlier"),       # G = 3, odd tile count
+    (1, 640, 2, 2, 192, True, "gaussian"),      # MLA shape, five tiles
 ])
 def test_fp8_matches_fp64_on_quantised_inputs(B, S, Hq, Hkv, dqk, causal, dist):
     _, dev, host = _fp8_inputs(B, S, Hq, Hkv, dqk, 7 + S, dist)
@@ -110,6 +114,7 @@ def test_fp8_matches_fp64_on_quantised_inputs(B, S, Hq, Hkv, dqk, causal, dist):
     (1, 384, 2, 1, 128, True, "gaussian"),
     (1, 256, 2, 2, 192, True, "outlier"),
     (2, 256, 2, 1, 128, False, "outlier"),
+    (1, 640, 3, 1, 128, True, "outlier"),      # G = 3 (rows mode), five tiles
 ])
 def test_fp8_leanp_codes_bit_exact(B, S, Hq, Hkv, dqk, causal, dist):
     _, dev, host = _fp8_inputs(B, S, Hq, Hkv, dqk, 100 + S, dist)

@@ -30,6 +30,7 @@ def test_wait_on_a_flag_nothing_sets_times_out():
     assert np.abs(o.float().cpu().numpy() - ref).max() <= 1e-2
 
 
+@pytest.mark.usefixtures("prefill_kernel")
 @pytest.mark.parametrize("fp8", [False, True])
 def test_attention_unwinds_when_its_waits_run_out(fp8):
     """The load warp stops before key tile 1, so the MMA warp's wait for that tile can never

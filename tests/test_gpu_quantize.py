@@ -44,3 +44,26 @@ def test_quantize_deterministic():
     for _ in range(20):
         c, d = pkg.attn_quantize_e4m3(x, hadamard=True)
         assert torch.equal(c, c0) and torch.equal(d, d0)
+
+
+@pytest.mark.parametrize("B,S,Hq,Hkv,dqk,rot,dist", [
+    (1, 1024, 8, 2, 128, False, "outlier"),
+    (2, 384, 4, 4, 128, True, "gaussian"),
+    (1, 257, 4, 2, 192, False, "outlier"),    # MLA shape, ragged token count
+    (1, 3, 2, 1, 128, True, "outlier"),       # fewer rows than one block
+])
+def test_quantize_qkv_batched_bit_exact(B, S, Hq, Hkv, dqk, rot, dist):
+    """The two-launch Q/K/V quantiser gives the oracle's codes and descales for each
+    tensor, bit for bit."""
+    q, k, v = synth.make_qkv(B, S, Hq, Hkv, dqk, 128, seed=S, dist=dist)
+    res = pkg.attn_quantize_qkv_e4m3(q.cuda(), k.cuda(), v.cuda(), hadamard=rot)
+    torch.cuda.synchronize()
+    for (codes, ds), x in zip(res, (q, k, v)):
+        ref_codes, ref_ds = quantize.quantize_e4m3(x.float().numpy(), rotate=rot)
+        assert np.array_equal(codes.cpu().numpy(), ref_codes)
+        assert ds.item() == float(ref_ds)
+    # an empty batch sets every descale to 1
+    e = [torch.zeros((0, h, d), dtype=torch.bfloat16, device="cuda")
+         for h, d in ((Hq, dqk), (Hkv, dqk), (Hkv, 128))]
+    for codes, ds in pkg.attn_quantize_qkv_e4m3(*e):
+        assert codes.numel() == 0 and ds.item() == 1.0
