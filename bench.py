@@ -584,7 +584,90 @@ def gpu_bench(args, rank, world, local_rank):
     }
     if energy is not None:
         result["energy"] = energy
+    if world == 1 and not args.no_extras and args.workload == "gqa16k_outlier":
+        with ClockSampler(gpu_selector(local_rank)) as xclk:
+            extras = headline_extras(args, dev, peaks, peak_src)
+        extras["clocks"] = xclk.summary()
+        result["extra"] = extras
     return result
+
+
+# ----------------------------------------------------------------------------- headline shapes
+EXTRA_PREFILL = ("mha32k_gaussian", "mla32k_outlier")
+EXTRA_DECODE = "decode_gqa_b64_s4k"
+
+
+def headline_extras(args, dev, peaks, peak_src):
+    """Kernel throughput on the pages' own headline shapes, next to the main workload:
+    MHA 32 heads at S = 32768 on Gaussian inputs (FP8 and BF16) and the MLA shape at
+    S = 32768 (FP8), each timed over a few launches with an L2 flush between them, and one
+    paged-decode workload (GB/s against the copy bandwidth)."""
+    import copy
+
+    import torch
+
+    import bf16_causal_prefill_attn_b200 as pkg
+    import synth
+
+    bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    out = {}
+
+    def time_kernel(fn, K=8, W=3):
+        for _ in range(W):
+            flush.zero_()
+            fn()
+        torch.cuda.synchronize(dev)
+        ms = []
+        for _ in range(K):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            ms.append(a.elapsed_time(b))
+        st = pkg.attn_device_status()
+        if st != pkg.ATTN_OK:
+            raise RuntimeError(f"device status {pkg.status_string(st)}")
+        return statistics.median(ms)
+
+    for name in EXTRA_PREFILL:
+        B, S, Hq, Hkv, dqk, dv, distn, desc = WORKLOADS[name]
+        flops = causal_flops(B, Hq, S, dqk, dv)
+        q, k, v = [t.to(dev) for t in synth.make_qkv(B, S, Hq, Hkv, dqk, dv, seed=0, dist=distn)]
+        (q8, dq), (k8, dk), (v8, dvs) = pkg.attn_quantize_qkv_e4m3(q, k, v)
+        o = torch.empty((B, S, Hq, dv), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((B, Hq, S), dtype=torch.float32, device=dev)
+        ms8 = time_kernel(lambda: pkg.attn_fwd(q8, k8, v8, descale_q=dq, descale_k=dk,
+                                               descale_v=dvs, out=o, lse=lse))
+        tf8 = flops / (ms8 * 1e-3) / 1e12
+        entry = {"workload": desc, "fp8": {
+            "kernel_ms": round(ms8, 4), "tflops": round(tf8, 1),
+            "roofline": {"bound": "tensor", "achieved": round(tf8, 1),
+                         "peak": round(2 * bf16_peak, 1), "unit": "TFLOP/s",
+                         "frac": round(tf8 / (2 * bf16_peak), 4),
+                         "frac_of_nominal_4500": round(tf8 / NOMINAL_FP8_TFLOPS, 4),
+                         "peak_source": f"{peak_src} bf16 cuBLAS burst x2"}}}
+        if dqk == 128:
+            msb = time_kernel(lambda: pkg.attn_fwd(q, k, v, out=o, lse=lse))
+            tfb = flops / (msb * 1e-3) / 1e12
+            entry["bf16"] = {"kernel_ms": round(msb, 4), "tflops": round(tfb, 1),
+                             "roofline": {"bound": "tensor", "achieved": round(tfb, 1),
+                                          "peak": round(bf16_peak, 1), "unit": "TFLOP/s",
+                                          "frac": round(tfb / bf16_peak, 4),
+                                          "frac_of_nominal_2250": round(tfb / NOMINAL_BF16_TFLOPS, 4),
+                                          "peak_source": f"{peak_src} bf16 cuBLAS burst"}}
+        out[name] = entry
+        del q, k, v, q8, k8, v8, o, lse
+        torch.cuda.empty_cache()
+    da = copy.copy(args)
+    da.workload, da.steps, da.warmup = EXTRA_DECODE, 10, 3
+    d = gpu_bench_decode(da, 0, 1, dev.index)
+    out[EXTRA_DECODE] = {"workload": d["config"]["workload"], "fp8": d["roofline"],
+                         "bf16": d["bf16"]["roofline"]}
+    return out
 
 
 PREFILL_SOURCES = ("attn_fwd.cuh", "ptx.cuh")
@@ -619,11 +702,35 @@ def load_traffic(workload, fname="traffic.json", names=PREFILL_SOURCES):
 _CPU_CACHE = {}
 
 
+def cpu_model():
+    """The host CPU's model name (first 'model name' entry of /proc/cpuinfo)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
 def cpu_reference(workload, budget_s, rank=0):
-    """The oracle (fp64 attention on the dequantised FP8 inputs), as it stands, on a bounded
-    sample of query rows of the workload, on this host's cores.  The e4m3 codes of the whole
-    tensors are made once (not timed); each sampled (batch, head) is dequantised and its
-    rows computed inside the timing."""
+    """The oracle (fp64 attention on the dequantised FP8 inputs), as it stands, on this
+    host's cores, on a stratified sample of the workload: every 64th query row (and the
+    last) of whole (batch, head) slices, slices taken in a seeded order until the time
+    budget is spent (at least one).  The value is the sample's causal FLOPs (sum over the
+    sampled rows of 2 (i + 1) (d_qk + d_v)) over its time, i.e. the full problem's time
+    extrapolated by the exact causal row-cost ratio.  The e4m3 codes of the whole tensors
+    are made once and each slice is dequantised before its timing starts."""
     import numpy as np
 
     import synth
@@ -635,36 +742,31 @@ def cpu_reference(workload, budget_s, rank=0):
         q, k, v = synth.make_qkv(B, S, Hq, Hkv, dqk, dv, seed=rank, dist=distn)
         _CPU_CACHE[key] = [quantize.quantize_e4m3(t.float().numpy()) for t in (q, k, v)]
     (qc, dq), (kc, dk), (vc, dvs) = _CPU_CACHE[key]
-    rng = np.random.default_rng(0)
     G = Hq // Hkv
-    # a few (batch, head) slices, dequantised before the timing
-    slices = []
-    for _ in range(4):
-        b = int(rng.integers(0, B))
-        h = int(rng.integers(0, Hq))
+    rows = np.unique(np.append(np.arange(0, S, 64), S - 1))
+    row_flops = float(sum(2.0 * (int(i) + 1) * (dqk + dv) for i in rows))
+    order = np.random.default_rng(0).permutation(B * Hq)
+    done_flops, dt, slices = 0.0, 0.0, 0
+    for idx in order:
+        b, h = divmod(int(idx), Hq)
         g = h // G
-        slices.append((quantize.dequantize(qc[b:b + 1, :, h:h + 1], dq),
-                       quantize.dequantize(kc[b:b + 1, :, g:g + 1], dk),
-                       quantize.dequantize(vc[b:b + 1, :, g:g + 1], dvs)))
-    done_flops = 0.0
-    rows_done = 0
-    t0 = time.perf_counter()
-    while time.perf_counter() - t0 < budget_s:
-        qd, kd, vd = slices[rows_done // 8 % len(slices)]
-        rows = np.sort(rng.integers(0, S, size=8))
+        qd = quantize.dequantize(qc[b:b + 1, :, h:h + 1], dq)
+        kd = quantize.dequantize(kc[b:b + 1, :, g:g + 1], dk)
+        vd = quantize.dequantize(vc[b:b + 1, :, g:g + 1], dvs)
+        t0 = time.perf_counter()
         attention.causal_attention_rows(qd, kd, vd, rows, [0], batch=0)
-        done_flops += sum(2.0 * (int(i) + 1) * (dqk + dv) for i in rows)
-        rows_done += len(rows)
-    dt = time.perf_counter() - t0
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    except Exception:
-        cores = os.cpu_count() or 1
-    return {"value": done_flops / dt / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"{rows_done} random causal query rows (fp64, all visible keys) of 4 "
-                      f"random (batch, head) slices of {desc}; {dt:.1f} s; input generation, "
-                      "quantisation and dequantisation not timed",
+        dt += time.perf_counter() - t0
+        done_flops += row_flops
+        slices += 1
+        if dt >= budget_s:
+            break
+    return {"value": done_flops / dt / 1e12, "unit": UNIT, "cores": oracle_threads(),
+            "cpu_model": cpu_model(), "kind": "oracle",
+            "sample": f"every 64th causal query row and the last ({len(rows)} rows) of "
+                      f"{slices} of the {B * Hq} (batch, head) slices of {desc}; fp64, all "
+                      f"visible keys; {dt:.1f} s; time extrapolated to the whole problem by "
+                      "the causal row-cost ratio; input generation, quantisation and "
+                      "dequantisation not timed",
             "seconds": dt}
 
 
@@ -691,13 +793,8 @@ def cpu_reference_decode(workload, budget_s):
         decode.decode_attention(q, kc, vc, table, lens, page)
         n += 1
     dt = time.perf_counter() - t0
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    except Exception:
-        cores = os.cpu_count() or 1
-    return {"value": n * 2.0 * L * Hkv * 128 / dt / 1e9, "unit": "GB/s", "cores": cores,
-            "kind": "oracle",
+    return {"value": n * 2.0 * L * Hkv * 128 / dt / 1e9, "unit": "GB/s",
+            "cores": oracle_threads(), "cpu_model": cpu_model(), "kind": "oracle",
             "sample": f"{n} sequences of {L} cached tokens (all {Hq} query heads each) of "
                       f"{desc}; {dt:.1f} s; cache generation not timed",
             "seconds": dt}
@@ -723,7 +820,8 @@ def reference_main(args, rank, world):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": desc, "name": args.workload},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": last["cores"],
-                             "kind": "oracle", "sample": last["sample"]},
+                             "cpu_model": last["cpu_model"], "kind": "oracle",
+                             "sample": last["sample"]},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -740,6 +838,9 @@ def main(argv=None):
     ap.add_argument("--hadamard", action="store_true")
     ap.add_argument("--no-energy", action="store_true",
                     help="skip the NVML energy windows (about 12 s of extra GPU time)")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the headline shapes (MHA 32K, MLA 32K, paged decode) timed after "
+                         "the default workload")
     ap.add_argument("--exact-p", action="store_true",
                     help="FP8 probabilities by exponential + e4m3 rounding (the ablation of lean P)")
     ap.add_argument("--kernel", default="single", choices=["pair", "single"],
