@@ -670,7 +670,7 @@ def headline_extras(args, dev, peaks, peak_src):
     return out
 
 
-PREFILL_SOURCES = ("attn_fwd.cuh", "ptx.cuh")
+PREFILL_SOURCES = ("attn_fwd.cuh", "attn_pair.cuh", "ptx.cuh")
 DECODE_SOURCES = ("decode.cuh", "ptx.cuh")
 
 

@@ -147,6 +147,14 @@ attn_status_t launch_pair(const void* q, const void* k, const void* v, attn::Fwd
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  // a pair of these CTAs must fit on the device at all (once per kernel instance)
+  static std::atomic<int> fits{0};  // 0 not yet checked, 1 yes, 2 no
+  if (fits.load(std::memory_order_relaxed) == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) return ATTN_ERR_CUDA;
+    fits.store(n > 0 ? 1 : 2, std::memory_order_relaxed);
+  }
+  if (fits.load(std::memory_order_relaxed) != 1) return ATTN_ERR_UNSUPPORTED;
   if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, pp) != cudaSuccess) return ATTN_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
