@@ -24,9 +24,11 @@
 //                   all 128 keys;
 //   O_t += P_t V    A = P_t (each CTA its own rows: FP8 in shared memory, BF16 in TMEM),
 //                   B = V tile (CTA c holds value columns 64 c .. 64 c + 63, MN-major);
-//                   FP8 extends each half by 8 columns of ones (64-byte swizzled atoms, the
-//                   ones one leading-byte offset away), so N = 144 and TMEM columns
-//                   [0,64) = O[:, 0:64], [64,72) = row sum, [72,136) = O[:, 64:128].
+//                   FP8 extends each half by 16 columns of ones (64-byte swizzled atoms,
+//                   the ones one leading-byte offset away), so N = 160 and TMEM columns
+//                   [0,64) = O[:, 0:64], [64,80) = row sum, [80,144) = O[:, 64:128].  (A
+//                   pair MMA with an MN-major B takes N in multiples of 32, 16 per CTA; the
+//                   single-CTA kernel's N = 144 is not one.)
 // Roles (384 threads per CTA, 12 warps):
 //   warps 0-7   softmax of slots 0 and 1 (thread r = query row r = TMEM lane r), both CTAs;
 //   warp 8      TMA producer of this CTA's operands (its Q rows, its K and V halves);
@@ -70,7 +72,7 @@ struct PairCfg {
   static constexpr int KSTEP = FP8 ? 32 : 16;
   static constexpr int QK_STEPS = DQK / KSTEP;
   static constexpr int PV_STEPS = BLOCK_N / KSTEP;
-  static constexpr int PV_N = FP8 ? 144 : 128;
+  static constexpr int PV_N = FP8 ? 160 : 128;
   static constexpr int OV1 = PV_N / 2;       // TMEM column of O[:, 64] within O_t
   static constexpr int RS = 64;              // FP8: row-sum column within O_t
   static constexpr int OFF_Q = 0;
@@ -94,11 +96,20 @@ struct PairCfg {
   static constexpr uint32_t IDESC_PV_BF16 = idesc_dense(1u, 1u, 0u, 1u, 2 * BLOCK_M, DV);
 };
 
-// FP8 TMEM columns per CTA: O_0 [0,144), P scale factors [144,152), V scale factors
-// [152,160), O_1 [160,304), S_0 [320,448), S_1 [384,512) (overlapping in [384,448)).
-// BF16: S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512); P_t over S_t.
+// TMEM columns per CTA.  FP8: O_0 [0,160), O_1 [160,320) (value columns and row sum as
+// above), P scale factors [320,324) and [324,328), V scale factors [328,336), S_0 [336,464),
+// S_1 [384,512) (overlapping in [384,464): an S MMA waits until both slots have read their
+// latest S).  BF16: S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512); P_t (bf16)
+// over the first columns of S_t.
 template <bool FP8>
-using PairTmem = TmemMap<FP8>;
+struct PairTmem {
+  __host__ __device__ static constexpr uint32_t S(int t) { return FP8 ? 336u + 48u * t : 128u * t; }
+  __host__ __device__ static constexpr uint32_t O(int t) { return FP8 ? 160u * t : 256u + 128u * t; }
+  __host__ __device__ static constexpr uint32_t P(int t) { return 128u * t; }       // BF16 only
+  __host__ __device__ static constexpr uint32_t SFA(int t) { return 320u + 4u * t; }  // FP8
+  static constexpr uint32_t SFB = 328;                                              // FP8
+};
+static_assert(PairTmem<true>::S(0) + 128 <= 512 && PairTmem<true>::S(1) + 128 == 512, "TMEM");
 
 template <bool FP8, int DQK, bool DUMP, bool EXACT = false, bool VARLEN = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)

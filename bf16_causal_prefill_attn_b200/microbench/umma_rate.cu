@@ -30,8 +30,11 @@ __device__ __forceinline__ uint64_t desc(uint32_t saddr, uint32_t lbo, uint32_t 
 
 // CG: CTAs per MMA (1 or 2); KIND: 0 bf16 (kind::f16), 1 e4m3 (kind::f8f6f4),
 // 2 block-scaled e4m3 (kind::mxf8f6f4.block_scale); ATM: A from tensor memory (bf16 only);
-// BMN: B MN-major (the V operand of P V), else K-major (the K operand of Q K^T).
-template <int CG, int KIND, bool ATM, int N, bool BMN>
+// BL: B layout -- 0 K-major, 128-B swizzle (the K operand of Q K^T); 1 MN-major, 128-B
+// swizzle, atoms 16 KB apart (the V operand of the single-CTA P V); 2 MN-major, 64-B swizzle,
+// a 64-column atom then a second atom 8 KB away (the pair kernel's V half + ones block).
+// A pair MMA with an MN-major B takes N in multiples of 32.
+template <int CG, int KIND, bool ATM, int N, int BL>
 __global__ void __launch_bounds__(128, 1) rate_kernel(long long* cycles, int ni) {
   extern __shared__ uint8_t raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
@@ -63,12 +66,15 @@ __global__ void __launch_bounds__(128, 1) rate_kernel(long long* cycles, int ni)
   constexpr uint32_t D1 = N <= 128 ? 128 : 256;
   static_assert(!ATM || N <= 128, "A in TMEM at column 384");
   static_assert(KIND != 2 || N <= 192, "scale factors at columns 448..463");
-  constexpr uint32_t IDESC = KIND == 2 ? idesc_mxf8(0, BMN ? 1 : 0, M, N, 0, 0)
+  static_assert(CG == 1 || BL == 0 || N % 32 == 0, "pair MMA, MN-major B: N % 32");
+  constexpr uint32_t BMN = BL != 0 ? 1u : 0u;
+  constexpr uint32_t IDESC = KIND == 2 ? idesc_mxf8(0, BMN, M, N, 0, 0)
                                        : idesc_dense(KIND == 0 ? 1 : 0, KIND == 0 ? 1 : 0, 0,
-                                                     BMN ? 1 : 0, M, N);
+                                                     BMN, M, N);
   const uint64_t ad = desc(smem_addr(smem + SMEM_A), 16, 1024);
-  const uint64_t bd = BMN ? desc(smem_addr(smem + SMEM_B), 16384, 1024)
-                          : desc(smem_addr(smem + SMEM_B), 16, 1024);
+  const uint64_t bd = BL == 1   ? desc(smem_addr(smem + SMEM_B), 16384, 1024)
+                      : BL == 2 ? smem_desc_sw64(smem_addr(smem + SMEM_B), 8192, 512)
+                                : desc(smem_addr(smem + SMEM_B), 16, 1024);
   long long t = 0;
   bool ok = true;
   if (warp == 0) {
@@ -131,9 +137,9 @@ __global__ void __launch_bounds__(128, 1) rate_kernel(long long* cycles, int ni)
   if (threadIdx.x == 0) cycles[blockIdx.x] = ok ? t : -1;
 }
 
-template <int CG, int KIND, bool ATM, int N, bool BMN>
+template <int CG, int KIND, bool ATM, int N, int BL>
 void run(const char* name, int sms, int ni) {
-  auto k = rate_kernel<CG, KIND, ATM, N, BMN>;
+  auto k = rate_kernel<CG, KIND, ATM, N, BL>;
   cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES + 1024);
   const int grid = sms / CG * CG;
   long long* d = nullptr;
@@ -194,25 +200,24 @@ int main() {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, 0);
   const int ni = 4096;
   // S = Q K^T shapes (A, B K-major in shared memory)
-  run<1, 0, false, 128, false>("bf16 QK^T", sms, ni);
-  run<1, 0, false, 256, false>("bf16 QK^T", sms, ni);
-  run<2, 0, false, 128, false>("bf16 QK^T", sms, ni);
-  run<2, 0, false, 256, false>("bf16 QK^T", sms, ni);
-  run<1, 1, false, 128, false>("e4m3 QK^T", sms, ni);
-  run<1, 1, false, 256, false>("e4m3 QK^T", sms, ni);
-  run<2, 1, false, 128, false>("e4m3 QK^T", sms, ni);
-  run<2, 1, false, 256, false>("e4m3 QK^T", sms, ni);
+  run<1, 0, false, 128, 0>("bf16 QK^T", sms, ni);
+  run<1, 0, false, 256, 0>("bf16 QK^T", sms, ni);
+  run<2, 0, false, 128, 0>("bf16 QK^T", sms, ni);
+  run<2, 0, false, 256, 0>("bf16 QK^T", sms, ni);
+  run<1, 1, false, 128, 0>("e4m3 QK^T", sms, ni);
+  run<1, 1, false, 256, 0>("e4m3 QK^T", sms, ni);
+  run<2, 1, false, 128, 0>("e4m3 QK^T", sms, ni);
+  run<2, 1, false, 256, 0>("e4m3 QK^T", sms, ni);
   // P V shapes (B MN-major)
-  run<1, 0, true, 128, true>("bf16 PV, P in TMEM", sms, ni);
-  run<2, 0, true, 128, true>("bf16 PV, P in TMEM", sms, ni);
-  run<1, 0, false, 128, true>("bf16 PV, P in smem", sms, ni);
-  run<2, 0, false, 128, true>("bf16 PV, P in smem", sms, ni);
-  run<1, 2, false, 128, true>("e4m3 block-scaled PV", sms, ni);
-  run<1, 2, false, 144, true>("e4m3 block-scaled PV + row sum", sms, ni);
-  run<2, 2, false, 128, true>("e4m3 block-scaled PV", sms, ni);
-  run<2, 2, false, 144, true>("e4m3 block-scaled PV + row sum", sms, ni);
-  run<2, 2, false, 160, true>("e4m3 block-scaled PV + row sum", sms, ni);
-  run<1, 1, false, 128, true>("e4m3 PV (no scales)", sms, ni);
-  run<2, 1, false, 128, true>("e4m3 PV (no scales)", sms, ni);
+  run<1, 0, true, 128, 1>("bf16 PV, P in TMEM", sms, ni);
+  run<2, 0, true, 128, 1>("bf16 PV, P in TMEM", sms, ni);
+  run<1, 0, false, 128, 1>("bf16 PV, P in smem", sms, ni);
+  run<2, 0, false, 128, 1>("bf16 PV, P in smem", sms, ni);
+  run<1, 1, false, 128, 1>("e4m3 PV (no scales)", sms, ni);
+  run<2, 1, false, 128, 1>("e4m3 PV (no scales)", sms, ni);
+  run<1, 2, false, 128, 1>("e4m3 block-scaled PV", sms, ni);
+  run<1, 2, false, 144, 1>("e4m3 block-scaled PV + row sum (single-CTA kernel)", sms, ni);
+  run<2, 2, false, 128, 1>("e4m3 block-scaled PV", sms, ni);
+  run<2, 2, false, 160, 2>("e4m3 block-scaled PV + row sum (pair kernel, 64-B swizzle)", sms, ni);
   return 0;
 }
