@@ -32,8 +32,8 @@
 // Roles (384 threads per CTA, 12 warps):
 //   warps 0-7   softmax of slots 0 and 1 (thread r = query row r = TMEM lane r), both CTAs;
 //   warp 8      TMA producer of this CTA's operands (its Q rows, its K and V halves);
-//   warp 9      leader: S MMA issuer (FP8), all MMAs (BF16); peer: idle;
-//   warp 10     leader, FP8: PV MMA issuer; otherwise idle;
+//   warp 9      leader: the MMA issuer (S and PV of both slots); peer: idle;
+//   warp 10     idle;
 //   warp 11     TMEM allocator (cta_group::2) and forwarder: each CTA's copies complete on
 //               its own barriers (so each CTA can drain its own copies on any exit path);
 //               the forwarder relays each completion to the leader's ready barriers
@@ -96,20 +96,22 @@ struct PairCfg {
   static constexpr uint32_t IDESC_PV_BF16 = idesc_dense(1u, 1u, 0u, 1u, 2 * BLOCK_M, DV);
 };
 
-// TMEM columns per CTA.  FP8: O_0 [0,160), O_1 [160,320) (value columns and row sum as
-// above), P scale factors [320,324) and [324,328), V scale factors [328,336), S_0 [336,464),
-// S_1 [384,512) (overlapping in [384,464): an S MMA waits until both slots have read their
-// latest S).  BF16: S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512); P_t (bf16)
-// over the first columns of S_t.
+// TMEM columns per CTA (every MMA accumulator at a multiple of 32 columns).  FP8: O_0
+// [0,160), O_1 [160,320) (value columns and row sum as above); scale factors of P at
+// [320,336): slot t, 64-key block b at 320 + 8 t + 4 b, one column per 32-row quadrant of the
+// datapath (row R's factor in byte 0 of lane R, column + R / 32); scale factors of [V | 1] at
+// [336,344); S_0 [352,480), S_1 [384,512) (overlapping in [384,480): an S MMA waits until
+// both slots have read their latest S).  BF16: S_0 [0,128), S_1 [128,256), O_0 [256,384),
+// O_1 [384,512); P_t (bf16) over the first columns of S_t.
 template <bool FP8>
 struct PairTmem {
-  __host__ __device__ static constexpr uint32_t S(int t) { return FP8 ? 336u + 48u * t : 128u * t; }
+  __host__ __device__ static constexpr uint32_t S(int t) { return FP8 ? 352u + 32u * t : 128u * t; }
   __host__ __device__ static constexpr uint32_t O(int t) { return FP8 ? 160u * t : 256u + 128u * t; }
   __host__ __device__ static constexpr uint32_t P(int t) { return 128u * t; }       // BF16 only
-  __host__ __device__ static constexpr uint32_t SFA(int t) { return 320u + 4u * t; }  // FP8
-  static constexpr uint32_t SFB = 328;                                              // FP8
+  __host__ __device__ static constexpr uint32_t SFA(int t, int b) { return 320u + 8u * t + 4u * b; }
+  static constexpr uint32_t SFB = 336;
 };
-static_assert(PairTmem<true>::S(0) + 128 <= 512 && PairTmem<true>::S(1) + 128 == 512, "TMEM");
+static_assert(PairTmem<true>::S(0) % 32 == 0 && PairTmem<true>::S(1) + 128 == 512, "TMEM");
 
 template <bool FP8, int DQK, bool DUMP, bool EXACT = false, bool VARLEN = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -290,8 +292,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       __syncwarp();
-    } else if (leader && (warp == 9 || (FP8 && warp == 10))) {
-      // ------------------------------------------------- pair MMA issuers (leader only)
+    } else if (leader && warp == 9) {
+      // ------------------------------------------------- pair MMA issuer (leader only; one
+      // warp issues every MMA of the pair, S and PV)
       auto nt = [&](int t) { return t == 0 ? n_t0 : n_t1; };
       const uint64_t dq0 = smem_desc_sw128(smem_addr(smem + C::OFF_Q), 16, 1024);
       const uint64_t dk0 = smem_desc_sw128(smem_addr(smem + C::OFF_K), 16, 1024);
@@ -340,10 +343,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint64_t pd = dp0 + static_cast<uint32_t>((t * C::Q_BOX_BYTES) >> 4);
 #pragma unroll
             for (int s = 0; s < C::PV_STEPS; ++s) {
-              const uint32_t sfa = (tmem + TM::SFA(t)) | (static_cast<uint32_t>(s) << 30);
-              const uint32_t sfb = (tmem + TM::SFB) | (static_cast<uint32_t>(s) << 30);
+              // 32 keys per step: block b = s / 2 of the tile; scale-factor id 0 (byte 0)
+              const uint32_t sfa = tmem + TM::SFA(t, s / 2);
+              const uint32_t sfb = tmem + TM::SFB;
               mma2_ss_mxf8(tm_o, pd + ((s * 32) >> 4), vd + ((s * 32 * C::V_ROW) >> 4),
-                           idesc_mxf8(0, 1, 2 * BLOCK_M, C::PV_N, s, s), sfa, sfb,
+                           idesc_mxf8(0, 1, 2 * BLOCK_M, C::PV_N, 0, 0), sfa, sfb,
                            (j > 0 || s > 0) ? 1u : 0u);
             }
           }
@@ -359,9 +363,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (jo < 0) return true;
         return mbar_wait<true>(s_read(1 - t), jo & 1, p.err, p.timeout_ns);
       };
-      const bool s_issuer = warp == 9;
       bool ok = true;
-      if (s_issuer) {
+      {
         ok = mbar_wait<true>(q_ready, 0, p.err, p.timeout_ns);
         if (__all_sync(0xffffffffu, ok)) {
           ok = n_max > 0 ? mbar_wait<true>(k_ready, 0, p.err, p.timeout_ns) : true;
@@ -384,23 +387,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (j >= nt(t)) continue;
           const bool next = j + 1 < nt(t);
           if constexpr (FP8) {
-            if (s_issuer) {
-              if (next) {
-                const int jo = t == 0 ? min(j, n_t1 - 1) : min(j + 1, n_t0 - 1);
-                ok = mbar_wait<true>(s_read(t), j & 1, p.err, p.timeout_ns);
-                if (ok) ok = wait_other_read(t, jo);
-                if (ok) ok = mbar_wait<true>(k_ready + (j + 1) % C::NK, ((j + 1) / C::NK) & 1, p.err, p.timeout_ns);
-                if (!__all_sync(0xffffffffu, ok)) break;
-                tc_fence_after();
-                issue_s(t, j + 1);
-              }
-            } else {
-              ok = mbar_wait<true>(p_full(t), j & 1, p.err, p.timeout_ns);
-              if (ok) ok = mbar_wait<true>(v_ready + j % C::NV, (j / C::NV) & 1, p.err, p.timeout_ns);
+            // S_t(j+1) as soon as S_t(j) and the other slot's latest S have been read (P is
+            // in shared memory, so S_t(j+1) need not wait for PV_t(j)), then PV_t(j)
+            if (next) {
+              const int jo = t == 0 ? min(j, n_t1 - 1) : min(j + 1, n_t0 - 1);
+              ok = mbar_wait<true>(s_read(t), j & 1, p.err, p.timeout_ns);
+              if (ok) ok = wait_other_read(t, jo);
+              if (ok) ok = mbar_wait<true>(k_ready + (j + 1) % C::NK, ((j + 1) / C::NK) & 1, p.err, p.timeout_ns);
               if (!__all_sync(0xffffffffu, ok)) break;
               tc_fence_after();
-              issue_pv(t, j);
+              issue_s(t, j + 1);
             }
+            ok = mbar_wait<true>(p_full(t), j & 1, p.err, p.timeout_ns);
+            if (ok) ok = mbar_wait<true>(v_ready + j % C::NV, (j / C::NV) & 1, p.err, p.timeout_ns);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            issue_pv(t, j);
           } else {
             if (next) ok = mbar_wait<true>(k_ready + (j + 1) % C::NK, ((j + 1) / C::NK) & 1, p.err, p.timeout_ns);
             if (ok) ok = mbar_wait<true>(p_full(t), j & 1, p.err, p.timeout_ns);
@@ -413,10 +415,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       // every MMA issued by this warp completes before the pair's TMEM is released
-      const int mine = s_issuer ? 0 : 1;
-      if (elect_one()) tc_commit2(mma_done(mine), 1);
+      if (elect_one()) tc_commit2(mma_done(0), 1);
       __syncwarp();
-      mbar_wait(mma_done(mine), 0, p.err, DRAIN_TIMEOUT_NS, false);
+      mbar_wait(mma_done(0), 0, p.err, DRAIN_TIMEOUT_NS, false);
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_SOFTMAX));
@@ -562,7 +563,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
         const uint32_t e0 = static_cast<uint32_t>(120 - k0), e1 = static_cast<uint32_t>(120 - k1);
-        const uint32_t sf_word = e0 | (e0 << 8) | (e1 << 16) | (e1 << 24);
+        // UE8M0 2^-(7+k) of the two 64-key blocks (byte 0 of each block's column)
+        const uint32_t sf_word = e0 | (e1 << 16);
         if constexpr (DUMP) {
           // key tiles past the row's causal extent (rows mode) are not part of its row
           if (slot_in && (!p.causal || j <= qt)) {
@@ -614,7 +616,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           st_shared_v4(prow + ((c ^ (r & 7)) << 4), pw[4 * c], pw[4 * c + 1], pw[4 * c + 2],
                        pw[4 * c + 3]);
         fence_proxy_async_smem();
-        tmem_st1(lane_base + TM::SFA(t) + (warp & 3), sf_w);
+        tmem_st1(lane_base + TM::SFA(t, 0) + (warp & 3), sf_w & 0xFFu);
+        tmem_st1(lane_base + TM::SFA(t, 1) + (warp & 3), sf_w >> 16);
       }
       tmem_wait_st();
       tc_fence_before();
