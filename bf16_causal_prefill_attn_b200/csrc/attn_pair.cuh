@@ -22,7 +22,8 @@
 //   S_t = Q_t K^T   A = Q_t (each CTA its own 128 rows), B = K tile (CTA c holds keys
 //                   64 c .. 64 c + 63, K-major), N = 128: each CTA's TMEM gets its rows x
 //                   all 128 keys;
-//   O_t += P_t V    A = P_t (each CTA its own rows: FP8 in shared memory, BF16 in TMEM),
+//   O_t += P_t V    A = P_t (each CTA its own rows, in shared memory; BF16 with d_qk = 192:
+//                   in TMEM over S_t),
 //                   B = V tile (CTA c holds value columns 64 c .. 64 c + 63, MN-major);
 //                   FP8 extends each half by 16 columns of ones (64-byte swizzled atoms,
 //                   the ones one leading-byte offset away), so N = 160 and TMEM columns
@@ -54,6 +55,15 @@
 
 namespace attn {
 
+// Register split after setmaxnreg: the pair kernel's MMA warp issues for both CTAs from
+// precomputed descriptors (more live registers than the single-CTA kernel's), so it takes
+// 104 per thread and the softmax warps 200; the launch needs 168 either way.
+constexpr int PAIR_REGS_SOFTMAX = 200;
+constexpr int PAIR_REGS_OTHER = 104;
+static_assert((2 * 128 * PAIR_REGS_SOFTMAX + 128 * PAIR_REGS_OTHER + NUM_THREADS - 1) /
+                      NUM_THREADS <= REGS_NEEDED_AT_LAUNCH,
+              "the pair split must fit the registers the launch checks for");
+
 template <bool FP8, int DQK>
 struct PairCfg {
   static constexpr int E = FP8 ? 1 : 2;                    // bytes per element
@@ -67,6 +77,11 @@ struct PairCfg {
   // BF16: 128 B rows, 128-B swizzle)
   static constexpr int V_BYTES = 128 * 64 * E;
   static constexpr int V_ROW = 64 * E;
+  // P_t in shared memory (the A operand of PV, K-major, 128-B swizzle): always for FP8
+  // (e4m3 codes), for BF16 with d_qk = 128 (with d_qk = 192 the bf16 P stays over S_t in
+  // TMEM: shared memory holds Q, the K/V ring and no more)
+  static constexpr bool PSMEM = FP8 || DQK == 128;
+  static constexpr int P_BYTES = FP8 ? 128 * 128 : (PSMEM ? 2 * 128 * 128 : 0);  // per slot
   static constexpr int NK = FP8 ? (DQK == 128 ? 6 : 4) : (DQK == 128 ? 3 : 2);
   static constexpr int NV = NK;
   static constexpr int KSTEP = FP8 ? 32 : 16;
@@ -79,8 +94,8 @@ struct PairCfg {
   static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
   static constexpr int OFF_V = OFF_K + NK * K_BYTES;
   static constexpr int OFF_ONES = OFF_V + NV * V_BYTES;           // FP8: 128 keys x 64 B
-  static constexpr int OFF_P = OFF_ONES + (FP8 ? 128 * 64 : 0);   // FP8: P_0, P_1
-  static constexpr int OFF_BAR = OFF_P + (FP8 ? 2 * Q_BOX_BYTES : 0);
+  static constexpr int OFF_P = OFF_ONES + (FP8 ? 128 * 64 : 0);   // P_0, P_1 (PSMEM)
+  static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
   // barriers, per CTA: q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV] (this
   // CTA's copies / the pair's MMAs), q_ready, k_ready[NK], v_ready[NV] (leader: both
   // halves landed), and per slot: s_full, p_full, pv_done, s_read, mma_done
@@ -102,7 +117,7 @@ struct PairCfg {
 // datapath (row R's factor in byte 0 of lane R, column + R / 32); scale factors of [V | 1] at
 // [336,344); S_0 [352,480), S_1 [384,512) (overlapping in [384,480): an S MMA waits until
 // both slots have read their latest S).  BF16: S_0 [0,128), S_1 [128,256), O_0 [256,384),
-// O_1 [384,512); P_t (bf16) over the first columns of S_t.
+// O_1 [384,512); with d_qk = 192 P_t (bf16) over the first columns of S_t.
 template <bool FP8>
 struct PairTmem {
   __host__ __device__ static constexpr uint32_t S(int t) { return FP8 ? 352u + 32u * t : 128u * t; }
@@ -232,7 +247,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem = *tmem_ptr;
 
   if (warp >= 8) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_OTHER));
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(PAIR_REGS_OTHER));
     if (warp == 8) {
       // ------------------------------------------------- TMA producer of this CTA's operands
       bool ok = true;
@@ -298,7 +313,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       auto nt = [&](int t) { return t == 0 ? n_t0 : n_t1; };
       const uint64_t dq0 = smem_desc_sw128(smem_addr(smem + C::OFF_Q), 16, 1024);
       const uint64_t dk0 = smem_desc_sw128(smem_addr(smem + C::OFF_K), 16, 1024);
-      const uint64_t dp0 = smem_desc_sw128(smem_addr(smem + C::OFF_P), 16, 1024);  // FP8
+      const uint64_t dp0 = smem_desc_sw128(smem_addr(smem + C::OFF_P), 16, 1024);  // PSMEM
       auto v_desc = [&](int sv) -> uint64_t {
         const uint32_t va = smem_addr(smem + C::OFF_V + sv * C::V_BYTES);
         if constexpr (FP8) {
@@ -333,14 +348,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint64_t vd = v_desc(sv);
         const uint32_t tm_o = tmem + TM::O(t);
         if (elect_one()) {
-          if constexpr (!FP8) {
+          if constexpr (!FP8 && C::PSMEM) {
+            // bf16 P_t from shared memory: 16 keys (32 B) per step, 64 keys per 128-B box
+            const uint64_t pd = dp0 + static_cast<uint32_t>((t * C::P_BYTES) >> 4);
+#pragma unroll
+            for (int s = 0; s < C::PV_STEPS; ++s)
+              mma2_ss<0>(tm_o, pd + (((s / 4) * C::Q_BOX_BYTES + (s % 4) * 32) >> 4),
+                         vd + ((s * 16 * C::V_ROW) >> 4), C::IDESC_PV_BF16,
+                         (j > 0 || s > 0) ? 1u : 0u);
+          } else if constexpr (!FP8) {
             const uint32_t tm_p = tmem + TM::P(t);
 #pragma unroll
             for (int s = 0; s < C::PV_STEPS; ++s)
               mma2_ts_f16(tm_o, tm_p + s * 8, vd + ((s * 16 * C::V_ROW) >> 4), C::IDESC_PV_BF16,
                           (j > 0 || s > 0) ? 1u : 0u);
           } else {
-            const uint64_t pd = dp0 + static_cast<uint32_t>((t * C::Q_BOX_BYTES) >> 4);
+            const uint64_t pd = dp0 + static_cast<uint32_t>((t * C::P_BYTES) >> 4);
 #pragma unroll
             for (int s = 0; s < C::PV_STEPS; ++s) {
               // 32 keys per step: block b = s / 2 of the tile; scale-factor id 0 (byte 0)
@@ -386,7 +409,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int t = 0; t < 2; ++t) {
           if (j >= nt(t)) continue;
           const bool next = j + 1 < nt(t);
-          if constexpr (FP8) {
+          if constexpr (C::PSMEM) {
             // S_t(j+1) as soon as S_t(j) and the other slot's latest S have been read (P is
             // in shared memory, so S_t(j+1) need not wait for PV_t(j)), then PV_t(j)
             if (next) {
@@ -420,7 +443,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_wait(mma_done(0), 0, p.err, DRAIN_TIMEOUT_NS, false);
     }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_SOFTMAX));
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(PAIR_REGS_SOFTMAX));
     // ------------------------------------------------------------- softmax of slot t
     const int t = warp >> 2;
     const int n_t = t == 0 ? n_t0 : n_t1;
@@ -457,8 +480,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(ts + c * 32, sraw + c * 32);
       tmem_wait_ld();
-      if constexpr (FP8) {
-        // S_t is in registers: the leader may now overwrite the shared columns
+      if constexpr (C::PSMEM) {
+        // S_t is in registers: the leader may now issue the next S into these columns
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(s_read_l);
@@ -580,7 +603,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         sf_w = sf_word;
       }
-      if constexpr (FP8) {
+      if constexpr (C::PSMEM) {
+        // S_t(j) may have been issued before PV_t(j-1): that PV must be complete before O_t
+        // is rescaled and before P_t (and its scale factors) are overwritten
         if (j > 0) {
           ok = mbar_wait(pv_done(t), (j - 1) & 1, p.err, p.timeout_ns);
           if (!__all_sync(0xffffffffu, ok)) break;
@@ -606,11 +631,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tmem_st1(to + C::RS, __float_as_uint(__uint_as_float(rs) * alpha));
         }
       }
-      if constexpr (!FP8) {
+      if constexpr (!FP8 && C::PSMEM) {
+        // row r of P_t: 128 bf16 = 16 chunks of 16 B; chunk c in 128-B box c / 8 at chunk
+        // position (c mod 8) ^ (r mod 8) of the row
+        const uint32_t prow = smem_addr(smem + C::OFF_P + t * C::P_BYTES) + r * 128;
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          st_shared_v4(prow + (c / 8) * C::Q_BOX_BYTES + (((c % 8) ^ (r & 7)) << 4), pw[4 * c],
+                       pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+        fence_proxy_async_smem();
+      } else if constexpr (!FP8) {
         tmem_st32(tp, pw);
         tmem_st32(tp + 32, pw + 32);
       } else {
-        const uint32_t prow = smem_addr(smem + C::OFF_P + t * C::Q_BOX_BYTES) + r * 128;
+        const uint32_t prow = smem_addr(smem + C::OFF_P + t * C::P_BYTES) + r * 128;
 #pragma unroll
         for (int c = 0; c < 8; ++c)
           st_shared_v4(prow + ((c ^ (r & 7)) << 4), pw[4 * c], pw[4 * c + 1], pw[4 * c + 2],
