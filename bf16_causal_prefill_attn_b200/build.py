@@ -6,8 +6,13 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libattn_b200.so")
-SOURCES = ["api.cu", "attn_fwd.cuh", "quantize.cuh", "ptx.cuh", "decode.cuh"]
 HEADER = os.path.join(ROOT, "include", "attn.h")
+
+
+def sources():
+    """Every file the library is compiled from: all of csrc/ and the public header."""
+    return sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC)
+                  if f.endswith((".cu", ".cuh", ".h")))
 
 
 def nvcc_cmd(out=LIB, extra=()):
@@ -20,7 +25,7 @@ def up_to_date():
     if not os.path.exists(LIB):
         return False
     t = os.path.getmtime(LIB)
-    deps = [os.path.join(CSRC, s) for s in SOURCES] + [HEADER, __file__]
+    deps = sources() + [HEADER, __file__]
     return all(os.path.getmtime(d) <= t for d in deps)
 
 

@@ -159,3 +159,14 @@ def test_decode_argument_validation(L):
     assert _decode(L, q=0) == pkg.ATTN_ERR_INVALID_ARG
     assert _decode(L, cache_off=8) == pkg.ATTN_ERR_ALIGNMENT
     assert _decode(L, B=0, q=0, o=0, table=0, lens=0, ws=0) == pkg.ATTN_OK
+
+
+def test_built_library_is_newer_than_every_source(L):
+    """The build's up-to-date check covers every file under csrc/ and the header, so the
+    library the tests load is never older than a source it was compiled from."""
+    lib_t = os.path.getmtime(B.LIB)
+    csrc = os.path.join(os.path.dirname(B.__file__), "csrc")
+    files = [os.path.join(csrc, f) for f in os.listdir(csrc)] + [HEADER]
+    assert set(B.sources()) >= {f for f in files if f.endswith((".cu", ".cuh", ".h"))} - {HEADER}
+    for f in files:
+        assert os.path.getmtime(f) <= lib_t, f
