@@ -24,6 +24,7 @@ ATTN_FLAG_UNROTATE_O = 1
 ATTN_FLAG_EXACT_P = 2
 ATTN_KERNEL_SINGLE = 0
 ATTN_KERNEL_PAIR = 1
+ATTN_KERNEL_HEADS = 2
 
 _lib = None
 

@@ -103,8 +103,14 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, attn::FwdP
     return ATTN_ERR_CUDA;
   const attn_status_t rs = register_split_ok(kern);
   if (rs != ATTN_OK) return rs;
-  const unsigned grid = static_cast<unsigned>(prm.n_pairs) * prm.B * prm.Hq;
-  kern<<<grid, attn::NUM_THREADS, C::SMEM_ALLOC, stream>>>(mq, mk, mv, prm);
+  // units: two query tiles of one head, or (ATTN_KERNEL_HEADS, Hq / Hkv even) one query
+  // tile of two heads of one kv group
+  attn::FwdParams pp = prm;
+  pp.head_pairs = (g_kernel == ATTN_KERNEL_HEADS && prm.G % 2 == 0) ? 1 : 0;
+  pp.n_pairs = pp.head_pairs ? prm.n_q_tiles : (prm.n_q_tiles + 1) / 2;
+  const unsigned grid = static_cast<unsigned>(pp.n_pairs) * prm.B *
+                        static_cast<unsigned>(pp.head_pairs ? prm.Hq / 2 : prm.Hq);
+  kern<<<grid, attn::NUM_THREADS, C::SMEM_ALLOC, stream>>>(mq, mk, mv, pp);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -262,7 +268,7 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, flo
   if ((S % 128) != 0 && (dump || (flags & ATTN_FLAG_EXACT_P))) return ATTN_ERR_UNSUPPORTED;
   const int n_q_tiles = (S + 127) / 128;
   if (static_cast<int64_t>(B) * S > INT32_MAX ||
-      static_cast<int64_t>((n_q_tiles + 1) / 2) * B * Hq > INT32_MAX)
+      static_cast<int64_t>(n_q_tiles) * B * Hq > INT32_MAX)
     return ATTN_ERR_UNSUPPORTED;
   e = pointer_args(q, k, v, o, lse, dtype, dq, dk, dv);
   if (e != ATTN_OK) return e;
@@ -298,7 +304,7 @@ attn_status_t varlen_impl(const void* q, const void* k, const void* v, void* o, 
   if (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) return ATTN_ERR_ALIGNMENT;
   const int n_q_tiles = (max_seqlen + 127) / 128;
   if (total_tokens > INT32_MAX || max_seqlen > total_tokens ||
-      static_cast<int64_t>((n_q_tiles + 1) / 2) * B * Hq > INT32_MAX)
+      static_cast<int64_t>(n_q_tiles) * B * Hq > INT32_MAX)
     return ATTN_ERR_UNSUPPORTED;
   e = pointer_args(q, k, v, o, lse, dtype, dq, dk, dv);
   if (e != ATTN_OK) return e;
@@ -612,7 +618,8 @@ void attn_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns = ns ? ns : kDefaultTi
 void attn_selftest_stall_tile(int tile) { g_stall_tile = tile < 0 ? -1 : tile; }
 
 attn_status_t attn_select_prefill_kernel(int kernel) {
-  if (kernel != ATTN_KERNEL_SINGLE && kernel != ATTN_KERNEL_PAIR) return ATTN_ERR_INVALID_ARG;
+  if (kernel != ATTN_KERNEL_SINGLE && kernel != ATTN_KERNEL_PAIR && kernel != ATTN_KERNEL_HEADS)
+    return ATTN_ERR_INVALID_ARG;
   g_kernel = kernel;
   return ATTN_OK;
 }

@@ -90,7 +90,10 @@ constexpr float EXP2_C3 = 0.05517097562551498f;
 
 struct FwdParams {
   int B, S, Hq, Hkv, G;
-  int n_q_tiles, n_pairs;  // VARLEN: of the longest sequence (max_seqlen)
+  int n_q_tiles, n_pairs;  // VARLEN: of the longest sequence (max_seqlen); n_pairs = units
+                           // along the queries (query-tile pairs, or query tiles with head_pairs)
+  int head_pairs;          // 1: a CTA's two slots are two query heads of one kv group at the
+                           // same query tile (Hq / Hkv even); 0: two query tiles of one head
   int causal;
   // VARLEN: sequence b is tokens [cu_seqlens[b], cu_seqlens[b+1]) of the packed tensors
   // (null: every sequence has S tokens, sequence b starting at token b S), at most
@@ -175,6 +178,21 @@ __device__ __forceinline__ float exp2_poly(float x) {
   return __int_as_float(__float_as_int(j) * (1 << 23) + __float_as_int(p));
 }
 
+// Two lanes of exp2_poly with the packed two-wide fp32 instructions of sm_100 (per lane the
+// same operations and roundings as exp2_poly, so the same results bit for bit).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 j = __fadd2_rn(x, make_float2(LEANP_MAGIC, LEANP_MAGIC));
+  const float2 n = __fadd2_rn(j, make_float2(-LEANP_MAGIC, -LEANP_MAGIC));
+  const float2 f = __fadd2_rn(x, make_float2(-n.x, -n.y));
+  float2 q = __ffma2_rn(make_float2(EXP2_C3, EXP2_C3), f, make_float2(EXP2_C2, EXP2_C2));
+  q = __ffma2_rn(q, f, make_float2(EXP2_C1, EXP2_C1));
+  q = __ffma2_rn(q, f, make_float2(EXP2_C0, EXP2_C0));
+  return make_float2(__int_as_float(__float_as_int(j.x) * (1 << 23) + __float_as_int(q.x)),
+                     __int_as_float(__float_as_int(j.y) * (1 << 23) + __float_as_int(q.y)));
+}
+
 // EXACT (FP8 only): the exact-P ablation -- P = e4m3_rn(2^((a s - m)/8 + 7 + k_b)) by the
 // MUFU exponential and the hardware e4m3 conversion, instead of the lean-P multiply-add and
 // integer conversion; everything else (reference max, block shifts, block-scaled PV, row
@@ -208,12 +226,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
-  // longest-processing-time order: the pairs with the largest causal extent first
-  const int nbh = p.B * p.Hq;
+  // longest-processing-time order: the units with the largest causal extent first.  A unit
+  // is two query tiles of one head, or (head_pairs) one query tile of two heads of one kv
+  // group, which then share every K/V tile with equal causal extents
+  const bool hp = p.head_pairs != 0;
+  const int heads_per_unit = hp ? p.Hq / 2 : p.Hq;
+  const int nbh = p.B * heads_per_unit;
   const int pr = p.n_pairs - 1 - static_cast<int>(blockIdx.x) / nbh;
   const int bh = static_cast<int>(blockIdx.x) % nbh;
-  const int b = bh / p.Hq;
-  const int h = bh % p.Hq;
+  const int b = bh / heads_per_unit;
+  const int h = hp ? 2 * (bh % heads_per_unit) : bh % heads_per_unit;  // head of slot 0
   const int g = h / p.G;
   int tok0 = b * p.S;       // first token of this sequence
   int seq_len = p.S;        // its length
@@ -230,12 +252,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       seq_len = c1 - c0;
     }
     n_q_tiles = (seq_len + BLOCK_M - 1) / BLOCK_M;
-    if (2 * pr >= n_q_tiles) return;  // this sequence has fewer query-tile pairs
+    if ((hp ? pr : 2 * pr) >= n_q_tiles) return;  // this sequence has fewer units
   }
-  const int qt0 = 2 * pr;                               // query tile of t = 0
-  const bool has1 = qt0 + 1 < n_q_tiles;                // t = 1 exists
+  const int qt0 = hp ? pr : 2 * pr;                     // query tile of t = 0
+  const int qt1 = hp ? pr : 2 * pr + 1;                 // query tile of t = 1
+  const bool has1 = qt1 < n_q_tiles;                    // t = 1 exists
   const int n_t0 = p.causal ? qt0 + 1 : n_q_tiles;      // key tiles of each query tile
-  const int n_t1 = has1 ? (p.causal ? qt0 + 2 : n_q_tiles) : 0;
+  const int n_t1 = has1 ? (p.causal ? qt1 + 1 : n_q_tiles) : 0;
   const int n_max = n_t1 > n_t0 ? n_t1 : n_t0;
 
   if (tid == 0) {
@@ -283,12 +306,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // ----------------------------------------------------------- TMA producer (warp-wide,
       // one elected lane issues)
       bool ok = true;
+      // Q is read once (evicted first); K and V are read by every CTA of the kv group and
+      // of later query tiles (kept in L2 longest)
+      const uint64_t pol_once = l2_policy_evict_first();
+      const uint64_t pol_keep = l2_policy_evict_last();
       if (elect_one()) {
         mbar_arrive_expect_tx(q_full, (has1 ? 2 : 1) * C::Q_BYTES);
         for (int t = 0; t < (has1 ? 2 : 1); ++t)
           for (int i = 0; i < C::Q_BOXES; ++i)
-            tma_load_3d(smem + C::OFF_Q + t * C::Q_BYTES + i * C::BOX_BYTES, &tm_q, q_full,
-                        i * C::BOX_COLS, h, tok0 + (qt0 + t) * BLOCK_M);
+            tma_load_3d_hint(smem + C::OFF_Q + t * C::Q_BYTES + i * C::BOX_BYTES, &tm_q, q_full,
+                             i * C::BOX_COLS, hp ? h + t : h, tok0 + (t ? qt1 : qt0) * BLOCK_M,
+                             pol_once);
       }
       __syncwarp();
       int jk = 0, jv = 0;  // K and V tiles issued
@@ -300,8 +328,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (elect_one()) {
           mbar_arrive_expect_tx(k_full + sk, C::K_BYTES);
           for (int i = 0; i < C::Q_BOXES; ++i)
-            tma_load_3d(smem + C::OFF_K + sk * C::K_BYTES + i * C::BOX_BYTES, &tm_k, k_full + sk,
-                        i * C::BOX_COLS, g, tok0 + j * BLOCK_N);
+            tma_load_3d_hint(smem + C::OFF_K + sk * C::K_BYTES + i * C::BOX_BYTES, &tm_k,
+                             k_full + sk, i * C::BOX_COLS, g, tok0 + j * BLOCK_N, pol_keep);
         }
         __syncwarp();
         jk = j + 1;
@@ -311,8 +339,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (elect_one()) {
           mbar_arrive_expect_tx(v_full + sv, C::V_BYTES);
           for (int i = 0; i < C::V_BOXES; ++i)
-            tma_load_3d(smem + C::OFF_V + sv * C::V_BYTES + i * C::BOX_BYTES, &tm_v, v_full + sv,
-                        i * C::BOX_COLS, g, tok0 + j * BLOCK_N);
+            tma_load_3d_hint(smem + C::OFF_V + sv * C::V_BYTES + i * C::BOX_BYTES, &tm_v,
+                             v_full + sv, i * C::BOX_COLS, g, tok0 + j * BLOCK_N, pol_keep);
         }
         __syncwarp();
         jv = j + 1;
@@ -472,7 +500,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ------------------------------------------------------------- softmax of tile t
     const int t = warp >> 2;
     const int n_t = t == 0 ? n_t0 : n_t1;
-    const int qt = qt0 + t;
+    const int qt = t ? qt1 : qt0;
+    const int hs = hp ? h + t : h;                // this slot's query head
     const int r = tid & 127;                      // row within the tile == TMEM lane
     const int q_pos = qt * BLOCK_M + r;           // query position in the sequence
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
@@ -549,31 +578,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const float ms_new = (j == 0 || cand > ms + BF16_HEADROOM) ? cand : ms;
         if (j > 0) alpha = ex2_approx(ms - ms_new);
         ms = ms_new;
-        float lsum0 = 0.0f, lsum1 = 0.0f;
+        // element pairs in packed two-wide fp32 (the even and odd sums are the two lanes)
+        const float2 c1x2 = make_float2(p.c1, p.c1);
+        const float2 nms2 = make_float2(-ms, -ms);
+        float2 lsum = make_float2(0.0f, 0.0f);
         if (diag) {
 #pragma unroll
           for (int c = 0; c < BLOCK_N; c += 2) {
-            const float p0 = ex2_approx(__fmaf_rn(s[c], p.c1, -ms));
-            const float p1 = ex2_approx(__fmaf_rn(s[c + 1], p.c1, -ms));
-            lsum0 += p0;
-            lsum1 += p1;
-            pw[c >> 1] = pack_bf16x2(p0, p1);
+            const float2 x = __ffma2_rn(make_float2(s[c], s[c + 1]), c1x2, nms2);
+            const float2 pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            lsum = __fadd2_rn(lsum, pp);
+            pw[c >> 1] = pack_bf16x2(pp.x, pp.y);
           }
         } else {
 #pragma unroll
           for (int c = 0; c < BLOCK_N; c += 2) {
-            const float x0 = __fmaf_rn(s[c], p.c1, -ms);
-            const float x1 = __fmaf_rn(s[c + 1], p.c1, -ms);
+            const float2 x = __ffma2_rn(make_float2(s[c], s[c + 1]), c1x2, nms2);
             // one element pair in four on the FMA pipe, the rest on the MUFU
             const bool poly = (c & 7) == 6;
-            const float p0 = poly ? exp2_poly(x0) : ex2_approx(x0);
-            const float p1 = poly ? exp2_poly(x1) : ex2_approx(x1);
-            lsum0 += p0;
-            lsum1 += p1;
-            pw[c >> 1] = pack_bf16x2(p0, p1);
+            const float2 pp = poly ? exp2_poly2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            lsum = __fadd2_rn(lsum, pp);
+            pw[c >> 1] = pack_bf16x2(pp.x, pp.y);
           }
         }
-        l = l * alpha + (lsum0 + lsum1);
+        l = l * alpha + (lsum.x + lsum.y);
       } else {
         const float mu = fmaxf(mu0, mu1);
         const int cand = __float2int_ru(__fmul_rn(a, mu));
@@ -599,21 +627,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         } else {
           const float cb0 = __int2float_rn(LEANP_TOP + 8 * k0 - m_new) * 0.00390625f;
           const float cb1 = __int2float_rn(LEANP_TOP + 8 * k1 - m_new) * 0.00390625f;
+          const float2 s256 = make_float2(256.0f, 256.0f);
+          const float2 magic = make_float2(LEANP_MAGIC, LEANP_MAGIC);
 #pragma unroll
           for (int c = 0; c < BLOCK_N; c += 4) {
             const float cb = c < 64 ? cb0 : cb1;
-            // multiply-add (saturating to [0,1]) and the integer conversion by a magic fma
-            const uint32_t b0 = __float_as_uint(__fmaf_rn(fma_sat(s[c + 0], a256, cb), 256.0f, LEANP_MAGIC));
-            const uint32_t b1 = __float_as_uint(__fmaf_rn(fma_sat(s[c + 1], a256, cb), 256.0f, LEANP_MAGIC));
-            const uint32_t b2 = __float_as_uint(__fmaf_rn(fma_sat(s[c + 2], a256, cb), 256.0f, LEANP_MAGIC));
-            const uint32_t b3 = __float_as_uint(__fmaf_rn(fma_sat(s[c + 3], a256, cb), 256.0f, LEANP_MAGIC));
-            pw[c >> 2] = pack_low_bytes(b0, b1, b2, b3);
+            // multiply-add (saturating to [0,1]), then the integer conversion by a magic fma,
+            // two lanes at a time
+            const float2 u01 = make_float2(fma_sat(s[c + 0], a256, cb), fma_sat(s[c + 1], a256, cb));
+            const float2 u23 = make_float2(fma_sat(s[c + 2], a256, cb), fma_sat(s[c + 3], a256, cb));
+            const float2 r01 = __ffma2_rn(u01, s256, magic);
+            const float2 r23 = __ffma2_rn(u23, s256, magic);
+            pw[c >> 2] = pack_low_bytes(__float_as_uint(r01.x), __float_as_uint(r01.y),
+                                        __float_as_uint(r23.x), __float_as_uint(r23.y));
           }
         }
         const uint32_t e0 = static_cast<uint32_t>(120 - k0), e1 = static_cast<uint32_t>(120 - k1);
         const uint32_t sf_word = e0 | (e0 << 8) | (e1 << 16) | (e1 << 24);  // UE8M0 2^-(7+k)
         if constexpr (DUMP) {
-          const size_t row = (static_cast<size_t>(b) * p.Hq + h) * p.S + q_pos;
+          const size_t row = (static_cast<size_t>(b) * p.Hq + hs) * p.S + q_pos;
           float* ds = p.dump_s + row * p.S + static_cast<size_t>(j) * BLOCK_N;
           uint8_t* dc = p.dump_codes + row * p.S + static_cast<size_t>(j) * BLOCK_N;
           for (int c = 0; c < BLOCK_N; ++c) ds[c] = s[c];
@@ -641,8 +673,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint32_t o[32];
           tmem_ld32(to + c * 32, o);
           tmem_wait_ld();
+          const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          for (int i = 0; i < 32; i += 2) {
+            const float2 r = __fmul2_rn(make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), a2);
+            o[i] = __float_as_uint(r.x);
+            o[i + 1] = __float_as_uint(r.y);
+          }
           tmem_st32(to + c * 32, o);
         }
         if constexpr (FP8) {
@@ -710,15 +747,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // VARLEN: rows past the end of the sequence hold another sequence's queries (or zero
       // fill) and are not written
       const bool row_in = !VARLEN || q_pos < seq_len;
-      __nv_bfloat16* orow = p.o + ((static_cast<size_t>(tok0) + q_pos) * p.Hq + h) * DV;
+      __nv_bfloat16* orow = p.o + ((static_cast<size_t>(tok0) + q_pos) * p.Hq + hs) * DV;
+      const uint64_t pol_once = l2_policy_evict_first();  // O is written once
+      const float2 inv2 = make_float2(inv, inv);
 #pragma unroll
       for (int c = 0; c < DV; c += 8) {
+        const float2 a0 = __fmul2_rn(make_float2(o[c + 0], o[c + 1]), inv2);
+        const float2 a1 = __fmul2_rn(make_float2(o[c + 2], o[c + 3]), inv2);
+        const float2 a2 = __fmul2_rn(make_float2(o[c + 4], o[c + 5]), inv2);
+        const float2 a3 = __fmul2_rn(make_float2(o[c + 6], o[c + 7]), inv2);
         uint4 v;
-        v.x = pack_bf16x2(o[c + 0] * inv, o[c + 1] * inv);
-        v.y = pack_bf16x2(o[c + 2] * inv, o[c + 3] * inv);
-        v.z = pack_bf16x2(o[c + 4] * inv, o[c + 5] * inv);
-        v.w = pack_bf16x2(o[c + 6] * inv, o[c + 7] * inv);
-        if (row_in) *reinterpret_cast<uint4*>(orow + c) = v;
+        v.x = pack_bf16x2(a0.x, a0.y);
+        v.y = pack_bf16x2(a1.x, a1.y);
+        v.z = pack_bf16x2(a2.x, a2.y);
+        v.w = pack_bf16x2(a3.x, a3.y);
+        if (row_in) st_global_v4_hint(orow + c, v, pol_once);
       }
       if (p.lse != nullptr && row_in) {
         float lse_v;
@@ -728,8 +771,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           lse_v = 0.69314718055994531f * (ms + __log2f(l));
         // lse [B, Hq, S], or [Hq, total tokens] for packed sequences
         const size_t li = (VARLEN && p.cu_seqlens != nullptr)
-                              ? static_cast<size_t>(h) * p.total_tokens + tok0 + q_pos
-                              : (static_cast<size_t>(b) * p.Hq + h) * p.S + q_pos;
+                              ? static_cast<size_t>(hs) * p.total_tokens + tok0 + q_pos
+                              : (static_cast<size_t>(b) * p.Hq + hs) * p.S + q_pos;
         p.lse[li] = lse_v;
       }
     }

@@ -235,13 +235,17 @@ attn_status_t attn_device_status(void* stream);
  *                       (tcgen05 cta_group::2): two query heads of one kv group, or four
  *                       query tiles of one head, per cluster, each K/V tile split between
  *                       the two CTAs;
- *   ATTN_KERNEL_SINGLE  (default) one CTA per two query tiles of one head, M = 128 MMAs.
- * Both compute the same function (bitwise the same lean-P codes; outputs equal up to the
+ *   ATTN_KERNEL_SINGLE  (default) one CTA per two query tiles of one head, M = 128 MMAs;
+ *   ATTN_KERNEL_HEADS   the single-CTA kernel with one query tile of two query heads of one
+ *                       kv group per CTA (equal causal extents, every K/V tile serving both
+ *                       heads); with Hq / Hkv odd it is ATTN_KERNEL_SINGLE.
+ * All compute the same function (bitwise the same lean-P codes; outputs equal up to the
  * tensor cores' fp32 summation order).  A process-wide setting, for measurement and tests;
  * returns ATTN_ERR_INVALID_ARG for another value.
  */
 #define ATTN_KERNEL_SINGLE 0
 #define ATTN_KERNEL_PAIR 1
+#define ATTN_KERNEL_HEADS 2
 attn_status_t attn_select_prefill_kernel(int kernel);
 
 /* Test-only: sets the bounded-wait limit in nanoseconds (0 restores the default, 2 s). */
