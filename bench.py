@@ -338,7 +338,7 @@ def gpu_bench(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    pkg.attn_select_prefill_kernel(pkg.ATTN_KERNEL_PAIR if args.kernel == "pair"
+    pkg.attn_select_prefill_kernel(pkg.ATTN_KERNEL_HEADS if args.kernel == "heads"
                                    else pkg.ATTN_KERNEL_SINGLE)
     B, S, Hq, Hkv, dqk, dv, distn, desc = WORKLOADS[args.workload]
     if args.split == "heads":
@@ -670,7 +670,7 @@ def headline_extras(args, dev, peaks, peak_src):
     return out
 
 
-PREFILL_SOURCES = ("attn_fwd.cuh", "attn_pair.cuh", "ptx.cuh")
+PREFILL_SOURCES = ("attn_fwd.cuh", "ptx.cuh")
 DECODE_SOURCES = ("decode.cuh", "ptx.cuh")
 
 
@@ -843,9 +843,9 @@ def main(argv=None):
                          "the default workload")
     ap.add_argument("--exact-p", action="store_true",
                     help="FP8 probabilities by exponential + e4m3 rounding (the ablation of lean P)")
-    ap.add_argument("--kernel", default="single", choices=["pair", "single"],
-                    help="prefill kernel family: CTA pairs with M = 256 MMAs (default) or "
-                         "single CTAs with M = 128 MMAs")
+    ap.add_argument("--kernel", default="single", choices=["single", "heads"],
+                    help="work unit of the prefill kernel: two query tiles of one head "
+                         "(default) or one query tile of two heads of one kv group")
     ap.add_argument("--split", default="replicas", choices=["replicas", "heads"],
                     help="multi-GPU: an independent problem per GPU (weak scaling), or one "
                          "problem divided by kv heads (strong scaling)")

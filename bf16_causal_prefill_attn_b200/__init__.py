@@ -23,7 +23,6 @@ ATTN_FP8_E4M3 = 1
 ATTN_FLAG_UNROTATE_O = 1
 ATTN_FLAG_EXACT_P = 2
 ATTN_KERNEL_SINGLE = 0
-ATTN_KERNEL_PAIR = 1
 ATTN_KERNEL_HEADS = 2
 
 _lib = None
@@ -301,8 +300,9 @@ def attn_set_wait_timeout_ns(ns):
 
 
 def attn_select_prefill_kernel(kernel):
-    """Prefill kernel family for later calls: ATTN_KERNEL_PAIR (default, CTA pairs with
-    M = 256 MMAs) or ATTN_KERNEL_SINGLE (one CTA, M = 128)."""
+    """Work unit of the prefill kernel for later calls: ATTN_KERNEL_SINGLE (two query tiles
+    of one head per CTA) or ATTN_KERNEL_HEADS (one query tile of two heads of one kv
+    group)."""
     _check(lib().attn_select_prefill_kernel(int(kernel)), "attn_select_prefill_kernel")
 
 

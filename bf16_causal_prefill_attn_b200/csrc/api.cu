@@ -13,7 +13,6 @@
 
 #include "../../include/attn.h"
 #include "attn_fwd.cuh"
-#include "attn_pair.cuh"
 #include "decode.cuh"
 #include "quantize.cuh"
 
@@ -114,64 +113,10 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, attn::FwdP
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-// The pair kernel: clusters of two CTAs, M = 256 MMAs (attn_pair.cuh).  Units along the
-// queries: pairs of query tiles (heads mode, Hq / Hkv even) or quads (rows mode).
-template <bool FP8, int DQK, bool DUMP, bool EXACT = false, bool VARLEN = false>
-attn_status_t launch_pair(const void* q, const void* k, const void* v, attn::FwdParams& prm,
-                          cudaStream_t stream) {
-  using C = attn::PairCfg<FP8, DQK>;
-  const CUtensorMapDataType dt =
-      FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  const uint64_t T = static_cast<uint64_t>(prm.total_tokens);
-  CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, dt, C::E, DQK, prm.Hq, T, C::BOX_COLS) ||
-      !make_map(&mk, k, dt, C::E, DQK, prm.Hkv, T, C::BOX_COLS, 64) ||
-      !make_map(&mv, v, dt, C::E, attn::DV, prm.Hkv, T, 64, 128,
-                FP8 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B))
-    return ATTN_ERR_CUDA;
-  auto kern = attn::attn_pair_kernel<FP8, DQK, DUMP, EXACT, VARLEN>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC) !=
-      cudaSuccess)
-    return ATTN_ERR_CUDA;
-  const attn_status_t rs = register_split_ok(kern);
-  if (rs != ATTN_OK) return rs;
-  const bool heads_mode = (prm.G % 2) == 0;
-  attn::FwdParams pp = prm;
-  pp.n_pairs = heads_mode ? (prm.n_q_tiles + 1) / 2 : (prm.n_q_tiles + 3) / 4;
-  const int64_t units =
-      static_cast<int64_t>(pp.n_pairs) * prm.B * (heads_mode ? prm.Hq / 2 : prm.Hq);
-  if (units * 2 > INT32_MAX) return ATTN_ERR_UNSUPPORTED;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(units * 2));
-  cfg.blockDim = dim3(attn::NUM_THREADS);
-  cfg.dynamicSmemBytes = C::SMEM_ALLOC;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  // a pair of these CTAs must fit on the device at all (once per kernel instance)
-  static std::atomic<int> fits{0};  // 0 not yet checked, 1 yes, 2 no
-  if (fits.load(std::memory_order_relaxed) == 0) {
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) return ATTN_ERR_CUDA;
-    fits.store(n > 0 ? 1 : 2, std::memory_order_relaxed);
-  }
-  if (fits.load(std::memory_order_relaxed) != 1) return ATTN_ERR_UNSUPPORTED;
-  if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, pp) != cudaSuccess) return ATTN_ERR_CUDA;
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
-}
-
-// Kernel family for one instantiation: the pair kernel unless the single-CTA one is
-// selected (attn_select_prefill_kernel).
+// The prefill kernel for one instantiation.
 template <bool FP8, int DQK, bool DUMP, bool EXACT = false, bool VARLEN = false>
 attn_status_t launch_prefill(const void* q, const void* k, const void* v, attn::FwdParams& prm,
                              cudaStream_t stream) {
-  if (g_kernel == ATTN_KERNEL_PAIR)
-    return launch_pair<FP8, DQK, DUMP, EXACT, VARLEN>(q, k, v, prm, stream);
   return launch_fwd<FP8, DQK, DUMP, EXACT, VARLEN>(q, k, v, prm, stream);
 }
 
@@ -618,8 +563,7 @@ void attn_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns = ns ? ns : kDefaultTi
 void attn_selftest_stall_tile(int tile) { g_stall_tile = tile < 0 ? -1 : tile; }
 
 attn_status_t attn_select_prefill_kernel(int kernel) {
-  if (kernel != ATTN_KERNEL_SINGLE && kernel != ATTN_KERNEL_PAIR && kernel != ATTN_KERNEL_HEADS)
-    return ATTN_ERR_INVALID_ARG;
+  if (kernel != ATTN_KERNEL_SINGLE && kernel != ATTN_KERNEL_HEADS) return ATTN_ERR_INVALID_ARG;
   g_kernel = kernel;
   return ATTN_OK;
 }

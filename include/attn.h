@@ -230,21 +230,16 @@ attn_status_t attn_fwd_fp8_dump(const void* q, const void* k, const void* v, voi
 attn_status_t attn_device_status(void* stream);
 
 /*
- * Prefill kernel family used by attn_fwd, attn_fwd_ex, attn_fwd_varlen and the dump:
- *   ATTN_KERNEL_PAIR    clusters of two CTAs on two SMs issuing M = 256 MMAs
- *                       (tcgen05 cta_group::2): two query heads of one kv group, or four
- *                       query tiles of one head, per cluster, each K/V tile split between
- *                       the two CTAs;
- *   ATTN_KERNEL_SINGLE  (default) one CTA per two query tiles of one head, M = 128 MMAs;
- *   ATTN_KERNEL_HEADS   the single-CTA kernel with one query tile of two query heads of one
- *                       kv group per CTA (equal causal extents, every K/V tile serving both
- *                       heads); with Hq / Hkv odd it is ATTN_KERNEL_SINGLE.
- * All compute the same function (bitwise the same lean-P codes; outputs equal up to the
+ * Work unit of the prefill kernel used by attn_fwd, attn_fwd_ex, attn_fwd_varlen and the
+ * dump (one CTA per unit, two 128-row query slots in ping-pong sharing every K/V tile):
+ *   ATTN_KERNEL_SINGLE  (default) two consecutive query tiles of one query head;
+ *   ATTN_KERNEL_HEADS   one query tile of two query heads of one kv group (equal causal
+ *                       extents); with Hq / Hkv odd it is ATTN_KERNEL_SINGLE.
+ * Both compute the same function (bitwise the same lean-P codes; outputs equal up to the
  * tensor cores' fp32 summation order).  A process-wide setting, for measurement and tests;
  * returns ATTN_ERR_INVALID_ARG for another value.
  */
 #define ATTN_KERNEL_SINGLE 0
-#define ATTN_KERNEL_PAIR 1
 #define ATTN_KERNEL_HEADS 2
 attn_status_t attn_select_prefill_kernel(int kernel);
 

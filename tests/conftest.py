@@ -26,14 +26,12 @@ def pytest_collection_modifyitems(config, items):
             item.add_marker(skip)
 
 
-@pytest.fixture(params=["pair", "single", "heads"])
+@pytest.fixture(params=["single", "heads"])
 def prefill_kernel(request):
-    """Runs a test under each prefill kernel family (CTA pairs with M = 256 MMAs; single CTAs
-    with M = 128 MMAs over two query tiles of one head, or over two heads of one kv group),
-    restoring the default afterwards."""
+    """Runs a test under each work unit of the prefill kernel (two query tiles of one head;
+    one query tile of two heads of one kv group), restoring the default afterwards."""
     import bf16_causal_prefill_attn_b200 as pkg
-    k = {"pair": pkg.ATTN_KERNEL_PAIR, "single": pkg.ATTN_KERNEL_SINGLE,
-         "heads": pkg.ATTN_KERNEL_HEADS}[request.param]
+    k = {"single": pkg.ATTN_KERNEL_SINGLE, "heads": pkg.ATTN_KERNEL_HEADS}[request.param]
     pkg.attn_select_prefill_kernel(k)
     yield request.param
     pkg.attn_select_prefill_kernel(pkg.ATTN_KERNEL_SINGLE)

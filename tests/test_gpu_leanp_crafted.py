@@ -157,8 +157,8 @@ def replay_and_count(scores, a):
 @pytest.mark.usefixtures("prefill_kernel")
 @pytest.mark.parametrize("d_qk,hq", [(128, 2), (192, 2), (128, 1)])
 def test_leanp_codes_bit_exact_on_crafted_edge_cases(d_qk, hq):
-    """hq = 2: two query heads share the kv head (the pair kernel's heads mode); hq = 1: one
-    head (its rows mode, four query tiles per pair)."""
+    """hq = 2: two query heads share the kv head (so the head-pair work unit applies); hq = 1:
+    one head (two query tiles per CTA in either setting)."""
     codes, (dq, dk, dv) = build_inputs(d_qk, seed=d_qk, hq=hq)
     a = leanp.slope(d_qk, dq, dk)
     assert a == np.float32(0.25)
