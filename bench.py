@@ -725,12 +725,13 @@ def oracle_threads():
 
 def cpu_reference(workload, budget_s, rank=0):
     """The oracle (fp64 attention on the dequantised FP8 inputs), as it stands, on this
-    host's cores, on a stratified sample of the workload: every 64th query row (and the
-    last) of whole (batch, head) slices, slices taken in a seeded order until the time
-    budget is spent (at least one).  The value is the sample's causal FLOPs (sum over the
-    sampled rows of 2 (i + 1) (d_qk + d_v)) over its time, i.e. the full problem's time
-    extrapolated by the exact causal row-cost ratio.  The e4m3 codes of the whole tensors
-    are made once and each slice is dequantised before its timing starts."""
+    host's cores, on a stratified sample of the workload: passes over every (batch, head)
+    slice, each pass taking every 64th query row from an offset (0, 32, 16, 48, 8, ... --
+    the first pass also the last row), until the time budget is spent (at least one pass
+    of one slice).  The value is the sample's causal FLOPs (sum over the sampled rows of
+    2 (i + 1) (d_qk + d_v)) over its time, i.e. the full problem's time extrapolated by the
+    exact causal row-cost ratio.  The e4m3 codes of the whole tensors are made once and each
+    slice is dequantised before its timing starts."""
     import numpy as np
 
     import synth
@@ -743,30 +744,41 @@ def cpu_reference(workload, budget_s, rank=0):
         _CPU_CACHE[key] = [quantize.quantize_e4m3(t.float().numpy()) for t in (q, k, v)]
     (qc, dq), (kc, dk), (vc, dvs) = _CPU_CACHE[key]
     G = Hq // Hkv
-    rows = np.unique(np.append(np.arange(0, S, 64), S - 1))
-    row_flops = float(sum(2.0 * (int(i) + 1) * (dqk + dv) for i in rows))
     order = np.random.default_rng(0).permutation(B * Hq)
-    done_flops, dt, slices = 0.0, 0.0, 0
-    for idx in order:
-        b, h = divmod(int(idx), Hq)
-        g = h // G
-        qd = quantize.dequantize(qc[b:b + 1, :, h:h + 1], dq)
-        kd = quantize.dequantize(kc[b:b + 1, :, g:g + 1], dk)
-        vd = quantize.dequantize(vc[b:b + 1, :, g:g + 1], dvs)
-        t0 = time.perf_counter()
-        attention.causal_attention_rows(qd, kd, vd, rows, [0], batch=0)
-        dt += time.perf_counter() - t0
-        done_flops += row_flops
-        slices += 1
+    # row offsets in bit-reversed order, so every prefix of passes is spread over the rows
+    offsets = [int(f"{i:06b}"[::-1], 2) for i in range(64)]
+    done_flops, dt, slices, rows_done, passes = 0.0, 0.0, 0, 0, 0
+    for off in offsets:
+        rows = np.arange(off, S, 64)
+        if off == 0:
+            rows = np.unique(np.append(rows, S - 1))
+        if rows.size == 0:
+            continue
+        row_flops = float(sum(2.0 * (int(i) + 1) * (dqk + dv) for i in rows))
+        for idx in order:
+            b, h = divmod(int(idx), Hq)
+            g = h // G
+            qd = quantize.dequantize(qc[b:b + 1, :, h:h + 1], dq)
+            kd = quantize.dequantize(kc[b:b + 1, :, g:g + 1], dk)
+            vd = quantize.dequantize(vc[b:b + 1, :, g:g + 1], dvs)
+            t0 = time.perf_counter()
+            attention.causal_attention_rows(qd, kd, vd, rows, [0], batch=0)
+            dt += time.perf_counter() - t0
+            done_flops += row_flops
+            rows_done += rows.size
+            slices += 1
+            if dt >= budget_s:
+                break
+        passes += 1
         if dt >= budget_s:
             break
     return {"value": done_flops / dt / 1e12, "unit": UNIT, "cores": oracle_threads(),
             "cpu_model": cpu_model(), "kind": "oracle",
-            "sample": f"every 64th causal query row and the last ({len(rows)} rows) of "
-                      f"{slices} of the {B * Hq} (batch, head) slices of {desc}; fp64, all "
-                      f"visible keys; {dt:.1f} s; time extrapolated to the whole problem by "
-                      "the causal row-cost ratio; input generation, quantisation and "
-                      "dequantisation not timed",
+            "sample": f"{rows_done} causal query rows of {desc}: {passes} stratified pass(es) "
+                      f"of every 64th row from an offset over the {B * Hq} (batch, head) "
+                      f"slices ({slices} slice visits); fp64, all visible keys; {dt:.1f} s; "
+                      "time extrapolated to the whole problem by the causal row-cost ratio; "
+                      "input generation, quantisation and dequantisation not timed",
             "seconds": dt}
 
 

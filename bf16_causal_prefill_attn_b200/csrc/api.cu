@@ -306,6 +306,53 @@ int num_sms() {
   return n;
 }
 
+// One amax launch and one conversion launch over n tensors (n <= 3): x[i] bf16 [el[i]
+// elements] -> y[i] e4m3 codes, ds[i] its descale, amax[i] a cleared word.  Blocks are split
+// among the tensors in proportion to their sizes; the conversion visits the tensors in the
+// reverse order, so those the amax pass read last are re-read first, while they may still
+// be in L2.
+attn_status_t launch_quantize(int n, const void* const* x, void* const* y, float* const* ds,
+                              const int64_t* el, int hadamard, uint32_t* amax,
+                              cudaStream_t st) {
+  const int threads = 256;
+  const int64_t per_block_items = hadamard ? threads / 32 : threads * 4;  // rows or chunks
+  const int64_t budget = int64_t(num_sms()) * 16;  // blocks per pass, split by size
+  int64_t total = 0;
+  for (int i = 0; i < n; ++i) total += el[i];
+  attn::QuantBatch fwd{}, rev{};
+  fwd.njobs = rev.njobs = n;
+  int end_f = 0, end_r = 0;
+  for (int o = 0; o < n; ++o) {
+    for (int pass = 0; pass < 2; ++pass) {
+      const int i = pass == 0 ? o : n - 1 - o;
+      const int64_t items = hadamard ? el[i] / 128 : el[i] / 8;
+      const int64_t want = (items + per_block_items - 1) / per_block_items;
+      const int64_t share = std::max<int64_t>(1, (budget * el[i] + total - 1) / total);
+      const int nb = static_cast<int>(std::max<int64_t>(1, std::min(want, share)));
+      attn::QuantJob jb{static_cast<const __nv_bfloat16*>(x[i]), static_cast<uint8_t*>(y[i]),
+                        items, amax + i, ds[i]};
+      if (pass == 0) {
+        fwd.job[o] = jb;
+        end_f += nb;
+        fwd.block_end[o] = end_f;
+      } else {
+        rev.job[o] = jb;
+        end_r += nb;
+        rev.block_end[o] = end_r;
+      }
+    }
+  }
+  if (cudaMemsetAsync(amax, 0, n * sizeof(uint32_t), st) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (hadamard) {
+    attn::amax_batch_kernel<true><<<end_f, threads, 0, st>>>(fwd);
+    attn::convert_batch_kernel<true><<<end_r, threads, 0, st>>>(rev);
+  } else {
+    attn::amax_batch_kernel<false><<<end_f, threads, 0, st>>>(fwd);
+    attn::convert_batch_kernel<false><<<end_r, threads, 0, st>>>(rev);
+  }
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -446,24 +493,11 @@ attn_status_t attn_quantize_e4m3(const void* x_bf16, void* x_e4m3, float* descal
   }
   if (!x_bf16 || !x_e4m3) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(x_bf16) || !aligned16(x_e4m3)) return ATTN_ERR_ALIGNMENT;
-  if (cudaMemsetAsync(amax, 0, sizeof(uint32_t), st) != cudaSuccess) return ATTN_ERR_CUDA;
-  const int threads = 256;
-  const int sms = num_sms();
-  const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(x_bf16);
-  uint8_t* y = static_cast<uint8_t*>(x_e4m3);
-  if (hadamard) {
-    const int64_t want = (rows + 7) / 8;  // 8 warps (rows) per block
-    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(want, int64_t(sms) * 16));
-    attn::amax_rot_kernel<<<grid, threads, 0, st>>>(x, rows, amax);
-    attn::convert_rot_kernel<<<grid, threads, 0, st>>>(x, y, rows, amax, descale_out);
-  } else {
-    const int64_t n8 = rows * d / 8;
-    const int64_t want = (n8 + threads - 1) / threads;
-    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(want, int64_t(sms) * 16));
-    attn::amax_flat_kernel<<<grid, threads, 0, st>>>(x, n8, amax);
-    attn::convert_flat_kernel<<<grid, threads, 0, st>>>(x, y, n8, amax, descale_out);
-  }
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  const void* xs[1] = {x_bf16};
+  void* ys[1] = {x_e4m3};
+  float* dss[1] = {descale_out};
+  const int64_t el[1] = {rows * d};
+  return launch_quantize(1, xs, ys, dss, el, hadamard, amax, st);
 }
 
 size_t attn_quantize_qkv_workspace_size(void) { return 16; }
@@ -497,52 +531,11 @@ attn_status_t attn_quantize_qkv_e4m3(const void* q, const void* k, const void* v
   for (const void* p : {q, k, v, static_cast<const void*>(q8), static_cast<const void*>(k8),
                         static_cast<const void*>(v8)})
     if (!aligned16(p)) return ATTN_ERR_ALIGNMENT;
-  uint32_t* amax = static_cast<uint32_t*>(workspace);
-  if (cudaMemsetAsync(amax, 0, 3 * sizeof(uint32_t), st) != cudaSuccess) return ATTN_ERR_CUDA;
-  // jobs in the order Q, K, V for the amax pass and V, K, Q for the convert pass: the
-  // tensors read last by the first pass are the first re-read by the second, while they
-  // may still be in L2
   const int64_t el[3] = {tokens * Hq * d_qk, tokens * Hkv * d_qk, tokens * Hkv * d_v};
   const void* xs[3] = {q, k, v};
   void* ys[3] = {q8, k8, v8};
-  float* ds[3] = {descale_q, descale_k, descale_v};
-  const int threads = 256;
-  const int64_t per_block_items = hadamard ? threads / 32 : threads;  // rows or chunks
-  const int sms = num_sms();
-  const int64_t budget = int64_t(sms) * 16;  // blocks per pass, split by size
-  int64_t total = 0;
-  for (int i = 0; i < 3; ++i) total += el[i];
-  attn::QuantBatch fwd{}, rev{};
-  fwd.njobs = rev.njobs = 3;
-  int end_f = 0, end_r = 0;
-  for (int o = 0; o < 3; ++o) {
-    for (int pass = 0; pass < 2; ++pass) {
-      const int i = pass == 0 ? o : 2 - o;
-      const int64_t n = hadamard ? el[i] / 128 : el[i] / 8;
-      const int64_t want = (n + per_block_items - 1) / per_block_items;
-      const int64_t share = std::max<int64_t>(1, (budget * el[i] + total - 1) / total);
-      const int nb = static_cast<int>(std::max<int64_t>(1, std::min(want, share)));
-      attn::QuantJob jb{static_cast<const __nv_bfloat16*>(xs[i]), static_cast<uint8_t*>(ys[i]),
-                        n, amax + i, ds[i]};
-      if (pass == 0) {
-        fwd.job[o] = jb;
-        end_f += nb;
-        fwd.block_end[o] = end_f;
-      } else {
-        rev.job[o] = jb;
-        end_r += nb;
-        rev.block_end[o] = end_r;
-      }
-    }
-  }
-  if (hadamard) {
-    attn::amax_batch_kernel<true><<<end_f, threads, 0, st>>>(fwd);
-    attn::convert_batch_kernel<true><<<end_r, threads, 0, st>>>(rev);
-  } else {
-    attn::amax_batch_kernel<false><<<end_f, threads, 0, st>>>(fwd);
-    attn::convert_batch_kernel<false><<<end_r, threads, 0, st>>>(rev);
-  }
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  float* dss[3] = {descale_q, descale_k, descale_v};
+  return launch_quantize(3, xs, ys, dss, el, hadamard, static_cast<uint32_t*>(workspace), st);
 }
 
 attn_status_t attn_device_status(void* stream) {

@@ -71,37 +71,6 @@ __device__ __forceinline__ void block_amax_atomic(float m, uint32_t* amax_bits) 
   }
 }
 
-__global__ void amax_rot_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows,
-                                uint32_t* amax_bits) {
-  const int lane = threadIdx.x & 31;
-  const int64_t warp_g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  float m = 0.0f;
-  for (int64_t row = warp_g; row < rows; row += nwarps) {
-    float v[4];
-    load_row4(x, row, lane, v);
-    hadamard_row4(v, lane);
-    m = fmaxf(m, fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3]))));
-  }
-  block_amax_atomic(m, amax_bits);
-}
-
-__global__ void amax_flat_kernel(const __nv_bfloat16* __restrict__ x, int64_t n8,
-                                 uint32_t* amax_bits) {
-  float m = 0.0f;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
-       i += stride) {
-    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(x) + i);
-    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      m = fmaxf(m, fmaxf(fabsf(__low2float(h2[k])), fabsf(__high2float(h2[k]))));
-    }
-  }
-  block_amax_atomic(m, amax_bits);
-}
-
 __device__ __forceinline__ float quant_scale(uint32_t amax_bits) {
   const float amax = __uint_as_float(amax_bits);
   return amax > 0.0f ? __fdiv_rn(448.0f, amax) : 1.0f;
@@ -110,52 +79,6 @@ __device__ __forceinline__ float quant_scale(uint32_t amax_bits) {
 // descale of an empty tensor (amax 0): 1, written on the device so the call stays
 // stream-ordered and capturable (no host-to-device copy)
 __global__ void descale_one_kernel(float* descale_out) { *descale_out = 1.0f; }
-
-__device__ __forceinline__ void write_descale(uint32_t amax_bits, float* descale_out) {
-  if (blockIdx.x == 0 && threadIdx.x == 0) {
-    const float amax = __uint_as_float(amax_bits);
-    *descale_out = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-  }
-}
-
-__global__ void convert_rot_kernel(const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ y,
-                                   int64_t rows, const uint32_t* amax_bits, float* descale_out) {
-  const uint32_t ab = *amax_bits;
-  const float sc = quant_scale(ab);
-  write_descale(ab, descale_out);
-  const int lane = threadIdx.x & 31;
-  const int64_t warp_g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  for (int64_t row = warp_g; row < rows; row += nwarps) {
-    float v[4];
-    load_row4(x, row, lane, v);
-    hadamard_row4(v, lane);
-    const uint32_t lo = f32_to_e4m3x2(__fmul_rn(v[0], sc), __fmul_rn(v[1], sc));
-    const uint32_t hi = f32_to_e4m3x2(__fmul_rn(v[2], sc), __fmul_rn(v[3], sc));
-    reinterpret_cast<uint32_t*>(y + row * 128)[lane] = lo | (hi << 16);
-  }
-}
-
-__global__ void convert_flat_kernel(const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ y,
-                                    int64_t n8, const uint32_t* amax_bits, float* descale_out) {
-  const uint32_t ab = *amax_bits;
-  const float sc = quant_scale(ab);
-  write_descale(ab, descale_out);
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
-       i += stride) {
-    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(x) + i);
-    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-    uint32_t w[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k)
-      w[k] = f32_to_e4m3x2(__fmul_rn(__low2float(h2[k]), sc), __fmul_rn(__high2float(h2[k]), sc));
-    uint2 out;
-    out.x = w[0] | (w[1] << 16);
-    out.y = w[2] | (w[3] << 16);
-    reinterpret_cast<uint2*>(y)[i] = out;
-  }
-}
 
 // ---- several tensors in one launch per pass (Q, K and V of one attention call): block b
 // works on job j for block_end[j-1] <= b < block_end[j], grid-striding over that job's
@@ -185,6 +108,16 @@ __device__ __forceinline__ int batch_job(const QuantBatch& b, int& first_block) 
   return j;
 }
 
+__device__ __forceinline__ float absmax8(const uint4 raw, float m) {
+  const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    m = fmaxf(m, fmaxf(fabsf(__low2float(h2[k])), fabsf(__high2float(h2[k]))));
+  return m;
+}
+
+// Four independent 16-byte loads (or rows) in flight per thread, then one per step for the
+// remainder: the passes are HBM-bound and need the bytes in flight.
 template <bool ROT>
 __global__ void amax_batch_kernel(const QuantBatch b) {
   int first = 0;
@@ -196,23 +129,52 @@ __global__ void amax_batch_kernel(const QuantBatch b) {
   if constexpr (ROT) {
     const int lane = threadIdx.x & 31;
     const int64_t nwarps = (static_cast<int64_t>(nblk) * blockDim.x) >> 5;
-    for (int64_t row = tid >> 5; row < jb.n; row += nwarps) {
+    int64_t row = tid >> 5;
+    for (; row + nwarps < jb.n; row += 2 * nwarps) {
+      float v[4], w[4];
+      load_row4(jb.x, row, lane, v);
+      load_row4(jb.x, row + nwarps, lane, w);
+      hadamard_row4(v, lane);
+      hadamard_row4(w, lane);
+      m = fmaxf(m, fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3]))));
+      m = fmaxf(m, fmaxf(fmaxf(fabsf(w[0]), fabsf(w[1])), fmaxf(fabsf(w[2]), fabsf(w[3]))));
+    }
+    for (; row < jb.n; row += nwarps) {
       float v[4];
       load_row4(jb.x, row, lane, v);
       hadamard_row4(v, lane);
       m = fmaxf(m, fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3]))));
     }
   } else {
-    const int64_t stride = static_cast<int64_t>(nblk) * blockDim.x;
-    for (int64_t i = tid; i < jb.n; i += stride) {
-      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(jb.x) + i);
-      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        m = fmaxf(m, fmaxf(fabsf(__low2float(h2[k])), fabsf(__high2float(h2[k]))));
+    const int64_t st = static_cast<int64_t>(nblk) * blockDim.x;
+    const uint4* x = reinterpret_cast<const uint4*>(jb.x);
+    int64_t i = tid;
+    for (; i + 3 * st < jb.n; i += 4 * st) {
+      const uint4 r0 = __ldg(x + i), r1 = __ldg(x + i + st), r2 = __ldg(x + i + 2 * st),
+                  r3 = __ldg(x + i + 3 * st);
+      m = absmax8(r3, absmax8(r2, absmax8(r1, absmax8(r0, m))));
     }
+    for (; i < jb.n; i += st) m = absmax8(__ldg(x + i), m);
   }
   block_amax_atomic(m, jb.amax);
+}
+
+__device__ __forceinline__ uint2 e4m3x8(const uint4 raw, float sc) {
+  const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+  uint32_t w[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    w[k] = f32_to_e4m3x2(__fmul_rn(__low2float(h2[k]), sc), __fmul_rn(__high2float(h2[k]), sc));
+  return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
+}
+
+__device__ __forceinline__ void convert_row(const QuantJob& jb, int64_t row, int lane, float sc) {
+  float v[4];
+  load_row4(jb.x, row, lane, v);
+  hadamard_row4(v, lane);
+  const uint32_t lo = f32_to_e4m3x2(__fmul_rn(v[0], sc), __fmul_rn(v[1], sc));
+  const uint32_t hi = f32_to_e4m3x2(__fmul_rn(v[2], sc), __fmul_rn(v[3], sc));
+  reinterpret_cast<uint32_t*>(jb.y + row * 128)[lane] = lo | (hi << 16);
 }
 
 template <bool ROT>
@@ -231,28 +193,26 @@ __global__ void convert_batch_kernel(const QuantBatch b) {
   if constexpr (ROT) {
     const int lane = threadIdx.x & 31;
     const int64_t nwarps = (static_cast<int64_t>(nblk) * blockDim.x) >> 5;
-    for (int64_t row = tid >> 5; row < jb.n; row += nwarps) {
-      float v[4];
-      load_row4(jb.x, row, lane, v);
-      hadamard_row4(v, lane);
-      const uint32_t lo = f32_to_e4m3x2(__fmul_rn(v[0], sc), __fmul_rn(v[1], sc));
-      const uint32_t hi = f32_to_e4m3x2(__fmul_rn(v[2], sc), __fmul_rn(v[3], sc));
-      reinterpret_cast<uint32_t*>(jb.y + row * 128)[lane] = lo | (hi << 16);
+    int64_t row = tid >> 5;
+    for (; row + nwarps < jb.n; row += 2 * nwarps) {
+      convert_row(jb, row, lane, sc);
+      convert_row(jb, row + nwarps, lane, sc);
     }
+    for (; row < jb.n; row += nwarps) convert_row(jb, row, lane, sc);
   } else {
-    const int64_t stride = static_cast<int64_t>(nblk) * blockDim.x;
-    for (int64_t i = tid; i < jb.n; i += stride) {
-      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(jb.x) + i);
-      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-      uint32_t w[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        w[k] = f32_to_e4m3x2(__fmul_rn(__low2float(h2[k]), sc), __fmul_rn(__high2float(h2[k]), sc));
-      uint2 out;
-      out.x = w[0] | (w[1] << 16);
-      out.y = w[2] | (w[3] << 16);
-      reinterpret_cast<uint2*>(jb.y)[i] = out;
+    const int64_t st = static_cast<int64_t>(nblk) * blockDim.x;
+    const uint4* x = reinterpret_cast<const uint4*>(jb.x);
+    uint2* y = reinterpret_cast<uint2*>(jb.y);
+    int64_t i = tid;
+    for (; i + 3 * st < jb.n; i += 4 * st) {
+      const uint4 r0 = __ldg(x + i), r1 = __ldg(x + i + st), r2 = __ldg(x + i + 2 * st),
+                  r3 = __ldg(x + i + 3 * st);
+      y[i] = e4m3x8(r0, sc);
+      y[i + st] = e4m3x8(r1, sc);
+      y[i + 2 * st] = e4m3x8(r2, sc);
+      y[i + 3 * st] = e4m3x8(r3, sc);
     }
+    for (; i < jb.n; i += st) y[i] = e4m3x8(__ldg(x + i), sc);
   }
 }
 
