@@ -49,10 +49,35 @@ bool dev_err_ptr(uint32_t** out) {
   return true;
 }
 
-// 3-D tiled map over [T, H, d] (d innermost), box = (box_cols, 1, box_rows).
+// 3-D tiled map over [T, H, d] (d innermost), box = (box_cols, 1, box_rows).  An encoded map
+// is a pure function of these arguments, so the last few are kept per host thread and
+// reused when the same tensor is passed again (no lock: the cache is thread-local).
+struct MapKey {
+  const void* base;
+  uint64_t d, H, T;
+  uint32_t box_cols, box_rows;
+  int dt, esize, swz;
+  bool operator==(const MapKey& o) const {
+    return base == o.base && d == o.d && H == o.H && T == o.T && box_cols == o.box_cols &&
+           box_rows == o.box_rows && dt == o.dt && esize == o.esize && swz == o.swz;
+  }
+};
+
 bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, uint64_t d,
               uint64_t H, uint64_t T, uint32_t box_cols, uint32_t box_rows = 128,
               CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
+  constexpr int kSlots = 8;
+  thread_local MapKey keys[kSlots] = {};
+  thread_local CUtensorMap maps[kSlots];
+  thread_local int next = 0;
+  const MapKey key{base, d, H, T, box_cols, box_rows, static_cast<int>(dt), esize,
+                   static_cast<int>(swz)};
+  for (int i = 0; i < kSlots; ++i) {
+    if (keys[i] == key && keys[i].base != nullptr) {
+      *m = maps[i];
+      return true;
+    }
+  }
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {d, H, T};
@@ -62,7 +87,49 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esiz
   CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  if (r != CUDA_SUCCESS) return false;
+  keys[next] = key;
+  maps[next] = *m;
+  next = (next + 1) % kSlots;
+  return true;
+}
+
+// The current context (driver API, through the runtime's entry-point query), to key state
+// that belongs to a context: a device's primary context is replaced by cudaDeviceReset.
+using PFN_ctxGetCurrent = CUresult (*)(CUcontext*);
+CUcontext current_context() {
+  static PFN_ctxGetCurrent fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_ctxGetCurrent>(p);
+  });
+  CUcontext c = nullptr;
+  if (fn == nullptr || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
+// cudaFuncSetAttribute(max dynamic shared memory) for kernel `kern`, skipped when it was
+// already done for the current context by this host thread.
+template <typename K>
+bool set_smem_attr(K kern, int bytes) {
+  thread_local CUcontext done_ctx[4] = {};
+  thread_local int next = 0;
+  const CUcontext c = current_context();
+  if (c != nullptr)
+    for (CUcontext d : done_ctx)
+      if (d == c) return true;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess)
+    return false;
+  if (c != nullptr) {
+    done_ctx[next] = c;
+    next = (next + 1) % 4;
+  }
+  return true;
 }
 
 // The prefill kernels move registers from their producer/MMA warps to their softmax warps
@@ -97,9 +164,7 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, attn::FwdP
       !make_map(&mv, v, dt, C::E, attn::DV, prm.Hkv, T, C::BOX_COLS))
     return ATTN_ERR_CUDA;
   auto kern = attn::attn_fwd_kernel<FP8, DQK, DUMP, EXACT, VARLEN>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC) !=
-      cudaSuccess)
-    return ATTN_ERR_CUDA;
+  if (!set_smem_attr(kern, C::SMEM_ALLOC)) return ATTN_ERR_CUDA;
   const attn_status_t rs = register_split_ok(kern);
   if (rs != ATTN_OK) return rs;
   // units: two query tiles of one head, or (ATTN_KERNEL_HEADS, Hq / Hkv even) one query
@@ -268,8 +333,7 @@ template <bool FP8, int G>
 attn_status_t launch_decode(attn::DecodeParams& prm, cudaStream_t st) {
   auto k1 = attn::decode_split_kernel<FP8, G>;
   constexpr int smem = attn::dec_smem_bytes<FP8, G>();
-  if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return ATTN_ERR_CUDA;
+  if (!set_smem_attr(k1, smem)) return ATTN_ERR_CUDA;
   const dim3 grid(static_cast<unsigned>(prm.Hkv), static_cast<unsigned>(prm.n_splits),
                   static_cast<unsigned>(prm.B));
   k1<<<grid, attn::DEC_THREADS, smem, st>>>(prm);
