@@ -37,6 +37,12 @@ NOMINAL_FP8_TFLOPS = 4500.0
 NOMINAL_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
+# prefill kernel families (attn_select_prefill_kernel)
+KERNEL_IDS = {"single": lambda pkg: pkg.ATTN_KERNEL_SINGLE,
+              "heads": lambda pkg: pkg.ATTN_KERNEL_HEADS,
+              "k64": lambda pkg: pkg.ATTN_KERNEL_K64,
+              "k64heads": lambda pkg: pkg.ATTN_KERNEL_K64_HEADS}
+
 WORKLOADS = {
     # name: (B, S, Hq, Hkv, d_qk, d_v, distribution, description)
     "small_s256": (1, 256, 1, 1, 128, 128, "gaussian",
@@ -338,8 +344,7 @@ def gpu_bench(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    pkg.attn_select_prefill_kernel(pkg.ATTN_KERNEL_HEADS if args.kernel == "heads"
-                                   else pkg.ATTN_KERNEL_SINGLE)
+    pkg.attn_select_prefill_kernel(KERNEL_IDS[args.kernel](pkg))
     B, S, Hq, Hkv, dqk, dv, distn, desc = WORKLOADS[args.workload]
     if args.split == "heads":
         # one problem shared by all ranks: rank r takes a contiguous range of kv heads and
@@ -855,9 +860,10 @@ def main(argv=None):
                          "the default workload")
     ap.add_argument("--exact-p", action="store_true",
                     help="FP8 probabilities by exponential + e4m3 rounding (the ablation of lean P)")
-    ap.add_argument("--kernel", default="single", choices=["single", "heads"],
-                    help="work unit of the prefill kernel: two query tiles of one head "
-                         "(default) or one query tile of two heads of one kv group")
+    ap.add_argument("--kernel", default="single", choices=list(KERNEL_IDS),
+                    help="prefill kernel: 128-key tiles with two query tiles of one head "
+                         "(single, default) or one query tile of two heads of one kv group "
+                         "(heads) per CTA; k64 / k64heads: the same units with 64-key tiles")
     ap.add_argument("--split", default="replicas", choices=["replicas", "heads"],
                     help="multi-GPU: an independent problem per GPU (weak scaling), or one "
                          "problem divided by kv heads (strong scaling)")

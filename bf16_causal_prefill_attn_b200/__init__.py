@@ -24,6 +24,8 @@ ATTN_FLAG_UNROTATE_O = 1
 ATTN_FLAG_EXACT_P = 2
 ATTN_KERNEL_SINGLE = 0
 ATTN_KERNEL_HEADS = 2
+ATTN_KERNEL_K64 = 3
+ATTN_KERNEL_K64_HEADS = 4
 
 _lib = None
 
@@ -300,9 +302,10 @@ def attn_set_wait_timeout_ns(ns):
 
 
 def attn_select_prefill_kernel(kernel):
-    """Work unit of the prefill kernel for later calls: ATTN_KERNEL_SINGLE (two query tiles
-    of one head per CTA) or ATTN_KERNEL_HEADS (one query tile of two heads of one kv
-    group)."""
+    """Prefill kernel for later calls: ATTN_KERNEL_SINGLE (128-key tiles, two query tiles
+    of one head per CTA), ATTN_KERNEL_HEADS (128-key tiles, one query tile of two heads of
+    one kv group), ATTN_KERNEL_K64 / ATTN_KERNEL_K64_HEADS (the same units with 64-key
+    tiles)."""
     _check(lib().attn_select_prefill_kernel(int(kernel)), "attn_select_prefill_kernel")
 
 

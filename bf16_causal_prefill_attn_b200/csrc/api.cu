@@ -13,6 +13,7 @@
 
 #include "../../include/attn.h"
 #include "attn_fwd.cuh"
+#include "attn_k64.cuh"
 #include "decode.cuh"
 #include "quantize.cuh"
 
@@ -112,17 +113,18 @@ CUcontext current_context() {
   return c;
 }
 
-// cudaFuncSetAttribute(max dynamic shared memory) for kernel `kern`, skipped when it was
-// already done for the current context by this host thread.
-template <typename K>
-bool set_smem_attr(K kern, int bytes) {
+// cudaFuncSetAttribute(max dynamic shared memory) for kernel KERN, skipped when it was
+// already done for the current context by this host thread.  The cache is per kernel (a
+// template on the kernel's address: the prefill kernels all share one function type).
+template <auto KERN>
+bool set_smem_attr(int bytes) {
   thread_local CUcontext done_ctx[4] = {};
   thread_local int next = 0;
   const CUcontext c = current_context();
   if (c != nullptr)
     for (CUcontext d : done_ctx)
       if (d == c) return true;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+  if (cudaFuncSetAttribute(KERN, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
       cudaSuccess)
     return false;
   if (c != nullptr) {
@@ -135,14 +137,15 @@ bool set_smem_attr(K kern, int bytes) {
 // The prefill kernels move registers from their producer/MMA warps to their softmax warps
 // (setmaxnreg); the increase only succeeds if the block was launched with at least
 // REGS_NEEDED_AT_LAUNCH registers per thread, so never launch one with fewer.  The count
-// is a property of the compiled kernel: checked once per kernel, then remembered.
-template <typename K>
-attn_status_t register_split_ok(K kern) {
+// is a property of the compiled kernel: checked once per kernel (a template on its
+// address), then remembered.
+template <auto KERN>
+attn_status_t register_split_ok() {
   static std::atomic<int> known{0};  // 0 not yet checked, 1 ok, 2 too few registers
   const int k = known.load(std::memory_order_relaxed);
   if (k != 0) return k == 1 ? ATTN_OK : ATTN_ERR_UNSUPPORTED;
   cudaFuncAttributes fa;
-  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return ATTN_ERR_CUDA;  // not cached
+  if (cudaFuncGetAttributes(&fa, KERN) != cudaSuccess) return ATTN_ERR_CUDA;  // not cached
   const bool ok = fa.numRegs >= attn::REGS_NEEDED_AT_LAUNCH &&
                   fa.numRegs * attn::NUM_THREADS <= 65536;
   known.store(ok ? 1 : 2, std::memory_order_relaxed);
@@ -163,9 +166,9 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, attn::FwdP
       !make_map(&mk, k, dt, C::E, DQK, prm.Hkv, T, C::BOX_COLS) ||
       !make_map(&mv, v, dt, C::E, attn::DV, prm.Hkv, T, C::BOX_COLS))
     return ATTN_ERR_CUDA;
-  auto kern = attn::attn_fwd_kernel<FP8, DQK, DUMP, EXACT, VARLEN>;
-  if (!set_smem_attr(kern, C::SMEM_ALLOC)) return ATTN_ERR_CUDA;
-  const attn_status_t rs = register_split_ok(kern);
+  constexpr auto kern = attn::attn_fwd_kernel<FP8, DQK, DUMP, EXACT, VARLEN>;
+  if (!set_smem_attr<kern>(C::SMEM_ALLOC)) return ATTN_ERR_CUDA;
+  const attn_status_t rs = register_split_ok<kern>();
   if (rs != ATTN_OK) return rs;
   // units: two query tiles of one head, or (ATTN_KERNEL_HEADS, Hq / Hkv even) one query
   // tile of two heads of one kv group
@@ -178,10 +181,38 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, attn::FwdP
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-// The prefill kernel for one instantiation.
+// The 64-key-tile kernel (attn_k64.cuh): K and V boxes of 64 rows, the same units.
+template <bool FP8, int DQK, bool DUMP, bool EXACT = false, bool VARLEN = false>
+attn_status_t launch_k64(const void* q, const void* k, const void* v, attn::FwdParams& prm,
+                         cudaStream_t stream) {
+  using C = attn::Cfg64<FP8, DQK>;
+  const CUtensorMapDataType dt =
+      FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const uint64_t T = static_cast<uint64_t>(prm.total_tokens);
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, dt, C::E, DQK, prm.Hq, T, C::BOX_COLS) ||
+      !make_map(&mk, k, dt, C::E, DQK, prm.Hkv, T, C::BOX_COLS, attn::KT) ||
+      !make_map(&mv, v, dt, C::E, attn::DV, prm.Hkv, T, C::BOX_COLS, attn::KT))
+    return ATTN_ERR_CUDA;
+  constexpr auto kern = attn::attn_k64_kernel<FP8, DQK, DUMP, EXACT, VARLEN>;
+  if (!set_smem_attr<kern>(C::SMEM_ALLOC)) return ATTN_ERR_CUDA;
+  const attn_status_t rs = register_split_ok<kern>();
+  if (rs != ATTN_OK) return rs;
+  attn::FwdParams pp = prm;
+  pp.head_pairs = (g_kernel == ATTN_KERNEL_K64_HEADS && prm.G % 2 == 0) ? 1 : 0;
+  pp.n_pairs = pp.head_pairs ? prm.n_q_tiles : (prm.n_q_tiles + 1) / 2;
+  const unsigned grid = static_cast<unsigned>(pp.n_pairs) * prm.B *
+                        static_cast<unsigned>(pp.head_pairs ? prm.Hq / 2 : prm.Hq);
+  kern<<<grid, attn::NUM_THREADS, C::SMEM_ALLOC, stream>>>(mq, mk, mv, pp);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// The prefill kernel for one instantiation, by the selected kernel family.
 template <bool FP8, int DQK, bool DUMP, bool EXACT = false, bool VARLEN = false>
 attn_status_t launch_prefill(const void* q, const void* k, const void* v, attn::FwdParams& prm,
                              cudaStream_t stream) {
+  if (g_kernel == ATTN_KERNEL_K64 || g_kernel == ATTN_KERNEL_K64_HEADS)
+    return launch_k64<FP8, DQK, DUMP, EXACT, VARLEN>(q, k, v, prm, stream);
   return launch_fwd<FP8, DQK, DUMP, EXACT, VARLEN>(q, k, v, prm, stream);
 }
 
@@ -331,9 +362,9 @@ attn_status_t varlen_impl(const void* q, const void* k, const void* v, void* o, 
 
 template <bool FP8, int G>
 attn_status_t launch_decode(attn::DecodeParams& prm, cudaStream_t st) {
-  auto k1 = attn::decode_split_kernel<FP8, G>;
+  constexpr auto k1 = attn::decode_split_kernel<FP8, G>;
   constexpr int smem = attn::dec_smem_bytes<FP8, G>();
-  if (!set_smem_attr(k1, smem)) return ATTN_ERR_CUDA;
+  if (!set_smem_attr<k1>(smem)) return ATTN_ERR_CUDA;
   const dim3 grid(static_cast<unsigned>(prm.Hkv), static_cast<unsigned>(prm.n_splits),
                   static_cast<unsigned>(prm.B));
   k1<<<grid, attn::DEC_THREADS, smem, st>>>(prm);
@@ -620,7 +651,9 @@ void attn_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns = ns ? ns : kDefaultTi
 void attn_selftest_stall_tile(int tile) { g_stall_tile = tile < 0 ? -1 : tile; }
 
 attn_status_t attn_select_prefill_kernel(int kernel) {
-  if (kernel != ATTN_KERNEL_SINGLE && kernel != ATTN_KERNEL_HEADS) return ATTN_ERR_INVALID_ARG;
+  if (kernel != ATTN_KERNEL_SINGLE && kernel != ATTN_KERNEL_HEADS && kernel != ATTN_KERNEL_K64 &&
+      kernel != ATTN_KERNEL_K64_HEADS)
+    return ATTN_ERR_INVALID_ARG;
   g_kernel = kernel;
   return ATTN_OK;
 }

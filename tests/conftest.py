@@ -26,12 +26,23 @@ def pytest_collection_modifyitems(config, items):
             item.add_marker(skip)
 
 
-@pytest.fixture(params=["single", "heads"])
+KERNELS = {"single": "ATTN_KERNEL_SINGLE", "heads": "ATTN_KERNEL_HEADS",
+           "k64": "ATTN_KERNEL_K64", "k64heads": "ATTN_KERNEL_K64_HEADS"}
+
+
+@pytest.fixture(params=list(KERNELS))
 def prefill_kernel(request):
-    """Runs a test under each work unit of the prefill kernel (two query tiles of one head;
-    one query tile of two heads of one kv group), restoring the default afterwards."""
+    """Runs a test under each prefill kernel (128-key tiles with two query tiles of one head
+    or one query tile of two heads of one kv group per CTA; 64-key tiles with either unit),
+    restoring the default afterwards."""
     import bf16_causal_prefill_attn_b200 as pkg
-    k = {"single": pkg.ATTN_KERNEL_SINGLE, "heads": pkg.ATTN_KERNEL_HEADS}[request.param]
-    pkg.attn_select_prefill_kernel(k)
+    pkg.attn_select_prefill_kernel(getattr(pkg, KERNELS[request.param]))
     yield request.param
     pkg.attn_select_prefill_kernel(pkg.ATTN_KERNEL_SINGLE)
+
+
+@pytest.fixture
+def key_tile(prefill_kernel):
+    """Keys per tile of the selected prefill kernel: the FP8 lean-P reference max is updated
+    once per key tile, so the emulator replays the kernel with this tile."""
+    return 64 if prefill_kernel.startswith("k64") else 128

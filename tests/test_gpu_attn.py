@@ -85,7 +85,7 @@ def _fp8_inputs(B, S, Hq, Hkv, dqk, seed, dist, rotate=False):
     (2, 384, 6, 2, 128, True, "outlier"),       # G = 3, odd tile count
     (1, 640, 2, 2, 192, True, "gaussian"),      # MLA shape, five tiles
 ])
-def test_fp8_matches_fp64_on_quantised_inputs(B, S, Hq, Hkv, dqk, causal, dist):
+def test_fp8_matches_fp64_on_quantised_inputs(B, S, Hq, Hkv, dqk, causal, dist, key_tile):
     _, dev, host = _fp8_inputs(B, S, Hq, Hkv, dqk, 7 + S, dist)
     (q8, dq), (k8, dk), (v8, dv) = dev
     o, lse = pkg.attn_fwd(q8, k8, v8, causal=causal, descale_q=dq, descale_k=dk, descale_v=dv)
@@ -99,7 +99,7 @@ def test_fp8_matches_fp64_on_quantised_inputs(B, S, Hq, Hkv, dqk, causal, dist):
     for b in range(B):
         eo, _ = leanp.attention_rows(host[0][0], host[1][0], host[2][0], host[0][1], host[1][1],
                                      host[2][1], np.arange(S), list(range(Hq)), batch=b,
-                                     causal=causal)
+                                     causal=causal, tile=key_tile)
         emu[b] = eo.transpose(1, 0, 2)
     assert rel_rms(got, emu) <= 5e-3
     # the FP8 bar holds on the causal contract; full attention over short rows is the
@@ -116,7 +116,7 @@ def test_fp8_matches_fp64_on_quantised_inputs(B, S, Hq, Hkv, dqk, causal, dist):
     (2, 256, 2, 1, 128, False, "outlier"),
     (1, 640, 3, 1, 128, True, "outlier"),      # G = 3 (rows mode), five tiles
 ])
-def test_fp8_leanp_codes_bit_exact(B, S, Hq, Hkv, dqk, causal, dist):
+def test_fp8_leanp_codes_bit_exact(B, S, Hq, Hkv, dqk, causal, dist, key_tile):
     _, dev, host = _fp8_inputs(B, S, Hq, Hkv, dqk, 100 + S, dist)
     (q8, dq), (k8, dk), (v8, dv) = dev
     o, lse, ds, dc, dks = pkg.attn_fwd_fp8_dump(q8, k8, v8, dq, dk, dv, causal=causal)
@@ -145,7 +145,7 @@ def test_fp8_leanp_codes_bit_exact(B, S, Hq, Hkv, dqk, causal, dist):
                 fin = np.isfinite(exact)
                 assert np.array_equal(np.isfinite(srow), fin)
                 np.testing.assert_allclose(srow[fin], exact[fin], rtol=1e-5, atol=1e-5 * np.abs(exact[fin]).max())
-                codes, ks, _ = leanp.encode_row(srow, a)
+                codes, ks, _ = leanp.encode_row(srow, a, key_tile)
                 assert np.array_equal(dc[b, h, i, : nt * 128], codes), (b, h, i)
                 assert np.array_equal(dks[b, h, i, : nt * 2], ks), (b, h, i)
             # O from the emulator driven by the kernel's own scores: equal up to fp32
@@ -159,7 +159,7 @@ def test_fp8_leanp_codes_bit_exact(B, S, Hq, Hkv, dqk, causal, dist):
                 srow = np.ascontiguousarray(ds[b, h, i, :nvis])
                 vv = np.ascontiguousarray(vd[b, :, g, :])
                 leanp.lib().leanp_attention_row(
-                    srow.ctypes.data_as(ctypes.POINTER(ctypes.c_float)), nvis, 128,
+                    srow.ctypes.data_as(ctypes.POINTER(ctypes.c_float)), nvis, key_tile,
                     vv.ctypes.data_as(ctypes.POINTER(ctypes.c_double)), 128, float(a), leanp.KMAX,
                     orow.ctypes.data_as(ctypes.POINTER(ctypes.c_double)),
                     lrow.ctypes.data_as(ctypes.POINTER(ctypes.c_double)))

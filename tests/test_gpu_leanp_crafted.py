@@ -122,7 +122,7 @@ def exact_scores(codes):
     return np.einsum("ihd,jd->hij", qd[0], kd[0, :, 0, :])
 
 
-def replay_and_count(scores, a):
+def replay_and_count(scores, a, tile):
     """Replay the emulator on every causal row; return the codes, shifts and counts of the
     edge cases met: rows with two or more mid-row raises, live blocks at k_b = 16, codes at
     126, and live codes formed from an exact .5 midpoint."""
@@ -135,7 +135,7 @@ def replay_and_count(scores, a):
             nt = i // 128 + 1
             row = np.full(nt * 128, -np.inf, dtype=np.float32)
             row[: i + 1] = scores[h, i, : i + 1]
-            codes, ks, mref = leanp.encode_row(row, a)
+            codes, ks, mref = leanp.encode_row(row, a, tile)
             out_codes[h, i, : nt * 128] = codes
             out_ks[h, i, : nt * 2] = ks
             n["raises2"] += int(np.count_nonzero(np.diff(mref)) >= 2)
@@ -147,7 +147,7 @@ def replay_and_count(scores, a):
             fin = np.isfinite(row)
             x = (np.float64(a) * row[fin].astype(np.float64)
                  + (top + 8 * ks[np.nonzero(fin)[0] // 64].astype(np.float64)
-                    - mref[np.nonzero(fin)[0] // 128]))
+                    - mref[np.nonzero(fin)[0] // tile]))
             live = (x > 0.5) & (x < 126)
             n["ties"] += int(((x - np.floor(x)) == 0.5)[live].sum())
     return out_codes, out_ks, n
@@ -156,7 +156,7 @@ def replay_and_count(scores, a):
 @pytest.mark.gpu
 @pytest.mark.usefixtures("prefill_kernel")
 @pytest.mark.parametrize("d_qk,hq", [(128, 2), (192, 2), (128, 1)])
-def test_leanp_codes_bit_exact_on_crafted_edge_cases(d_qk, hq):
+def test_leanp_codes_bit_exact_on_crafted_edge_cases(d_qk, hq, key_tile):
     """hq = 2: two query heads share the kv head (so the head-pair work unit applies); hq = 1:
     one head (two query tiles per CTA in either setting)."""
     codes, (dq, dk, dv) = build_inputs(d_qk, seed=d_qk, hq=hq)
@@ -176,7 +176,7 @@ def test_leanp_codes_bit_exact_on_crafted_edge_cases(d_qk, hq):
         for i in range(S):
             nt = i // 128 + 1
             assert np.isneginf(d_s[h, i, i + 1: nt * 128]).all()
-    exp_codes, exp_ks, n = replay_and_count(d_s, a)
+    exp_codes, exp_ks, n = replay_and_count(d_s, a, key_tile)
     # every edge case the inputs were built for occurs
     assert n["raises2"] >= 100 * hq and n["k16_live"] >= 100 * hq and n["code126"] >= 50 * hq
     assert n["ties"] >= 1000, n
@@ -194,7 +194,7 @@ def test_leanp_codes_bit_exact_on_crafted_edge_cases(d_qk, hq):
             srow = np.ascontiguousarray(d_s[h, i, : i + 1])
             orow, lrow = np.zeros(128), np.zeros(1)
             leanp.lib().leanp_attention_row(
-                srow.ctypes.data_as(ctypes.POINTER(ctypes.c_float)), i + 1, 128,
+                srow.ctypes.data_as(ctypes.POINTER(ctypes.c_float)), i + 1, key_tile,
                 vd.ctypes.data_as(ctypes.POINTER(ctypes.c_double)), 128, float(a), leanp.KMAX,
                 orow.ctypes.data_as(ctypes.POINTER(ctypes.c_double)),
                 lrow.ctypes.data_as(ctypes.POINTER(ctypes.c_double)))
