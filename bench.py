@@ -39,9 +39,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # prefill kernel families (attn_select_prefill_kernel)
 KERNEL_IDS = {"single": lambda pkg: pkg.ATTN_KERNEL_SINGLE,
-              "heads": lambda pkg: pkg.ATTN_KERNEL_HEADS,
-              "k64": lambda pkg: pkg.ATTN_KERNEL_K64,
-              "k64heads": lambda pkg: pkg.ATTN_KERNEL_K64_HEADS}
+              "heads": lambda pkg: pkg.ATTN_KERNEL_HEADS}
 
 WORKLOADS = {
     # name: (B, S, Hq, Hkv, d_qk, d_v, distribution, description)
@@ -861,9 +859,8 @@ def main(argv=None):
     ap.add_argument("--exact-p", action="store_true",
                     help="FP8 probabilities by exponential + e4m3 rounding (the ablation of lean P)")
     ap.add_argument("--kernel", default="single", choices=list(KERNEL_IDS),
-                    help="prefill kernel: 128-key tiles with two query tiles of one head "
-                         "(single, default) or one query tile of two heads of one kv group "
-                         "(heads) per CTA; k64 / k64heads: the same units with 64-key tiles")
+                    help="work unit of the prefill kernel: two query tiles of one head "
+                         "(default) or one query tile of two heads of one kv group")
     ap.add_argument("--split", default="replicas", choices=["replicas", "heads"],
                     help="multi-GPU: an independent problem per GPU (weak scaling), or one "
                          "problem divided by kv heads (strong scaling)")

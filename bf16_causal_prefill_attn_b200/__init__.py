@@ -24,8 +24,7 @@ ATTN_FLAG_UNROTATE_O = 1
 ATTN_FLAG_EXACT_P = 2
 ATTN_KERNEL_SINGLE = 0
 ATTN_KERNEL_HEADS = 2
-ATTN_KERNEL_K64 = 3
-ATTN_KERNEL_K64_HEADS = 4
+ATTN_KERNEL_PERSISTENT = 4
 
 _lib = None
 
@@ -81,6 +80,8 @@ def lib():
         L.attn_select_prefill_kernel.restype = i32
         L.attn_selftest_stall_tile.argtypes = [i32]
         L.attn_selftest_stall_tile.restype = None
+        L.attn_selftest_max_ctas.argtypes = [i32]
+        L.attn_selftest_max_ctas.restype = None
         L.attn_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
         L.attn_selftest_wait_timeout.restype = i32
         L.attn_status_string.argtypes = [i32]
@@ -302,11 +303,16 @@ def attn_set_wait_timeout_ns(ns):
 
 
 def attn_select_prefill_kernel(kernel):
-    """Prefill kernel for later calls: ATTN_KERNEL_SINGLE (128-key tiles, two query tiles
-    of one head per CTA), ATTN_KERNEL_HEADS (128-key tiles, one query tile of two heads of
-    one kv group), ATTN_KERNEL_K64 / ATTN_KERNEL_K64_HEADS (the same units with 64-key
-    tiles)."""
+    """Work unit and schedule of the prefill kernel for later calls: ATTN_KERNEL_SINGLE (two
+    query tiles of one head per unit) or ATTN_KERNEL_HEADS (one query tile of two heads of
+    one kv group), optionally OR ATTN_KERNEL_PERSISTENT (one CTA per SM looping over the
+    units instead of one CTA per unit)."""
     _check(lib().attn_select_prefill_kernel(int(kernel)), "attn_select_prefill_kernel")
+
+
+def attn_selftest_max_ctas(n):
+    """Test-only: cap the persistent grid at n CTAs (n <= 0: no cap)."""
+    lib().attn_selftest_max_ctas(int(n))
 
 
 def attn_selftest_stall_tile(tile):

@@ -13,7 +13,6 @@
 
 #include "../../include/attn.h"
 #include "attn_fwd.cuh"
-#include "attn_k64.cuh"
 #include "decode.cuh"
 #include "quantize.cuh"
 
@@ -28,6 +27,7 @@ __device__ uint32_t g_dev_err = 0;
 uint64_t g_timeout_ns = kDefaultTimeoutNs;
 int g_stall_tile = -1;  // test-only (attn_selftest_stall_tile)
 int g_kernel = ATTN_KERNEL_SINGLE;  // prefill kernel family (attn_select_prefill_kernel)
+int g_max_ctas = 0;  // test-only cap on the persistent grid (attn_selftest_max_ctas; 0: none)
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -152,6 +152,22 @@ attn_status_t register_split_ok() {
   return ok ? ATTN_OK : ATTN_ERR_UNSUPPORTED;
 }
 
+// Multiprocessors of the current device (cached per device; devices are few).
+int sm_count() {
+  constexpr int kMaxDev = 64;
+  static std::atomic<int> cache[kMaxDev] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (dev >= 0 && dev < kMaxDev) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  if (dev >= 0 && dev < kMaxDev) cache[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 template <bool FP8, int DQK, bool DUMP, bool EXACT = false, bool VARLEN = false>
@@ -171,48 +187,30 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, attn::FwdP
   const attn_status_t rs = register_split_ok<kern>();
   if (rs != ATTN_OK) return rs;
   // units: two query tiles of one head, or (ATTN_KERNEL_HEADS, Hq / Hkv even) one query
-  // tile of two heads of one kv group
+  // tile of two heads of one kv group; one CTA per unit, or (ATTN_KERNEL_PERSISTENT) one
+  // CTA per SM running every SM-count-th unit
   attn::FwdParams pp = prm;
-  pp.head_pairs = (g_kernel == ATTN_KERNEL_HEADS && prm.G % 2 == 0) ? 1 : 0;
+  pp.head_pairs = ((g_kernel & ATTN_KERNEL_HEADS) && prm.G % 2 == 0) ? 1 : 0;
   pp.n_pairs = pp.head_pairs ? prm.n_q_tiles : (prm.n_q_tiles + 1) / 2;
-  const unsigned grid = static_cast<unsigned>(pp.n_pairs) * prm.B *
-                        static_cast<unsigned>(pp.head_pairs ? prm.Hq / 2 : prm.Hq);
+  const int64_t units = static_cast<int64_t>(pp.n_pairs) * prm.B *
+                        (pp.head_pairs ? prm.Hq / 2 : prm.Hq);
+  if (units <= 0 || units > INT32_MAX) return ATTN_ERR_INVALID_ARG;
+  pp.n_units = static_cast<int>(units);
+  unsigned grid = static_cast<unsigned>(units);
+  if (g_kernel & ATTN_KERNEL_PERSISTENT) {
+    const int sms = sm_count();
+    if (sms <= 0) return ATTN_ERR_CUDA;
+    grid = static_cast<unsigned>(std::min<int64_t>(units, sms));
+    if (g_max_ctas > 0) grid = std::min(grid, static_cast<unsigned>(g_max_ctas));
+  }
   kern<<<grid, attn::NUM_THREADS, C::SMEM_ALLOC, stream>>>(mq, mk, mv, pp);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-// The 64-key-tile kernel (attn_k64.cuh): K and V boxes of 64 rows, the same units.
-template <bool FP8, int DQK, bool DUMP, bool EXACT = false, bool VARLEN = false>
-attn_status_t launch_k64(const void* q, const void* k, const void* v, attn::FwdParams& prm,
-                         cudaStream_t stream) {
-  using C = attn::Cfg64<FP8, DQK>;
-  const CUtensorMapDataType dt =
-      FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  const uint64_t T = static_cast<uint64_t>(prm.total_tokens);
-  CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, dt, C::E, DQK, prm.Hq, T, C::BOX_COLS) ||
-      !make_map(&mk, k, dt, C::E, DQK, prm.Hkv, T, C::BOX_COLS, attn::KT) ||
-      !make_map(&mv, v, dt, C::E, attn::DV, prm.Hkv, T, C::BOX_COLS, attn::KT))
-    return ATTN_ERR_CUDA;
-  constexpr auto kern = attn::attn_k64_kernel<FP8, DQK, DUMP, EXACT, VARLEN>;
-  if (!set_smem_attr<kern>(C::SMEM_ALLOC)) return ATTN_ERR_CUDA;
-  const attn_status_t rs = register_split_ok<kern>();
-  if (rs != ATTN_OK) return rs;
-  attn::FwdParams pp = prm;
-  pp.head_pairs = (g_kernel == ATTN_KERNEL_K64_HEADS && prm.G % 2 == 0) ? 1 : 0;
-  pp.n_pairs = pp.head_pairs ? prm.n_q_tiles : (prm.n_q_tiles + 1) / 2;
-  const unsigned grid = static_cast<unsigned>(pp.n_pairs) * prm.B *
-                        static_cast<unsigned>(pp.head_pairs ? prm.Hq / 2 : prm.Hq);
-  kern<<<grid, attn::NUM_THREADS, C::SMEM_ALLOC, stream>>>(mq, mk, mv, pp);
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
-}
-
-// The prefill kernel for one instantiation, by the selected kernel family.
+// The prefill kernel for one instantiation.
 template <bool FP8, int DQK, bool DUMP, bool EXACT = false, bool VARLEN = false>
 attn_status_t launch_prefill(const void* q, const void* k, const void* v, attn::FwdParams& prm,
                              cudaStream_t stream) {
-  if (g_kernel == ATTN_KERNEL_K64 || g_kernel == ATTN_KERNEL_K64_HEADS)
-    return launch_k64<FP8, DQK, DUMP, EXACT, VARLEN>(q, k, v, prm, stream);
   return launch_fwd<FP8, DQK, DUMP, EXACT, VARLEN>(q, k, v, prm, stream);
 }
 
@@ -650,10 +648,10 @@ void attn_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns = ns ? ns : kDefaultTi
 
 void attn_selftest_stall_tile(int tile) { g_stall_tile = tile < 0 ? -1 : tile; }
 
+void attn_selftest_max_ctas(int n) { g_max_ctas = n > 0 ? n : 0; }
+
 attn_status_t attn_select_prefill_kernel(int kernel) {
-  if (kernel != ATTN_KERNEL_SINGLE && kernel != ATTN_KERNEL_HEADS && kernel != ATTN_KERNEL_K64 &&
-      kernel != ATTN_KERNEL_K64_HEADS)
-    return ATTN_ERR_INVALID_ARG;
+  if ((kernel & ~(ATTN_KERNEL_HEADS | ATTN_KERNEL_PERSISTENT)) != 0) return ATTN_ERR_INVALID_ARG;
   g_kernel = kernel;
   return ATTN_OK;
 }

@@ -14,8 +14,13 @@
 //         normaliser is the sum of the rounded probabilities, formed by one extra MMA per
 //         key tile against a matrix of ones.
 //
-// A CTA owns two 128-row query tiles t = 0, 1 of one (batch, head): rows
-// [256 p + 128 t, +128) of query-tile pair p.  They share every K/V tile in shared memory.
+// A work unit is two 128-row query tiles (slots t = 0, 1) that share every K/V tile in
+// shared memory: rows [256 p + 128 t, +128) of query-tile pair p of one (batch, head), or
+// (head pairs) one query tile of two query heads of one kv group.  Units are numbered
+// longest first; a CTA runs units blockIdx.x, then (in the next round of gridDim.x units)
+// the mirrored index, and so on.  With one CTA per unit that is one unit per CTA; with one
+// CTA per SM (persistent) a CTA's setup is paid once and each slot's epilogue overlaps the
+// other slot's work and the next unit's first S.  All barrier phases are running counts.
 // Roles (384 threads, 12 warps):
 //   warps 0-3   softmax of tile 0, warps 4-7 softmax of tile 1: thread r of the group owns
 //               query row r (TMEM lane r); reads S, updates the reference max (lazily:
@@ -23,7 +28,7 @@
 //               in TMEM when it does, writes P (BF16: into the S columns it has consumed;
 //               FP8: into shared memory, with its scale factors in TMEM), and finally
 //               writes O and lse;
-//   warp 8      TMA producer: both Q tiles once, then K and V through NK / NV stages;
+//   warp 8      TMA producer of K and V (NK / NV stages, continuing across units);
 //   warp 9      MMA issuer (warp-wide control flow, one elected lane issues).  One tile's
 //               softmax overlaps the other tile's MMAs (ping-pong).  Order per key tile j:
 //                 BF16  PV_0(j), S_0(j+1), PV_1(j), S_1(j+1)  (P_t aliases S_t, so
@@ -32,7 +37,8 @@
 //                       read into registers, so it runs during the softmax of S_t(j): each
 //                       softmax group then has a whole period, not half, for its tile);
 //   warp 10     FP8: PV MMA issuer (warp 9 then issues only the S MMAs); BF16: idle;
-//   warp 11     TMEM allocator.
+//   warp 11     TMEM allocator, then the Q loader: slot t's Q tile of the next unit as soon
+//               as the slot's last S MMA of the current unit has completed (q_empty).
 // TMEM (512 columns x 128 lanes, see TmemMap):
 //   BF16  S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512); P_t (bf16, 64
 //         columns) overwrites the first columns of S_t.
@@ -59,8 +65,8 @@ constexpr int BLOCK_M = 128;
 constexpr int BLOCK_N = 128;
 constexpr int DV = 128;
 constexpr int NUM_THREADS = 384;
-constexpr int REGS_SOFTMAX = 208;  // per thread of warps 0-7 after setmaxnreg
-constexpr int REGS_OTHER = 88;     // per thread of warps 8-11
+constexpr int REGS_SOFTMAX = 200;  // per thread of warps 0-7 after setmaxnreg
+constexpr int REGS_OTHER = 104;    // per thread of warps 8-11 (unit loop state)
 // registers per thread the launch must provide at least for that split
 constexpr int REGS_NEEDED_AT_LAUNCH =
     (2 * 128 * REGS_SOFTMAX + 128 * REGS_OTHER + NUM_THREADS - 1) / NUM_THREADS;
@@ -92,6 +98,7 @@ struct FwdParams {
   int B, S, Hq, Hkv, G;
   int n_q_tiles, n_pairs;  // VARLEN: of the longest sequence (max_seqlen); n_pairs = units
                            // along the queries (query-tile pairs, or query tiles with head_pairs)
+  int n_units;             // n_pairs * B * (head_pairs ? Hq / 2 : Hq)
   int head_pairs;          // 1: a CTA's two slots are two query heads of one kv group at the
                            // same query tile (Hq / Hkv even); 0: two query tiles of one head
   int causal;
@@ -138,9 +145,9 @@ struct FwdCfg {
   static constexpr int OFF_ONES = OFF_V + NV * V_BYTES;  // FP8: 128 keys x 128 B of 1.0
   static constexpr int OFF_P = OFF_ONES + (FP8 ? BOX_BYTES : 0);  // FP8: P_0, P_1
   static constexpr int OFF_BAR = OFF_P + (FP8 ? 2 * BOX_BYTES : 0);
-  // barriers: q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], and per tile:
-  //           s_full, p_full, pv_done, s_read, mma_done
-  static constexpr int NUM_BARS = 1 + 2 * NK + 2 * NV + 2 * 5;
+  // barriers: k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], and per slot:
+  //           q_full, q_empty, s_full, p_full, pv_done, s_read, mma_done
+  static constexpr int NUM_BARS = 2 * NK + 2 * NV + 2 * 7;
   static constexpr int OFF_TMEMPTR = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_TMEMPTR + 16;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;           // 1024-B alignment slack
@@ -193,6 +200,58 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
                      __int_as_float(__float_as_int(j.y) * (1 << 23) + __float_as_int(q.y)));
 }
 
+// One work unit: its sequence and the query tiles / heads of its two slots.
+struct Unit {
+  int b, h, g;        // batch, query head of slot 0 (slot 1: h + 1 with head pairs), kv head
+  int tok0, seq_len;  // first token and length of the sequence
+  int qt0, qt1;       // query tile of each slot
+  int n_t0, n_t1;     // key tiles of each slot (0: the slot has no query tile in this unit)
+};
+
+// Unit u (0 = the longest).  Returns 1, 0 if the unit has no query tile in its sequence
+// (packed sequences shorter than the longest), -1 if the sequence bounds are invalid.
+template <bool VARLEN>
+__device__ __forceinline__ int unit_info(const FwdParams& p, int u, Unit& U) {
+  const bool hp = p.head_pairs != 0;
+  const int heads_per_unit = hp ? p.Hq / 2 : p.Hq;
+  const int nbh = p.B * heads_per_unit;
+  const int pr = p.n_pairs - 1 - u / nbh;
+  const int bh = u % nbh;
+  U.b = bh / heads_per_unit;
+  U.h = hp ? 2 * (bh % heads_per_unit) : bh % heads_per_unit;
+  U.g = U.h / p.G;
+  U.tok0 = U.b * p.S;
+  U.seq_len = p.S;
+  int n_q_tiles = p.n_q_tiles;
+  if constexpr (VARLEN) {
+    if (p.cu_seqlens != nullptr) {
+      const int c0 = __ldg(p.cu_seqlens + U.b), c1 = __ldg(p.cu_seqlens + U.b + 1);
+      if (c0 < 0 || c1 < c0 || static_cast<int64_t>(c1) > p.total_tokens ||
+          c1 - c0 > p.max_seqlen)
+        return -1;
+      U.tok0 = c0;
+      U.seq_len = c1 - c0;
+    }
+    n_q_tiles = (U.seq_len + BLOCK_M - 1) / BLOCK_M;
+    if ((hp ? pr : 2 * pr) >= n_q_tiles) return 0;
+  }
+  U.qt0 = hp ? pr : 2 * pr;
+  U.qt1 = hp ? pr : 2 * pr + 1;
+  const bool has1 = U.qt1 < n_q_tiles;
+  U.n_t0 = p.causal ? U.qt0 + 1 : n_q_tiles;
+  U.n_t1 = has1 ? (p.causal ? U.qt1 + 1 : n_q_tiles) : 0;
+  return 1;
+}
+
+// The k-th unit of this CTA: round k holds units [k G, (k+1) G) (G = gridDim.x), taken in
+// CTA order in even rounds and in reverse CTA order in odd rounds, which evens out the
+// decreasing unit lengths.  Every role of the CTA walks the same list.
+__device__ __forceinline__ int cta_unit(int k) {
+  const int G = static_cast<int>(gridDim.x);
+  const int c = static_cast<int>(blockIdx.x);
+  return k * G + ((k & 1) ? G - 1 - c : c);
+}
+
 // EXACT (FP8 only): the exact-P ablation -- P = e4m3_rn(2^((a s - m)/8 + 7 + k_b)) by the
 // MUFU exponential and the hardware e4m3 conversion, instead of the lean-P multiply-add and
 // integer conversion; everything else (reference max, block shifts, block-scaled PV, row
@@ -205,64 +264,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using C = FwdCfg<FP8, DQK>;
+  using TM = TmemMap<FP8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* q_full = bars;
-  uint64_t* k_full = bars + 1;
+  uint64_t* k_full = bars;
   uint64_t* k_empty = k_full + C::NK;
   uint64_t* v_full = k_empty + C::NK;
   uint64_t* v_empty = v_full + C::NV;
-  uint64_t* tbar = v_empty + C::NV;  // per tile: 5 barriers
-  auto s_full = [&](int t) { return tbar + 5 * t + 0; };
-  auto p_full = [&](int t) { return tbar + 5 * t + 1; };
-  auto pv_done = [&](int t) { return tbar + 5 * t + 2; };
-  auto s_read = [&](int t) { return tbar + 5 * t + 3; };
-  auto mma_done = [&](int t) { return tbar + 5 * t + 4; };
+  uint64_t* tbar = v_empty + C::NV;  // per slot: 7 barriers
+  auto q_full = [&](int t) { return tbar + 7 * t + 0; };
+  auto q_empty = [&](int t) { return tbar + 7 * t + 1; };
+  auto s_full = [&](int t) { return tbar + 7 * t + 2; };
+  auto p_full = [&](int t) { return tbar + 7 * t + 3; };
+  auto pv_done = [&](int t) { return tbar + 7 * t + 4; };
+  auto s_read = [&](int t) { return tbar + 7 * t + 5; };
+  auto mma_done = [&](int t) { return tbar + 7 * t + 6; };
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEMPTR);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-
-  // longest-processing-time order: the units with the largest causal extent first.  A unit
-  // is two query tiles of one head, or (head_pairs) one query tile of two heads of one kv
-  // group, which then share every K/V tile with equal causal extents
   const bool hp = p.head_pairs != 0;
-  const int heads_per_unit = hp ? p.Hq / 2 : p.Hq;
-  const int nbh = p.B * heads_per_unit;
-  const int pr = p.n_pairs - 1 - static_cast<int>(blockIdx.x) / nbh;
-  const int bh = static_cast<int>(blockIdx.x) % nbh;
-  const int b = bh / heads_per_unit;
-  const int h = hp ? 2 * (bh % heads_per_unit) : bh % heads_per_unit;  // head of slot 0
-  const int g = h / p.G;
-  int tok0 = b * p.S;       // first token of this sequence
-  int seq_len = p.S;        // its length
-  int n_q_tiles = p.n_q_tiles;
-  if constexpr (VARLEN) {
-    if (p.cu_seqlens != nullptr) {
-      const int c0 = p.cu_seqlens[b], c1 = p.cu_seqlens[b + 1];
-      if (c0 < 0 || c1 < c0 || static_cast<int64_t>(c1) > p.total_tokens ||
-          c1 - c0 > p.max_seqlen) {
-        if (threadIdx.x == 0) atomicCAS(p.err, DEV_OK, DEV_BAD_SEQLENS);
-        return;  // the whole CTA, before any barrier or allocation
-      }
-      tok0 = c0;
-      seq_len = c1 - c0;
-    }
-    n_q_tiles = (seq_len + BLOCK_M - 1) / BLOCK_M;
-    if ((hp ? pr : 2 * pr) >= n_q_tiles) return;  // this sequence has fewer units
-  }
-  const int qt0 = hp ? pr : 2 * pr;                     // query tile of t = 0
-  const int qt1 = hp ? pr : 2 * pr + 1;                 // query tile of t = 1
-  const bool has1 = qt1 < n_q_tiles;                    // t = 1 exists
-  const int n_t0 = p.causal ? qt0 + 1 : n_q_tiles;      // key tiles of each query tile
-  const int n_t1 = has1 ? (p.causal ? qt1 + 1 : n_q_tiles) : 0;
-  const int n_max = n_t1 > n_t0 ? n_t1 : n_t0;
 
   if (tid == 0) {
-    mbar_init(q_full, 1);
     for (int i = 0; i < C::NK; ++i) {
       mbar_init(k_full + i, 1);
       mbar_init(k_empty + i, 1);
@@ -272,6 +298,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(v_empty + i, 1);
     }
     for (int t = 0; t < 2; ++t) {
+      mbar_init(q_full(t), 1);
+      mbar_init(q_empty(t), 1);
       mbar_init(s_full(t), 1);
       mbar_init(p_full(t), 128);
       mbar_init(pv_done(t), 1);
@@ -302,55 +330,83 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp >= 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_OTHER));
+    // Q is read once (evicted first); K and V are read by every CTA of the kv group and
+    // of later query tiles (kept in L2 longest)
     if (warp == 8) {
-      // ----------------------------------------------------------- TMA producer (warp-wide,
-      // one elected lane issues)
-      bool ok = true;
-      // Q is read once (evicted first); K and V are read by every CTA of the kv group and
-      // of later query tiles (kept in L2 longest)
-      const uint64_t pol_once = l2_policy_evict_first();
+      // ----------------------------------------------------------- K/V producer (warp-wide,
+      // one elected lane issues); gk / gv count the tiles issued by this CTA
       const uint64_t pol_keep = l2_policy_evict_last();
-      if (elect_one()) {
-        mbar_arrive_expect_tx(q_full, (has1 ? 2 : 1) * C::Q_BYTES);
-        for (int t = 0; t < (has1 ? 2 : 1); ++t)
-          for (int i = 0; i < C::Q_BOXES; ++i)
-            tma_load_3d_hint(smem + C::OFF_Q + t * C::Q_BYTES + i * C::BOX_BYTES, &tm_q, q_full,
-                             i * C::BOX_COLS, hp ? h + t : h, tok0 + (t ? qt1 : qt0) * BLOCK_M,
-                             pol_once);
-      }
-      __syncwarp();
-      int jk = 0, jv = 0;  // K and V tiles issued
-      for (int j = 0; j < n_max && ok; ++j) {
-        if (j == p.stall_tile) break;  // test-only: the waits on this tile must run out
-        const int sk = j % C::NK;
-        if (j >= C::NK) ok = mbar_wait(k_empty + sk, ((j / C::NK) - 1) & 1, p.err, p.timeout_ns);
-        if (!__all_sync(0xffffffffu, ok)) break;
-        if (elect_one()) {
-          mbar_arrive_expect_tx(k_full + sk, C::K_BYTES);
-          for (int i = 0; i < C::Q_BOXES; ++i)
-            tma_load_3d_hint(smem + C::OFF_K + sk * C::K_BYTES + i * C::BOX_BYTES, &tm_k,
-                             k_full + sk, i * C::BOX_COLS, g, tok0 + j * BLOCK_N, pol_keep);
+      bool ok = true;
+      int gk = 0, gv = 0;
+      for (int k = 0; ok; ++k) {
+        const int u = cta_unit(k);
+        if (u >= p.n_units) break;
+        Unit U;
+        if (unit_info<VARLEN>(p, u, U) <= 0) continue;
+        const int n_max = max(U.n_t0, U.n_t1);
+        for (int j = 0; j < n_max; ++j) {
+          if (j == p.stall_tile) {  // test-only: the waits on this tile must run out
+            ok = false;
+            break;
+          }
+          const int sk = gk % C::NK;
+          if (gk >= C::NK) ok = mbar_wait(k_empty + sk, ((gk / C::NK) - 1) & 1, p.err, p.timeout_ns);
+          if (!__all_sync(0xffffffffu, ok)) break;
+          if (elect_one()) {
+            mbar_arrive_expect_tx(k_full + sk, C::K_BYTES);
+            for (int i = 0; i < C::Q_BOXES; ++i)
+              tma_load_3d_hint(smem + C::OFF_K + sk * C::K_BYTES + i * C::BOX_BYTES, &tm_k,
+                               k_full + sk, i * C::BOX_COLS, U.g, U.tok0 + j * BLOCK_N, pol_keep);
+          }
+          __syncwarp();
+          ++gk;
+          const int sv = gv % C::NV;
+          if (gv >= C::NV) ok = mbar_wait(v_empty + sv, ((gv / C::NV) - 1) & 1, p.err, p.timeout_ns);
+          if (!__all_sync(0xffffffffu, ok)) break;
+          if (elect_one()) {
+            mbar_arrive_expect_tx(v_full + sv, C::V_BYTES);
+            for (int i = 0; i < C::V_BOXES; ++i)
+              tma_load_3d_hint(smem + C::OFF_V + sv * C::V_BYTES + i * C::BOX_BYTES, &tm_v,
+                               v_full + sv, i * C::BOX_COLS, U.g, U.tok0 + j * BLOCK_N, pol_keep);
+          }
+          __syncwarp();
+          ++gv;
         }
-        __syncwarp();
-        jk = j + 1;
-        const int sv = j % C::NV;
-        if (j >= C::NV) ok = mbar_wait(v_empty + sv, ((j / C::NV) - 1) & 1, p.err, p.timeout_ns);
-        if (!__all_sync(0xffffffffu, ok)) break;
-        if (elect_one()) {
-          mbar_arrive_expect_tx(v_full + sv, C::V_BYTES);
-          for (int i = 0; i < C::V_BOXES; ++i)
-            tma_load_3d_hint(smem + C::OFF_V + sv * C::V_BYTES + i * C::BOX_BYTES, &tm_v,
-                             v_full + sv, i * C::BOX_COLS, g, tok0 + j * BLOCK_N, pol_keep);
-        }
-        __syncwarp();
-        jv = j + 1;
       }
       // drain: no copy issued by this CTA may still be in flight at exit
-      mbar_wait(q_full, 0, p.err, DRAIN_TIMEOUT_NS, false);
-      for (int jj = (jk > C::NK ? jk - C::NK : 0); jj < jk; ++jj)
-        mbar_wait(k_full + jj % C::NK, (jj / C::NK) & 1, p.err, DRAIN_TIMEOUT_NS, false);
-      for (int jj = (jv > C::NV ? jv - C::NV : 0); jj < jv; ++jj)
-        mbar_wait(v_full + jj % C::NV, (jj / C::NV) & 1, p.err, DRAIN_TIMEOUT_NS, false);
+      for (int i = (gk > C::NK ? gk - C::NK : 0); i < gk; ++i)
+        mbar_wait(k_full + i % C::NK, (i / C::NK) & 1, p.err, DRAIN_TIMEOUT_NS, false);
+      for (int i = (gv > C::NV ? gv - C::NV : 0); i < gv; ++i)
+        mbar_wait(v_full + i % C::NV, (i / C::NV) & 1, p.err, DRAIN_TIMEOUT_NS, false);
+    } else if (warp == 11) {
+      // ----------------------------------------------------------- Q loader: slot t's tile
+      // of each unit once the slot's last S MMA of its previous unit has completed
+      const uint64_t pol_once = l2_policy_evict_first();
+      bool ok = true;
+      int nq[2] = {0, 0};  // Q tiles loaded per slot
+      for (int k = 0; ok; ++k) {
+        const int u = cta_unit(k);
+        if (u >= p.n_units) break;
+        Unit U;
+        if (unit_info<VARLEN>(p, u, U) <= 0) continue;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if ((t ? U.n_t1 : U.n_t0) == 0) continue;
+          if (nq[t] > 0) ok = mbar_wait(q_empty(t), (nq[t] - 1) & 1, p.err, p.timeout_ns);
+          if (!__all_sync(0xffffffffu, ok)) break;
+          if (elect_one()) {
+            mbar_arrive_expect_tx(q_full(t), C::Q_BYTES);
+            for (int i = 0; i < C::Q_BOXES; ++i)
+              tma_load_3d_hint(smem + C::OFF_Q + t * C::Q_BYTES + i * C::BOX_BYTES, &tm_q,
+                               q_full(t), i * C::BOX_COLS, hp ? U.h + t : U.h,
+                               U.tok0 + (t ? U.qt1 : U.qt0) * BLOCK_M, pol_once);
+          }
+          __syncwarp();
+          ++nq[t];
+        }
+      }
+      for (int t = 0; t < 2; ++t)
+        if (nq[t] > 0) mbar_wait(q_full(t), (nq[t] - 1) & 1, p.err, DRAIN_TIMEOUT_NS, false);
     } else if (warp == 9 || (FP8 && warp == 10)) {
       // ----------------------------------------------------------- MMA issuers (warp-wide
       // control flow, one elected lane issues); the order per key tile is in the header.
@@ -358,8 +414,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // columns and P is in shared memory, so only mbarriers order them), so that one
       // warp's waits and control flow overlap the other warp's issue.  BF16: warp 9 issues
       // both (P_t aliases S_t, so S_t(j+1) must follow PV_t(j) in one issue stream).
-      using TM = TmemMap<FP8>;
-      auto nt = [&](int t) { return t == 0 ? n_t0 : n_t1; };
       // Descriptors are built once; advancing an operand by `off` bytes adds off >> 4 to
       // the start-address field (shared-memory addresses stay below 2^18, so the 14-bit
       // field never carries into its neighbours).
@@ -375,25 +429,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           return smem_desc_sw128(va, C::BOX_BYTES, 1024);  // two 64-column atoms of V
         }
       };
-      auto issue_s = [&](int t, int j) {
-        const int sk = j % C::NK;
+      // S_t(j) of a unit whose key tiles start at ring position g0; commits s_full, q_empty
+      // after the slot's last S of the unit, and k_empty after the tile's last S (slot 1's,
+      // or slot 0's where slot 1 does not use the tile)
+      auto issue_s = [&](int t, int j, int g0, const Unit& U) {
+        const int sk = (g0 + j) % C::NK;
         const uint64_t qd = dq0 + static_cast<uint32_t>((t * C::Q_BYTES) >> 4);
         const uint64_t kd = dk0 + static_cast<uint32_t>((sk * C::K_BYTES) >> 4);
         const uint32_t tm_s = tmem + TM::S(t);
         if (elect_one()) {
-#pragma unroll
+          // unrolled per 128-byte box: fully unrolled, d_qk = 192 runs out of the issuing
+          // warps' registers
+#pragma unroll 4
           for (int s = 0; s < C::QK_STEPS; ++s) {
             const uint32_t off = ((s / 4) * C::BOX_BYTES + (s % 4) * 32) >> 4;
             mma_ss<FP8 ? 1 : 0>(tm_s, qd + off, kd + off, C::IDESC_S, s > 0 ? 1u : 0u);
           }
           tc_commit(s_full(t));
-          // K(j) is free once its last S has run: tile 1's, or tile 0's if tile 1 skips j
-          if (t == 1 || j >= n_t1) tc_commit(k_empty + sk);
+          if (j == (t ? U.n_t1 : U.n_t0) - 1) tc_commit(q_empty(t));
+          if (t == 1 || j >= U.n_t1) tc_commit(k_empty + sk);
         }
         __syncwarp();
       };
-      auto issue_pv = [&](int t, int j) {
-        const int sv = j % C::NV;
+      auto issue_pv = [&](int t, int j, int g0, const Unit& U) {
+        const int sv = (g0 + j) % C::NV;
         const uint64_t vd = v_desc(sv);
         const uint32_t tm_o = tmem + TM::O(t);
         if (elect_one()) {
@@ -419,75 +478,105 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           }
           tc_commit(pv_done(t));
-          if (t == 1 || j >= n_t1) tc_commit(v_empty + sv);
+          if (t == 1 || j >= U.n_t1) tc_commit(v_empty + sv);
         }
         __syncwarp();
       };
-      // FP8: S_0 and S_1 share 64 TMEM columns; before writing S_t, the other tile's
-      // softmax group must have read its latest S (the index of that S is passed)
-      auto wait_other_read = [&](int t, int jo) -> bool {
-        if constexpr (!FP8) return true;
-        if (jo < 0) return true;
-        return mbar_wait(s_read(1 - t), jo & 1, p.err, p.timeout_ns);
-      };
       const bool s_issuer = warp == 9;  // FP8: S MMAs; BF16: all MMAs
       bool ok = true;
-      if (s_issuer) {
-        ok = mbar_wait(q_full, 0, p.err, p.timeout_ns);
-        if (__all_sync(0xffffffffu, ok)) {
-          ok = mbar_wait(k_full, 0, p.err, p.timeout_ns);
-          if (__all_sync(0xffffffffu, ok)) {
-            tc_fence_after();
-            if (n_t0 > 0) issue_s(0, 0);
-            if (n_t1 > 0) {
-              ok = wait_other_read(1, n_t0 > 0 ? 0 : -1);
-              if (__all_sync(0xffffffffu, ok)) {
-                tc_fence_after();
-                issue_s(1, 0);
-              }
-            }
-          }
-        }
-      }
-      for (int j = 0; j < n_max && __all_sync(0xffffffffu, ok); ++j) {
+      int cs[2] = {0, 0};  // S MMAs issued per slot
+      int cp[2] = {0, 0};  // PV MMAs issued per slot
+      int nq[2] = {0, 0};  // units begun per slot (Q tiles consumed)
+      int g0 = 0;          // ring position of the current unit's key tile 0
+      // the Q tile of slot t for its current unit has landed
+      auto wait_q = [&](int t) { return mbar_wait(q_full(t), nq[t] & 1, p.err, p.timeout_ns); };
+      auto wait_k = [&](int g) {
+        return mbar_wait(k_full + g % C::NK, (g / C::NK) & 1, p.err, p.timeout_ns);
+      };
+      // FP8: before writing S_t, both slots must have read every S issued to them (S_0 and
+      // S_1 share 64 TMEM columns)
+      auto wait_reads = [&]() {
+        bool r = true;
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          if (j >= nt(t)) continue;
-          const bool next = j + 1 < nt(t);
-          if constexpr (FP8) {
-            if (s_issuer) {
-              // S_t(j+1) once S_t(j) and the other tile's latest S (S_1(j) or S_0(j+1))
-              // have been read into registers and K(j+1) has landed
-              if (next) {
-                const int jo = t == 0 ? min(j, n_t1 - 1) : min(j + 1, n_t0 - 1);
-                ok = mbar_wait(s_read(t), j & 1, p.err, p.timeout_ns);
-                if (ok) ok = wait_other_read(t, jo);
-                if (ok) ok = mbar_wait(k_full + (j + 1) % C::NK, ((j + 1) / C::NK) & 1, p.err, p.timeout_ns);
+        for (int x = 0; x < 2; ++x)
+          if (r && cs[x] > 0) r = mbar_wait(s_read(x), (cs[x] - 1) & 1, p.err, p.timeout_ns);
+        return r;
+      };
+      for (int k = 0; ok; ++k) {
+        const int u = cta_unit(k);
+        if (u >= p.n_units) break;
+        Unit U;
+        if (unit_info<VARLEN>(p, u, U) <= 0) continue;
+        const int n_max = max(U.n_t0, U.n_t1);
+        auto nt = [&](int t) { return t == 0 ? U.n_t0 : U.n_t1; };
+        if constexpr (FP8) {
+          if (s_issuer) {
+            // S_t(j) in the order S_0(0), S_1(0), S_0(1), S_1(1), ...
+            for (int j = 0; j < n_max && ok; ++j) {
+#pragma unroll
+              for (int t = 0; t < 2; ++t) {
+                if (j >= nt(t)) continue;
+                ok = wait_reads();
+                if (ok && j == 0) ok = wait_q(t);
+                if (ok) ok = wait_k(g0 + j);
                 if (!__all_sync(0xffffffffu, ok)) break;
                 tc_fence_after();
-                issue_s(t, j + 1);
+                issue_s(t, j, g0, U);
+                ++cs[t];
               }
-            } else {
-              // PV_t(j) once P_t(j) is in shared memory and V(j) has landed
-              ok = mbar_wait(p_full(t), j & 1, p.err, p.timeout_ns);
-              if (ok) ok = mbar_wait(v_full + j % C::NV, (j / C::NV) & 1, p.err, p.timeout_ns);
-              if (!__all_sync(0xffffffffu, ok)) break;
-              tc_fence_after();
-              issue_pv(t, j);
             }
           } else {
-            if (next) {
-              // prerequisites of S_t(j+1), normally met long before P_t(j) is ready
-              ok = mbar_wait(k_full + (j + 1) % C::NK, ((j + 1) / C::NK) & 1, p.err, p.timeout_ns);
+            // PV_t(j) once P_t(j) is in shared memory and V(j) has landed
+            for (int j = 0; j < n_max && ok; ++j) {
+#pragma unroll
+              for (int t = 0; t < 2; ++t) {
+                if (j >= nt(t)) continue;
+                ok = mbar_wait(p_full(t), cp[t] & 1, p.err, p.timeout_ns);
+                if (ok) ok = mbar_wait(v_full + (g0 + j) % C::NV, ((g0 + j) / C::NV) & 1, p.err, p.timeout_ns);
+                if (!__all_sync(0xffffffffu, ok)) break;
+                tc_fence_after();
+                issue_pv(t, j, g0, U);
+                ++cp[t];
+              }
             }
-            if (ok) ok = mbar_wait(p_full(t), j & 1, p.err, p.timeout_ns);
-            if (ok) ok = mbar_wait(v_full + j % C::NV, (j / C::NV) & 1, p.err, p.timeout_ns);
+          }
+        } else {
+          // S_0(0), S_1(0); then per key tile j and slot t: PV_t(j), S_t(j+1).  S_t(0) of a
+          // unit follows the slot's last PV of the previous unit in this issue stream, so it
+          // overwrites P_t only after that PV has read it.
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            if (!ok || nt(t) == 0) continue;
+            ok = wait_q(t);
+            if (ok) ok = wait_k(g0);
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
-            issue_pv(t, j);
-            if (next) issue_s(t, j + 1);
+            issue_s(t, 0, g0, U);
+            ++cs[t];
+          }
+          for (int j = 0; j < n_max && ok; ++j) {
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              if (j >= nt(t)) continue;
+              const bool next = j + 1 < nt(t);
+              // prerequisites of S_t(j+1), normally met long before P_t(j) is ready
+              if (next) ok = wait_k(g0 + j + 1);
+              if (ok) ok = mbar_wait(p_full(t), cp[t] & 1, p.err, p.timeout_ns);
+              if (ok) ok = mbar_wait(v_full + (g0 + j) % C::NV, ((g0 + j) / C::NV) & 1, p.err, p.timeout_ns);
+              if (!__all_sync(0xffffffffu, ok)) break;
+              tc_fence_after();
+              issue_pv(t, j, g0, U);
+              ++cp[t];
+              if (next) {
+                issue_s(t, j + 1, g0, U);
+                ++cs[t];
+              }
+            }
           }
         }
+#pragma unroll
+        for (int t = 0; t < 2; ++t) nq[t] += nt(t) > 0 ? 1 : 0;
+        g0 += n_max;
       }
       // every MMA issued by this warp completes before TMEM is released
       const int mine = s_issuer ? 0 : 1;
@@ -497,15 +586,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_SOFTMAX));
-    // ------------------------------------------------------------- softmax of tile t
+    // ------------------------------------------------------------- softmax of slot t
     const int t = warp >> 2;
-    const int n_t = t == 0 ? n_t0 : n_t1;
-    const int qt = t ? qt1 : qt0;
-    const int hs = hp ? h + t : h;                // this slot's query head
     const int r = tid & 127;                      // row within the tile == TMEM lane
-    const int q_pos = qt * BLOCK_M + r;           // query position in the sequence
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    using TM = TmemMap<FP8>;
     const uint32_t ts = lane_base + TM::S(t);     // S_t columns of this lane
     const uint32_t tp = lane_base + TM::P(t);     // BF16: P_t columns
     const uint32_t to = lane_base + TM::O(t);     // O_t (FP8: and the row sum) columns
@@ -514,209 +598,222 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       a = static_cast<float>(p.leanp_c * static_cast<double>(*p.descale_q) *
                              static_cast<double>(*p.descale_k));
       a256 = a * 0.00390625f;
-    }
-    float ms = -INFINITY;  // BF16 reference max, scaled to log2 units
-    int m_i = 0;           // FP8 reference max, code units
-    float l = 0.0f;        // running row sum
-    if constexpr (FP8) {
       // scale factors of the B operand [V | 1]: 2^0, for every PV of this CTA
       const uint32_t sfb = lane_base + TM::SFB;
       tmem_st4(sfb, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
       tmem_st4(sfb + 4, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
     }
     bool ok = true;
-    for (int j = 0; j < n_t; ++j) {
-      ok = mbar_wait(s_full(t), j & 1, p.err, p.timeout_ns);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tc_fence_after();
-      uint32_t sraw[BLOCK_N];
+    int c = 0;  // key tiles of this slot processed so far (all units)
+    for (int k = 0; ok; ++k) {
+      const int u = cta_unit(k);
+      if (u >= p.n_units) break;
+      Unit U;
+      const int st = unit_info<VARLEN>(p, u, U);
+      if (st < 0 && tid == 0) atomicCAS(p.err, DEV_OK, DEV_BAD_SEQLENS);
+      if (st <= 0) continue;
+      const int n_t = t == 0 ? U.n_t0 : U.n_t1;
+      if (n_t == 0) continue;
+      const int qt = t ? U.qt1 : U.qt0;
+      const int hs = hp ? U.h + t : U.h;            // this slot's query head
+      const int q_pos = qt * BLOCK_M + r;           // query position in the sequence
+      float ms = -INFINITY;  // BF16 reference max, scaled to log2 units
+      int m_i = 0;           // FP8 reference max, code units
+      float l = 0.0f;        // running row sum
+      for (int j = 0; j < n_t; ++j, ++c) {
+        ok = mbar_wait(s_full(t), c & 1, p.err, p.timeout_ns);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        tc_fence_after();
+        uint32_t sraw[BLOCK_N];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(ts + c * 32, sraw + c * 32);
-      tmem_wait_ld();
-      if constexpr (FP8) {
-        // S_t is in registers: the other tile may now overwrite the shared columns
-        tc_fence_before();
-        mbar_arrive(s_read(t));
-      }
-      float s[BLOCK_N];
-#pragma unroll
-      for (int c = 0; c < BLOCK_N; ++c) s[c] = __uint_as_float(sraw[c]);
-      const bool diag = p.causal && j == qt;
-      if (diag) {
-#pragma unroll
-        for (int c = 0; c < BLOCK_N; ++c)
-          if (c > r) s[c] = -INFINITY;
-      }
-      if constexpr (VARLEN) {
-        // keys past the end of the sequence (the next sequence's, or zero fill)
-        const int kvalid = seq_len - j * BLOCK_N;
-        if (kvalid < BLOCK_N) {
-#pragma unroll
-          for (int c = 0; c < BLOCK_N; ++c)
-            if (c >= kvalid) s[c] = -INFINITY;
+        for (int cc = 0; cc < 4; ++cc) tmem_ld32(ts + cc * 32, sraw + cc * 32);
+        tmem_wait_ld();
+        if constexpr (FP8) {
+          // S_t is in registers: the other slot may now overwrite the shared columns
+          tc_fence_before();
+          mbar_arrive(s_read(t));
         }
-      }
-      // block maxima with two independent chains per 64-key block
-      float mx[4];
+        float s[BLOCK_N];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) mx[i] = s[i * 32];
-#pragma unroll
-      for (int c = 1; c < 31; c += 2) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) mx[i] = fmax3(mx[i], s[i * 32 + c], s[i * 32 + c + 1]);
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) mx[i] = fmaxf(mx[i], s[i * 32 + 31]);
-      const float mu0 = fmaxf(mx[0], mx[1]);
-      const float mu1 = fmaxf(mx[2], mx[3]);
-
-      uint32_t pw[FP8 ? 32 : 64];
-      float alpha = 1.0f;
-      uint32_t sf_w = 0;
-      if constexpr (!FP8) {
-        const float cand = fmaxf(mu0, mu1) * p.c1;
-        const float ms_new = (j == 0 || cand > ms + BF16_HEADROOM) ? cand : ms;
-        if (j > 0) alpha = ex2_approx(ms - ms_new);
-        ms = ms_new;
-        // element pairs in packed two-wide fp32 (the even and odd sums are the two lanes)
-        const float2 c1x2 = make_float2(p.c1, p.c1);
-        const float2 nms2 = make_float2(-ms, -ms);
-        float2 lsum = make_float2(0.0f, 0.0f);
+        for (int cc = 0; cc < BLOCK_N; ++cc) s[cc] = __uint_as_float(sraw[cc]);
+        const bool diag = p.causal && j == qt;
         if (diag) {
 #pragma unroll
-          for (int c = 0; c < BLOCK_N; c += 2) {
-            const float2 x = __ffma2_rn(make_float2(s[c], s[c + 1]), c1x2, nms2);
-            const float2 pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-            lsum = __fadd2_rn(lsum, pp);
-            pw[c >> 1] = pack_bf16x2(pp.x, pp.y);
+          for (int cc = 0; cc < BLOCK_N; ++cc)
+            if (cc > r) s[cc] = -INFINITY;
+        }
+        if constexpr (VARLEN) {
+          // keys past the end of the sequence (the next sequence's, or zero fill)
+          const int kvalid = U.seq_len - j * BLOCK_N;
+          if (kvalid < BLOCK_N) {
+#pragma unroll
+            for (int cc = 0; cc < BLOCK_N; ++cc)
+              if (cc >= kvalid) s[cc] = -INFINITY;
           }
+        }
+        // block maxima with two independent chains per 64-key block
+        float mx[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) mx[i] = s[i * 32];
+#pragma unroll
+        for (int cc = 1; cc < 31; cc += 2) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) mx[i] = fmax3(mx[i], s[i * 32 + cc], s[i * 32 + cc + 1]);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) mx[i] = fmaxf(mx[i], s[i * 32 + 31]);
+        const float mu0 = fmaxf(mx[0], mx[1]);
+        const float mu1 = fmaxf(mx[2], mx[3]);
+
+        uint32_t pw[FP8 ? 32 : 64];
+        float alpha = 1.0f;
+        uint32_t sf_w = 0;
+        if constexpr (!FP8) {
+          const float cand = fmaxf(mu0, mu1) * p.c1;
+          const float ms_new = (j == 0 || cand > ms + BF16_HEADROOM) ? cand : ms;
+          if (j > 0) alpha = ex2_approx(ms - ms_new);
+          ms = ms_new;
+          // element pairs in packed two-wide fp32 (the even and odd sums are the two lanes)
+          const float2 c1x2 = make_float2(p.c1, p.c1);
+          const float2 nms2 = make_float2(-ms, -ms);
+          float2 lsum = make_float2(0.0f, 0.0f);
+          if (diag) {
+#pragma unroll
+            for (int cc = 0; cc < BLOCK_N; cc += 2) {
+              const float2 x = __ffma2_rn(make_float2(s[cc], s[cc + 1]), c1x2, nms2);
+              const float2 pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+              lsum = __fadd2_rn(lsum, pp);
+              pw[cc >> 1] = pack_bf16x2(pp.x, pp.y);
+            }
+          } else {
+#pragma unroll
+            for (int cc = 0; cc < BLOCK_N; cc += 2) {
+              const float2 x = __ffma2_rn(make_float2(s[cc], s[cc + 1]), c1x2, nms2);
+              // one element pair in four on the FMA pipe, the rest on the MUFU
+              const bool poly = (cc & 7) == 6;
+              const float2 pp = poly ? exp2_poly2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+              lsum = __fadd2_rn(lsum, pp);
+              pw[cc >> 1] = pack_bf16x2(pp.x, pp.y);
+            }
+          }
+          l = l * alpha + (lsum.x + lsum.y);
         } else {
+          const float mu = fmaxf(mu0, mu1);
+          const int cand = __float2int_ru(__fmul_rn(a, mu));
+          const int m_new = (j == 0 || cand > m_i + LEANP_HEADROOM) ? cand : m_i;
+          if (j > 0) alpha = ex2_approx(static_cast<float>(m_i - m_new) * 0.125f);
+          m_i = m_new;
+          const int k0 = leanp_kshift(mu0, a, m_new);
+          const int k1 = leanp_kshift(mu1, a, m_new);
+          if constexpr (EXACT) {
+            // x = fmaf(s, a/8, (8 (7 + k_b) - m)/8); P code = e4m3_rn(2^x)
+            const float a8 = a * 0.125f;
+            const float cx0 = __int2float_rn(8 * (7 + k0) - m_new) * 0.125f;
+            const float cx1 = __int2float_rn(8 * (7 + k1) - m_new) * 0.125f;
 #pragma unroll
-          for (int c = 0; c < BLOCK_N; c += 2) {
-            const float2 x = __ffma2_rn(make_float2(s[c], s[c + 1]), c1x2, nms2);
-            // one element pair in four on the FMA pipe, the rest on the MUFU
-            const bool poly = (c & 7) == 6;
-            const float2 pp = poly ? exp2_poly2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
-            lsum = __fadd2_rn(lsum, pp);
-            pw[c >> 1] = pack_bf16x2(pp.x, pp.y);
+            for (int cc = 0; cc < BLOCK_N; cc += 4) {
+              const float cx = cc < 64 ? cx0 : cx1;
+              const float p0 = ex2_approx(__fmaf_rn(s[cc + 0], a8, cx));
+              const float p1 = ex2_approx(__fmaf_rn(s[cc + 1], a8, cx));
+              const float p2 = ex2_approx(__fmaf_rn(s[cc + 2], a8, cx));
+              const float p3 = ex2_approx(__fmaf_rn(s[cc + 3], a8, cx));
+              pw[cc >> 2] = f32_to_e4m3x2(p0, p1) | (f32_to_e4m3x2(p2, p3) << 16);
+            }
+          } else {
+            const float cb0 = __int2float_rn(LEANP_TOP + 8 * k0 - m_new) * 0.00390625f;
+            const float cb1 = __int2float_rn(LEANP_TOP + 8 * k1 - m_new) * 0.00390625f;
+            const float2 s256 = make_float2(256.0f, 256.0f);
+            const float2 magic = make_float2(LEANP_MAGIC, LEANP_MAGIC);
+#pragma unroll
+            for (int cc = 0; cc < BLOCK_N; cc += 4) {
+              const float cb = cc < 64 ? cb0 : cb1;
+              // multiply-add (saturating to [0,1]), then the integer conversion by a magic
+              // fma, two lanes at a time
+              const float2 u01 = make_float2(fma_sat(s[cc + 0], a256, cb), fma_sat(s[cc + 1], a256, cb));
+              const float2 u23 = make_float2(fma_sat(s[cc + 2], a256, cb), fma_sat(s[cc + 3], a256, cb));
+              const float2 r01 = __ffma2_rn(u01, s256, magic);
+              const float2 r23 = __ffma2_rn(u23, s256, magic);
+              pw[cc >> 2] = pack_low_bytes(__float_as_uint(r01.x), __float_as_uint(r01.y),
+                                           __float_as_uint(r23.x), __float_as_uint(r23.y));
+            }
           }
-        }
-        l = l * alpha + (lsum.x + lsum.y);
-      } else {
-        const float mu = fmaxf(mu0, mu1);
-        const int cand = __float2int_ru(__fmul_rn(a, mu));
-        const int m_new = (j == 0 || cand > m_i + LEANP_HEADROOM) ? cand : m_i;
-        if (j > 0) alpha = ex2_approx(static_cast<float>(m_i - m_new) * 0.125f);
-        m_i = m_new;
-        const int k0 = leanp_kshift(mu0, a, m_new);
-        const int k1 = leanp_kshift(mu1, a, m_new);
-        if constexpr (EXACT) {
-          // x = fmaf(s, a/8, (8 (7 + k_b) - m)/8); P code = e4m3_rn(2^x)
-          const float a8 = a * 0.125f;
-          const float cx0 = __int2float_rn(8 * (7 + k0) - m_new) * 0.125f;
-          const float cx1 = __int2float_rn(8 * (7 + k1) - m_new) * 0.125f;
-#pragma unroll
-          for (int c = 0; c < BLOCK_N; c += 4) {
-            const float cx = c < 64 ? cx0 : cx1;
-            const float p0 = ex2_approx(__fmaf_rn(s[c + 0], a8, cx));
-            const float p1 = ex2_approx(__fmaf_rn(s[c + 1], a8, cx));
-            const float p2 = ex2_approx(__fmaf_rn(s[c + 2], a8, cx));
-            const float p3 = ex2_approx(__fmaf_rn(s[c + 3], a8, cx));
-            pw[c >> 2] = f32_to_e4m3x2(p0, p1) | (f32_to_e4m3x2(p2, p3) << 16);
+          const uint32_t e0 = static_cast<uint32_t>(120 - k0), e1 = static_cast<uint32_t>(120 - k1);
+          const uint32_t sf_word = e0 | (e0 << 8) | (e1 << 16) | (e1 << 24);  // UE8M0 2^-(7+k)
+          if constexpr (DUMP) {
+            const size_t row = (static_cast<size_t>(U.b) * p.Hq + hs) * p.S + q_pos;
+            float* ds = p.dump_s + row * p.S + static_cast<size_t>(j) * BLOCK_N;
+            uint8_t* dc = p.dump_codes + row * p.S + static_cast<size_t>(j) * BLOCK_N;
+            for (int cc = 0; cc < BLOCK_N; ++cc) ds[cc] = s[cc];
+            for (int cc = 0; cc < BLOCK_N / 4; ++cc) reinterpret_cast<uint32_t*>(dc)[cc] = pw[cc];
+            uint8_t* dk = p.dump_kshift + row * (p.S / 64) + j * 2;
+            dk[0] = static_cast<uint8_t>(k0);
+            dk[1] = static_cast<uint8_t>(k1);
           }
-        } else {
-          const float cb0 = __int2float_rn(LEANP_TOP + 8 * k0 - m_new) * 0.00390625f;
-          const float cb1 = __int2float_rn(LEANP_TOP + 8 * k1 - m_new) * 0.00390625f;
-          const float2 s256 = make_float2(256.0f, 256.0f);
-          const float2 magic = make_float2(LEANP_MAGIC, LEANP_MAGIC);
-#pragma unroll
-          for (int c = 0; c < BLOCK_N; c += 4) {
-            const float cb = c < 64 ? cb0 : cb1;
-            // multiply-add (saturating to [0,1]), then the integer conversion by a magic fma,
-            // two lanes at a time
-            const float2 u01 = make_float2(fma_sat(s[c + 0], a256, cb), fma_sat(s[c + 1], a256, cb));
-            const float2 u23 = make_float2(fma_sat(s[c + 2], a256, cb), fma_sat(s[c + 3], a256, cb));
-            const float2 r01 = __ffma2_rn(u01, s256, magic);
-            const float2 r23 = __ffma2_rn(u23, s256, magic);
-            pw[c >> 2] = pack_low_bytes(__float_as_uint(r01.x), __float_as_uint(r01.y),
-                                        __float_as_uint(r23.x), __float_as_uint(r23.y));
-          }
-        }
-        const uint32_t e0 = static_cast<uint32_t>(120 - k0), e1 = static_cast<uint32_t>(120 - k1);
-        const uint32_t sf_word = e0 | (e0 << 8) | (e1 << 16) | (e1 << 24);  // UE8M0 2^-(7+k)
-        if constexpr (DUMP) {
-          const size_t row = (static_cast<size_t>(b) * p.Hq + hs) * p.S + q_pos;
-          float* ds = p.dump_s + row * p.S + static_cast<size_t>(j) * BLOCK_N;
-          uint8_t* dc = p.dump_codes + row * p.S + static_cast<size_t>(j) * BLOCK_N;
-          for (int c = 0; c < BLOCK_N; ++c) ds[c] = s[c];
-          for (int c = 0; c < BLOCK_N / 4; ++c) reinterpret_cast<uint32_t*>(dc)[c] = pw[c];
-          uint8_t* dk = p.dump_kshift + row * (p.S / 64) + j * 2;
-          dk[0] = static_cast<uint8_t>(k0);
-          dk[1] = static_cast<uint8_t>(k1);
-        }
-        sf_w = sf_word;
-      }
-      if constexpr (FP8) {
-        // S_t(j) may have been issued before PV_t(j-1): that PV must be complete before
-        // O_t is rescaled and before P_t and its scale factors are overwritten
-        if (j > 0) {
-          ok = mbar_wait(pv_done(t), (j - 1) & 1, p.err, p.timeout_ns);
-          if (!__all_sync(0xffffffffu, ok)) break;
-          tc_fence_after();
-        }
-      }
-      // BF16: the previous PV of this tile is complete here (S_t(j) was issued after it
-      // and has completed).  O_t (and the FP8 row sum) may be rescaled.
-      if (__any_sync(0xffffffffu, alpha != 1.0f)) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t o[32];
-          tmem_ld32(to + c * 32, o);
-          tmem_wait_ld();
-          const float2 a2 = make_float2(alpha, alpha);
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            const float2 r = __fmul2_rn(make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), a2);
-            o[i] = __float_as_uint(r.x);
-            o[i + 1] = __float_as_uint(r.y);
-          }
-          tmem_st32(to + c * 32, o);
+          sf_w = sf_word;
         }
         if constexpr (FP8) {
-          uint32_t rs;
-          tmem_ld1(to + TM::RS, rs);
-          tmem_wait_ld();
-          tmem_st1(to + TM::RS, __float_as_uint(__uint_as_float(rs) * alpha));
+          // S_t(j) may have been issued before PV_t(j-1): that PV must be complete before
+          // O_t is rescaled and before P_t and its scale factors are overwritten (the
+          // previous unit's last PV was waited for by its epilogue)
+          if (j > 0) {
+            ok = mbar_wait(pv_done(t), (c - 1) & 1, p.err, p.timeout_ns);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+          }
         }
-      }
-      if constexpr (!FP8) {
-        tmem_st32(tp, pw);
-        tmem_st32(tp + 32, pw + 32);
-      } else {
-        // row r of P_t: 128 codes = 8 chunks of 16 B; chunk c sits at chunk position
-        // c ^ (r mod 8) of the row (128-byte swizzle, rows 128 B apart)
-        const uint32_t prow = smem_addr(smem + C::OFF_P + t * C::BOX_BYTES) + r * 128;
+        // BF16: the previous PV of this slot is complete here (S_t(j) was issued after it
+        // and has completed).  O_t (and the FP8 row sum) may be rescaled.
+        if (__any_sync(0xffffffffu, alpha != 1.0f)) {
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          st_shared_v4(prow + ((c ^ (r & 7)) << 4), pw[4 * c], pw[4 * c + 1], pw[4 * c + 2],
-                       pw[4 * c + 3]);
-        fence_proxy_async_smem();
-        // scale factors of P: row R's word (byte k = 32-key block k of the tile) at lane R,
-        // column SFA + R/32 -- the quadrant of the MMA datapath that computes row R
-        tmem_st1(lane_base + TM::SFA(t) + (warp & 3), sf_w);
+          for (int cc = 0; cc < 4; ++cc) {
+            uint32_t o[32];
+            tmem_ld32(to + cc * 32, o);
+            tmem_wait_ld();
+            const float2 a2 = make_float2(alpha, alpha);
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+              const float2 rr = __fmul2_rn(make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), a2);
+              o[i] = __float_as_uint(rr.x);
+              o[i + 1] = __float_as_uint(rr.y);
+            }
+            tmem_st32(to + cc * 32, o);
+          }
+          if constexpr (FP8) {
+            uint32_t rs;
+            tmem_ld1(to + TM::RS, rs);
+            tmem_wait_ld();
+            tmem_st1(to + TM::RS, __float_as_uint(__uint_as_float(rs) * alpha));
+          }
+        }
+        if constexpr (!FP8) {
+          tmem_st32(tp, pw);
+          tmem_st32(tp + 32, pw + 32);
+        } else {
+          // row r of P_t: 128 codes = 8 chunks of 16 B; chunk cc sits at chunk position
+          // cc ^ (r mod 8) of the row (128-byte swizzle, rows 128 B apart)
+          const uint32_t prow = smem_addr(smem + C::OFF_P + t * C::BOX_BYTES) + r * 128;
+#pragma unroll
+          for (int cc = 0; cc < 8; ++cc)
+            st_shared_v4(prow + ((cc ^ (r & 7)) << 4), pw[4 * cc], pw[4 * cc + 1], pw[4 * cc + 2],
+                         pw[4 * cc + 3]);
+          fence_proxy_async_smem();
+          // scale factors of P: row R's word (byte k = 32-key block k of the tile) at lane R,
+          // column SFA + R/32 -- the quadrant of the MMA datapath that computes row R
+          tmem_st1(lane_base + TM::SFA(t) + (warp & 3), sf_w);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(p_full(t));
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(p_full(t));
-    }
-    tmem_wait_st();  // nothing of this thread may still be writing TMEM on any exit path
-    // ------------------------------------------------------------- epilogue
-    if (ok && n_t > 0) ok = mbar_wait(pv_done(t), (n_t - 1) & 1, p.err, p.timeout_ns);
-    if (ok && n_t > 0) {
+      tmem_wait_st();  // nothing of this thread may still be writing TMEM on any exit path
+      if (!ok) break;
+      // ----------------------------------------------------------- epilogue of the unit
+      ok = mbar_wait(pv_done(t), (c - 1) & 1, p.err, p.timeout_ns);
+      if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       uint32_t oraw[DV];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(to + c * 32, oraw + c * 32);
+      for (int cc = 0; cc < 4; ++cc) tmem_ld32(to + cc * 32, oraw + cc * 32);
       if constexpr (FP8) {
         uint32_t rs;
         tmem_ld1(to + TM::RS, rs);
@@ -724,9 +821,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         l = __uint_as_float(rs);  // sum of the rounded probabilities, 2^-(7+k) scaled
       }
       tmem_wait_ld();
+      // O_t is in registers: the next unit's first PV may overwrite it once this slot
+      // signals P_t(0) of that unit (after its own fence and arrive)
       float o[DV];
 #pragma unroll
-      for (int c = 0; c < DV; ++c) o[c] = __uint_as_float(oraw[c]);
+      for (int cc = 0; cc < DV; ++cc) o[cc] = __uint_as_float(oraw[cc]);
       float inv = 1.0f / l;
       if constexpr (FP8) inv *= *p.descale_v;
       if (p.unrotate) {
@@ -736,9 +835,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int i = 0; i < DV; ++i) {
             if ((i & hh) == 0) {
-              const float u = o[i], w = o[i + hh];
-              o[i] = u + w;
-              o[i + hh] = u - w;
+              const float x0 = o[i], x1 = o[i + hh];
+              o[i] = x0 + x1;
+              o[i + hh] = x0 - x1;
             }
           }
         }
@@ -746,22 +845,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       // VARLEN: rows past the end of the sequence hold another sequence's queries (or zero
       // fill) and are not written
-      const bool row_in = !VARLEN || q_pos < seq_len;
-      __nv_bfloat16* orow = p.o + ((static_cast<size_t>(tok0) + q_pos) * p.Hq + hs) * DV;
+      const bool row_in = !VARLEN || q_pos < U.seq_len;
+      __nv_bfloat16* orow = p.o + ((static_cast<size_t>(U.tok0) + q_pos) * p.Hq + hs) * DV;
       const uint64_t pol_once = l2_policy_evict_first();  // O is written once
       const float2 inv2 = make_float2(inv, inv);
 #pragma unroll
-      for (int c = 0; c < DV; c += 8) {
-        const float2 a0 = __fmul2_rn(make_float2(o[c + 0], o[c + 1]), inv2);
-        const float2 a1 = __fmul2_rn(make_float2(o[c + 2], o[c + 3]), inv2);
-        const float2 a2 = __fmul2_rn(make_float2(o[c + 4], o[c + 5]), inv2);
-        const float2 a3 = __fmul2_rn(make_float2(o[c + 6], o[c + 7]), inv2);
+      for (int cc = 0; cc < DV; cc += 8) {
+        const float2 a0 = __fmul2_rn(make_float2(o[cc + 0], o[cc + 1]), inv2);
+        const float2 a1 = __fmul2_rn(make_float2(o[cc + 2], o[cc + 3]), inv2);
+        const float2 a2 = __fmul2_rn(make_float2(o[cc + 4], o[cc + 5]), inv2);
+        const float2 a3 = __fmul2_rn(make_float2(o[cc + 6], o[cc + 7]), inv2);
         uint4 v;
         v.x = pack_bf16x2(a0.x, a0.y);
         v.y = pack_bf16x2(a1.x, a1.y);
         v.z = pack_bf16x2(a2.x, a2.y);
         v.w = pack_bf16x2(a3.x, a3.y);
-        if (row_in) st_global_v4_hint(orow + c, v, pol_once);
+        if (row_in) st_global_v4_hint(orow + cc, v, pol_once);
       }
       if (p.lse != nullptr && row_in) {
         float lse_v;
@@ -771,8 +870,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           lse_v = 0.69314718055994531f * (ms + __log2f(l));
         // lse [B, Hq, S], or [Hq, total tokens] for packed sequences
         const size_t li = (VARLEN && p.cu_seqlens != nullptr)
-                              ? static_cast<size_t>(hs) * p.total_tokens + tok0 + q_pos
-                              : (static_cast<size_t>(b) * p.Hq + hs) * p.S + q_pos;
+                              ? static_cast<size_t>(hs) * p.total_tokens + U.tok0 + q_pos
+                              : (static_cast<size_t>(U.b) * p.Hq + hs) * p.S + q_pos;
         p.lse[li] = lse_v;
       }
     }

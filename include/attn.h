@@ -230,27 +230,21 @@ attn_status_t attn_fwd_fp8_dump(const void* q, const void* k, const void* v, voi
 attn_status_t attn_device_status(void* stream);
 
 /*
- * Prefill kernel used by attn_fwd, attn_fwd_ex, attn_fwd_varlen and the dump (one CTA per
- * unit, two 128-row query slots in ping-pong sharing every K/V tile):
- *   ATTN_KERNEL_SINGLE     (default) 128-key tiles; a unit is two consecutive query tiles
- *                          of one query head;
- *   ATTN_KERNEL_HEADS      128-key tiles; a unit is one query tile of two query heads of
- *                          one kv group (equal causal extents); with Hq / Hkv odd it is
- *                          ATTN_KERNEL_SINGLE;
- *   ATTN_KERNEL_K64        64-key tiles (every TMEM buffer separate, P double-buffered);
- *                          units as ATTN_KERNEL_SINGLE;
- *   ATTN_KERNEL_K64_HEADS  64-key tiles, units as ATTN_KERNEL_HEADS.
- * The two unit kinds compute the same function (bitwise the same lean-P codes; outputs
- * equal up to the tensor cores' fp32 summation order).  The tile size changes one step of
- * the FP8 lean-P reading: the lazy reference max is updated once per key tile, so 64-key
- * tiles may update it at other keys than 128-key tiles (both within the same bounds).  A
- * process-wide setting, for measurement and tests; returns ATTN_ERR_INVALID_ARG for
- * another value.
+ * Work unit and schedule of the prefill kernel used by attn_fwd, attn_fwd_ex,
+ * attn_fwd_varlen and the dump: the bitwise OR of a unit (a CTA's two 128-row query slots
+ * in ping-pong sharing every K/V tile) and a schedule:
+ *   ATTN_KERNEL_SINGLE      (0) two consecutive query tiles of one query head;
+ *   ATTN_KERNEL_HEADS       (2) one query tile of two query heads of one kv group (equal
+ *                           causal extents); with Hq / Hkv odd it is ATTN_KERNEL_SINGLE;
+ *   ATTN_KERNEL_PERSISTENT  (4) one CTA per SM, each running every SM-count-th unit
+ *                           (longest first), instead of one CTA per unit.
+ * All compute the same function (bitwise the same lean-P codes; outputs equal up to the
+ * tensor cores' fp32 summation order).  A process-wide setting, for measurement and tests;
+ * returns ATTN_ERR_INVALID_ARG for another value.  Default: ATTN_KERNEL_SINGLE.
  */
 #define ATTN_KERNEL_SINGLE 0
 #define ATTN_KERNEL_HEADS 2
-#define ATTN_KERNEL_K64 3
-#define ATTN_KERNEL_K64_HEADS 4
+#define ATTN_KERNEL_PERSISTENT 4
 attn_status_t attn_select_prefill_kernel(int kernel);
 
 /* Test-only: sets the bounded-wait limit in nanoseconds (0 restores the default, 2 s). */
@@ -264,6 +258,12 @@ void attn_set_wait_timeout_ns(uint64_t ns);
  * Applies to the attn_fwd* calls made while it is set.
  */
 void attn_selftest_stall_tile(int tile);
+
+/*
+ * Test-only: caps the grid of the persistent schedule (ATTN_KERNEL_PERSISTENT) at n CTAs, so
+ * that small problems run many units per CTA (n <= 0 removes the cap).
+ */
+void attn_selftest_max_ctas(int n);
 
 /*
  * Test-only: launches one thread that waits, with the bounded wait the kernels use, on an

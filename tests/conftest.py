@@ -26,23 +26,37 @@ def pytest_collection_modifyitems(config, items):
             item.add_marker(skip)
 
 
-KERNELS = {"single": "ATTN_KERNEL_SINGLE", "heads": "ATTN_KERNEL_HEADS",
-           "k64": "ATTN_KERNEL_K64", "k64heads": "ATTN_KERNEL_K64_HEADS"}
+# prefill kernel settings: (unit and schedule flags, cap on the persistent grid).  The caps
+# make the small test problems run several units per CTA on the persistent schedule.
+KERNELS = {"single": (("ATTN_KERNEL_SINGLE",), 0),
+           "heads": (("ATTN_KERNEL_HEADS",), 0),
+           "persistent": (("ATTN_KERNEL_SINGLE", "ATTN_KERNEL_PERSISTENT"), 5),
+           "heads_persistent": (("ATTN_KERNEL_HEADS", "ATTN_KERNEL_PERSISTENT"), 3)}
+
+
+def select_kernel(pkg, name):
+    flags, cap = KERNELS[name]
+    k = 0
+    for f in flags:
+        k |= getattr(pkg, f)
+    pkg.attn_select_prefill_kernel(k)
+    pkg.attn_selftest_max_ctas(cap)
 
 
 @pytest.fixture(params=list(KERNELS))
 def prefill_kernel(request):
-    """Runs a test under each prefill kernel (128-key tiles with two query tiles of one head
-    or one query tile of two heads of one kv group per CTA; 64-key tiles with either unit),
-    restoring the default afterwards."""
+    """Runs a test under each work unit (two query tiles of one head; one query tile of two
+    heads of one kv group) and schedule (one CTA per unit; a persistent grid, capped so that
+    CTAs run several units) of the prefill kernel, restoring the default afterwards."""
     import bf16_causal_prefill_attn_b200 as pkg
-    pkg.attn_select_prefill_kernel(getattr(pkg, KERNELS[request.param]))
+    select_kernel(pkg, request.param)
     yield request.param
     pkg.attn_select_prefill_kernel(pkg.ATTN_KERNEL_SINGLE)
+    pkg.attn_selftest_max_ctas(0)
 
 
 @pytest.fixture
 def key_tile(prefill_kernel):
     """Keys per tile of the selected prefill kernel: the FP8 lean-P reference max is updated
     once per key tile, so the emulator replays the kernel with this tile."""
-    return 64 if prefill_kernel.startswith("k64") else 128
+    return 128
