@@ -37,9 +37,17 @@ NOMINAL_FP8_TFLOPS = 4500.0
 NOMINAL_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# prefill kernel families (attn_select_prefill_kernel)
-KERNEL_IDS = {"single": lambda pkg: pkg.ATTN_KERNEL_SINGLE,
-              "heads": lambda pkg: pkg.ATTN_KERNEL_HEADS}
+# prefill work unit and schedule (attn_select_prefill_kernel): auto (the library default:
+# dynamic take-over of units, head pairs for FP8, tile pairs for BF16); a unit (tile pairs
+# "single", head pairs "heads") with one CTA per unit, a static persistent grid ("-static")
+# or dynamic take-over ("-dynamic")
+KERNEL_IDS = {"auto": lambda pkg: pkg.ATTN_KERNEL_AUTO,
+              "single": lambda pkg: pkg.ATTN_KERNEL_SINGLE,
+              "heads": lambda pkg: pkg.ATTN_KERNEL_HEADS,
+              "single-static": lambda pkg: pkg.ATTN_KERNEL_SINGLE | pkg.ATTN_KERNEL_PERSISTENT,
+              "heads-static": lambda pkg: pkg.ATTN_KERNEL_HEADS | pkg.ATTN_KERNEL_PERSISTENT,
+              "single-dynamic": lambda pkg: pkg.ATTN_KERNEL_SINGLE | pkg.ATTN_KERNEL_DYNAMIC,
+              "heads-dynamic": lambda pkg: pkg.ATTN_KERNEL_HEADS | pkg.ATTN_KERNEL_DYNAMIC}
 
 WORKLOADS = {
     # name: (B, S, Hq, Hkv, d_qk, d_v, distribution, description)
@@ -858,9 +866,9 @@ def main(argv=None):
                          "the default workload")
     ap.add_argument("--exact-p", action="store_true",
                     help="FP8 probabilities by exponential + e4m3 rounding (the ablation of lean P)")
-    ap.add_argument("--kernel", default="single", choices=list(KERNEL_IDS),
-                    help="work unit of the prefill kernel: two query tiles of one head "
-                         "(default) or one query tile of two heads of one kv group")
+    ap.add_argument("--kernel", default="auto", choices=list(KERNEL_IDS),
+                    help="work unit and schedule of the prefill kernel (default: the "
+                         "library's automatic choice)")
     ap.add_argument("--split", default="replicas", choices=["replicas", "heads"],
                     help="multi-GPU: an independent problem per GPU (weak scaling), or one "
                          "problem divided by kv heads (strong scaling)")

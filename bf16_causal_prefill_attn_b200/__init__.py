@@ -25,6 +25,8 @@ ATTN_FLAG_EXACT_P = 2
 ATTN_KERNEL_SINGLE = 0
 ATTN_KERNEL_HEADS = 2
 ATTN_KERNEL_PERSISTENT = 4
+ATTN_KERNEL_DYNAMIC = 8
+ATTN_KERNEL_AUTO = 16
 
 _lib = None
 
@@ -305,8 +307,10 @@ def attn_set_wait_timeout_ns(ns):
 def attn_select_prefill_kernel(kernel):
     """Work unit and schedule of the prefill kernel for later calls: ATTN_KERNEL_SINGLE (two
     query tiles of one head per unit) or ATTN_KERNEL_HEADS (one query tile of two heads of
-    one kv group), optionally OR ATTN_KERNEL_PERSISTENT (one CTA per SM looping over the
-    units instead of one CTA per unit)."""
+    one kv group), optionally OR one schedule: ATTN_KERNEL_PERSISTENT (one CTA per SM
+    running a static list of units) or ATTN_KERNEL_DYNAMIC (one CTA per unit; running CTAs
+    take over the units of CTAs not yet started); or ATTN_KERNEL_AUTO (the default:
+    dynamic, head pairs for FP8, tile pairs for BF16)."""
     _check(lib().attn_select_prefill_kernel(int(kernel)), "attn_select_prefill_kernel")
 
 

@@ -26,7 +26,7 @@ __device__ uint32_t g_dev_err = 0;
 
 uint64_t g_timeout_ns = kDefaultTimeoutNs;
 int g_stall_tile = -1;  // test-only (attn_selftest_stall_tile)
-int g_kernel = ATTN_KERNEL_SINGLE;  // prefill kernel family (attn_select_prefill_kernel)
+int g_kernel = ATTN_KERNEL_AUTO;  // prefill unit and schedule (attn_select_prefill_kernel)
 int g_max_ctas = 0;  // test-only cap on the persistent grid (attn_selftest_max_ctas; 0: none)
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -187,17 +187,21 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, attn::FwdP
   const attn_status_t rs = register_split_ok<kern>();
   if (rs != ATTN_OK) return rs;
   // units: two query tiles of one head, or (ATTN_KERNEL_HEADS, Hq / Hkv even) one query
-  // tile of two heads of one kv group; one CTA per unit, or (ATTN_KERNEL_PERSISTENT) one
-  // CTA per SM running every SM-count-th unit
+  // tile of two heads of one kv group; one CTA per unit (ATTN_KERNEL_DYNAMIC: running CTAs
+  // take over the units of CTAs not yet started), or (ATTN_KERNEL_PERSISTENT) one CTA per
+  // SM running a static list of units
   attn::FwdParams pp = prm;
-  pp.head_pairs = ((g_kernel & ATTN_KERNEL_HEADS) && prm.G % 2 == 0) ? 1 : 0;
+  const int kernel =
+      g_kernel == ATTN_KERNEL_AUTO ? (ATTN_KERNEL_DYNAMIC | (FP8 ? ATTN_KERNEL_HEADS : 0)) : g_kernel;
+  pp.head_pairs = ((kernel & ATTN_KERNEL_HEADS) && prm.G % 2 == 0) ? 1 : 0;
   pp.n_pairs = pp.head_pairs ? prm.n_q_tiles : (prm.n_q_tiles + 1) / 2;
   const int64_t units = static_cast<int64_t>(pp.n_pairs) * prm.B *
                         (pp.head_pairs ? prm.Hq / 2 : prm.Hq);
   if (units <= 0 || units > INT32_MAX) return ATTN_ERR_INVALID_ARG;
   pp.n_units = static_cast<int>(units);
   unsigned grid = static_cast<unsigned>(units);
-  if (g_kernel & ATTN_KERNEL_PERSISTENT) {
+  pp.dynamic = (kernel & ATTN_KERNEL_DYNAMIC) ? 1 : 0;
+  if (kernel & ATTN_KERNEL_PERSISTENT) {
     const int sms = sm_count();
     if (sms <= 0) return ATTN_ERR_CUDA;
     grid = static_cast<unsigned>(std::min<int64_t>(units, sms));
@@ -651,7 +655,10 @@ void attn_selftest_stall_tile(int tile) { g_stall_tile = tile < 0 ? -1 : tile; }
 void attn_selftest_max_ctas(int n) { g_max_ctas = n > 0 ? n : 0; }
 
 attn_status_t attn_select_prefill_kernel(int kernel) {
-  if ((kernel & ~(ATTN_KERNEL_HEADS | ATTN_KERNEL_PERSISTENT)) != 0) return ATTN_ERR_INVALID_ARG;
+  if (kernel != ATTN_KERNEL_AUTO &&
+      ((kernel & ~(ATTN_KERNEL_HEADS | ATTN_KERNEL_PERSISTENT | ATTN_KERNEL_DYNAMIC)) != 0 ||
+       ((kernel & ATTN_KERNEL_PERSISTENT) && (kernel & ATTN_KERNEL_DYNAMIC))))
+    return ATTN_ERR_INVALID_ARG;
   g_kernel = kernel;
   return ATTN_OK;
 }

@@ -118,6 +118,34 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
 }
 
 // ------------------------------------------------------------------ TMA
+// Cluster launch control (sm_100): ask the hardware to cancel the launch of a CTA that has
+// not started yet; the 16-byte response lands at `resp` (16-byte aligned shared memory) and
+// completes 16 transaction bytes on `bar` (the caller arms it with mbar_arrive_expect_tx).
+// After a request that found nothing to cancel, no further request may be made.
+__device__ __forceinline__ void clc_try_cancel(void* resp, uint64_t* bar) {
+  asm volatile(
+      "clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 "
+      "[%0], [%1];" ::"r"(smem_addr(resp)),
+      "r"(smem_addr(bar))
+      : "memory");
+}
+
+// Decodes a response: true and the cancelled CTA's blockIdx.x, or false (nothing left).
+__device__ __forceinline__ bool clc_query(const void* resp, int* ctaid_x) {
+  uint32_t ok, x;
+  asm volatile(
+      "{.reg .b128 r; .reg .pred p;\n\t"
+      "ld.shared.b128 r, [%2];\n\t"
+      "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, r;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t"
+      "clusterlaunchcontrol.query_cancel.get_first_ctaid::x.b32.b128 %1, r;}"
+      : "=r"(ok), "=r"(x)
+      : "r"(smem_addr(resp))
+      : "memory");
+  *ctaid_x = static_cast<int>(x);
+  return ok != 0;
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const void* desc) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(desc)) : "memory");
 }

@@ -232,19 +232,27 @@ attn_status_t attn_device_status(void* stream);
 /*
  * Work unit and schedule of the prefill kernel used by attn_fwd, attn_fwd_ex,
  * attn_fwd_varlen and the dump: the bitwise OR of a unit (a CTA's two 128-row query slots
- * in ping-pong sharing every K/V tile) and a schedule:
+ * in ping-pong sharing every K/V tile) and at most one schedule flag:
  *   ATTN_KERNEL_SINGLE      (0) two consecutive query tiles of one query head;
  *   ATTN_KERNEL_HEADS       (2) one query tile of two query heads of one kv group (equal
  *                           causal extents); with Hq / Hkv odd it is ATTN_KERNEL_SINGLE;
- *   ATTN_KERNEL_PERSISTENT  (4) one CTA per SM, each running every SM-count-th unit
- *                           (longest first), instead of one CTA per unit.
- * All compute the same function (bitwise the same lean-P codes; outputs equal up to the
- * tensor cores' fp32 summation order).  A process-wide setting, for measurement and tests;
- * returns ATTN_ERR_INVALID_ARG for another value.  Default: ATTN_KERNEL_SINGLE.
+ *   ATTN_KERNEL_PERSISTENT  (4) one CTA per SM, each running a static list of units
+ *                           (rounds of SM-count units, alternate rounds mirrored);
+ *   ATTN_KERNEL_DYNAMIC     (8) one CTA launched per unit (longest first); a CTA that
+ *                           finishes its unit takes over the unit of a CTA that has not
+ *                           started yet (cluster launch control), so each SM keeps one CTA
+ *                           running unit after unit.
+ * Without a schedule flag every CTA runs one unit.  ATTN_KERNEL_AUTO (16, alone; the
+ * default) is ATTN_KERNEL_DYNAMIC with head pairs for FP8 and tile pairs for BF16.  All
+ * compute the same function (bitwise the same outputs and lean-P codes: a unit is computed
+ * by the same code whichever CTA runs it).  A process-wide setting, for measurement and
+ * tests; returns ATTN_ERR_INVALID_ARG for another value.
  */
 #define ATTN_KERNEL_SINGLE 0
 #define ATTN_KERNEL_HEADS 2
 #define ATTN_KERNEL_PERSISTENT 4
+#define ATTN_KERNEL_DYNAMIC 8
+#define ATTN_KERNEL_AUTO 16
 attn_status_t attn_select_prefill_kernel(int kernel);
 
 /* Test-only: sets the bounded-wait limit in nanoseconds (0 restores the default, 2 s). */

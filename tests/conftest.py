@@ -31,7 +31,9 @@ def pytest_collection_modifyitems(config, items):
 KERNELS = {"single": (("ATTN_KERNEL_SINGLE",), 0),
            "heads": (("ATTN_KERNEL_HEADS",), 0),
            "persistent": (("ATTN_KERNEL_SINGLE", "ATTN_KERNEL_PERSISTENT"), 5),
-           "heads_persistent": (("ATTN_KERNEL_HEADS", "ATTN_KERNEL_PERSISTENT"), 3)}
+           "heads_persistent": (("ATTN_KERNEL_HEADS", "ATTN_KERNEL_PERSISTENT"), 3),
+           "dynamic": (("ATTN_KERNEL_SINGLE", "ATTN_KERNEL_DYNAMIC"), 0),
+           "auto": (("ATTN_KERNEL_AUTO",), 0)}
 
 
 def select_kernel(pkg, name):
@@ -46,12 +48,13 @@ def select_kernel(pkg, name):
 @pytest.fixture(params=list(KERNELS))
 def prefill_kernel(request):
     """Runs a test under each work unit (two query tiles of one head; one query tile of two
-    heads of one kv group) and schedule (one CTA per unit; a persistent grid, capped so that
-    CTAs run several units) of the prefill kernel, restoring the default afterwards."""
+    heads of one kv group) and schedule (one CTA per unit; a static persistent grid, capped
+    so that CTAs run several units; dynamic take-over of units) of the prefill kernel,
+    restoring the default afterwards."""
     import bf16_causal_prefill_attn_b200 as pkg
     select_kernel(pkg, request.param)
     yield request.param
-    pkg.attn_select_prefill_kernel(pkg.ATTN_KERNEL_SINGLE)
+    pkg.attn_select_prefill_kernel(pkg.ATTN_KERNEL_AUTO)
     pkg.attn_selftest_max_ctas(0)
 
 

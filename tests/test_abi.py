@@ -170,3 +170,21 @@ def test_built_library_is_newer_than_every_source(L):
     assert set(B.sources()) >= {f for f in files if f.endswith((".cu", ".cuh", ".h"))} - {HEADER}
     for f in files:
         assert os.path.getmtime(f) <= lib_t, f
+
+
+def test_prefill_kernel_selection_validated(L):
+    """Units and schedules combine by OR; both schedule flags at once, or an unknown bit,
+    are rejected (no GPU call is made)."""
+    import bf16_causal_prefill_attn_b200 as pkg
+    good = [pkg.ATTN_KERNEL_SINGLE, pkg.ATTN_KERNEL_HEADS,
+            pkg.ATTN_KERNEL_PERSISTENT, pkg.ATTN_KERNEL_HEADS | pkg.ATTN_KERNEL_PERSISTENT,
+            pkg.ATTN_KERNEL_DYNAMIC, pkg.ATTN_KERNEL_HEADS | pkg.ATTN_KERNEL_DYNAMIC,
+            pkg.ATTN_KERNEL_AUTO]
+    try:
+        for k in good:
+            assert L.attn_select_prefill_kernel(k) == pkg.ATTN_OK
+        for bad in (pkg.ATTN_KERNEL_PERSISTENT | pkg.ATTN_KERNEL_DYNAMIC, 1, 32, -1,
+                    pkg.ATTN_KERNEL_AUTO | pkg.ATTN_KERNEL_HEADS):
+            assert L.attn_select_prefill_kernel(bad) == pkg.ATTN_ERR_INVALID_ARG
+    finally:
+        L.attn_select_prefill_kernel(pkg.ATTN_KERNEL_AUTO)

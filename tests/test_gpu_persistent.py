@@ -1,8 +1,10 @@
-"""The persistent schedule (one CTA per SM running every SM-count-th unit) against one CTA
-per unit: the units are computed by the same code in the same order, so outputs, lse and
-the lean-P dumps must be bitwise identical.  Small grids (down to a single CTA running
-every unit) carry the per-slot phase counts, the K/V ring positions and the Q hand-over
-through many units."""
+"""The multi-unit schedules against one CTA per unit: the static persistent grid (one CTA
+per SM running a list of units) and the dynamic one (CTAs taking over the units of CTAs not
+yet started, by cluster launch control).  A unit is computed by the same code whichever
+CTA runs it, so outputs, lse and the lean-P dumps must be bitwise identical.  Small static
+grids (down to a single CTA running every unit) carry the per-slot phase counts, the K/V
+ring positions, the unit queue and the Q hand-over through many units; problems with more
+units than SMs make the dynamic schedule take units over."""
 import numpy as np
 import pytest
 import torch
@@ -24,7 +26,7 @@ def _run(fn, kernel, cap):
         assert pkg.attn_device_status() == pkg.ATTN_OK
         return out
     finally:
-        pkg.attn_select_prefill_kernel(pkg.ATTN_KERNEL_SINGLE)
+        pkg.attn_select_prefill_kernel(pkg.ATTN_KERNEL_AUTO)
         pkg.attn_selftest_max_ctas(0)
 
 
@@ -45,6 +47,8 @@ def _same(a, b):
     (1, 512, 4, 4, 192, True, True),      # MLA head dimension
     (3, 384, 6, 2, 128, False, False),    # full attention, G = 3
     (4, 1024, 8, 2, 128, True, True),     # 128 units: several per CTA at every cap
+    (8, 1024, 8, 2, 128, True, False),    # 256 units: more than SMs (dynamic take-over)
+    (8, 1024, 8, 2, 128, True, True),
 ])
 def test_persistent_equals_one_cta_per_unit(unit, B, S, Hq, Hkv, dqk, causal, fp8):
     q, k, v = [t.cuda() for t in synth.make_qkv(B, S, Hq, Hkv, dqk, 128, seed=S + Hq, dist="outlier")]
@@ -57,13 +61,15 @@ def test_persistent_equals_one_cta_per_unit(unit, B, S, Hq, Hkv, dqk, causal, fp
     ref = _run(fn, u, 0)
     for cap in CAPS:
         _same(_run(fn, u | pkg.ATTN_KERNEL_PERSISTENT, cap), ref)
+    for _ in range(3):   # which CTA takes which unit varies from run to run
+        _same(_run(fn, u | pkg.ATTN_KERNEL_DYNAMIC, 0), ref)
 
 
 @pytest.mark.parametrize("fp8", [False, True])
 def test_persistent_varlen_equals_one_cta_per_unit(fp8):
     """Packed sequences with empty, one-token and ragged members: the units that a short
     sequence lacks are skipped by every role of the CTA alike."""
-    lengths = [129, 1, 300, 0, 128, 64, 513, 127, 0, 700]
+    lengths = [129, 1, 300, 0, 128, 64, 513, 127, 0, 700] * 6
     lead, tail, Hq, Hkv = 16, 40, 4, 2
     T = lead + sum(lengths) + tail
     q, k, v = [t[0].cuda() for t in synth.make_qkv(1, T, Hq, Hkv, 128, 128, seed=5, dist="gaussian")]
@@ -83,6 +89,8 @@ def test_persistent_varlen_equals_one_cta_per_unit(fp8):
     for cap in CAPS:
         _same(_run(fn, pkg.ATTN_KERNEL_SINGLE | pkg.ATTN_KERNEL_PERSISTENT, cap), ref)
         _same(_run(fn, pkg.ATTN_KERNEL_HEADS | pkg.ATTN_KERNEL_PERSISTENT, cap), ref)
+    for u in (pkg.ATTN_KERNEL_SINGLE, pkg.ATTN_KERNEL_HEADS):
+        _same(_run(fn, u | pkg.ATTN_KERNEL_DYNAMIC, 0), ref)
 
 
 def test_persistent_dump_equals_one_cta_per_unit():
@@ -93,3 +101,5 @@ def test_persistent_dump_equals_one_cta_per_unit():
     ref = _run(fn, pkg.ATTN_KERNEL_SINGLE, 0)
     for cap in (1, 3):
         _same(_run(fn, pkg.ATTN_KERNEL_SINGLE | pkg.ATTN_KERNEL_PERSISTENT, cap), ref)
+    _same(_run(fn, pkg.ATTN_KERNEL_SINGLE | pkg.ATTN_KERNEL_DYNAMIC, 0), ref)
+
