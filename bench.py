@@ -604,15 +604,16 @@ def gpu_bench(args, rank, world, local_rank):
 
 
 # ----------------------------------------------------------------------------- headline shapes
-EXTRA_PREFILL = ("mha32k_gaussian", "mla32k_outlier")
+EXTRA_PREFILL = ("mha32k_gaussian", "mla32k_outlier", "sweep_s1k", "sweep_s4k")
 EXTRA_DECODE = "decode_gqa_b64_s4k"
 
 
 def headline_extras(args, dev, peaks, peak_src):
     """Kernel throughput on the pages' own headline shapes, next to the main workload:
-    MHA 32 heads at S = 32768 on Gaussian inputs (FP8 and BF16) and the MLA shape at
-    S = 32768 (FP8), each timed over a few launches with an L2 flush between them, and one
-    paged-decode workload (GB/s against the copy bandwidth)."""
+    MHA 32 heads at S = 32768 on Gaussian inputs (FP8 and BF16), the MLA shape at
+    S = 32768 (FP8) and two points of the sequence-length sweep (B * S = 32768 at S = 1024
+    and 4096, FP8 and BF16), each timed over a few launches with an L2 flush between them,
+    and one paged-decode workload (GB/s against the copy bandwidth)."""
     import copy
 
     import torch
