@@ -177,11 +177,18 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, attn::FwdP
   const CUtensorMapDataType dt =
       FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const uint64_t T = static_cast<uint64_t>(prm.total_tokens);
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   if (!make_map(&mq, q, dt, C::E, DQK, prm.Hq, T, C::BOX_COLS) ||
       !make_map(&mk, k, dt, C::E, DQK, prm.Hkv, T, C::BOX_COLS) ||
       !make_map(&mv, v, dt, C::E, attn::DV, prm.Hkv, T, C::BOX_COLS))
     return ATTN_ERR_CUDA;
+  // O [T, Hq, 128] bf16 in boxes of 64 columns x 128 rows (stored through shared memory)
+  if (C::TMA_O && !VARLEN) {
+    if (!make_map(&mo, prm.o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, attn::DV, prm.Hq, T, 64))
+      return ATTN_ERR_CUDA;
+  } else {
+    mo = mq;  // unused
+  }
   constexpr auto kern = attn::attn_fwd_kernel<FP8, DQK, DUMP, EXACT, VARLEN>;
   if (!set_smem_attr<kern>(C::SMEM_ALLOC)) return ATTN_ERR_CUDA;
   const attn_status_t rs = register_split_ok<kern>();
@@ -207,7 +214,7 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, attn::FwdP
     grid = static_cast<unsigned>(std::min<int64_t>(units, sms));
     if (g_max_ctas > 0) grid = std::min(grid, static_cast<unsigned>(g_max_ctas));
   }
-  kern<<<grid, attn::NUM_THREADS, C::SMEM_ALLOC, stream>>>(mq, mk, mv, pp);
+  kern<<<grid, attn::NUM_THREADS, C::SMEM_ALLOC, stream>>>(mq, mk, mv, mo, pp);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

@@ -163,11 +163,17 @@ struct FwdCfg {
   static constexpr int OFF_V = OFF_K + NK * K_BYTES;
   static constexpr int OFF_ONES = OFF_V + NV * V_BYTES;  // FP8: 128 keys x 128 B of 1.0
   static constexpr int OFF_P = OFF_ONES + (FP8 ? BOX_BYTES : 0);  // FP8: P_0, P_1
-  static constexpr int OFF_BAR = OFF_P + (FP8 ? 2 * BOX_BYTES : 0);
+  // O leaves through shared memory and a TMA store (64 columns, 16 KB per slot at a time):
+  // FP8 stages in P_t (free once the slot's last PV has completed); BF16 with d_qk = 128
+  // has a staging area of its own; BF16 with d_qk = 192 has no room and stores rows directly
+  static constexpr bool TMA_O = FP8 || DQK == 128;
+  static constexpr int OFF_OST = OFF_P;                        // slot t at OFF_OST + t BOX_BYTES
+  static constexpr int OFF_BAR = OFF_P + (TMA_O ? 2 * BOX_BYTES : 0);
   // barriers: k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], per slot q_full, q_empty,
   //           s_full, p_full, pv_done, s_read, mma_done, then unit_full[UQ],
-  //           unit_empty[UQ] and the launch-control barrier
-  static constexpr int NUM_BARS = 2 * NK + 2 * NV + 2 * 7 + 2 * UQ + 1;
+  //           unit_empty[UQ], the launch-control barrier and per slot the O-staging
+  //           barrier
+  static constexpr int NUM_BARS = 2 * NK + 2 * NV + 2 * 7 + 2 * UQ + 1 + 2;
   static constexpr int OFF_UNITQ = OFF_BAR + NUM_BARS * 8;              // int[UQ]
   static constexpr int OFF_CLC = (OFF_UNITQ + UQ * 4 + 15) / 16 * 16;   // 16-byte response
   static constexpr int OFF_TMEMPTR = OFF_CLC + 16;
@@ -280,11 +286,14 @@ __device__ __forceinline__ int cta_unit(int k) {
 // sum) is shared.
 // VARLEN: sequences of any length (packed, or a fixed S not a multiple of 128): keys past
 // the end of the sequence are masked, rows past it are not written.
+// tm_o: O [tokens, Hq, 128] bf16, boxes of 64 columns x 128 rows with the 128-byte swizzle
+// (used when C::TMA_O and not VARLEN).
 template <bool FP8, int DQK, bool DUMP, bool EXACT = false, bool VARLEN = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+                    const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_o, const FwdParams p) {
   using C = FwdCfg<FP8, DQK>;
   using TM = TmemMap<FP8>;
   extern __shared__ uint8_t smem_raw[];
@@ -306,6 +315,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* unit_full = tbar + 14;       // [UQ] unit index published by the producer
   uint64_t* unit_empty = unit_full + UQ;  // [UQ] read by every consumer warp
   uint64_t* clc_bar = unit_empty + UQ;   // launch-control response landed
+  uint64_t* o_sync = clc_bar + 1;        // [2] the four warps of slot t at the O staging
   int* unit_q = reinterpret_cast<int*>(smem + C::OFF_UNITQ);
   void* clc_resp = smem + C::OFF_CLC;
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEMPTR);
@@ -340,6 +350,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(unit_empty + i, UNIT_CONSUMERS);
     }
     mbar_init(clc_bar, 1);
+    mbar_init(o_sync + 0, 4);
+    mbar_init(o_sync + 1, 4);
     fence_barrier_init();
   }
   if (warp == 11) {
@@ -350,6 +362,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
+    if (C::TMA_O && !VARLEN) tma_prefetch_desc(&tm_o);
   }
   if constexpr (FP8) {
     // the ones block (e4m3 1.0 = 0x38) that extends every V tile to N = 144 for the row
@@ -704,6 +717,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     bool ok = true;
     int c = 0;  // key tiles of this slot processed so far (all units)
+    constexpr bool TMA_O = C::TMA_O && !VARLEN;
+    const bool o_issuer = (tid & 127) == 0;  // issues this slot's O stores
+    bool o_pending = false;  // FP8: a store from P_t may still be reading it
+    int o_phase = 0;         // completed phases of o_sync(t)
+    // the slot's four warps meet (bounded, so that a warp that has given up cannot leave the
+    // others waiting for ever); orders the issuer's and the other threads' shared-memory
+    // accesses through the barrier's release / acquire
+    auto slot_sync = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(o_sync + t);
+      const bool r = mbar_wait(o_sync + t, o_phase & 1, p.err, p.timeout_ns);
+      ++o_phase;
+      return __all_sync(0xffffffffu, r);
+    };
     for (int k = 0; ok; ++k) {
       int u = -1;
       ok = take_unit(k, u);
@@ -891,6 +918,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         } else {
           // row r of P_t: 128 codes = 8 chunks of 16 B; chunk cc sits at chunk position
           // cc ^ (r mod 8) of the row (128-byte swizzle, rows 128 B apart)
+          if (o_pending) {
+            // P_t held the previous unit's O on its way out: that store must have read it
+            if (o_issuer) bulk_wait_read_all();
+            o_pending = false;
+            ok = slot_sync();
+            if (!ok) break;
+          }
           const uint32_t prow = smem_addr(smem + C::OFF_P + t * C::BOX_BYTES) + r * 128;
 #pragma unroll
           for (int cc = 0; cc < 8; ++cc)
@@ -910,6 +944,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // ----------------------------------------------------------- epilogue of the unit
       ok = mbar_wait(pv_done(t), (c - 1) & 1, p.err, p.timeout_ns);
       if (!__all_sync(0xffffffffu, ok)) break;
+      if constexpr (TMA_O && !FP8) {
+        // the staging buffer's previous store (the previous unit's second half) must have
+        // read it; waited for here, before O occupies the registers
+        if (o_issuer) bulk_wait_read_all();
+        ok = slot_sync();
+        if (!ok) break;
+      }
       tc_fence_after();
       uint32_t oraw[DV];
 #pragma unroll
@@ -946,21 +987,58 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // VARLEN: rows past the end of the sequence hold another sequence's queries (or zero
       // fill) and are not written
       const bool row_in = !VARLEN || q_pos < U.seq_len;
-      __nv_bfloat16* orow = p.o + ((static_cast<size_t>(U.tok0) + q_pos) * p.Hq + hs) * DV;
       const uint64_t pol_once = l2_policy_evict_first();  // O is written once
       const float2 inv2 = make_float2(inv, inv);
+      if constexpr (TMA_O) {
+        // 64 columns at a time: row r's 128 bytes as 8 chunks at positions cc ^ (r mod 8) of
+        // the slot's staging buffer (the tensor map's swizzle), then one thread stores the
+        // 128 x 64 box; rows of O are 8 KB apart, so per-thread row stores would touch a
+        // separate line per lane
+        uint8_t* ost = smem + C::OFF_OST + t * C::BOX_BYTES;
+        const uint32_t srow = smem_addr(ost) + r * 128;
 #pragma unroll
-      for (int cc = 0; cc < DV; cc += 8) {
-        const float2 a0 = __fmul2_rn(make_float2(o[cc + 0], o[cc + 1]), inv2);
-        const float2 a1 = __fmul2_rn(make_float2(o[cc + 2], o[cc + 3]), inv2);
-        const float2 a2 = __fmul2_rn(make_float2(o[cc + 4], o[cc + 5]), inv2);
-        const float2 a3 = __fmul2_rn(make_float2(o[cc + 6], o[cc + 7]), inv2);
-        uint4 v;
-        v.x = pack_bf16x2(a0.x, a0.y);
-        v.y = pack_bf16x2(a1.x, a1.y);
-        v.z = pack_bf16x2(a2.x, a2.y);
-        v.w = pack_bf16x2(a3.x, a3.y);
-        if (row_in) st_global_v4_hint(orow + cc, v, pol_once);
+        for (int h = 0; h < 2 && ok; ++h) {
+          if (h == 1) {
+            // the buffer's previous store (this unit's first half) must have read it
+            if (o_issuer) bulk_wait_read_all();
+            ok = slot_sync();
+            if (!ok) break;
+          }
+#pragma unroll
+          for (int cc = 0; cc < 8; ++cc) {
+            const int col = 64 * h + 8 * cc;
+            const float2 a0 = __fmul2_rn(make_float2(o[col + 0], o[col + 1]), inv2);
+            const float2 a1 = __fmul2_rn(make_float2(o[col + 2], o[col + 3]), inv2);
+            const float2 a2 = __fmul2_rn(make_float2(o[col + 4], o[col + 5]), inv2);
+            const float2 a3 = __fmul2_rn(make_float2(o[col + 6], o[col + 7]), inv2);
+            st_shared_v4(srow + ((cc ^ (r & 7)) << 4), pack_bf16x2(a0.x, a0.y), pack_bf16x2(a1.x, a1.y),
+                         pack_bf16x2(a2.x, a2.y), pack_bf16x2(a3.x, a3.y));
+          }
+          fence_proxy_async_smem();
+          ok = slot_sync();
+          if (!ok) break;
+          if (o_issuer) {
+            tma_store_3d_hint(&tm_o, ost, 64 * h, hs, U.tok0 + qt * BLOCK_M, pol_once);
+            bulk_commit_group();
+          }
+        }
+        o_pending = FP8;
+        if (!ok) break;
+      } else {
+        __nv_bfloat16* orow = p.o + ((static_cast<size_t>(U.tok0) + q_pos) * p.Hq + hs) * DV;
+#pragma unroll
+        for (int cc = 0; cc < DV; cc += 8) {
+          const float2 a0 = __fmul2_rn(make_float2(o[cc + 0], o[cc + 1]), inv2);
+          const float2 a1 = __fmul2_rn(make_float2(o[cc + 2], o[cc + 3]), inv2);
+          const float2 a2 = __fmul2_rn(make_float2(o[cc + 4], o[cc + 5]), inv2);
+          const float2 a3 = __fmul2_rn(make_float2(o[cc + 6], o[cc + 7]), inv2);
+          uint4 v;
+          v.x = pack_bf16x2(a0.x, a0.y);
+          v.y = pack_bf16x2(a1.x, a1.y);
+          v.z = pack_bf16x2(a2.x, a2.y);
+          v.w = pack_bf16x2(a3.x, a3.y);
+          if (row_in) st_global_v4_hint(orow + cc, v, pol_once);
+        }
       }
       if (p.lse != nullptr && row_in) {
         float lse_v;
@@ -975,6 +1053,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         p.lse[li] = lse_v;
       }
     }
+    // the O stores complete before the CTA exits (their source is this CTA's shared memory)
+    if (TMA_O && o_issuer) bulk_wait_all();
   }
   __syncthreads();
   if (warp == 11) {

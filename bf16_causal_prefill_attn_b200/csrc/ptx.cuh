@@ -185,6 +185,28 @@ __device__ __forceinline__ void tma_load_3d_hint(void* smem_dst, const void* des
       : "memory");
 }
 
+// 3-D tiled tensor store shared -> global with an L2 eviction policy, tracked as a bulk
+// async-group of the issuing thread (source: 1024-byte aligned, in the tensor map's swizzle).
+__device__ __forceinline__ void tma_store_3d_hint(const void* desc, const void* smem_src, int32_t c0,
+                                                  int32_t c1, int32_t c2, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group.L2::cache_hint"
+      " [%0, {%2, %3, %4}], [%1], %5;" ::"l"(reinterpret_cast<uint64_t>(desc)),
+      "r"(smem_addr(smem_src)), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// the issuing thread's bulk stores have finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// the issuing thread's bulk stores have completed
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 // 16-byte global store with an L2 eviction policy
 __device__ __forceinline__ void st_global_v4_hint(void* ptr, uint4 v, uint64_t policy) {
   asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(ptr),
