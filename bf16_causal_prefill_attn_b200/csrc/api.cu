@@ -43,10 +43,30 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+unsigned long long current_context_id();
+
+// Device address of the error word in the current context, looked up once per context by
+// this host thread (the last few contexts are kept, by their unique ids).
 bool dev_err_ptr(uint32_t** out) {
+  constexpr int kSlots = 4;
+  thread_local unsigned long long ctxs[kSlots] = {};
+  thread_local uint32_t* ptrs[kSlots] = {};
+  thread_local int next = 0;
+  const unsigned long long c = current_context_id();
+  if (c != 0)
+    for (int i = 0; i < kSlots; ++i)
+      if (ctxs[i] == c) {
+        *out = ptrs[i];
+        return true;
+      }
   void* p = nullptr;
   if (cudaGetSymbolAddress(&p, g_dev_err) != cudaSuccess) return false;
   *out = static_cast<uint32_t*>(p);
+  if (c != 0) {
+    ctxs[next] = c;
+    ptrs[next] = *out;
+    next = (next + 1) % kSlots;
+  }
   return true;
 }
 
@@ -95,22 +115,34 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esiz
   return true;
 }
 
-// The current context (driver API, through the runtime's entry-point query), to key state
-// that belongs to a context: a device's primary context is replaced by cudaDeviceReset.
+// The unique id of the current context (driver API through the runtime's entry-point
+// query), to key state that belongs to a context.  Ids are never reused, unlike context
+// handles: after cudaDeviceReset the new primary context may have the old handle.  0: no
+// context, or the driver offers no id (callers then cache nothing).
 using PFN_ctxGetCurrent = CUresult (*)(CUcontext*);
-CUcontext current_context() {
-  static PFN_ctxGetCurrent fn = nullptr;
+using PFN_ctxGetId = CUresult (*)(CUcontext, unsigned long long*);
+unsigned long long current_context_id() {
+  static PFN_ctxGetCurrent get_current = nullptr;
+  static PFN_ctxGetId get_id = nullptr;
   static std::once_flag once;
   std::call_once(once, [] {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_ctxGetCurrent>(p);
+      get_current = reinterpret_cast<PFN_ctxGetCurrent>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_ctxGetId>(p);
   });
   CUcontext c = nullptr;
-  if (fn == nullptr || fn(&c) != CUDA_SUCCESS) return nullptr;
-  return c;
+  if (get_current == nullptr || get_id == nullptr || get_current(&c) != CUDA_SUCCESS ||
+      c == nullptr)
+    return 0;
+  unsigned long long id = 0;
+  if (get_id(c, &id) != CUDA_SUCCESS) return 0;
+  return id;
 }
 
 // cudaFuncSetAttribute(max dynamic shared memory) for kernel KERN, skipped when it was
@@ -118,16 +150,16 @@ CUcontext current_context() {
 // template on the kernel's address: the prefill kernels all share one function type).
 template <auto KERN>
 bool set_smem_attr(int bytes) {
-  thread_local CUcontext done_ctx[4] = {};
+  thread_local unsigned long long done_ctx[4] = {};
   thread_local int next = 0;
-  const CUcontext c = current_context();
-  if (c != nullptr)
-    for (CUcontext d : done_ctx)
+  const unsigned long long c = current_context_id();
+  if (c != 0)
+    for (unsigned long long d : done_ctx)
       if (d == c) return true;
   if (cudaFuncSetAttribute(KERN, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
       cudaSuccess)
     return false;
-  if (c != nullptr) {
+  if (c != 0) {
     done_ctx[next] = c;
     next = (next + 1) % 4;
   }
