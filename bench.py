@@ -311,12 +311,7 @@ def gpu_bench_decode(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "e4m3",
         "data": "synthetic",
-        "config": {"workload": desc, "name": args.workload, "B": B, "L": L, "Hq": Hq, "Hkv": Hkv,
-                   "d": 128, "page_size": page,
-                   "step": "one decode call (split-KV kernel + combine kernel)",
-                   "l2": f"no flush: the caches ({kv_bytes(1) / 1e9:.2f} GB FP8, "
-                         f"{kv_bytes(2) / 1e9:.2f} GB BF16) exceed the 126 MB L2",
-                   "parallelism": f"replicas x{world} (independent problems per GPU)"},
+        "config": decode_config(args, world),
         "roofline": {"bound": "hbm", "achieved": round(fp8_gbs, 1), "peak": hbm,
                      "unit": "GB/s", "frac": round(fp8_gbs / hbm, 4),
                      "peak_source": f"{peak_src} copy bandwidth",
@@ -550,17 +545,7 @@ def gpu_bench(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "e4m3",
         "data": "synthetic",
-        "config": {"workload": desc, "name": args.workload, "B": B, "S": S,
-                   "Hq": WORKLOADS[args.workload][2], "Hkv": WORKLOADS[args.workload][3],
-                   "d_qk": dqk, "d_v": dv, "hadamard": bool(args.hadamard),
-                   "kernel": args.kernel,
-                   "step": "e4m3 quantisation of Q, K, V + "
-                           + ("exact-P attention (ablation)" if args.exact_p else "lean-P attention"),
-                   "l2": "256 MiB L2 flush written between steps, outside the timed step",
-                   "parallelism": (f"heads split x{world} (one problem; each GPU {Hkv} kv heads "
-                                   f"and their {Hq} query heads; no data-path collective)"
-                                   if args.split == "heads" else
-                                   f"replicas x{world} (independent problems per GPU)")},
+        "config": prefill_config(args, world, Hq, Hkv),
         "roofline": {"bound": "tensor", "achieved": round(fp8_kern_tf, 2),
                      "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
                      "frac": round(fp8_kern_tf / fp8_peak, 4),
@@ -824,6 +809,34 @@ def cpu_reference_decode(workload, budget_s):
             "seconds": dt}
 
 
+def decode_config(args, world):
+    """The `config` object of a decode line (the same for the GPU arm and the reference arm)."""
+    B, L, Hq, Hkv, page, desc = DECODE_WORKLOADS[args.workload]
+    kv = lambda e: 2.0 * B * L * Hkv * 128 * e
+    return {"workload": desc, "name": args.workload, "B": B, "L": L, "Hq": Hq, "Hkv": Hkv,
+            "d": 128, "page_size": page,
+            "step": "one decode call (split-KV kernel + combine kernel)",
+            "l2": f"no flush: the caches ({kv(1) / 1e9:.2f} GB FP8, "
+                  f"{kv(2) / 1e9:.2f} GB BF16) exceed the 126 MB L2",
+            "parallelism": f"replicas x{world} (independent problems per GPU)"}
+
+
+def prefill_config(args, world, rank_hq, rank_hkv):
+    """The `config` object of a prefill line (the same for the GPU arm and the reference
+    arm); rank_hq / rank_hkv: the heads one rank computes."""
+    B, S, Hq, Hkv, dqk, dv, distn, desc = WORKLOADS[args.workload]
+    return {"workload": desc, "name": args.workload, "B": B, "S": S, "Hq": Hq, "Hkv": Hkv,
+            "d_qk": dqk, "d_v": dv, "hadamard": bool(args.hadamard),
+            "kernel": args.kernel,
+            "step": "e4m3 quantisation of Q, K, V + "
+                    + ("exact-P attention (ablation)" if args.exact_p else "lean-P attention"),
+            "l2": "256 MiB L2 flush written between steps, outside the timed step",
+            "parallelism": (f"heads split x{world} (one problem; each GPU {rank_hkv} kv heads "
+                            f"and their {rank_hq} query heads; no data-path collective)"
+                            if args.split == "heads" else
+                            f"replicas x{world} (independent problems per GPU)")}
+
+
 def reference_main(args, rank, world):
     if rank != 0:
         return 0
@@ -837,12 +850,18 @@ def reference_main(args, rank, world):
         vals.append(last["value"])
         secs += last["seconds"]
     B, S, Hq, Hkv, dqk, dv, distn, desc = WORKLOADS[args.workload]
+    rank_hq, rank_hkv = Hq, Hkv
+    if args.split == "heads":
+        from bf16_causal_prefill_attn_b200 import shard
+        kv_lo, kv_hi, q_lo, q_hi = shard.head_partition(Hq, Hkv, world, 0)
+        rank_hq, rank_hkv = q_hi - q_lo, kv_hi - kv_lo
     value = statistics.mean(vals)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": secs * 1e3 / max(1, args.steps), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": desc, "name": args.workload},
+            "scaling": "strong" if args.split == "heads" else "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic",
+            "config": prefill_config(args, world, rank_hq, rank_hkv),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": last["cores"],
                              "cpu_model": last["cpu_model"], "kind": "oracle",
                              "sample": last["sample"]},
@@ -897,7 +916,7 @@ def main(argv=None):
                                   "steps": args.steps, "warmup": args.warmup,
                                   "higher_is_better": True, "scaling": "weak",
                                   "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                                  "config": {"workload": desc, "name": args.workload},
+                                  "config": decode_config(args, world),
                                   "cpu_baseline": c,
                                   "e2e": {"value": c["value"], "unit": "GB/s",
                                           "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
