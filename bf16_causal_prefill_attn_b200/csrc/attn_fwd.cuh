@@ -174,8 +174,10 @@ struct FwdCfg {
   //           unit_empty[UQ], the launch-control barrier and per slot the O-staging
   //           barrier
   static constexpr int NUM_BARS = 2 * NK + 2 * NV + 2 * 7 + 2 * UQ + 1 + 2;
-  static constexpr int OFF_UNITQ = OFF_BAR + NUM_BARS * 8;              // int[UQ]
-  static constexpr int OFF_CLC = (OFF_UNITQ + UQ * 4 + 15) / 16 * 16;   // 16-byte response
+  // unit queue: UQ entries of 12 ints (the unit, its status, the decoded Unit)
+  static constexpr int UQ_INTS = 12;
+  static constexpr int OFF_UNITQ = (OFF_BAR + NUM_BARS * 8 + 15) / 16 * 16;
+  static constexpr int OFF_CLC = OFF_UNITQ + UQ * UQ_INTS * 4;         // 16-byte response
   static constexpr int OFF_TMEMPTR = OFF_CLC + 16;
   static constexpr int SMEM_BYTES = OFF_TMEMPTR + 16;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;           // 1024-B alignment slack
@@ -374,16 +376,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_ptr;
-  // the k-th unit of this CTA from the queue (warp-wide; -1: no more units); false if the
-  // wait ran out
-  auto take_unit = [&](int k, int& u) -> bool {
+  // the k-th unit of this CTA from the queue (warp-wide; u = -1: no more units), decoded
+  // once by the producer: st is unit_info's result, U its unit; false if the wait ran out.
+  // Without `release` the caller keeps the entry (and may read it again) until
+  // release_unit(k).
+  auto take_unit = [&](int k, int& u, int& st, Unit& U, bool release = true) -> bool {
     const int slot = k % UQ;
     const bool r = mbar_wait(unit_full + slot, (k / UQ) & 1, p.err, p.timeout_ns);
     if (!__all_sync(0xffffffffu, r)) return false;
-    u = *reinterpret_cast<volatile int*>(unit_q + slot);
+    // scalar loads: a role's unused fields are never loaded
+    const int* e = unit_q + slot * C::UQ_INTS;
+    u = e[0];
+    st = e[1];
+    U.b = e[2];
+    U.h = e[3];
+    U.g = e[4];
+    U.tok0 = e[5];
+    U.seq_len = e[6];
+    U.qt0 = e[7];
+    U.qt1 = e[8];
+    U.n_t0 = e[9];
+    U.n_t1 = e[10];
     __syncwarp();
-    if (lane == 0) mbar_arrive(unit_empty + slot);
+    if (release && lane == 0) mbar_arrive(unit_empty + slot);
     return true;
+  };
+  auto release_unit = [&](int k) {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(unit_empty + k % UQ);
   };
 
   if (warp >= 8) {
@@ -417,14 +437,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int slot = k % UQ;
         if (k >= UQ) ok = mbar_wait(unit_empty + slot, ((k / UQ) - 1) & 1, p.err, p.timeout_ns);
         if (!__all_sync(0xffffffffu, ok)) break;
+        Unit U = {};
+        const int st = u >= 0 ? unit_info<VARLEN>(p, u, U) : 0;
         if (lane == 0) {
-          unit_q[slot] = u;
+          int4* e = reinterpret_cast<int4*>(unit_q + slot * C::UQ_INTS);
+          e[0] = make_int4(u, st, U.b, U.h);
+          e[1] = make_int4(U.g, U.tok0, U.seq_len, U.qt0);
+          e[2] = make_int4(U.qt1, U.n_t0, U.n_t1, 0);
           mbar_arrive(unit_full + slot);
         }
         __syncwarp();
         if (u < 0) break;
-        Unit U;
-        const int n_max = unit_info<VARLEN>(p, u, U) > 0 ? max(U.n_t0, U.n_t1) : 0;
+        const int n_max = st > 0 ? max(U.n_t0, U.n_t1) : 0;
         for (int j = 0; j < n_max; ++j) {
           if (j == p.stall_tile) {  // test-only: the waits on this tile must run out
             ok = false;
@@ -481,11 +505,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       int nq[2] = {0, 0};  // Q tiles loaded per slot
       for (int k = 0; ok; ++k) {
-        int u = -1;
-        ok = take_unit(k, u);
-        if (!ok || u < 0) break;
+        int u = -1, st = 0;
         Unit U;
-        if (unit_info<VARLEN>(p, u, U) <= 0) continue;
+        ok = take_unit(k, u, st, U);
+        if (!ok || u < 0) break;
+        if (st <= 0) continue;
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
           if ((t ? U.n_t1 : U.n_t0) == 0) continue;
@@ -600,11 +624,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         return r;
       };
       for (int k = 0; ok; ++k) {
-        int u = -1;
-        ok = take_unit(k, u);
-        if (!ok || u < 0) break;
+        int u = -1, st = 0;
         Unit U;
-        if (unit_info<VARLEN>(p, u, U) <= 0) continue;
+        ok = take_unit(k, u, st, U);
+        if (!ok || u < 0) break;
+        if (st <= 0) continue;
         const int n_max = max(U.n_t0, U.n_t1);
         auto nt = [&](int t) { return t == 0 ? U.n_t0 : U.n_t1; };
         if constexpr (FP8) {
@@ -732,17 +756,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       return __all_sync(0xffffffffu, r);
     };
     for (int k = 0; ok; ++k) {
-      int u = -1;
-      ok = take_unit(k, u);
-      if (!ok || u < 0) break;
+      // the unit's queue entry is kept until the end of its epilogue, which reads the
+      // head, batch and first token from it again (fewer values live through the tiles)
+      int u = -1, st = 0;
       Unit U;
-      const int st = unit_info<VARLEN>(p, u, U);
+      ok = take_unit(k, u, st, U, false);
+      if (!ok || u < 0) break;
       if (st < 0 && tid == 0) atomicCAS(p.err, DEV_OK, DEV_BAD_SEQLENS);
-      if (st <= 0) continue;
       const int n_t = t == 0 ? U.n_t0 : U.n_t1;
-      if (n_t == 0) continue;
+      if (st <= 0 || n_t == 0) {
+        release_unit(k);
+        continue;
+      }
       const int qt = t ? U.qt1 : U.qt0;
-      const int hs = hp ? U.h + t : U.h;            // this slot's query head
       const int q_pos = qt * BLOCK_M + r;           // query position in the sequence
       float ms = -INFINITY;  // BF16 reference max, scaled to log2 units
       int m_i = 0;           // FP8 reference max, code units
@@ -867,7 +893,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t e0 = static_cast<uint32_t>(120 - k0), e1 = static_cast<uint32_t>(120 - k1);
           const uint32_t sf_word = e0 | (e0 << 8) | (e1 << 16) | (e1 << 24);  // UE8M0 2^-(7+k)
           if constexpr (DUMP) {
-            const size_t row = (static_cast<size_t>(U.b) * p.Hq + hs) * p.S + q_pos;
+            const int* ue = unit_q + (k % UQ) * C::UQ_INTS;
+            const size_t row = (static_cast<size_t>(ue[2]) * p.Hq + (hp ? ue[3] + t : ue[3])) * p.S + q_pos;
             float* ds = p.dump_s + row * p.S + static_cast<size_t>(j) * BLOCK_N;
             uint8_t* dc = p.dump_codes + row * p.S + static_cast<size_t>(j) * BLOCK_N;
             for (int cc = 0; cc < BLOCK_N; ++cc) ds[cc] = s[cc];
@@ -986,6 +1013,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       // VARLEN: rows past the end of the sequence hold another sequence's queries (or zero
       // fill) and are not written
+      const int* ue = unit_q + (k % UQ) * C::UQ_INTS;
+      const int hs = hp ? ue[3] + t : ue[3];  // this slot's query head
+      U.b = ue[2];
+      U.tok0 = ue[5];
       const bool row_in = !VARLEN || q_pos < U.seq_len;
       const uint64_t pol_once = l2_policy_evict_first();  // O is written once
       const float2 inv2 = make_float2(inv, inv);
@@ -1052,6 +1083,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                               : (static_cast<size_t>(U.b) * p.Hq + hs) * p.S + q_pos;
         p.lse[li] = lse_v;
       }
+      release_unit(k);
     }
     // the O stores complete before the CTA exits (their source is this CTA's shared memory)
     if (TMA_O && o_issuer) bulk_wait_all();
