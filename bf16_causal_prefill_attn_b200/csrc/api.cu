@@ -214,9 +214,10 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, attn::FwdP
       !make_map(&mk, k, dt, C::E, DQK, prm.Hkv, T, C::BOX_COLS) ||
       !make_map(&mv, v, dt, C::E, attn::DV, prm.Hkv, T, C::BOX_COLS))
     return ATTN_ERR_CUDA;
-  // O [T, Hq, 128] bf16 in boxes of 64 columns x 128 rows (stored through shared memory)
+  // O [T, Hq, 128] bf16 in boxes of 64 columns x 128 rows (FP8) or 32 rows (BF16: one box
+  // per softmax warp), stored through shared memory
   if (C::TMA_O && !VARLEN) {
-    if (!make_map(&mo, prm.o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, attn::DV, prm.Hq, T, 64))
+    if (!make_map(&mo, prm.o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, attn::DV, prm.Hq, T, 64, C::O_BOX_ROWS))
       return ATTN_ERR_CUDA;
   } else {
     mo = mq;  // unused

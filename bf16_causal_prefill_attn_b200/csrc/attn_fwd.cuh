@@ -167,6 +167,11 @@ struct FwdCfg {
   // FP8 stages in P_t (free once the slot's last PV has completed); BF16 with d_qk = 128
   // has a staging area of its own; BF16 with d_qk = 192 has no room and stores rows directly
   static constexpr bool TMA_O = FP8 || DQK == 128;
+  // BF16: each softmax warp stores its own 32 rows (no warp waits for another; measured
+  // faster); FP8: one thread per slot stores 128 rows (the per-warp form measured slower
+  // there: the FP8 softmax sits at its register limit)
+  static constexpr bool WARP_O = !FP8;
+  static constexpr int O_BOX_ROWS = WARP_O ? 32 : 128;
   static constexpr int OFF_OST = OFF_P;                        // slot t at OFF_OST + t BOX_BYTES
   static constexpr int OFF_BAR = OFF_P + (TMA_O ? 2 * BOX_BYTES : 0);
   // barriers: k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], per slot q_full, q_empty,
@@ -288,7 +293,8 @@ __device__ __forceinline__ int cta_unit(int k) {
 // sum) is shared.
 // VARLEN: sequences of any length (packed, or a fixed S not a multiple of 128): keys past
 // the end of the sequence are masked, rows past it are not written.
-// tm_o: O [tokens, Hq, 128] bf16, boxes of 64 columns x 128 rows with the 128-byte swizzle
+// tm_o: O [tokens, Hq, 128] bf16, boxes of 64 columns x C::O_BOX_ROWS rows (FP8 128, BF16
+// 32) with the 128-byte swizzle
 // (used when C::TMA_O and not VARLEN).
 template <bool FP8, int DQK, bool DUMP, bool EXACT = false, bool VARLEN = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -352,7 +358,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(unit_empty + i, UNIT_CONSUMERS);
     }
     mbar_init(clc_bar, 1);
-    mbar_init(o_sync + 0, 4);
+    mbar_init(o_sync + 0, 4);  // FP8 only
     mbar_init(o_sync + 1, 4);
     fence_barrier_init();
   }
@@ -742,7 +748,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     bool ok = true;
     int c = 0;  // key tiles of this slot processed so far (all units)
     constexpr bool TMA_O = C::TMA_O && !VARLEN;
-    const bool o_issuer = (tid & 127) == 0;  // issues this slot's O stores
+    constexpr bool WARP_O = C::WARP_O;
+    // issues this slot's O stores (BF16: this warp's)
+    const bool o_issuer = WARP_O ? lane == 0 : (tid & 127) == 0;
     bool o_pending = false;  // FP8: a store from P_t may still be reading it
     int o_phase = 0;         // completed phases of o_sync(t)
     // the slot's four warps meet (bounded, so that a warp that has given up cannot leave the
@@ -972,11 +980,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ok = mbar_wait(pv_done(t), (c - 1) & 1, p.err, p.timeout_ns);
       if (!__all_sync(0xffffffffu, ok)) break;
       if constexpr (TMA_O && !FP8) {
-        // the staging buffer's previous store (the previous unit's second half) must have
-        // read it; waited for here, before O occupies the registers
+        // this warp's previous store from the staging buffer (the previous unit's second
+        // half) must have read its rows; waited for here, before O occupies the registers
         if (o_issuer) bulk_wait_read_all();
-        ok = slot_sync();
-        if (!ok) break;
+        __syncwarp();
       }
       tc_fence_after();
       uint32_t oraw[DV];
@@ -1023,16 +1030,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if constexpr (TMA_O) {
         // 64 columns at a time: row r's 128 bytes as 8 chunks at positions cc ^ (r mod 8) of
         // the slot's staging buffer (the tensor map's swizzle), then one thread stores the
-        // 128 x 64 box; rows of O are 8 KB apart, so per-thread row stores would touch a
-        // separate line per lane
+        // 128 x 64 box (BF16: lane 0 of each warp its 32 x 64 box, 4 KB and 1 KB aligned);
+        // rows of O are 8 KB apart, so per-thread row stores would touch a separate line
+        // per lane
+        const int wr = WARP_O ? (warp & 3) * 32 : 0;  // first row of the stored box
         uint8_t* ost = smem + C::OFF_OST + t * C::BOX_BYTES;
         const uint32_t srow = smem_addr(ost) + r * 128;
+        auto staging_sync = [&]() -> bool {
+          if constexpr (WARP_O) {
+            __syncwarp();
+            return true;
+          } else {
+            return slot_sync();
+          }
+        };
 #pragma unroll
         for (int h = 0; h < 2 && ok; ++h) {
           if (h == 1) {
             // the buffer's previous store (this unit's first half) must have read it
             if (o_issuer) bulk_wait_read_all();
-            ok = slot_sync();
+            ok = staging_sync();
             if (!ok) break;
           }
 #pragma unroll
@@ -1046,10 +1063,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                          pack_bf16x2(a2.x, a2.y), pack_bf16x2(a3.x, a3.y));
           }
           fence_proxy_async_smem();
-          ok = slot_sync();
+          ok = staging_sync();
           if (!ok) break;
           if (o_issuer) {
-            tma_store_3d_hint(&tm_o, ost, 64 * h, hs, U.tok0 + qt * BLOCK_M, pol_once);
+            tma_store_3d_hint(&tm_o, ost + wr * 128, 64 * h, hs, U.tok0 + qt * BLOCK_M + wr, pol_once);
             bulk_commit_group();
           }
         }
