@@ -5,6 +5,8 @@
 // (M = 256 over two SMs).  Every SM runs one CTA (or half a pair); operands are zeros (the
 // rate does not depend on the values).  Prints one JSON line per shape.
 //
+// Also: the round trip of a dependent MMA group (issue, commit, wait for the commit).
+//
 // Build and run: python -m bf16_causal_prefill_attn_b200.microbench.umma_rate
 #include <cuda_runtime.h>
 
@@ -137,6 +139,95 @@ __global__ void __launch_bounds__(128, 1) rate_kernel(long long* cycles, int ni)
   if (threadIdx.x == 0) cycles[blockIdx.x] = ok ? t : -1;
 }
 
+// Round trip of a dependent group: one thread issues G MMAs (K-major A and B from shared
+// memory) and a commit, waits for the commit's arrival, and repeats -- the latency an S MMA
+// group pays between its issue and the softmax seeing it.  Every wait is bounded (a second
+// in all); after a timeout the thread stops issuing and the MMAs in flight drain (again
+// bounded) before TMEM is released.
+template <int KIND, int N, int G>
+__global__ void __launch_bounds__(128, 1) lat_kernel(long long* cycles, int ni) {
+  extern __shared__ uint8_t raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + SMEM_BAR);
+  uint32_t* tptr = reinterpret_cast<uint32_t*>(smem + SMEM_BAR + 16);
+  const int warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < SMEM_BAR / 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(smem)[i] = make_uint4(0, 0, 0, 0);
+  fence_proxy_async_smem();
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    mbar_init(bar + 1, 1);
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tptr, 512);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tptr;
+  constexpr uint32_t IDESC = idesc_dense(KIND == 0 ? 1 : 0, KIND == 0 ? 1 : 0, 0, 0, 128, N);
+  const uint64_t ad = desc(smem_addr(smem + SMEM_A), 16, 1024);
+  const uint64_t bd = desc(smem_addr(smem + SMEM_B), 16, 1024);
+  long long t = 0;
+  bool ok = true;
+  if (threadIdx.x == 0) {
+    const uint64_t g0 = globaltimer_ns();
+    const long long t0 = clock64();
+    for (int i = 0; i < ni && ok; ++i) {
+      for (int g = 0; g < G; ++g) mma_ss<KIND>(tmem, ad, bd, IDESC, g > 0 ? 1u : 0u);
+      tc_commit(bar);
+      while (!mbar_try_wait(bar, static_cast<uint32_t>(i & 1))) {
+        if (globaltimer_ns() - g0 > 1000000000ull) {
+          ok = false;
+          break;
+        }
+      }
+    }
+    t = clock64() - t0;
+    tc_commit(bar + 1);
+    const uint64_t g1 = globaltimer_ns();
+    while (!mbar_try_wait(bar + 1, 0))
+      if (globaltimer_ns() - g1 > 1000000000ull) break;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+  if (threadIdx.x == 0) cycles[blockIdx.x] = ok ? t : -1;
+}
+
+template <int KIND, int N, int G>
+void run_lat(const char* name, int sms, int ni) {
+  auto k = lat_kernel<KIND, N, G>;
+  cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES + 1024);
+  long long* d = nullptr;
+  cudaMalloc(&d, sms * sizeof(long long));
+  for (int rep = 0; rep < 3; ++rep) k<<<sms, 128, SMEM_BYTES + 1024>>>(d, ni);
+  cudaDeviceSynchronize();
+  cudaError_t err = cudaGetLastError();
+  std::vector<long long> h(sms);
+  cudaMemcpy(h.data(), d, sms * sizeof(long long), cudaMemcpyDeviceToHost);
+  cudaFree(d);
+  double sum = 0;
+  int n = 0, bad = 0;
+  for (long long v : h) {
+    if (v > 0) {
+      sum += double(v);
+      ++n;
+    } else if (v < 0) {
+      ++bad;
+    }
+  }
+  const double cyc = n ? sum / n / ni : 0.0;
+  std::printf(
+      "{\"latency\": \"%s\", \"N\": %d, \"mmas_per_group\": %d, \"cycles_per_round_trip\": %.1f, "
+      "\"timeouts\": %d, \"error\": \"%s\"}\n",
+      name, N, G, cyc, bad, cudaGetErrorString(err));
+  std::fflush(stdout);
+}
+
 template <int CG, int KIND, bool ATM, int N, int BL>
 void run(const char* name, int sms, int ni) {
   auto k = rate_kernel<CG, KIND, ATM, N, BL>;
@@ -200,10 +291,17 @@ int main() {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, 0);
   const int ni = 4096;
   // S = Q K^T shapes (A, B K-major in shared memory)
+  // below N = 128: where the instruction stops being bound by its own work
+  run<1, 0, false, 16, 0>("bf16 QK^T", sms, ni);
+  run<1, 0, false, 32, 0>("bf16 QK^T", sms, ni);
+  run<1, 0, false, 64, 0>("bf16 QK^T", sms, ni);
   run<1, 0, false, 128, 0>("bf16 QK^T", sms, ni);
   run<1, 0, false, 256, 0>("bf16 QK^T", sms, ni);
   run<2, 0, false, 128, 0>("bf16 QK^T", sms, ni);
   run<2, 0, false, 256, 0>("bf16 QK^T", sms, ni);
+  run<1, 1, false, 16, 0>("e4m3 QK^T", sms, ni);
+  run<1, 1, false, 32, 0>("e4m3 QK^T", sms, ni);
+  run<1, 1, false, 64, 0>("e4m3 QK^T", sms, ni);
   run<1, 1, false, 128, 0>("e4m3 QK^T", sms, ni);
   run<1, 1, false, 256, 0>("e4m3 QK^T", sms, ni);
   run<2, 1, false, 128, 0>("e4m3 QK^T", sms, ni);
@@ -219,5 +317,11 @@ int main() {
   run<1, 2, false, 144, 1>("e4m3 block-scaled PV + row sum (single-CTA kernel)", sms, ni);
   run<2, 2, false, 128, 1>("e4m3 block-scaled PV", sms, ni);
   run<2, 2, false, 160, 2>("e4m3 block-scaled PV + row sum (pair kernel, 64-B swizzle)", sms, ni);
+  // dependent round trips: the S group of each kernel (d = 128) and its key halves
+  run_lat<0, 128, 8>("bf16 S group", sms, 1024);
+  run_lat<0, 64, 8>("bf16 S key half", sms, 1024);
+  run_lat<1, 128, 4>("e4m3 S group", sms, 1024);
+  run_lat<1, 64, 4>("e4m3 S key half", sms, 1024);
+  run_lat<0, 128, 1>("bf16 one MMA", sms, 1024);
   return 0;
 }
