@@ -27,6 +27,8 @@ ATTN_KERNEL_HEADS = 2
 ATTN_KERNEL_PERSISTENT = 4
 ATTN_KERNEL_DYNAMIC = 8
 ATTN_KERNEL_AUTO = 16
+ATTN_KERNEL_BF16_S_AHEAD = 32
+ATTN_KERNEL_BF16_P_OVER_S = 64
 
 _lib = None
 
@@ -309,8 +311,10 @@ def attn_select_prefill_kernel(kernel):
     query tiles of one head per unit) or ATTN_KERNEL_HEADS (one query tile of two heads of
     one kv group), optionally OR one schedule: ATTN_KERNEL_PERSISTENT (one CTA per SM
     running a static list of units) or ATTN_KERNEL_DYNAMIC (one CTA per unit; running CTAs
-    take over the units of CTAs not yet started); or ATTN_KERNEL_AUTO (the default:
-    dynamic, head pairs for FP8, tile pairs for BF16)."""
+    take over the units of CTAs not yet started), and for BF16 optionally OR one pipeline:
+    ATTN_KERNEL_BF16_S_AHEAD or ATTN_KERNEL_BF16_P_OVER_S (without one: S-ahead when
+    Hq > Hkv); or ATTN_KERNEL_AUTO (the default: dynamic, head pairs for FP8, tile pairs for
+    BF16, the BF16 pipeline by Hq / Hkv)."""
     _check(lib().attn_select_prefill_kernel(int(kernel)), "attn_select_prefill_kernel")
 
 

@@ -202,7 +202,7 @@ int sm_count() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-template <bool FP8, int DQK, bool DUMP, bool EXACT = false, bool VARLEN = false>
+template <bool FP8, int DQK, bool DUMP, bool EXACT, bool VARLEN, bool BSA>
 attn_status_t launch_fwd(const void* q, const void* k, const void* v, attn::FwdParams& prm,
                          cudaStream_t stream) {
   using C = attn::FwdCfg<FP8, DQK>;
@@ -222,7 +222,7 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, attn::FwdP
   } else {
     mo = mq;  // unused
   }
-  constexpr auto kern = attn::attn_fwd_kernel<FP8, DQK, DUMP, EXACT, VARLEN>;
+  constexpr auto kern = attn::attn_fwd_kernel<FP8, DQK, DUMP, EXACT, VARLEN, BSA>;
   if (!set_smem_attr<kern>(C::SMEM_ALLOC)) return ATTN_ERR_CUDA;
   const attn_status_t rs = register_split_ok<kern>();
   if (rs != ATTN_OK) return rs;
@@ -251,11 +251,23 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, attn::FwdP
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+// BF16 pipeline: the S-ahead one when selected, or by default with grouped-query heads
+// (Hq > Hkv: its earlier K loads are mostly L2 hits there; with as many kv heads as query
+// heads every CTA streams its own K and V, and the P-over-S pipeline measured faster)
+bool bf16_s_ahead(const attn::FwdParams& prm) {
+  if (g_kernel != ATTN_KERNEL_AUTO && (g_kernel & ATTN_KERNEL_BF16_S_AHEAD)) return true;
+  if (g_kernel != ATTN_KERNEL_AUTO && (g_kernel & ATTN_KERNEL_BF16_P_OVER_S)) return false;
+  return prm.Hq > prm.Hkv;
+}
+
 // The prefill kernel for one instantiation.
 template <bool FP8, int DQK, bool DUMP, bool EXACT = false, bool VARLEN = false>
 attn_status_t launch_prefill(const void* q, const void* k, const void* v, attn::FwdParams& prm,
                              cudaStream_t stream) {
-  return launch_fwd<FP8, DQK, DUMP, EXACT, VARLEN>(q, k, v, prm, stream);
+  if constexpr (!FP8) {
+    if (bf16_s_ahead(prm)) return launch_fwd<FP8, DQK, DUMP, EXACT, VARLEN, true>(q, k, v, prm, stream);
+  }
+  return launch_fwd<FP8, DQK, DUMP, EXACT, VARLEN, false>(q, k, v, prm, stream);
 }
 
 // Checks shared by the fixed-length and packed entry points; fills the parameters that
@@ -696,8 +708,10 @@ void attn_selftest_max_ctas(int n) { g_max_ctas = n > 0 ? n : 0; }
 
 attn_status_t attn_select_prefill_kernel(int kernel) {
   if (kernel != ATTN_KERNEL_AUTO &&
-      ((kernel & ~(ATTN_KERNEL_HEADS | ATTN_KERNEL_PERSISTENT | ATTN_KERNEL_DYNAMIC)) != 0 ||
-       ((kernel & ATTN_KERNEL_PERSISTENT) && (kernel & ATTN_KERNEL_DYNAMIC))))
+      ((kernel & ~(ATTN_KERNEL_HEADS | ATTN_KERNEL_PERSISTENT | ATTN_KERNEL_DYNAMIC |
+                   ATTN_KERNEL_BF16_S_AHEAD | ATTN_KERNEL_BF16_P_OVER_S)) != 0 ||
+       ((kernel & ATTN_KERNEL_PERSISTENT) && (kernel & ATTN_KERNEL_DYNAMIC)) ||
+       ((kernel & ATTN_KERNEL_BF16_S_AHEAD) && (kernel & ATTN_KERNEL_BF16_P_OVER_S))))
     return ATTN_ERR_INVALID_ARG;
   g_kernel = kernel;
   return ATTN_OK;

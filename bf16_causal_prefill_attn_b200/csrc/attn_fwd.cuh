@@ -28,24 +28,26 @@
 //   warps 0-3   softmax of tile 0, warps 4-7 softmax of tile 1: thread r of the group owns
 //               query row r (TMEM lane r); reads S, updates the reference max (lazily:
 //               only when the tile max exceeds it by more than the headroom), rescales O
-//               in TMEM when it does, writes P (BF16: into the S columns it has consumed;
-//               FP8: into shared memory, with its scale factors in TMEM), and finally
-//               writes O and lse;
+//               in TMEM when it does, writes P (BF16: into TMEM, over the S columns it has
+//               consumed or, S-ahead, into columns of its own; FP8: into shared memory,
+//               with its scale factors in TMEM), and finally writes O and lse;
 //   warp 8      TMA producer of K and V (NK / NV stages, continuing across units) and the
 //               CTA's scheduler (publishes each unit to the other roles);
 //   warp 9      MMA issuer (warp-wide control flow, one elected lane issues).  One tile's
-//               softmax overlaps the other tile's MMAs (ping-pong).  Order per key tile j:
-//                 BF16  PV_0(j), S_0(j+1), PV_1(j), S_1(j+1)  (P_t aliases S_t, so
-//                       S_t(j+1) must follow PV_t(j));
-//                 FP8   S_0(j+1), PV_0(j), S_1(j+1), PV_1(j)  (S_t(j+1) only needs S_t(j)
-//                       read into registers, so it runs during the softmax of S_t(j): each
-//                       softmax group then has a whole period, not half, for its tile);
-//   warp 10     FP8: PV MMA issuer (warp 9 then issues only the S MMAs); BF16: idle;
+//               softmax overlaps the other tile's MMAs (ping-pong).  Two pipelines:
+//                 S-ahead (FP8; BF16 with BSA): warp 9 issues S_t(j+1) as soon as both
+//                       slots have read their latest S (S_t(j+1) only needs S_t(j) read into
+//                       registers, so it runs during the softmax of S_t(j): each softmax
+//                       group has a whole period, not half, for its tile), warp 10 PV_t(j);
+//                 P over S (BF16 without BSA): warp 9 issues PV_0(j), S_0(j+1), PV_1(j),
+//                       S_1(j+1) (P_t aliases S_t, so S_t(j+1) must follow PV_t(j));
+//   warp 10     S-ahead: PV MMA issuer; otherwise idle;
 //   warp 11     TMEM allocator, then the Q loader: slot t's Q tile of the next unit as soon
 //               as the slot's last S MMA of the current unit has completed (q_empty).
 // TMEM (512 columns x 128 lanes, see TmemMap):
-//   BF16  S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512); P_t (bf16, 64
-//         columns) overwrites the first columns of S_t.
+//   BF16  P over S: S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512); P_t (bf16,
+//         64 columns) overwrites the first columns of S_t.  S-ahead: S [0,128) shared by
+//         both slots in turn, P_0 [128,192), P_1 [192,256), O_0 [256,384), O_1 [384,512).
 //   FP8   O_0 [0,144), O_1 [160,304): the PV MMA has N = 144, V extended by a 16-column
 //         block of ones, so columns 128..143 accumulate the row sum of the rounded P with
 //         the same block scales (the "extra matrix instruction" costs no extra issue);
@@ -70,11 +72,13 @@ constexpr int BLOCK_N = 128;
 constexpr int DV = 128;
 constexpr int NUM_THREADS = 384;
 // Registers per thread after setmaxnreg: warps 0-7 (softmax) and warps 8-11 (producer, MMA
-// issuers, Q loader), per precision -- the FP8 issuing warps need more for their unit
-// loop state, the BF16 softmax more for its exponentials (either way no spills)
-template <bool FP8> struct RegSplit {
-  static constexpr int SOFTMAX = FP8 ? 200 : 208;
-  static constexpr int OTHER = FP8 ? 104 : 88;
+// issuers, Q loader), per pipeline -- SAHEAD (the S MMAs a key tile ahead of the PV MMAs,
+// on an issuing warp of their own: FP8, and BF16 with BSA) needs more in the issuing warps
+// for their unit-loop state; the other (BF16: one warp issues PV_t(j) then S_t(j+1)) gives
+// the BF16 softmax more for its exponentials.  The d_qk = 128 kernels do not spill.
+template <bool SAHEAD> struct RegSplit {
+  static constexpr int SOFTMAX = SAHEAD ? 200 : 208;
+  static constexpr int OTHER = SAHEAD ? 104 : 88;
 };
 // registers per thread the launch must provide at least for either split
 constexpr int regs_needed_at_launch(int softmax, int other) {
@@ -87,11 +91,17 @@ constexpr int REGS_NEEDED_AT_LAUNCH =
         : regs_needed_at_launch(RegSplit<false>::SOFTMAX, RegSplit<false>::OTHER);
 static_assert(REGS_NEEDED_AT_LAUNCH * NUM_THREADS <= 65536, "register split exceeds the SM");
 // TMEM column map per precision (see the layout above)
-template <bool FP8>
+template <bool FP8, bool SAHEAD>
 struct TmemMap {
-  __host__ __device__ static constexpr uint32_t S(int t) { return FP8 ? 320u + 64u * t : 128u * t; }
+  // BF16 with SAHEAD: one S buffer for both slots (S_0 and S_1 alternate in it), P_t of its
+  // own; BF16 otherwise: S_t of its own, P_t written over the first 64 columns of S_t
+  __host__ __device__ static constexpr uint32_t S(int t) {
+    return FP8 ? 320u + 64u * t : (SAHEAD ? 0u : 128u * t);
+  }
   __host__ __device__ static constexpr uint32_t O(int t) { return FP8 ? 160u * t : 256u + 128u * t; }
-  __host__ __device__ static constexpr uint32_t P(int t) { return 128u * t; }     // BF16 only
+  __host__ __device__ static constexpr uint32_t P(int t) {  // BF16 only
+    return SAHEAD ? 128u + 64u * t : 128u * t;
+  }
   __host__ __device__ static constexpr uint32_t SFA(int t) { return 144u + 4u * t; }  // FP8, 4 columns
   static constexpr uint32_t SFB = 152;                         // FP8, 8 columns
   static constexpr uint32_t RS = 128;                          // row-sum column of O(t)
@@ -296,14 +306,19 @@ __device__ __forceinline__ int cta_unit(int k) {
 // tm_o: O [tokens, Hq, 128] bf16, boxes of 64 columns x C::O_BOX_ROWS rows (FP8 128, BF16
 // 32) with the 128-byte swizzle
 // (used when C::TMA_O and not VARLEN).
-template <bool FP8, int DQK, bool DUMP, bool EXACT = false, bool VARLEN = false>
+// BSA (BF16 only): the S-ahead pipeline of FP8 -- warp 9 issues S_t(j+1) as soon as both
+// slots have read their latest S (they alternate in one S buffer), warp 10 issues PV_t(j)
+// from P_t in TMEM columns of its own.  Without it one warp issues PV_t(j) then S_t(j+1)
+// (P_t is written over S_t).  Results are the same bits either way.
+template <bool FP8, int DQK, bool DUMP, bool EXACT = false, bool VARLEN = false, bool BSA = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_o, const FwdParams p) {
   using C = FwdCfg<FP8, DQK>;
-  using TM = TmemMap<FP8>;
+  constexpr bool SAHEAD = FP8 || BSA;
+  using TM = TmemMap<FP8, SAHEAD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -328,7 +343,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   void* clc_resp = smem + C::OFF_CLC;
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEMPTR);
   // warps that read the unit queue: the Q loader, the MMA warps and the softmax warps
-  constexpr int UNIT_CONSUMERS = 1 + (FP8 ? 2 : 1) + 8;
+  constexpr int UNIT_CONSUMERS = 1 + (SAHEAD ? 2 : 1) + 8;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -413,7 +428,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   };
 
   if (warp >= 8) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(RegSplit<FP8>::OTHER));
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(RegSplit<SAHEAD>::OTHER));
     // Q is read once (evicted first); K and V are read by every CTA of the kv group and
     // of later query tiles (kept in L2 longest)
     if (warp == 8) {
@@ -455,34 +470,43 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         __syncwarp();
         if (u < 0) break;
         const int n_max = st > 0 ? max(U.n_t0, U.n_t1) : 0;
-        for (int j = 0; j < n_max; ++j) {
-          if (j == p.stall_tile) {  // test-only: the waits on this tile must run out
-            ok = false;
-            break;
+        // K leads V by KLEAD tiles (BF16 S-ahead: 1): there S_t(j+1) needs K(j+1) about a tile
+        // before PV_t(j) needs V(j), and with two-stage rings a V load waiting for its slot
+        // would otherwise hold the next K load back
+        constexpr int KLEAD = (!FP8 && BSA) ? 1 : 0;
+        for (int i = 0; i < n_max + KLEAD; ++i) {
+          if (i < n_max) {
+            const int j = i;
+            if (j == p.stall_tile) {  // test-only: the waits on this tile must run out
+              ok = false;
+              break;
+            }
+            const int sk = gk % C::NK;
+            if (gk >= C::NK) ok = mbar_wait(k_empty + sk, ((gk / C::NK) - 1) & 1, p.err, p.timeout_ns);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            if (elect_one()) {
+              mbar_arrive_expect_tx(k_full + sk, C::K_BYTES);
+              for (int b = 0; b < C::Q_BOXES; ++b)
+                tma_load_3d_hint(smem + C::OFF_K + sk * C::K_BYTES + b * C::BOX_BYTES, &tm_k,
+                                 k_full + sk, b * C::BOX_COLS, U.g, U.tok0 + j * BLOCK_N, pol_keep);
+            }
+            __syncwarp();
+            ++gk;
           }
-          const int sk = gk % C::NK;
-          if (gk >= C::NK) ok = mbar_wait(k_empty + sk, ((gk / C::NK) - 1) & 1, p.err, p.timeout_ns);
-          if (!__all_sync(0xffffffffu, ok)) break;
-          if (elect_one()) {
-            mbar_arrive_expect_tx(k_full + sk, C::K_BYTES);
-            for (int i = 0; i < C::Q_BOXES; ++i)
-              tma_load_3d_hint(smem + C::OFF_K + sk * C::K_BYTES + i * C::BOX_BYTES, &tm_k,
-                               k_full + sk, i * C::BOX_COLS, U.g, U.tok0 + j * BLOCK_N, pol_keep);
+          if (i >= KLEAD) {
+            const int j = i - KLEAD;
+            const int sv = gv % C::NV;
+            if (gv >= C::NV) ok = mbar_wait(v_empty + sv, ((gv / C::NV) - 1) & 1, p.err, p.timeout_ns);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            if (elect_one()) {
+              mbar_arrive_expect_tx(v_full + sv, C::V_BYTES);
+              for (int b = 0; b < C::V_BOXES; ++b)
+                tma_load_3d_hint(smem + C::OFF_V + sv * C::V_BYTES + b * C::BOX_BYTES, &tm_v,
+                                 v_full + sv, b * C::BOX_COLS, U.g, U.tok0 + j * BLOCK_N, pol_keep);
+            }
+            __syncwarp();
+            ++gv;
           }
-          __syncwarp();
-          ++gk;
-          const int sv = gv % C::NV;
-          if (gv >= C::NV) ok = mbar_wait(v_empty + sv, ((gv / C::NV) - 1) & 1, p.err, p.timeout_ns);
-          if (!__all_sync(0xffffffffu, ok)) break;
-          if (elect_one()) {
-            mbar_arrive_expect_tx(v_full + sv, C::V_BYTES);
-            for (int i = 0; i < C::V_BOXES; ++i)
-              tma_load_3d_hint(smem + C::OFF_V + sv * C::V_BYTES + i * C::BOX_BYTES, &tm_v,
-                               v_full + sv, i * C::BOX_COLS, U.g, U.tok0 + j * BLOCK_N, pol_keep);
-          }
-          __syncwarp();
-          ++gv;
-          if (p.dynamic && j == n_max - 1) request();
         }
         if (!ok) break;
         if (p.dynamic) {
@@ -534,7 +558,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       for (int t = 0; t < 2; ++t)
         if (nq[t] > 0) mbar_wait(q_full(t), (nq[t] - 1) & 1, p.err, DRAIN_TIMEOUT_NS, false);
-    } else if (warp == 9 || (FP8 && warp == 10)) {
+    } else if (warp == 9 || (SAHEAD && warp == 10)) {
       // ----------------------------------------------------------- MMA issuers (warp-wide
       // control flow, one elected lane issues); the order per key tile is in the header.
       // FP8: warp 9 issues the S MMAs, warp 10 the PV MMAs (they touch disjoint TMEM
@@ -609,7 +633,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         __syncwarp();
       };
-      const bool s_issuer = warp == 9;  // FP8: S MMAs; BF16: all MMAs
+      const bool s_issuer = warp == 9;  // S MMAs (warp 10: PV MMAs)
       bool ok = true;
       int cs[2] = {0, 0};  // S MMAs issued per slot
       int cp[2] = {0, 0};  // PV MMAs issued per slot
@@ -620,8 +644,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       auto wait_k = [&](int g) {
         return mbar_wait(k_full + g % C::NK, (g / C::NK) & 1, p.err, p.timeout_ns);
       };
-      // FP8: before writing S_t, both slots must have read every S issued to them (S_0 and
-      // S_1 share 64 TMEM columns)
+      // before writing S_t, both slots must have read every S issued to them (S_0 and S_1
+      // share TMEM columns: 64 for FP8, all 128 for BF16)
       auto wait_reads = [&]() {
         bool r = true;
 #pragma unroll
@@ -637,7 +661,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (st <= 0) continue;
         const int n_max = max(U.n_t0, U.n_t1);
         auto nt = [&](int t) { return t == 0 ? U.n_t0 : U.n_t1; };
-        if constexpr (FP8) {
+        if constexpr (SAHEAD) {
           if (s_issuer) {
             // S_0(0), S_1(0), then S_t(j+1) in iteration j (this loop shape measured ~12%
             // faster than issuing S_t(j) in iteration j, with the same waits)
@@ -668,7 +692,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               }
             }
           } else {
-            // PV_t(j) once P_t(j) is in shared memory and V(j) has landed
+            // PV_t(j) once P_t(j) is written (FP8: shared memory; BF16: TMEM) and V(j) has
+            // landed
             for (int j = 0; j < n_max && ok; ++j) {
 #pragma unroll
               for (int t = 0; t < 2; ++t) {
@@ -727,7 +752,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_wait(mma_done(mine), 0, p.err, DRAIN_TIMEOUT_NS, false);
     }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(RegSplit<FP8>::SOFTMAX));
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(RegSplit<SAHEAD>::SOFTMAX));
     // ------------------------------------------------------------- softmax of slot t
     const int t = warp >> 2;
     const int r = tid & 127;                      // row within the tile == TMEM lane
@@ -789,8 +814,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) tmem_ld32(ts + cc * 32, sraw + cc * 32);
         tmem_wait_ld();
-        if constexpr (FP8) {
-          // S_t is in registers: the other slot may now overwrite the shared columns
+        if constexpr (SAHEAD) {
+          // S_t is in registers: the next S (of either slot) may now overwrite the columns
           tc_fence_before();
           mbar_arrive(s_read(t));
         }
@@ -908,9 +933,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           sf_w = sf_word;
         }
-        if constexpr (FP8) {
+        if constexpr (SAHEAD) {
           // S_t(j) may have been issued before PV_t(j-1): that PV must be complete before
-          // O_t is rescaled and before P_t and its scale factors are overwritten (the
+          // O_t is rescaled and before P_t (FP8: and its scale factors) is overwritten (the
           // previous unit's last PV was waited for by its epilogue)
           if (j > 0) {
             ok = mbar_wait(pv_done(t), (c - 1) & 1, p.err, p.timeout_ns);
@@ -918,8 +943,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tc_fence_after();
           }
         }
-        // BF16: the previous PV of this slot is complete here (S_t(j) was issued after it
-        // and has completed).  O_t (and the FP8 row sum) may be rescaled.
+        // O_t (and the FP8 row sum) may be rescaled (without SAHEAD, PV_t(j-1) has completed:
+        // S_t(j) was issued after it and has completed)
         if (__any_sync(0xffffffffu, alpha != 1.0f)) {
 #pragma unroll
           for (int cc = 0; cc < 4; ++cc) {

@@ -242,17 +242,29 @@ attn_status_t attn_device_status(void* stream);
  *                           finishes its unit takes over the unit of a CTA that has not
  *                           started yet (cluster launch control), so each SM keeps one CTA
  *                           running unit after unit.
- * Without a schedule flag every CTA runs one unit.  ATTN_KERNEL_AUTO (16, alone; the
- * default) is ATTN_KERNEL_DYNAMIC with head pairs for FP8 and tile pairs for BF16.  All
- * compute the same function (bitwise the same outputs and lean-P codes: a unit is computed
- * by the same code whichever CTA runs it).  A process-wide setting, for measurement and
- * tests; returns ATTN_ERR_INVALID_ARG for another value.
+ * Without a schedule flag every CTA runs one unit.  For BF16, at most one pipeline flag:
+ *   ATTN_KERNEL_BF16_S_AHEAD  (32) the pipeline of the FP8 kernel: one warp issues S_t(j+1)
+ *                             as soon as both slots have read their latest S (the two
+ *                             slots alternate in one S buffer in TMEM), another PV_t(j)
+ *                             from P_t in TMEM columns of its own;
+ *   ATTN_KERNEL_BF16_P_OVER_S (64) P_t written over the S_t columns it came from, one warp
+ *                             issuing PV_t(j) then S_t(j+1).
+ * Without one (and with ATTN_KERNEL_AUTO) BF16 uses S-ahead when Hq > Hkv, P-over-S when
+ * Hq == Hkv (measured faster there: with a kv head per query head the K/V tiles stream from
+ * HBM and S-ahead needs them earlier).  FP8 ignores the pipeline flags.  ATTN_KERNEL_AUTO
+ * (16, alone; the default) is ATTN_KERNEL_DYNAMIC with head pairs for FP8 and tile pairs
+ * for BF16.  All compute the same function (bitwise the same outputs and lean-P codes: a
+ * unit is computed by the same code whichever CTA runs it, and both BF16 pipelines issue the
+ * same MMAs in the same order per slot).  A process-wide setting, for measurement and tests;
+ * returns ATTN_ERR_INVALID_ARG for another value.
  */
 #define ATTN_KERNEL_SINGLE 0
 #define ATTN_KERNEL_HEADS 2
 #define ATTN_KERNEL_PERSISTENT 4
 #define ATTN_KERNEL_DYNAMIC 8
 #define ATTN_KERNEL_AUTO 16
+#define ATTN_KERNEL_BF16_S_AHEAD 32
+#define ATTN_KERNEL_BF16_P_OVER_S 64
 attn_status_t attn_select_prefill_kernel(int kernel);
 
 /* Test-only: sets the bounded-wait limit in nanoseconds (0 restores the default, 2 s). */

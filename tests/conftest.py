@@ -33,6 +33,11 @@ KERNELS = {"single": (("ATTN_KERNEL_SINGLE",), 0),
            "persistent": (("ATTN_KERNEL_SINGLE", "ATTN_KERNEL_PERSISTENT"), 5),
            "heads_persistent": (("ATTN_KERNEL_HEADS", "ATTN_KERNEL_PERSISTENT"), 3),
            "dynamic": (("ATTN_KERNEL_SINGLE", "ATTN_KERNEL_DYNAMIC"), 0),
+           # both BF16 pipelines on every shape (without a flag the pipeline follows Hq / Hkv)
+           "dynamic_bf16_s_ahead": (("ATTN_KERNEL_SINGLE", "ATTN_KERNEL_DYNAMIC",
+                                     "ATTN_KERNEL_BF16_S_AHEAD"), 0),
+           "persistent_bf16_p_over_s": (("ATTN_KERNEL_SINGLE", "ATTN_KERNEL_PERSISTENT",
+                                         "ATTN_KERNEL_BF16_P_OVER_S"), 5),
            "auto": (("ATTN_KERNEL_AUTO",), 0)}
 
 

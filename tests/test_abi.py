@@ -173,18 +173,21 @@ def test_built_library_is_newer_than_every_source(L):
 
 
 def test_prefill_kernel_selection_validated(L):
-    """Units and schedules combine by OR; both schedule flags at once, or an unknown bit,
-    are rejected (no GPU call is made)."""
+    """Units, schedules and the BF16 pipeline combine by OR; both schedule flags or both
+    pipeline flags at once, or an unknown bit, are rejected (no GPU call is made)."""
     import bf16_causal_prefill_attn_b200 as pkg
     good = [pkg.ATTN_KERNEL_SINGLE, pkg.ATTN_KERNEL_HEADS,
             pkg.ATTN_KERNEL_PERSISTENT, pkg.ATTN_KERNEL_HEADS | pkg.ATTN_KERNEL_PERSISTENT,
             pkg.ATTN_KERNEL_DYNAMIC, pkg.ATTN_KERNEL_HEADS | pkg.ATTN_KERNEL_DYNAMIC,
-            pkg.ATTN_KERNEL_AUTO]
+            pkg.ATTN_KERNEL_AUTO, pkg.ATTN_KERNEL_BF16_S_AHEAD,
+            pkg.ATTN_KERNEL_BF16_P_OVER_S | pkg.ATTN_KERNEL_HEADS | pkg.ATTN_KERNEL_DYNAMIC]
     try:
         for k in good:
             assert L.attn_select_prefill_kernel(k) == pkg.ATTN_OK
-        for bad in (pkg.ATTN_KERNEL_PERSISTENT | pkg.ATTN_KERNEL_DYNAMIC, 1, 32, -1,
-                    pkg.ATTN_KERNEL_AUTO | pkg.ATTN_KERNEL_HEADS):
+        for bad in (pkg.ATTN_KERNEL_PERSISTENT | pkg.ATTN_KERNEL_DYNAMIC, 1, 128, -1,
+                    pkg.ATTN_KERNEL_AUTO | pkg.ATTN_KERNEL_HEADS,
+                    pkg.ATTN_KERNEL_AUTO | pkg.ATTN_KERNEL_BF16_S_AHEAD,
+                    pkg.ATTN_KERNEL_BF16_S_AHEAD | pkg.ATTN_KERNEL_BF16_P_OVER_S):
             assert L.attn_select_prefill_kernel(bad) == pkg.ATTN_ERR_INVALID_ARG
     finally:
         L.attn_select_prefill_kernel(pkg.ATTN_KERNEL_AUTO)

@@ -103,3 +103,48 @@ def test_persistent_dump_equals_one_cta_per_unit():
         _same(_run(fn, pkg.ATTN_KERNEL_SINGLE | pkg.ATTN_KERNEL_PERSISTENT, cap), ref)
     _same(_run(fn, pkg.ATTN_KERNEL_SINGLE | pkg.ATTN_KERNEL_DYNAMIC, 0), ref)
 
+
+
+@pytest.mark.parametrize("B,S,Hq,Hkv,dqk,causal", [
+    (2, 640, 4, 2, 128, True),      # grouped heads (S-ahead by default), odd tile count
+    (2, 512, 4, 4, 128, True),      # a kv head per query head (P over S by default)
+    (1, 512, 4, 4, 192, True),      # MLA head dimension
+    (3, 384, 6, 2, 128, False),     # full attention, G = 3
+    (8, 1024, 8, 2, 128, True),     # more units than SMs
+])
+def test_bf16_pipelines_equal(B, S, Hq, Hkv, dqk, causal):
+    """The two BF16 pipelines (S ahead of PV on its own warp, P in TMEM columns of its own;
+    P written over S, PV then S from one warp) issue the same MMAs in the same order per
+    slot on the same P: outputs and lse are bitwise identical, on every unit and schedule."""
+    q, k, v = [t.cuda() for t in synth.make_qkv(B, S, Hq, Hkv, dqk, 128, seed=S + 7 * Hq, dist="outlier")]
+    fn = lambda: pkg.attn_fwd(q, k, v, causal=causal)
+    ref = _run(fn, pkg.ATTN_KERNEL_SINGLE | pkg.ATTN_KERNEL_BF16_P_OVER_S, 0)
+    for u in (pkg.ATTN_KERNEL_SINGLE, pkg.ATTN_KERNEL_HEADS):
+        for pipe in (pkg.ATTN_KERNEL_BF16_S_AHEAD, pkg.ATTN_KERNEL_BF16_P_OVER_S):
+            _same(_run(fn, u | pipe, 0), ref)
+            _same(_run(fn, u | pipe | pkg.ATTN_KERNEL_DYNAMIC, 0), ref)
+            for cap in (1, 3):
+                _same(_run(fn, u | pipe | pkg.ATTN_KERNEL_PERSISTENT, cap), ref)
+    _same(_run(fn, pkg.ATTN_KERNEL_AUTO, 0), ref)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(4, 2), (4, 4)])
+def test_bf16_pipelines_equal_varlen(Hq, Hkv):
+    """The same for packed sequences with empty, one-token and ragged members."""
+    lengths = [129, 1, 300, 0, 128, 64, 513, 127, 0, 700] * 3
+    lead, tail = 16, 40
+    T = lead + sum(lengths) + tail
+    q, k, v = [t[0].cuda() for t in synth.make_qkv(1, T, Hq, Hkv, 128, 128, seed=9, dist="gaussian")]
+    cu = torch.from_numpy(np.concatenate([[lead], lead + np.cumsum(lengths)]).astype(np.int32)).cuda()
+
+    def fn():
+        o = torch.full((T, Hq, 128), 7.0, dtype=torch.bfloat16, device="cuda")
+        lse = torch.full((Hq, T), 7.0, dtype=torch.float32, device="cuda")
+        pkg.attn_fwd_varlen(q, k, v, cu, max(lengths), causal=True, out=o, lse=lse)
+        return o, lse
+
+    ref = _run(fn, pkg.ATTN_KERNEL_SINGLE | pkg.ATTN_KERNEL_BF16_P_OVER_S, 0)
+    for pipe in (pkg.ATTN_KERNEL_BF16_S_AHEAD, pkg.ATTN_KERNEL_BF16_P_OVER_S):
+        for u in (pkg.ATTN_KERNEL_SINGLE, pkg.ATTN_KERNEL_HEADS):
+            _same(_run(fn, u | pipe | pkg.ATTN_KERNEL_DYNAMIC, 0), ref)
+            _same(_run(fn, u | pipe | pkg.ATTN_KERNEL_PERSISTENT, 2), ref)
