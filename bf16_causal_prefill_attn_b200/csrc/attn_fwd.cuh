@@ -470,13 +470,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         __syncwarp();
         if (u < 0) break;
         const int n_max = st > 0 ? max(U.n_t0, U.n_t1) : 0;
-        // K leads V by KLEAD tiles (BF16 S-ahead: 1): there S_t(j+1) needs K(j+1) about a tile
-        // before PV_t(j) needs V(j), and with two-stage rings a V load waiting for its slot
-        // would otherwise hold the next K load back
-        constexpr int KLEAD = (!FP8 && BSA) ? 1 : 0;
-        for (int i = 0; i < n_max + KLEAD; ++i) {
-          if (i < n_max) {
-            const int j = i;
+        if constexpr (FP8 || !BSA) {
+          for (int j = 0; j < n_max; ++j) {
             if (j == p.stall_tile) {  // test-only: the waits on this tile must run out
               ok = false;
               break;
@@ -486,26 +481,63 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (!__all_sync(0xffffffffu, ok)) break;
             if (elect_one()) {
               mbar_arrive_expect_tx(k_full + sk, C::K_BYTES);
-              for (int b = 0; b < C::Q_BOXES; ++b)
-                tma_load_3d_hint(smem + C::OFF_K + sk * C::K_BYTES + b * C::BOX_BYTES, &tm_k,
-                                 k_full + sk, b * C::BOX_COLS, U.g, U.tok0 + j * BLOCK_N, pol_keep);
+              for (int i = 0; i < C::Q_BOXES; ++i)
+                tma_load_3d_hint(smem + C::OFF_K + sk * C::K_BYTES + i * C::BOX_BYTES, &tm_k,
+                                 k_full + sk, i * C::BOX_COLS, U.g, U.tok0 + j * BLOCK_N, pol_keep);
             }
             __syncwarp();
             ++gk;
-          }
-          if (i >= KLEAD) {
-            const int j = i - KLEAD;
             const int sv = gv % C::NV;
             if (gv >= C::NV) ok = mbar_wait(v_empty + sv, ((gv / C::NV) - 1) & 1, p.err, p.timeout_ns);
             if (!__all_sync(0xffffffffu, ok)) break;
             if (elect_one()) {
               mbar_arrive_expect_tx(v_full + sv, C::V_BYTES);
-              for (int b = 0; b < C::V_BOXES; ++b)
-                tma_load_3d_hint(smem + C::OFF_V + sv * C::V_BYTES + b * C::BOX_BYTES, &tm_v,
-                                 v_full + sv, b * C::BOX_COLS, U.g, U.tok0 + j * BLOCK_N, pol_keep);
+              for (int i = 0; i < C::V_BOXES; ++i)
+                tma_load_3d_hint(smem + C::OFF_V + sv * C::V_BYTES + i * C::BOX_BYTES, &tm_v,
+                                 v_full + sv, i * C::BOX_COLS, U.g, U.tok0 + j * BLOCK_N, pol_keep);
             }
             __syncwarp();
             ++gv;
+            if (p.dynamic && j == n_max - 1) request();
+          }
+        } else {
+          // BF16 S-ahead: K leads V by a tile.  S_t(j+1) needs K(j+1) about a tile
+          // before PV_t(j) needs V(j), and with two-stage rings a V load waiting for its slot
+          // would otherwise hold the next K load back
+          constexpr int KLEAD = 1;
+          for (int i = 0; i < n_max + KLEAD; ++i) {
+            if (i < n_max) {
+              const int j = i;
+              if (j == p.stall_tile) {  // test-only: the waits on this tile must run out
+                ok = false;
+                break;
+              }
+              const int sk = gk % C::NK;
+              if (gk >= C::NK) ok = mbar_wait(k_empty + sk, ((gk / C::NK) - 1) & 1, p.err, p.timeout_ns);
+              if (!__all_sync(0xffffffffu, ok)) break;
+              if (elect_one()) {
+                mbar_arrive_expect_tx(k_full + sk, C::K_BYTES);
+                for (int b = 0; b < C::Q_BOXES; ++b)
+                  tma_load_3d_hint(smem + C::OFF_K + sk * C::K_BYTES + b * C::BOX_BYTES, &tm_k,
+                                   k_full + sk, b * C::BOX_COLS, U.g, U.tok0 + j * BLOCK_N, pol_keep);
+              }
+              __syncwarp();
+              ++gk;
+            }
+            if (i >= KLEAD) {
+              const int j = i - KLEAD;
+              const int sv = gv % C::NV;
+              if (gv >= C::NV) ok = mbar_wait(v_empty + sv, ((gv / C::NV) - 1) & 1, p.err, p.timeout_ns);
+              if (!__all_sync(0xffffffffu, ok)) break;
+              if (elect_one()) {
+                mbar_arrive_expect_tx(v_full + sv, C::V_BYTES);
+                for (int b = 0; b < C::V_BOXES; ++b)
+                  tma_load_3d_hint(smem + C::OFF_V + sv * C::V_BYTES + b * C::BOX_BYTES, &tm_v,
+                                   v_full + sv, b * C::BOX_COLS, U.g, U.tok0 + j * BLOCK_N, pol_keep);
+              }
+              __syncwarp();
+              ++gv;
+            }
           }
         }
         if (!ok) break;
