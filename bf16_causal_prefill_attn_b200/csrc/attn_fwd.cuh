@@ -75,7 +75,7 @@ constexpr int NUM_THREADS = 384;
 // issuers, Q loader), per pipeline -- SAHEAD (the S MMAs a key tile ahead of the PV MMAs,
 // on an issuing warp of their own: FP8, and BF16 with BSA) needs more in the issuing warps
 // for their unit-loop state; the other (BF16: one warp issues PV_t(j) then S_t(j+1)) gives
-// the BF16 softmax more for its exponentials.  The d_qk = 128 kernels do not spill.
+// the BF16 softmax more for its exponentials.
 template <bool SAHEAD> struct RegSplit {
   static constexpr int SOFTMAX = SAHEAD ? 200 : 208;
   static constexpr int OTHER = SAHEAD ? 104 : 88;
