@@ -49,6 +49,12 @@ KERNEL_IDS = {"auto": lambda pkg: pkg.ATTN_KERNEL_AUTO,
               "single-dynamic": lambda pkg: pkg.ATTN_KERNEL_SINGLE | pkg.ATTN_KERNEL_DYNAMIC,
               "heads-dynamic": lambda pkg: pkg.ATTN_KERNEL_HEADS | pkg.ATTN_KERNEL_DYNAMIC}
 
+def bf16_pipeline(Hq, Hkv):
+    """The BF16 prefill pipeline the library picks when no pipeline flag is selected (the
+    bench selects none): S-ahead with grouped-query heads, P over S otherwise."""
+    return "S-ahead" if Hq > Hkv else "P over S"
+
+
 WORKLOADS = {
     # name: (B, S, Hq, Hkv, d_qk, d_v, distribution, description)
     "small_s256": (1, 256, 1, 1, 128, 128, "gaussian",
@@ -562,6 +568,7 @@ def gpu_bench(args, rank, world, local_rank):
                               "frac": round(bf16_kern_tf / bf16_peak, 4),
                               "peak_source": f"{peak_src} bf16 cuBLAS burst",
                               "frac_of_nominal_2250": round(bf16_kern_tf / NOMINAL_BF16_TFLOPS, 4),
+                              "kernel": f"attn_fwd_kernel<bf16>, {bf16_pipeline(Hq, Hkv)} pipeline",
                               "kernel_ms": round(bf16_kern, 4),
                               "kernel_ms_median": round(statistics.median(bf16_kern_ms), 4),
                               "kernel_ms_min": round(min(bf16_kern_ms), 4),
@@ -655,7 +662,8 @@ def headline_extras(args, dev, peaks, peak_src):
                                           "peak": round(bf16_peak, 1), "unit": "TFLOP/s",
                                           "frac": round(tfb / bf16_peak, 4),
                                           "frac_of_nominal_2250": round(tfb / NOMINAL_BF16_TFLOPS, 4),
-                                          "peak_source": f"{peak_src} bf16 cuBLAS burst"}}
+                                          "peak_source": f"{peak_src} bf16 cuBLAS burst",
+                                          "kernel": f"attn_fwd_kernel<bf16>, {bf16_pipeline(Hq, Hkv)} pipeline"}}
         out[name] = entry
         del q, k, v, q8, k8, v8, o, lse
         torch.cuda.empty_cache()
